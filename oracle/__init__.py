@@ -1,0 +1,58 @@
+"""Plain fp64 CPU oracle for exact blockwise ring attention and the blockwise FFN.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import this package:
+only the test-suite, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` use it.  It shares no code with the
+CUDA library (no kernels, headers, helpers, tables or constants) and imports
+nothing from ``exact_blockwise_long_b200``.
+
+What it computes follows the pages on Ring Attention:
+
+* "Ring Attention with Blockwise Transformers for Near-Infinite Context"
+  (paper abstract): blockwise self-attention and feed-forward, exact, "without
+  resorting to approximations".
+* chapterpal keyword page "Ring Attention" (definition paragraph): the
+  sequence is partitioned into blocks, each block keeps its queries while the
+  key/value blocks circulate around a ring.
+* darcstar.tech research note on the same paper, "DarcStar commentary",
+  paragraphs one and two: online softmax is associative, partial attention of
+  separate shards combines exactly; the causal mask and the softmax
+  denominator must be combined across chunks exactly.
+
+Every function here is either the plain mathematical definition (full-matrix
+softmax attention, its gradient, a SwiGLU feed-forward) or the method's steps
+written out in the pages' terms (shards, ring order, chunk tiles, log-sum-exp
+merge) for pinning the definition against the method.
+
+Parity status per function (what pins it is in ``tests/test_oracle.py``):
+
+* ``attention_forward``          pinned (hand-derived golden values, closed
+                                 forms, brute force, scipy softmax/logsumexp)
+* ``attention_backward``         pinned (central finite differences, shift and
+                                 homogeneity invariants)
+* ``ring_blockwise_forward``     pinned (equals the full matrix for every S
+                                 and chunk size, order invariant)
+* ``lse_merge``                  pinned (closed form of two-part softmax,
+                                 associativity, neutral element)
+* ``attention_rows`` / ``attention_backward_key_rows`` /
+  ``attention_backward_query_rows``
+                                 pinned (equal to the full functions on the
+                                 sampled subset)
+* ``swiglu_ffn`` / ``blockwise_ffn``
+                                 pinned (zero inputs, chunk invariance,
+                                 explicit loop, scipy expit)
+"""
+
+from .attention import (  # noqa: F401
+    attention_forward,
+    attention_backward,
+    ring_blockwise_forward,
+    ring_blockwise_step,
+    lse_merge,
+    attention_rows,
+    attention_backward_query_rows,
+    attention_backward_key_rows,
+    ring_visit_order,
+    ring_visit_order_bwd,
+)
+from .ffn import swiglu_ffn, blockwise_ffn, silu  # noqa: F401

@@ -1,0 +1,396 @@
+"""Pins for the fp64 oracle: each check is fixed by the pages or by mathematics,
+not by re-running the oracle's own formula.
+
+* hand-derived golden values (tests/golden/*.txt)
+* closed forms: q = 0 gives mean(V) and lse = ln N; causal row 0 gives v_0
+* library routines: scipy.special.softmax / logsumexp / expit
+* brute force with explicit Python loops on tiny inputs
+* the method itself: ring/blockwise result equals the full matrix for every
+  S and chunk size, in any ring visiting order, and the step partials merge
+  to it in any order
+* gradients: central finite differences, shift and homogeneity invariants
+"""
+
+import itertools
+import math
+
+import numpy as np
+import pytest
+import scipy.special
+
+import oracle
+from golden_io import golden_path, load, stack
+
+
+def _rand(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+# ---------------------------------------------------------------------------
+# Golden worked examples
+# ---------------------------------------------------------------------------
+
+def _hand_attention():
+    g = load(golden_path("attention_hand.txt"))
+    q = stack(g, "q", 3)[None, None]
+    k = stack(g, "k", 3)[None, None]
+    v = stack(g, "v", 3)[None, None]
+    do = stack(g, "do", 3)[None, None]
+    return g, q, k, v, do
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_golden_forward(causal):
+    g, q, k, v, _ = _hand_attention()
+    o, lse = oracle.attention_forward(q, k, v, causal)
+    p = "c_" if causal else "nc_"
+    np.testing.assert_allclose(o[0, 0], stack(g, p + "o", 3), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse[0, 0], g[p + "lse"], rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_golden_backward(causal):
+    g, q, k, v, do = _hand_attention()
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, causal)
+    p = "c_" if causal else "nc_"
+    np.testing.assert_allclose(dq[0, 0], stack(g, p + "dq", 3), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dk[0, 0], stack(g, p + "dk", 3), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dv[0, 0], stack(g, p + "dv", 3), rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_golden_ring_blockwise(causal):
+    g, q, k, v, _ = _hand_attention()
+    # N = 3: three shards of one token each, chunks of one token.
+    o, lse = oracle.ring_blockwise_forward(q, k, v, S=3, q_chunk=1, k_chunk=1, causal=causal)
+    p = "c_" if causal else "nc_"
+    np.testing.assert_allclose(o[0, 0], stack(g, p + "o", 3), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse[0, 0], g[p + "lse"], rtol=0, atol=1e-13)
+
+
+def test_golden_wrong_scale_is_caught():
+    """A dropped softmax scale (a plausible slip) moves the golden values."""
+    g, q, k, v, _ = _hand_attention()
+    o, _ = oracle.attention_forward(q, k, v, False, scale=1.0)
+    assert np.abs(o[0, 0] - stack(g, "nc_o", 3)).max() > 0.1
+
+
+def test_golden_ffn():
+    g = load(golden_path("ffn_hand.txt"))
+    x = stack(g, "x", 2)
+    w1 = stack(g, "w1_", 2)
+    w3 = stack(g, "w3_", 2)
+    w2 = stack(g, "w2_", 2)
+    y = oracle.swiglu_ffn(x, w1, w2, w3)
+    np.testing.assert_allclose(y, stack(g, "y", 2), rtol=0, atol=1e-13)
+    yb = oracle.blockwise_ffn(x, w1, w2, w3, chunk=1)
+    np.testing.assert_allclose(yb, stack(g, "y", 2), rtol=0, atol=1e-13)
+    # swapping the gate and up weights (a plausible slip) is caught
+    assert np.abs(oracle.swiglu_ffn(x, w3, w2, w1) - stack(g, "y", 2)).max() > 0.1
+
+
+# ---------------------------------------------------------------------------
+# Closed forms and library routines
+# ---------------------------------------------------------------------------
+
+def test_zero_query_gives_mean_of_v():
+    B, H, N, d = 2, 3, 37, 8
+    q = np.zeros((B, H, N, d))
+    k = _rand((B, H, N, d), 1)
+    v = _rand((B, H, N, d), 2)
+    o, lse = oracle.attention_forward(q, k, v, causal=False)
+    np.testing.assert_allclose(o, np.broadcast_to(v.mean(axis=2, keepdims=True), o.shape), atol=1e-13)
+    np.testing.assert_allclose(lse, np.log(N), atol=1e-13)
+
+
+def test_zero_query_causal_gives_prefix_mean():
+    N, d = 23, 4
+    q = np.zeros((1, 1, N, d))
+    k = _rand((1, 1, N, d), 3)
+    v = _rand((1, 1, N, d), 4)
+    o, lse = oracle.attention_forward(q, k, v, causal=True)
+    prefix = np.cumsum(v[0, 0], axis=0) / np.arange(1, N + 1)[:, None]
+    np.testing.assert_allclose(o[0, 0], prefix, atol=1e-13)
+    np.testing.assert_allclose(lse[0, 0], np.log(np.arange(1, N + 1)), atol=1e-13)
+
+
+def test_causal_row0_is_v0():
+    B, H, N, d = 2, 2, 16, 8
+    q, k, v = _rand((B, H, N, d), 5), _rand((B, H, N, d), 6), _rand((B, H, N, d), 7)
+    o, lse = oracle.attention_forward(q, k, v, causal=True)
+    np.testing.assert_allclose(o[:, :, 0], v[:, :, 0], atol=1e-14)
+    s00 = (q[:, :, 0] * k[:, :, 0]).sum(-1) / np.sqrt(d)
+    np.testing.assert_allclose(lse[:, :, 0], s00, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_matches_scipy_softmax(causal):
+    B, H, N, d = 1, 2, 40, 16
+    q, k, v = _rand((B, H, N, d), 8), _rand((B, H, N, d), 9, 2.0), _rand((B, H, N, d), 10)
+    o, lse = oracle.attention_forward(q, k, v, causal)
+    for h in range(H):
+        s = q[0, h] @ k[0, h].T / math.sqrt(d)
+        if causal:
+            s = np.where(np.tril(np.ones((N, N), bool)), s, -np.inf)
+        p = scipy.special.softmax(s, axis=1)
+        np.testing.assert_allclose(o[0, h], p @ v[0, h], atol=1e-12)
+        np.testing.assert_allclose(lse[0, h], scipy.special.logsumexp(s, axis=1), atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_brute_force_loops(causal):
+    """Explicit enumeration of visible pairs with math.exp, no arrays."""
+    N, d = 7, 3
+    q, k, v = _rand((1, 1, N, d), 11), _rand((1, 1, N, d), 12), _rand((1, 1, N, d), 13)
+    o, lse = oracle.attention_forward(q, k, v, causal)
+    sc = 1.0 / math.sqrt(d)
+    for i in range(N):
+        pairs = [j for j in range(N) if (j <= i or not causal)]
+        w = [math.exp(sc * sum(q[0, 0, i, c] * k[0, 0, j, c] for c in range(d))) for j in pairs]
+        tot = sum(w)
+        for c in range(d):
+            ref = sum(wj * v[0, 0, j, c] for wj, j in zip(w, pairs)) / tot
+            assert abs(o[0, 0, i, c] - ref) < 1e-13
+        assert abs(lse[0, 0, i] - math.log(tot)) < 1e-13
+
+
+def test_sharp_scores_select_argmax():
+    """A key aligned with the query and 100x longer dominates the softmax."""
+    N, d = 16, 8
+    rng = np.random.default_rng(14)
+    q = rng.standard_normal((1, 1, N, d))
+    k = rng.standard_normal((1, 1, N, d)) * 0.01
+    v = rng.standard_normal((1, 1, N, d))
+    k[0, 0, 5] = 100.0 * q[0, 0, 9] / np.linalg.norm(q[0, 0, 9])
+    o, _ = oracle.attention_forward(q, k, v, causal=False)
+    np.testing.assert_allclose(o[0, 0, 9], v[0, 0, 5], atol=1e-8)
+
+
+def test_causal_locality():
+    """Row i depends only on keys/values j <= i."""
+    B, H, N, d = 1, 2, 24, 8
+    q, k, v = _rand((B, H, N, d), 15), _rand((B, H, N, d), 16), _rand((B, H, N, d), 17)
+    o1, l1 = oracle.attention_forward(q, k, v, causal=True)
+    i = 10
+    k2, v2 = k.copy(), v.copy()
+    k2[:, :, i + 1:] += 5.0
+    v2[:, :, i + 1:] -= 3.0
+    o2, l2 = oracle.attention_forward(q, k2, v2, causal=True)
+    np.testing.assert_array_equal(o1[:, :, : i + 1], o2[:, :, : i + 1])
+    np.testing.assert_array_equal(l1[:, :, : i + 1], l2[:, :, : i + 1])
+    assert np.abs(o1[:, :, i + 1:] - o2[:, :, i + 1:]).max() > 1e-3
+
+
+# ---------------------------------------------------------------------------
+# The method against the definition
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("S", [1, 2, 4, 8, 16])
+def test_ring_blockwise_equals_full(S, causal):
+    B, H, N, d = 1, 2, 64, 8
+    q, k, v = _rand((B, H, N, d), 18), _rand((B, H, N, d), 19, 2.0), _rand((B, H, N, d), 20)
+    o_ref, l_ref = oracle.attention_forward(q, k, v, causal)
+    L = N // S
+    chunks = [c for c in (1, 2, 4, 8, 16, 32, 64) if L % c == 0]
+    for qc, kc in itertools.product(chunks, chunks):
+        if qc < L // 4 and kc < L // 4 and L > 8:
+            continue  # keep the sweep small; tiny chunks are covered at small L
+        o, lse = oracle.ring_blockwise_forward(q, k, v, S, qc, kc, causal)
+        np.testing.assert_allclose(o, o_ref, atol=1e-12, rtol=0)
+        np.testing.assert_allclose(lse, l_ref, atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_order_invariance(causal):
+    B, H, N, d, S = 1, 1, 48, 4, 6
+    q, k, v = _rand((B, H, N, d), 21), _rand((B, H, N, d), 22), _rand((B, H, N, d), 23)
+    o_ref, l_ref = oracle.attention_forward(q, k, v, causal)
+    rng = np.random.default_rng(24)
+    for _ in range(5):
+        perms = {}
+        for i in range(S):
+            vis = oracle.ring_visit_order(i, S, causal)
+            perms[i] = list(rng.permutation(vis))
+        o, lse = oracle.ring_blockwise_forward(q, k, v, S, 4, 2, causal, order=lambda i: perms[i])
+        np.testing.assert_allclose(o, o_ref, atol=1e-12)
+        np.testing.assert_allclose(lse, l_ref, atol=1e-12)
+
+
+def test_ring_visit_order_matches_statement():
+    # step t: shard i holds KV shard (i - t) mod S
+    assert oracle.ring_visit_order(2, 4, False) == [2, 1, 0, 3]
+    assert oracle.ring_visit_order(2, 4, True) == [2, 1, 0]
+    assert oracle.ring_visit_order(0, 4, True) == [0]
+    assert oracle.ring_visit_order_bwd(1, 4, False) == [1, 2, 3, 0]
+    assert oracle.ring_visit_order_bwd(1, 4, True) == [1, 2, 3]
+    # forward and backward loop nests cover the same causal pairs
+    S = 7
+    fwd = {(i, j) for i in range(S) for j in oracle.ring_visit_order(i, S, True)}
+    bwd = {(i, j) for j in range(S) for i in oracle.ring_visit_order_bwd(j, S, True)}
+    assert fwd == bwd and len(fwd) == S * (S + 1) // 2
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_step_partials_merge_to_full(causal):
+    """Materialise each ring step, merge the partials in any order."""
+    B, H, N, d, S = 1, 2, 32, 4, 4
+    q, k, v = _rand((B, H, N, d), 25), _rand((B, H, N, d), 26), _rand((B, H, N, d), 27)
+    o_ref, l_ref = oracle.attention_forward(q, k, v, causal)
+    parts = [oracle.ring_blockwise_step(q, k, v, S, t, causal) for t in range(S)]
+    for order in ([0, 1, 2, 3], [3, 1, 0, 2]):
+        o = np.zeros_like(o_ref)
+        lse = np.full(l_ref.shape, -np.inf)
+        for t in order:
+            o, lse = oracle.lse_merge(o, lse, *parts[t])
+        np.testing.assert_allclose(o, o_ref, atol=1e-12)
+        np.testing.assert_allclose(lse, l_ref, atol=1e-12)
+
+
+def test_lse_merge_closed_form_and_algebra():
+    rng = np.random.default_rng(28)
+    n, d = 10, 5
+    s = rng.standard_normal((n, 9)) * 3
+    v = rng.standard_normal((9, d))
+    # two disjoint key sets
+    a, b = slice(0, 4), slice(4, 9)
+    def part(sl):
+        lse = scipy.special.logsumexp(s[:, sl], axis=1)
+        return scipy.special.softmax(s[:, sl], axis=1) @ v[sl], lse
+    oa, la = part(a)
+    ob, lb = part(b)
+    o, lse = oracle.lse_merge(oa, la, ob, lb)
+    np.testing.assert_allclose(o, scipy.special.softmax(s, axis=1) @ v, atol=1e-13)
+    np.testing.assert_allclose(lse, scipy.special.logsumexp(s, axis=1), atol=1e-13)
+    # commutative
+    o2, l2 = oracle.lse_merge(ob, lb, oa, la)
+    np.testing.assert_allclose(o2, o, atol=1e-14)
+    np.testing.assert_allclose(l2, lse, atol=1e-14)
+    # associative over three parts
+    c = [slice(0, 2), slice(2, 6), slice(6, 9)]
+    p = [part(sl) for sl in c]
+    left = oracle.lse_merge(*oracle.lse_merge(*p[0], *p[1]), *p[2])
+    right = oracle.lse_merge(*p[0], *oracle.lse_merge(*p[1], *p[2]))
+    np.testing.assert_allclose(left[0], right[0], atol=1e-13)
+    np.testing.assert_allclose(left[1], right[1], atol=1e-13)
+    # neutral element (o anything, lse = -inf), including both empty
+    on, ln_ = oracle.lse_merge(oa, la, np.full_like(oa, 7.0), np.full(n, -np.inf))
+    np.testing.assert_array_equal(on, oa)
+    np.testing.assert_array_equal(ln_, la)
+    oe, le = oracle.lse_merge(np.zeros((2, d)), np.full(2, -np.inf), np.zeros((2, d)), np.full(2, -np.inf))
+    assert np.all(oe == 0) and np.all(np.isneginf(le))
+    # large offsets do not overflow
+    o3, l3 = oracle.lse_merge(oa, la + 800.0, ob, lb + 800.0)
+    np.testing.assert_allclose(o3, o, atol=1e-12)
+    np.testing.assert_allclose(l3, lse + 800.0, atol=1e-10)
+
+
+# ---------------------------------------------------------------------------
+# Gradients
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_finite_differences(causal):
+    B, H, N, d = 1, 1, 9, 5
+    q, k, v = _rand((B, H, N, d), 29), _rand((B, H, N, d), 30), _rand((B, H, N, d), 31)
+    do = _rand((B, H, N, d), 32)
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, causal)
+
+    def loss(q_, k_, v_):
+        return float((oracle.attention_forward(q_, k_, v_, causal)[0] * do).sum())
+
+    eps = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = {"q": q, "k": k, "v": v}
+            args_m = dict(args_p)
+            args_p[name], args_m[name] = xp, xm
+            num[idx] = (loss(**{f"{a}_": b for a, b in args_p.items()})
+                        - loss(**{f"{a}_": b for a, b in args_m.items()})) / (2 * eps)
+        err = np.abs(num - g).max() / max(1.0, np.abs(g).max())
+        assert err < 1e-6, (name, err)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_invariants(causal):
+    B, H, N, d = 2, 2, 20, 6
+    q, k, v = _rand((B, H, N, d), 33), _rand((B, H, N, d), 34), _rand((B, H, N, d), 35)
+    do = _rand((B, H, N, d), 36)
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, causal)
+    # adding one vector to every key shifts each score row by a constant:
+    # the loss does not move, so the key gradients sum to zero
+    np.testing.assert_allclose(dk.sum(axis=2), 0.0, atol=1e-12)
+    # q -> a q, k -> k / a leaves every score unchanged
+    np.testing.assert_allclose((q * dq).sum(axis=(2, 3)), (k * dk).sum(axis=(2, 3)), atol=1e-11)
+    # upstream dO = 1 gives dv_j = column sums of the attention matrix
+    ones = np.ones_like(do)
+    _, _, dv1 = oracle.attention_backward(q, k, v, ones, causal)
+    sc = 1 / math.sqrt(d)
+    for b, h in itertools.product(range(B), range(H)):
+        s = sc * q[b, h] @ k[b, h].T
+        if causal:
+            s = np.where(np.tril(np.ones((N, N), bool)), s, -np.inf)
+        p = scipy.special.softmax(s, axis=1)
+        np.testing.assert_allclose(dv1[b, h], np.repeat(p.sum(0)[:, None], d, 1), atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Sampled-row routines equal the full functions on the sample
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sampled_rows(causal):
+    B, H, N, d = 2, 3, 50, 8
+    q, k, v = _rand((B, H, N, d), 37), _rand((B, H, N, d), 38), _rand((B, H, N, d), 39)
+    do = _rand((B, H, N, d), 40)
+    o, lse = oracle.attention_forward(q, k, v, causal)
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, causal)
+    rng = np.random.default_rng(41)
+    rows = np.stack([rng.integers(0, B, 20), rng.integers(0, H, 20), rng.integers(0, N, 20)], 1)
+    rows[0] = (0, 0, 0)
+    rows[1] = (1, 2, N - 1)
+    o_r, l_r = oracle.attention_rows(q, k, v, rows, causal)
+    np.testing.assert_allclose(o_r, o[rows[:, 0], rows[:, 1], rows[:, 2]], atol=1e-13)
+    np.testing.assert_allclose(l_r, lse[rows[:, 0], rows[:, 1], rows[:, 2]], atol=1e-13)
+    dq_r = oracle.attention_backward_query_rows(q, k, v, do, rows, causal)
+    np.testing.assert_allclose(dq_r, dq[rows[:, 0], rows[:, 1], rows[:, 2]], atol=1e-12)
+    keys = np.array([0, 3, 17, N - 1])
+    dk_r, dv_r = oracle.attention_backward_key_rows(q, k, v, do, 1, 2, keys, causal, q_block=7)
+    np.testing.assert_allclose(dk_r, dk[1, 2, keys], atol=1e-12)
+    np.testing.assert_allclose(dv_r, dv[1, 2, keys], atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Feed-forward
+# ---------------------------------------------------------------------------
+
+def test_ffn_zero_cases_and_chunking():
+    T, dm, dff = 24, 8, 12
+    x = _rand((T, dm), 42)
+    w1, w3 = _rand((dff, dm), 43), _rand((dff, dm), 44)
+    w2 = _rand((dm, dff), 45)
+    assert np.all(oracle.swiglu_ffn(np.zeros_like(x), w1, w2, w3) == 0)
+    assert np.all(oracle.swiglu_ffn(x, w1, w2, np.zeros_like(w3)) == 0)
+    y = oracle.swiglu_ffn(x, w1, w2, w3)
+    for c in (1, 2, 3, 4, 6, 8, 12, 24):
+        np.testing.assert_allclose(oracle.blockwise_ffn(x, w1, w2, w3, c), y, atol=1e-13)
+    # explicit loops
+    ref = np.zeros((T, dm))
+    for t in range(T):
+        h = []
+        for f in range(dff):
+            g = sum(x[t, a] * w1[f, a] for a in range(dm))
+            u = sum(x[t, a] * w3[f, a] for a in range(dm))
+            h.append(g / (1 + math.exp(-g)) * u)
+        for a in range(dm):
+            ref[t, a] = sum(h[f] * w2[a, f] for f in range(dff))
+    np.testing.assert_allclose(y, ref, atol=1e-12)
+
+
+def test_silu_matches_expit():
+    z = np.linspace(-40, 40, 1001)
+    np.testing.assert_allclose(oracle.silu(z), z * scipy.special.expit(z), rtol=1e-14, atol=1e-300)
