@@ -1,0 +1,26 @@
+"""B200 (sm_100a) exact blockwise ring attention and blockwise feed-forward.
+
+Thin Python binding over the C ABI of ``libringattn.so`` (include/ringattn.h).
+Functions take torch CUDA tensors and only marshal pointers, sizes and the
+current CUDA stream; every step of the computation runs in the library's
+kernels.  PyTorch is used for device memory and streams only.
+"""
+
+from ._lib import RA_BF16, RA_F32, RingAttnError, lib  # noqa: F401
+from .api import (  # noqa: F401
+    ringattn_fwd,
+    ringattn_fwd_step,
+    ringattn_merge,
+    ringattn_bwd,
+    ringattn_bwd_workspace_size,
+    blockwise_ffn,
+    blockwise_ffn_workspace_size,
+    ringattn_get_error,
+    ringattn_selftest_timeout,
+)
+
+__all__ = [
+    "ringattn_fwd", "ringattn_fwd_step", "ringattn_merge", "ringattn_bwd", "ringattn_bwd_workspace_size",
+    "blockwise_ffn", "blockwise_ffn_workspace_size", "ringattn_get_error", "ringattn_selftest_timeout",
+    "RA_BF16", "RA_F32", "RingAttnError", "lib",
+]

@@ -1,0 +1,129 @@
+"""torch-tensor front end of the C ABI: argument marshalling only.
+
+Each function checks that its tensors are CUDA, contiguous and of the
+expected dtype, passes their device pointers and sizes to the library entry
+point of the same name on the current CUDA stream, and raises
+``RingAttnError`` on a non-zero status.  Nothing is computed here.
+"""
+
+from __future__ import annotations
+
+import torch
+
+from ._lib import RA_BF16, RA_F32, call, lib
+
+_DT = {torch.bfloat16: RA_BF16, torch.float32: RA_F32}
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _bhnd(q: torch.Tensor):
+    if q.dim() != 4:
+        raise ValueError("attention tensors are [B, H, N, D]")
+    return tuple(int(x) for x in q.shape)
+
+
+def _dtype(q: torch.Tensor) -> int:
+    if q.dtype not in _DT:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    return _DT[q.dtype]
+
+
+def ringattn_fwd(q, k, v, out, lse, S, q_chunk, k_chunk, causal, scale=0.0, stream=None):
+    """out, lse <- exact ring blockwise attention of (q, k, v)."""
+    B, H, N, D = _bhnd(q)
+    for t in (k, v, out):
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("q, k, v, out must share shape and dtype")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N):
+        raise ValueError("lse must be float32 [B, H, N]")
+    call("ringattn_fwd", _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), _dev(lse, "lse"),
+         B, H, N, D, _dtype(q), int(S), int(q_chunk), int(k_chunk), int(bool(causal)), float(scale),
+         _stream(stream))
+    return out, lse
+
+
+def ringattn_fwd_step(q, k, v, o_acc, lse_acc, S, q_chunk, k_chunk, causal, t, scale=0.0, stream=None):
+    """Merge ring step t of (q, k, v) into the fp32 accumulators (o_acc, lse_acc)."""
+    B, H, N, D = _bhnd(q)
+    if o_acc.dtype != torch.float32 or tuple(o_acc.shape) != (B, H, N, D):
+        raise ValueError("o_acc must be float32 [B, H, N, D]")
+    if lse_acc.dtype != torch.float32 or tuple(lse_acc.shape) != (B, H, N):
+        raise ValueError("lse_acc must be float32 [B, H, N]")
+    call("ringattn_fwd_step", _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o_acc, "o_acc"),
+         _dev(lse_acc, "lse_acc"), B, H, N, D, _dtype(q), int(S), int(q_chunk), int(k_chunk),
+         int(bool(causal)), float(scale), int(t), _stream(stream))
+    return o_acc, lse_acc
+
+
+def ringattn_merge(o_a, lse_a, o_b, lse_b, stream=None):
+    """(o_a, lse_a) <- exact log-sum-exp merge with (o_b, lse_b); fp32, [rows, D] / [rows]."""
+    D = int(o_a.shape[-1])
+    rows = o_a.numel() // D
+    if o_b.shape != o_a.shape or lse_a.numel() != rows or lse_b.numel() != rows:
+        raise ValueError("merge operands disagree in shape")
+    for x in (o_a, o_b, lse_a, lse_b):
+        if x.dtype != torch.float32:
+            raise ValueError("merge operands are float32")
+    call("ringattn_merge", _dev(o_a, "o_a"), _dev(lse_a, "lse_a"), _dev(o_b, "o_b"), _dev(lse_b, "lse_b"),
+         rows, D, _stream(stream))
+    return o_a, lse_a
+
+
+def ringattn_bwd_workspace_size(B, H, N, D) -> int:
+    return int(lib().ringattn_bwd_workspace_size(int(B), int(H), int(N), int(D)))
+
+
+def ringattn_bwd(q, k, v, out, lse, dout, dq, dk, dv, S, q_chunk, k_chunk, causal, workspace,
+                 scale=0.0, stream=None):
+    """dq, dk, dv <- gradient of sum(dout * out) through ringattn_fwd."""
+    B, H, N, D = _bhnd(q)
+    for t in (k, v, out, dout, dq, dk, dv):
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("attention tensors must share shape and dtype")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N):
+        raise ValueError("lse must be float32 [B, H, N]")
+    nbytes = workspace.numel() * workspace.element_size()
+    call("ringattn_bwd", _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), _dev(lse, "lse"),
+         _dev(dout, "dout"), _dev(dq, "dq"), _dev(dk, "dk"), _dev(dv, "dv"), B, H, N, D, _dtype(q),
+         int(S), int(q_chunk), int(k_chunk), int(bool(causal)), float(scale), _dev(workspace, "workspace"),
+         nbytes, _stream(stream))
+    return dq, dk, dv
+
+
+def blockwise_ffn_workspace_size(chunk, d_ff, dtype=torch.bfloat16) -> int:
+    return int(lib().blockwise_ffn_workspace_size(int(chunk), int(d_ff), _DT[dtype]))
+
+
+def blockwise_ffn(x, w1, w2, w3, y, chunk, workspace, stream=None):
+    """y <- (silu(x w1^T) * (x w3^T)) w2^T, chunk tokens at a time."""
+    T, d_model = (int(s) for s in x.shape)
+    d_ff = int(w1.shape[0])
+    if tuple(w1.shape) != (d_ff, d_model) or tuple(w3.shape) != (d_ff, d_model):
+        raise ValueError("w1, w3 are [d_ff, d_model]")
+    if tuple(w2.shape) != (d_model, d_ff) or tuple(y.shape) != (T, d_model):
+        raise ValueError("w2 is [d_model, d_ff], y is [T, d_model]")
+    nbytes = workspace.numel() * workspace.element_size()
+    call("blockwise_ffn", _dev(x, "x"), _dev(w1, "w1"), _dev(w2, "w2"), _dev(w3, "w3"), _dev(y, "y"),
+         T, d_model, d_ff, int(chunk), _dtype(x), _dev(workspace, "workspace"), nbytes, _stream(stream))
+    return y
+
+
+def ringattn_get_error(stream=None) -> int:
+    """Synchronise the stream; return and clear the device status word."""
+    return int(lib().ringattn_get_error(_stream(stream)))
+
+
+def ringattn_selftest_timeout(timeout_us: int, stream=None) -> None:
+    call("ringattn_selftest_timeout", int(timeout_us), _stream(stream))

@@ -1,0 +1,60 @@
+// Internal launch interface between the C ABI (abi.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "ringattn.h"
+
+namespace ra {
+
+struct DevStatus;
+
+// Status word of the current device plus the bounded-wait limit.  Returns
+// RA_OK or RA_ERR_CUDA.
+int current_status(DevStatus* out);
+
+struct AttnArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int64_t B, H, N, D;
+  int dtype;
+  int S, q_chunk, k_chunk, causal;
+  float scale;  // already resolved (> 0)
+};
+
+// Exact fp32 CUDA-core ring forward (whole ring, or one step merged into
+// fp32 accumulators when step >= 0).  Inputs fp32 or bf16.
+int launch_fwd_simt(const AttnArgs& a, void* out, float* lse, float* o_acc, float* lse_acc, int step,
+                    cudaStream_t stream);
+
+// tcgen05 ring forward, bf16 inputs (whole ring, or one step merged into
+// fp32 accumulators when step >= 0).
+int launch_fwd_tc(const AttnArgs& a, void* out, float* lse, float* o_acc, float* lse_acc, int step,
+                  cudaStream_t stream);
+
+int launch_merge(float* o_a, float* lse_a, const float* o_b, const float* lse_b, int64_t rows, int64_t D,
+                 cudaStream_t stream);
+
+// Backward: preprocess, KV-stationary tcgen05 main loop, dQ conversion.
+int launch_bwd_tc(const AttnArgs& a, const void* out, const float* lse, const void* dout, void* dq, void* dk,
+                  void* dv, void* workspace, cudaStream_t stream);
+
+// Blockwise SwiGLU FFN on the tensor cores.
+int launch_ffn_tc(const void* x, const void* w1, const void* w2, const void* w3, void* y, int64_t T,
+                  int64_t d_model, int64_t d_ff, int64_t chunk, void* workspace, cudaStream_t stream);
+
+int launch_selftest_timeout(int timeout_us, cudaStream_t stream);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point.
+// 2-D bf16 map over a row-major [rows, inner] matrix with the given row
+// pitch, box [box_rows, box_inner], 128-byte swizzle.
+int make_tmap_bf16_2d(void* tmap /* CUtensorMap* */, const void* base, uint64_t inner, uint64_t rows,
+                      uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_rows);
+
+// Opt a kernel into more than 48 KB of dynamic shared memory.
+int set_smem_attr(const void* func, int bytes);
+
+}  // namespace ra

@@ -1,0 +1,131 @@
+"""Seeded synthetic inputs shared by the tests, the bench and the oracle side.
+
+This module holds no part of the method's arithmetic: it only draws random
+tensors and picks sample rows.  Both the CUDA path and the oracle receive
+the very same bits (bf16 inputs are rounded once, here, and the oracle
+upcasts those bf16 values exactly to float64).
+
+Recipe (per workload): a torch.Generator on the target device seeded with
+the workload seed draws float32 standard normals in the order q, k, v, dO
+(then x, w1, w3, w2 for the feed-forward), each scaled as the workload says
+(k by 2 for the sharpened 32k workload, weights by 0.02), then rounded to the
+compute dtype with round-to-nearest-even.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+
+@dataclass(frozen=True)
+class AttnWorkload:
+    name: str
+    B: int
+    H: int
+    N: int
+    D: int
+    S: int
+    q_chunk: int
+    k_chunk: int
+    causal: bool
+    seed: int
+    dtype: torch.dtype = torch.bfloat16
+    k_scale: float = 1.0
+    bwd: bool = True
+
+
+@dataclass(frozen=True)
+class FFNWorkload:
+    name: str
+    T: int
+    d_model: int
+    d_ff: int
+    chunk: int
+    seed: int
+    w_std: float = 0.02
+    dtype: torch.dtype = torch.bfloat16
+
+
+WORKLOADS = {
+    # tiny exact check, fp32, forward only
+    "tiny_f32": AttnWorkload("tiny_f32", 1, 1, 512, 64, 4, 64, 64, True, 0, torch.float32, bwd=False),
+    # B=2, H=16, N=8192, d=64, S=8, chunks 128, causal and non-causal
+    "n8k_d64_causal": AttnWorkload("n8k_d64_causal", 2, 16, 8192, 64, 8, 128, 128, True, 1),
+    "n8k_d64_full": AttnWorkload("n8k_d64_full", 2, 16, 8192, 64, 8, 128, 128, False, 1),
+    # B=1, H=32, N=32768, d=128, S=16, q_chunk 512, k_chunk 1024, K scaled by 2
+    "n32k_d128": AttnWorkload("n32k_d128", 1, 32, 32768, 128, 16, 512, 1024, True, 2, k_scale=2.0),
+    # attention of the 7B-shaped layer: N=131072, 32 heads x 128, S=32, chunks 2048
+    "layer7b_attn": AttnWorkload("layer7b_attn", 1, 32, 131072, 128, 32, 2048, 2048, True, 3),
+    # million-token causal forward: S=64, q_chunk 1024, k_chunk 4096
+    "n1m_d128": AttnWorkload("n1m_d128", 1, 32, 1048576, 128, 64, 1024, 4096, True, 4, bwd=False),
+}
+
+FFN_WORKLOADS = {
+    # SwiGLU 4096 -> 11008 -> 4096 over N=131072 tokens in 2048-token chunks
+    "layer7b_ffn": FFNWorkload("layer7b_ffn", 131072, 4096, 11008, 2048, 3),
+}
+
+
+def _gen(device, seed: int) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def _draw(shape, g, device, scale, dtype):
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    if scale != 1.0:
+        x.mul_(scale)
+    return x.to(dtype)
+
+
+def attention_inputs(w: AttnWorkload, device="cuda", with_dout: bool | None = None):
+    """q, k, v (and dO when the workload has a backward) as [B,H,N,D] tensors."""
+    shape = (w.B, w.H, w.N, w.D)
+    g = _gen(device, w.seed)
+    q = _draw(shape, g, device, 1.0, w.dtype)
+    k = _draw(shape, g, device, w.k_scale, w.dtype)
+    v = _draw(shape, g, device, 1.0, w.dtype)
+    want_do = w.bwd if with_dout is None else with_dout
+    do = _draw(shape, g, device, 1.0, w.dtype) if want_do else None
+    return q, k, v, do
+
+
+def small_attention_inputs(B, H, N, D, seed, dtype=torch.bfloat16, device="cuda", k_scale=1.0):
+    """q, k, v, dO for ad-hoc test shapes (same recipe as the workloads)."""
+    w = AttnWorkload("adhoc", B, H, N, D, 1, N, N, True, seed, dtype, k_scale)
+    return attention_inputs(w, device, with_dout=True)
+
+
+def ffn_inputs(w: FFNWorkload, device="cuda", T: int | None = None):
+    """x [T, d_model], w1 [d_ff, d_model], w3 [d_ff, d_model], w2 [d_model, d_ff]."""
+    T = w.T if T is None else T
+    g = _gen(device, w.seed)
+    x = _draw((T, w.d_model), g, device, 1.0, w.dtype)
+    w1 = _draw((w.d_ff, w.d_model), g, device, w.w_std, w.dtype)
+    w3 = _draw((w.d_ff, w.d_model), g, device, w.w_std, w.dtype)
+    w2 = _draw((w.d_model, w.d_ff), g, device, w.w_std, w.dtype)
+    return x, w1, w2, w3
+
+
+def sample_rows(B: int, H: int, N: int, n: int, seed: int, include_ends: bool = True) -> np.ndarray:
+    """n seeded (b, h, i) triples (numpy default_rng(seed + 1000)).
+
+    With include_ends the first two are the first and the last token of a
+    head, so the first row of the causal diagonal and the longest row are
+    always checked.
+    """
+    rng = np.random.default_rng(seed + 1000)
+    rows = np.stack([rng.integers(0, B, n), rng.integers(0, H, n), rng.integers(0, N, n)], axis=1)
+    if include_ends and n >= 2:
+        rows[0] = (0, 0, 0)
+        rows[1] = (B - 1, H - 1, N - 1)
+    return rows.astype(np.int64)
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    """Exact upcast of a (bf16 / fp32) tensor to a float64 numpy array."""
+    return t.detach().to("cpu", torch.float32).numpy().astype(np.float64)

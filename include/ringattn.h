@@ -1,0 +1,209 @@
+/*
+ * ringattn.h -- C ABI of the B200 (sm_100a) library for exact blockwise ring
+ * attention and the blockwise feed-forward.
+ *
+ * What it computes (sources by page title and section):
+ *
+ *  - "Ring Attention with Blockwise Transformers for Near-Infinite Context",
+ *    abstract: self-attention and the feed-forward computed blockwise, with
+ *    no approximation, for training and inference.
+ *  - chapterpal keyword page "Ring Attention", definition: the sequence is
+ *    cut into blocks placed on a logical ring; each block keeps its queries
+ *    while key/value blocks circulate around the ring.
+ *  - sourcepulse project summary of the RingAttention package, "Highlighted
+ *    Details": the query_chunk_size and key_chunk_size knobs.
+ *  - darcstar.tech note on the paper, "DarcStar commentary", paragraphs one
+ *    and two: online softmax is associative, so partial attention of separate
+ *    shards combines exactly; the causal mask and the softmax denominator
+ *    must be combined across chunks exactly; no all-gather of K/V.
+ *
+ * On one GPU the ring is virtual: the S shards are slices of the [B,H,N,D]
+ * tensors in HBM and query shard i visits KV shard j = (i - t) mod S at ring
+ * step t = 0..S-1.  Under the causal mask pairs j > i are skipped and the
+ * diagonal pair j == i is masked inside its tiles.
+ *
+ * Conventions common to every call
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never frees or retains them.  The library allocates nothing per call.
+ *    Its only persistent device state is one status word per device.
+ *  - Attention tensors are contiguous [B, H, N, D] (D innermost).  LSE and
+ *    the backward's D-vector are contiguous fp32 [B, H, N].  Pointers must be
+ *    16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *    only enqueues work and returns; argument and launch errors come back
+ *    synchronously as a negative ra_status, device-side failures (a bounded
+ *    wait that ran out) are latched in the device status word and read back
+ *    by ringattn_get_error().
+ *  - Returns RA_OK (0) on success.  A request with an empty extent
+ *    (B, H, N or T equal to 0) is valid and returns RA_OK without launching
+ *    anything; negative sizes are RA_ERR_ARG.
+ */
+#ifndef RINGATTN_H_
+#define RINGATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RA_API __attribute__((visibility("default")))
+#else
+#define RA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { RA_BF16 = 0, RA_F32 = 1 } ra_dtype;
+
+typedef enum {
+  RA_OK = 0,
+  RA_ERR_ARG = -1,         /* null pointer or non-positive size             */
+  RA_ERR_SHAPE = -2,       /* N % S, shard % chunk or chunk % tile != 0     */
+  RA_ERR_DTYPE = -3,       /* dtype not RA_BF16 / RA_F32                    */
+  RA_ERR_ALIGN = -4,       /* a pointer is not 16-byte aligned             */
+  RA_ERR_UNSUPPORTED = -5, /* valid request this build does not implement   */
+  RA_ERR_CUDA = -6,        /* a CUDA runtime call failed                    */
+  RA_ERR_TIMEOUT = -7,     /* a kernel's bounded wait ran out (device word) */
+  RA_ERR_WORKSPACE = -8    /* workspace missing or smaller than required    */
+} ra_status;
+
+/* Library ABI version (major*100 + minor). */
+RA_API int ringattn_version(void);
+
+/* Human-readable text for an ra_status value (static storage). */
+RA_API const char* ringattn_status_string(int status);
+
+/*
+ * ringattn_fwd -- exact ring blockwise attention forward.
+ *
+ * For every (b, h) and query token i:
+ *   s_ij = scale * q_i . k_j ;  visible(i, j) = !causal || j <= i
+ *   lse_i = ln sum_{visible j} exp(s_ij)
+ *   out_i = sum_{visible j} exp(s_ij - lse_i) v_j
+ * computed shard by shard in ring order with an exact log-sum-exp merge of
+ * the partial (max, denominator, unnormalised output) states.
+ *
+ *   q, k, v  [B,H,N,D] inputs of `dtype`                         (read)
+ *   out      [B,H,N,D] output of `dtype` (bf16 rounded to nearest even)
+ *   lse      [B,H,N] fp32 natural-log softmax denominator        (written)
+ *   S        number of ring shards, N % S == 0, shard L = N / S
+ *   q_chunk, k_chunk  query / key chunk sizes; both divide L.  RA_BF16 runs
+ *            on the tensor cores in 128x128 tiles: chunks must be multiples
+ *            of 128.  RA_F32 runs in exact fp32 on CUDA cores in 64-row
+ *            tiles: chunks must be multiples of 64.
+ *   causal   0 or 1 (mask j > i on global token indices)
+ *   scale    softmax scale; <= 0 selects 1/sqrt(D)
+ *   D        64 or 128
+ * Errors: RA_ERR_ARG, RA_ERR_SHAPE, RA_ERR_DTYPE, RA_ERR_ALIGN, RA_ERR_CUDA.
+ */
+RA_API int ringattn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                 int64_t B, int64_t H, int64_t N, int64_t D, int dtype,
+                 int S, int q_chunk, int k_chunk, int causal, float scale,
+                 void* stream);
+
+/*
+ * ringattn_fwd_step -- one ring step t with a fused merge into running
+ * fp32 accumulators (the per-step building block of a multi-device ring).
+ *
+ * Query shard i attends to KV shard j = (i - t) mod S only, and the partial
+ * result is merged exactly into (o_acc, lse_acc):
+ *   lse' = ln(e^lse_acc + e^lse_t),
+ *   o'   = e^(lse_acc - lse') o_acc + e^(lse_t - lse') o_t
+ * where (o_t, lse_t) is the normalised attention of the pair.  Pairs that
+ * the causal mask skips (j > i) leave the accumulators unchanged.
+ * Start from o_acc = 0 and lse_acc = -inf (the neutral element) and run
+ * t = 0..S-1 in any order: the result equals ringattn_fwd's (in fp32).
+ *
+ *   o_acc    [B,H,N,D] fp32, read and written
+ *   lse_acc  [B,H,N]   fp32, read and written
+ * Other arguments as for ringattn_fwd; 0 <= t < S.
+ */
+RA_API int ringattn_fwd_step(const void* q, const void* k, const void* v,
+                      float* o_acc, float* lse_acc,
+                      int64_t B, int64_t H, int64_t N, int64_t D, int dtype,
+                      int S, int q_chunk, int k_chunk, int causal, float scale,
+                      int t, void* stream);
+
+/*
+ * ringattn_merge -- standalone exact log-sum-exp merge of two partials,
+ * (o_a, lse_a) <- (o_a, lse_a) (+) (o_b, lse_b), all fp32:
+ *   lse = ln(e^lse_a + e^lse_b);  o_a = e^(lse_a-lse) o_a + e^(lse_b-lse) o_b
+ * (-inf, any) is the neutral element; two -inf rows give (0, -inf).
+ *   o_a, o_b  [rows, D] fp32;  lse_a, lse_b  [rows] fp32;  D % 4 == 0.
+ * Darcstar note, DarcStar commentary, paragraph one (associative combine).
+ */
+RA_API int ringattn_merge(float* o_a, float* lse_a, const float* o_b, const float* lse_b,
+                   int64_t rows, int64_t D, void* stream);
+
+/* Bytes of device workspace ringattn_bwd needs: fp32 dQ accumulator
+ * [B,H,N,D] plus the fp32 row vector D_i = dO_i . O_i [B,H,N]. */
+RA_API size_t ringattn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D);
+
+/*
+ * ringattn_bwd -- gradient of sum(dout * out) for ringattn_fwd.
+ *
+ * With P_ij = exp(s_ij - lse_i) on visible pairs and D_i = dout_i . out_i:
+ *   dv_j = sum_i P_ij dout_i
+ *   dS_ij = P_ij (dout_i . v_j - D_i)
+ *   dq_i = scale sum_j dS_ij k_j ;  dk_j = scale sum_i dS_ij q_i
+ * Each key/value shard stays put while the query shards pass by in ring
+ * order i = (j + t) mod S (causal: pairs i < j skipped).
+ *
+ *   q,k,v,out,dout [B,H,N,D] of `dtype` (out and lse from ringattn_fwd)
+ *   lse            [B,H,N] fp32
+ *   dq,dk,dv       [B,H,N,D] of `dtype`, written
+ *   workspace      device buffer of ringattn_bwd_workspace_size() bytes,
+ *                  16-byte aligned; its contents on entry do not matter
+ * Only RA_BF16 is implemented (RA_F32 returns RA_ERR_UNSUPPORTED).
+ * Chunk rules as for ringattn_fwd with RA_BF16.
+ */
+RA_API int ringattn_bwd(const void* q, const void* k, const void* v, const void* out,
+                 const float* lse, const void* dout,
+                 void* dq, void* dk, void* dv,
+                 int64_t B, int64_t H, int64_t N, int64_t D, int dtype,
+                 int S, int q_chunk, int k_chunk, int causal, float scale,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace blockwise_ffn needs for one chunk's hidden
+ * activation h [chunk, d_ff] in `dtype`. */
+RA_API size_t blockwise_ffn_workspace_size(int64_t chunk, int64_t d_ff, int dtype);
+
+/*
+ * blockwise_ffn -- SwiGLU feed-forward applied `chunk` tokens at a time.
+ *
+ *   y = (silu(x w1^T) * (x w3^T)) w2^T,   silu(z) = z / (1 + e^-z)
+ * paper abstract: the feed-forward is computed blockwise, so only one
+ * chunk's hidden activation [chunk, d_ff] exists at a time (in workspace).
+ *
+ *   x   [T, d_model]     w1, w3 [d_ff, d_model]     w2 [d_model, d_ff]
+ *   y   [T, d_model] written.  Row-major, weights in [out, in] layout.
+ *   T % chunk == 0; chunk, d_model multiples of 128; d_ff multiple of 128.
+ *   workspace: blockwise_ffn_workspace_size(chunk, d_ff, dtype) bytes.
+ * Only RA_BF16 is implemented (fp32 accumulation, h rounded to bf16).
+ */
+RA_API int blockwise_ffn(const void* x, const void* w1, const void* w2, const void* w3, void* y,
+                  int64_t T, int64_t d_model, int64_t d_ff, int64_t chunk, int dtype,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * ringattn_get_error -- synchronise `stream`, return the device status word
+ * of the current device (RA_OK or RA_ERR_TIMEOUT) and clear it.  Also
+ * reports a pending CUDA error as RA_ERR_CUDA.
+ */
+RA_API int ringattn_get_error(void* stream);
+
+/*
+ * ringattn_selftest_timeout -- launch one tiny kernel whose bounded wait on
+ * an mbarrier that nothing arrives at runs out after `timeout_us`
+ * microseconds; the kernel then latches RA_ERR_TIMEOUT in the device status
+ * word and returns normally.  Lets a test exercise the timeout path without
+ * hanging or faulting the GPU.  Read the result with ringattn_get_error().
+ */
+RA_API int ringattn_selftest_timeout(int timeout_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RINGATTN_H_ */

@@ -34,7 +34,8 @@ Parity status per function (what pins it is in ``tests/test_oracle.py``):
                                  and chunk size, order invariant)
 * ``lse_merge``                  pinned (closed form of two-part softmax,
                                  associativity, neutral element)
-* ``attention_rows`` / ``attention_backward_key_rows`` /
+* ``attention_rows`` / ``attention_head_rows`` /
+  ``attention_backward_key_rows`` /
   ``attention_backward_query_rows``
                                  pinned (equal to the full functions on the
                                  sampled subset)
@@ -50,6 +51,7 @@ from .attention import (  # noqa: F401
     ring_blockwise_step,
     lse_merge,
     attention_rows,
+    attention_head_rows,
     attention_backward_query_rows,
     attention_backward_key_rows,
     ring_visit_order,

@@ -116,31 +116,41 @@ def attention_backward(q, k, v, do, causal: bool, scale=None):
 # Sampled rows: the same definition restricted to chosen rows.
 # ---------------------------------------------------------------------------
 
-def attention_rows(q, k, v, rows, causal: bool, scale=None):
-    """Forward definition for selected query rows only.
+def attention_head_rows(q_sel, K, V, idx, causal: bool, scale=None):
+    """Forward definition for chosen query rows of one head.
 
-    rows: integer array [n, 3] of (b, h, i).  Returns (o [n, d], lse [n]).
-    Each row is computed on its own from the full key/value sequence of its
-    head, so the result is exact for that row, not an estimate.
+    q_sel: [n, d] query vectors of tokens idx [n]; K, V: [N, d] of the head.
+    Each row is computed on its own from the full key/value sequence, so the
+    result is exact for that row, not an estimate.  Returns (o [n, d], lse [n]).
     """
-    rows = np.asarray(rows, dtype=np.int64)
-    d = q.shape[3]
-    sc = _scale(d, scale)
-    o = np.empty((len(rows), v.shape[3]))
-    lse = np.empty(len(rows))
-    for r, (b, h, i) in enumerate(rows):
-        kk = _f64(k[b, h])
-        vv = _f64(v[b, h])
-        qi = _f64(q[b, h, i])
-        if causal:
-            kk = kk[: i + 1]
-            vv = vv[: i + 1]
-        s = sc * (kk @ qi)
+    q_sel = _f64(q_sel)
+    K = _f64(K)
+    V = _f64(V)
+    sc = _scale(q_sel.shape[1], scale)
+    o = np.empty((len(idx), V.shape[1]))
+    lse = np.empty(len(idx))
+    for r, i in enumerate(np.asarray(idx, dtype=np.int64)):
+        kk, vv = (K[: i + 1], V[: i + 1]) if causal else (K, V)
+        s = sc * (kk @ q_sel[r])
         m = s.max()
         e = np.exp(s - m)
         den = e.sum()
         o[r] = (e / den) @ vv
         lse[r] = m + np.log(den)
+    return o, lse
+
+
+def attention_rows(q, k, v, rows, causal: bool, scale=None):
+    """Forward definition for selected query rows only.
+
+    rows: integer array [n, 3] of (b, h, i).  Returns (o [n, d], lse [n]).
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    o = np.empty((len(rows), v.shape[3]))
+    lse = np.empty(len(rows))
+    for r, (b, h, i) in enumerate(rows):
+        o[r:r + 1], lse[r:r + 1] = attention_head_rows(_f64(q[b, h, i])[None], k[b, h], v[b, h], [i],
+                                                       causal, scale)
     return o, lse
 
 

@@ -1,0 +1,126 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/ringattn.h declares, and rejects bad arguments
+before touching the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from exact_blockwise_long_b200 import build
+    build.build()
+    from exact_blockwise_long_b200 import _lib
+    return _lib.lib()
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "ringattn.h")).read()
+    return sorted(set(re.findall(r"RA_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_symbols()
+    for must in ("ringattn_fwd", "ringattn_bwd", "blockwise_ffn", "ringattn_merge", "ringattn_fwd_step"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    from exact_blockwise_long_b200 import _lib
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+        assert name in _lib.SIGNATURES, f"binding lacks {name}"
+
+
+def test_only_declared_symbols_are_exported():
+    """Hidden visibility: the dynamic symbol table holds only the ABI."""
+    import subprocess
+    from exact_blockwise_long_b200 import _lib
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True).stdout
+    ours = {ln.split()[-1] for ln in out.splitlines() if " T " in ln and ("ringattn" in ln or "ffn" in ln)}
+    assert ours == set(declared_symbols())
+
+
+FAKE = 0x10000  # aligned, never dereferenced: validation fails first
+MIS = 0x10001
+
+
+def fwd(L, q=FAKE, out=FAKE, lse=FAKE, B=1, H=1, N=1024, D=128, dtype=0, S=4, qc=128, kc=128, causal=1):
+    return L.ringattn_fwd(q, FAKE, FAKE, out, lse, B, H, N, D, dtype, S, qc, kc, causal, 0.0, None)
+
+
+def test_fwd_argument_errors(L):
+    assert fwd(L, q=None) == -1                     # null pointer
+    assert fwd(L, N=-128) == -1                     # negative size
+    assert fwd(L, causal=2) == -1
+    assert fwd(L, dtype=7) == -3                    # dtype
+    assert fwd(L, D=96) == -5                       # head dim not built
+    assert fwd(L, N=1000) == -2                     # N % S
+    assert fwd(L, N=1024, S=8, qc=256) == -2        # chunk larger than shard
+    assert fwd(L, N=1536, S=4, qc=256) == -2        # shard 384 not divisible by 256
+    assert fwd(L, qc=64) == -2                      # bf16 tiles are 128
+    assert fwd(L, q=MIS) == -4                      # alignment
+    assert fwd(L, lse=MIS) == -4
+    assert fwd(L, out=None) == -1
+
+
+def test_fwd_empty_extents_are_noops(L):
+    assert fwd(L, B=0, q=None, out=None, lse=None) == 0
+    assert fwd(L, N=0, q=None, out=None, lse=None) == 0
+    assert fwd(L, H=0) == 0
+
+
+def test_step_and_merge_argument_errors(L):
+    st = L.ringattn_fwd_step
+    assert st(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 1024, 128, 0, 4, 128, 128, 1, 0.0, 4, None) == -1  # t >= S
+    assert st(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 1024, 128, 0, 4, 128, 128, 1, 0.0, -1, None) == -1
+    assert st(FAKE, FAKE, FAKE, None, FAKE, 1, 1, 1024, 128, 0, 4, 128, 128, 1, 0.0, 0, None) == -1
+    m = L.ringattn_merge
+    assert m(FAKE, FAKE, FAKE, FAKE, 10, 6, None) == -2     # D % 4
+    assert m(None, FAKE, FAKE, FAKE, 10, 8, None) == -1
+    assert m(MIS, FAKE, FAKE, FAKE, 10, 8, None) == -4
+    assert m(FAKE, FAKE, FAKE, FAKE, 0, 8, None) == 0       # nothing to merge
+
+
+def test_bwd_workspace_contract(L):
+    ws = L.ringattn_bwd_workspace_size(1, 32, 32768, 128)
+    assert ws >= 32 * 32768 * 128 * 4 + 32 * 32768 * 4
+    assert L.ringattn_bwd_workspace_size(0, 1, 1, 1) == 0
+    b = L.ringattn_bwd
+    ws = L.ringattn_bwd_workspace_size(1, 1, 1024, 128)
+    args = [FAKE] * 9 + [1, 1, 1024, 128, 0, 4, 128, 128, 1, 0.0]
+    assert b(*args, FAKE, ws - 1, None) == -8          # too small
+    assert b(*args, None, ws, None) == -8              # missing
+    assert b(*(args[:13] + [1] + args[14:]), FAKE, ws, None) == -5  # fp32 backward not built
+
+
+def test_ffn_contract(L):
+    assert L.blockwise_ffn_workspace_size(2048, 11008, 0) == 2048 * 11008 * 2
+    f = L.blockwise_ffn
+    good = [FAKE] * 5 + [4096, 4096, 11008, 2048, 0]
+    ws = L.blockwise_ffn_workspace_size(2048, 11008, 0)
+    assert f(*good[:5], 4000, 4096, 11008, 2048, 0, FAKE, ws, None) == -2   # T % chunk
+    assert f(*good[:5], 4096, 4096, 11000, 2048, 0, FAKE, ws, None) == -2   # d_ff % 128
+    assert f(*good, FAKE, ws - 2, None) == -8
+    assert f(*good[:9], 5, FAKE, ws, None) == -3
+    assert f(*good[:5], 0, 4096, 11008, 2048, 0, None, 0, None) == 0        # no tokens
+
+
+def test_status_strings(L):
+    for code in range(-8, 1):
+        assert L.ringattn_status_string(code)
+    assert L.ringattn_version() >= 100
+
+
+def test_product_path_has_no_oracle_or_fallback():
+    """The package never imports the oracle and has no CPU fallback."""
+    pkg = os.path.join(ROOT, "exact_blockwise_long_b200")
+    for fn in os.listdir(pkg):
+        if fn.endswith(".py"):
+            src = open(os.path.join(pkg, fn)).read()
+            assert "import oracle" not in src and "from oracle" not in src, fn

@@ -354,6 +354,9 @@ def test_sampled_rows(causal):
     rows[0] = (0, 0, 0)
     rows[1] = (1, 2, N - 1)
     o_r, l_r = oracle.attention_rows(q, k, v, rows, causal)
+    o_h, l_h = oracle.attention_head_rows(q[1, 2, [3, 9]], k[1, 2], v[1, 2], [3, 9], causal)
+    np.testing.assert_allclose(o_h, o[1, 2, [3, 9]], atol=1e-13)
+    np.testing.assert_allclose(l_h, lse[1, 2, [3, 9]], atol=1e-13)
     np.testing.assert_allclose(o_r, o[rows[:, 0], rows[:, 1], rows[:, 2]], atol=1e-13)
     np.testing.assert_allclose(l_r, lse[rows[:, 0], rows[:, 1], rows[:, 2]], atol=1e-13)
     dq_r = oracle.attention_backward_query_rows(q, k, v, do, rows, causal)
