@@ -249,7 +249,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool ok = walk.run([&](int, bool diag) {
       const int sb = n & 1;
       const uint32_t tS = (sb ? tS1 : tS0) + lane_off;
-      if (!mbar_wait(&bar_sf[sb], (n >> 1) & 1, p.st, abort_flag)) return false;
+      // tcgen05.ld/st are warp-collective: every branch below that reaches
+      // them is taken by the whole warp.
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar_sf[sb], (n >> 1) & 1, p.st, abort_flag))) return false;
       tc_fence_after();
       float s[kBN];
 #pragma unroll
@@ -271,9 +273,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_new = fmaxf(m_run, mx * sl2);
       if (n == 0) {
         m_run = m_new;
-      } else if (m_new > m_run + kRescaleLog2) {
-        // O holds P V of every earlier tile once the last one has landed.
-        if (!mbar_wait(bar_od, (n - 1) & 1, p.st, abort_flag)) return false;
+      } else if (__any_sync(0xffffffffu, m_new > m_run + kRescaleLog2)) {
+        // Some row of this warp saw its max grow by more than 2^8: the whole
+        // warp moves to its new maxima (exact for every row).  O holds P V of
+        // every earlier tile once the last one has landed.
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_od, (n - 1) & 1, p.st, abort_flag))) return false;
         tc_fence_after();
         const float alpha = ex2_approx(m_run - m_new);
         l_run *= alpha;
@@ -309,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++n;
       return true;
     });
-    if (ok && mbar_wait(bar_od, (n - 1) & 1, p.st, abort_flag)) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(bar_od, (n - 1) & 1, p.st, abort_flag))) {
       tc_fence_after();
       const int grow = qrow0 + r;  // row of the [BH*N, D] view
       const float lse_t = (m_run + __log2f(l_run)) * kLn2;

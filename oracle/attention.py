@@ -397,5 +397,10 @@ def lse_merge(o_a, lse_a, o_b, lse_b):
         lse = np.where(fin, msafe + np.log(np.where(fin, tot, 1.0)), NEG_INF)
         wa = np.where(fin, ea / np.where(fin, tot, 1.0), 0.0)
         wb = np.where(fin, eb / np.where(fin, tot, 1.0), 0.0)
-    o = wa[..., None] * o_a + wb[..., None] * o_b
+    # an empty partial (lse = -inf) contributes nothing, whatever o it holds
+    a_in = np.isfinite(lse_a)[..., None]
+    b_in = np.isfinite(lse_b)[..., None]
+    with np.errstate(invalid="ignore"):
+        o = np.where(a_in, wa[..., None] * np.where(a_in, o_a, 0.0), 0.0) + \
+            np.where(b_in, wb[..., None] * np.where(b_in, o_b, 0.0), 0.0)
     return o, lse

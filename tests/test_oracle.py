@@ -279,6 +279,13 @@ def test_lse_merge_closed_form_and_algebra():
     np.testing.assert_array_equal(ln_, la)
     oe, le = oracle.lse_merge(np.zeros((2, d)), np.full(2, -np.inf), np.zeros((2, d)), np.full(2, -np.inf))
     assert np.all(oe == 0) and np.all(np.isneginf(le))
+    # the neutral element is neutral whatever output it carries (even NaN)
+    junk = np.full_like(oa, np.nan)
+    oj, lj = oracle.lse_merge(junk, np.full(n, -np.inf), ob, lb)
+    np.testing.assert_array_equal(oj, ob)
+    np.testing.assert_array_equal(lj, lb)
+    oj2, lj2 = oracle.lse_merge(junk, np.full(n, -np.inf), junk, np.full(n, -np.inf))
+    assert np.all(oj2 == 0) and np.all(np.isneginf(lj2))
     # large offsets do not overflow
     o3, l3 = oracle.lse_merge(oa, la + 800.0, ob, lb + 800.0)
     np.testing.assert_allclose(o3, o, atol=1e-12)
