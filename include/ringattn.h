@@ -136,8 +136,9 @@ RA_API int ringattn_fwd_step(const void* q, const void* k, const void* v,
 RA_API int ringattn_merge(float* o_a, float* lse_a, const float* o_b, const float* lse_b,
                    int64_t rows, int64_t D, void* stream);
 
-/* Bytes of device workspace ringattn_bwd needs: fp32 dQ accumulator
- * [B,H,N,D] plus the fp32 row vector D_i = dO_i . O_i [B,H,N]. */
+/* Bytes of device workspace ringattn_bwd needs: the fp32 dQ accumulator
+ * [B,H,N,D] plus two fp32 row vectors [B,H,N] (D_i = dO_i . O_i and
+ * lse_i * log2(e)), each region 256-byte aligned.  0 for empty problems. */
 RA_API size_t ringattn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D);
 
 /*

@@ -1,0 +1,96 @@
+"""GPU parity of the tcgen05 ring backward against the fp64 oracle gradient
+(dq, dk, dv of sum(dO * O)) on the same seeded input bits."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_blockwise_long_b200.synthetic import WORKLOADS, attention_inputs, sample_rows, small_attention_inputs, to_f64
+from helpers import TOL_BF16_GRAD, max_abs, run_fwd
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from exact_blockwise_long_b200 import build
+    build.build()
+    import exact_blockwise_long_b200 as ra
+    ra.lib()
+    torch.cuda.set_device(0)
+
+
+def run_bwd(q, k, v, do, S, qc, kc, causal):
+    import exact_blockwise_long_b200 as ra
+    o, lse = run_fwd(q, k, v, S, qc, kc, causal)
+    B, H, N, D = q.shape
+    ws = torch.empty(ra.ringattn_bwd_workspace_size(B, H, N, D), device="cuda", dtype=torch.uint8)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ra.ringattn_bwd(q, k, v, o, lse, do, dq, dk, dv, S, qc, kc, causal, ws)
+    assert ra.ringattn_get_error() == 0
+    return dq, dk, dv
+
+
+CASES = [
+    # (B, H, N, D, S, qc, kc, causal)
+    (1, 2, 1024, 128, 4, 128, 128, True),
+    (1, 2, 1024, 128, 4, 128, 256, False),
+    (2, 1, 1024, 64, 2, 256, 128, True),
+    (1, 3, 768, 64, 3, 128, 256, False),
+    (1, 1, 128, 128, 1, 128, 128, True),    # a single tile
+    (1, 1, 2048, 128, 16, 128, 128, True),  # one tile per shard
+    (1, 2, 1536, 64, 1, 512, 1536, True),   # no ring
+]
+
+
+@pytest.mark.parametrize("B,H,N,D,S,qc,kc,causal", CASES)
+def test_bwd_full_oracle(B, H, N, D, S, qc, kc, causal):
+    q, k, v, do = small_attention_inputs(B, H, N, D, 100 + N + D + S, k_scale=2.0 if causal else 1.0)
+    dq, dk, dv = run_bwd(q, k, v, do, S, qc, kc, causal)
+    gq, gk, gv = oracle.attention_backward(to_f64(q), to_f64(k), to_f64(v), to_f64(do), causal)
+    errs = [max_abs(to_f64(a), b) for a, b in ((dq, gq), (dk, gk), (dv, gv))]
+    assert max(errs) <= TOL_BF16_GRAD, errs
+
+
+def test_bwd_repeatable_within_atomics_noise():
+    """dK, dV are written once per key tile (deterministic); dQ sums fp32
+    atomics, so only its last bits may change between runs."""
+    q, k, v, do = small_attention_inputs(1, 2, 1024, 128, 5)
+    a = run_bwd(q, k, v, do, 4, 128, 128, True)
+    b = run_bwd(q, k, v, do, 4, 128, 128, True)
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+    assert (a[0].float() - b[0].float()).abs().max().item() <= 1e-2
+
+
+@pytest.mark.parametrize("name", ["n8k_d64_causal", "n8k_d64_full", "n32k_d128"])
+def test_workload_bwd_sampled(name):
+    w = WORKLOADS[name]
+    q, k, v, do = attention_inputs(w)
+    dq, dk, dv = run_bwd(q, k, v, do, w.S, w.q_chunk, w.k_chunk, w.causal)
+    rows = sample_rows(w.B, w.H, w.N, 256, w.seed)
+    # dq on 256 sampled query rows (each exact on its own)
+    err_q = 0.0
+    for b, h in sorted({(int(b), int(h)) for b, h, _ in rows}):
+        sel = rows[(rows[:, 0] == b) & (rows[:, 1] == h)]
+        local = np.stack([np.zeros(len(sel), np.int64), np.zeros(len(sel), np.int64), sel[:, 2]], 1)
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        ref = oracle.attention_backward_query_rows(to_f64(q[sl]), to_f64(k[sl]), to_f64(v[sl]), to_f64(do[sl]),
+                                                   local, w.causal)
+        got = to_f64(dq[b, h][torch.as_tensor(sel[:, 2], device="cuda")])
+        err_q = max(err_q, max_abs(got, ref))
+    assert err_q <= TOL_BF16_GRAD, err_q
+    # dk, dv on 128 seeded key rows of two sampled heads
+    rng = np.random.default_rng(w.seed + 2000)
+    for b, h in [(0, 0), (w.B - 1, w.H - 1)]:
+        keys = np.sort(rng.choice(w.N, 128, replace=False))
+        keys[0] = 0
+        keys[-1] = w.N - 1
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        gk, gv = oracle.attention_backward_key_rows(to_f64(q[sl]), to_f64(k[sl]), to_f64(v[sl]), to_f64(do[sl]),
+                                                    0, 0, keys, w.causal)
+        kidx = torch.as_tensor(keys, device="cuda")
+        assert max_abs(to_f64(dk[b, h][kidx]), gk) <= TOL_BF16_GRAD
+        assert max_abs(to_f64(dv[b, h][kidx]), gv) <= TOL_BF16_GRAD
