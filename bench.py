@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Benchmark of exact ring blockwise attention (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl native|reference]
+
+A step is one pass of the hot path over one batch of synthetic input:
+ring forward (ringattn_fwd) and ring backward (ringattn_bwd's three phases)
+of the attention workload, plus, for the layer workload, the blockwise SwiGLU
+feed-forward.  Inputs are resident in HBM when the timed region starts and
+are larger than the 126 MB L2.  The timed region is bracketed by a barrier and
+a device synchronise on both sides and timed with CUDA events on the launch
+stream; with several GPUs every rank runs its own batch (weak scaling, no
+data-path collective) and the maximum time over ranks is taken.
+
+Under ``--impl reference`` the fp64 CPU oracle is timed instead (rank 0
+only), on a bounded sample of the same workload.
+
+Prints one JSON line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "ring-attn fwd+bwd TFLOP/s & tokens/s on 1 B200; % of BF16 tensor peak"
+
+# DRAM traffic per launch of the dominant kernel, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
+# source it was taken on (sha256 of the source file).
+NCU_TRAFFIC = {}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="n32k_d128",
+                    choices=["n32k_d128", "n8k_d64_causal", "n8k_d64_full", "layer7b", "n1m_d128"])
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--heads", type=int, default=0, help="override the head count (smaller profiling cases)")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# workload description and FLOP counts
+# ---------------------------------------------------------------------------
+
+def workload(name):
+    from exact_blockwise_long_b200.synthetic import FFN_WORKLOADS, WORKLOADS
+    if name == "layer7b":
+        return WORKLOADS["layer7b_attn"], FFN_WORKLOADS["layer7b_ffn"]
+    return WORKLOADS[name], None
+
+
+def attn_fwd_flops(w):
+    """4 B H N^2 d, halved under the causal mask (causal FLOPs counted once)."""
+    f = 4.0 * w.B * w.H * w.N * w.N * w.D
+    return f * 0.5 if w.causal else f
+
+
+def attn_step_flops(w):
+    return attn_fwd_flops(w) * (3.5 if w.bwd else 1.0)  # backward = 2.5 x forward (5 MMAs vs 2)
+
+
+def ffn_flops(f):
+    return 6.0 * f.T * f.d_model * f.d_ff
+
+
+def describe(aw, fw):
+    d = {"workload": f"{aw.name}: ring attention {'fwd+bwd' if aw.bwd else 'fwd'}, B={aw.B}, H={aw.H}, "
+                     f"N={aw.N}, d={aw.D}, S={aw.S}, q_chunk={aw.q_chunk}, k_chunk={aw.k_chunk}, "
+                     f"{'causal' if aw.causal else 'non-causal'}"
+                     + (f"; blockwise SwiGLU FFN {fw.d_model}->{fw.d_ff}->{fw.d_model}, chunk {fw.chunk}"
+                        if fw else ""),
+         "B": aw.B, "H": aw.H, "seq_len": aw.N, "head_dim": aw.D, "shards": aw.S,
+         "q_chunk": aw.q_chunk, "k_chunk": aw.k_chunk, "causal": aw.causal,
+         "l2": "inputs larger than L2 (no flush between steps)"}
+    return d
+
+
+# ---------------------------------------------------------------------------
+# peaks, clocks
+# ---------------------------------------------------------------------------
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return {"bf16_burst": float(j["bf16_tflops"]), "bf16_sustained": float(j["bf16_tflops_sustained"]),
+                "hbm_gbs": float(j["hbm_gbs"]), "source": "measured"}
+    except Exception:
+        return {"bf16_burst": 1590.0, "bf16_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"ra_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        loaded = [s for s, p in zip(sm, power) if p > 300] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "samples_under_load": len(loaded)}
+
+
+# ---------------------------------------------------------------------------
+# the oracle on a bounded sample (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(aw, fw, n_tokens=4096, min_seconds=0.0, max_heads=32):
+    """Time the fp64 oracle on heads of the workload cut to their first
+    n_tokens tokens (a causal prefix is a complete sub-problem), adding heads
+    until min_seconds of CPU time have been spent.
+
+    Returns (seconds, counted FLOPs, description, threads)."""
+    import oracle
+    from dataclasses import replace
+    from exact_blockwise_long_b200.synthetic import attention_inputs, to_f64
+    n = min(aw.N, n_tokens)
+    small = replace(aw, B=1, H=1, N=n)
+    dt, heads = 0.0, 0
+    while heads < max_heads and (heads == 0 or dt < min_seconds):
+        q, k, v, do = attention_inputs(replace(small, seed=aw.seed + 7919 * heads), device="cpu",
+                                       with_dout=aw.bwd)
+        q, k, v = to_f64(q), to_f64(k), to_f64(v)
+        t0 = time.perf_counter()
+        oracle.attention_forward(q, k, v, aw.causal)
+        if aw.bwd:
+            oracle.attention_backward(q, k, v, to_f64(do), aw.causal)
+        dt += time.perf_counter() - t0
+        heads += 1
+    flops = attn_step_flops(small) * heads
+    desc = (f"fp64 oracle (numpy) {'forward+backward' if aw.bwd else 'forward'} of {heads} head(s) cut to "
+            f"their first {n} tokens, same workload recipe; causal FLOPs counted once")
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    return dt, flops, desc, threads
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from dataclasses import replace
+    aw, fw = workload(args.workload)
+    if args.heads:
+        aw = replace(aw, H=args.heads)
+    times, flops, desc, threads = [], 0.0, "", 1
+    for i in range(args.warmup + args.steps):
+        dt, flops, desc, threads = oracle_sample(aw, fw)
+        if i >= args.warmup:
+            times.append(dt)
+    t = sum(times) / len(times)
+    value = flops / t / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": describe(aw, fw),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": desc + f"; {args.steps} timed samples"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# the native arm
+# ---------------------------------------------------------------------------
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    from exact_blockwise_long_b200 import build
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    import exact_blockwise_long_b200 as ra
+    from dataclasses import replace
+    from exact_blockwise_long_b200.synthetic import attention_inputs, ffn_inputs
+
+    aw, fw = workload(args.workload)
+    if args.heads:
+        aw = replace(aw, H=args.heads)
+    # each rank draws its own batch (weak scaling): seed offset by rank
+    aw_r = replace(aw, seed=aw.seed + 1000 * rank)
+    q, k, v, do = attention_inputs(aw_r, device=dev)
+    B, H, N, D = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+    if aw.bwd:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(ra.ringattn_bwd_workspace_size(B, H, N, D), device=dev, dtype=torch.uint8)
+    if fw is not None:
+        x, w1, w2, w3 = ffn_inputs(replace(fw, seed=fw.seed + 1000 * rank), device=dev)
+        y = torch.empty_like(x)
+        ffn_ws = torch.empty(ra.blockwise_ffn_workspace_size(fw.chunk, fw.d_ff), device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream()
+    cfg = (aw.S, aw.q_chunk, aw.k_chunk, aw.causal)
+
+    ev = {}
+
+    def event():
+        return torch.cuda.Event(enable_timing=True)
+
+    def step(timed=False):
+        if timed:
+            e = [event() for _ in range(4)]
+            e[0].record(stream)
+        ra.ringattn_fwd(q, k, v, o, lse, *cfg)
+        launches = 1
+        if timed:
+            e[1].record(stream)
+        if aw.bwd:
+            ra.ringattn_bwd_phase(q, k, v, o, lse, do, dq, dk, dv, *cfg, ws, 1)
+            if timed:
+                e[2].record(stream)
+            ra.ringattn_bwd_phase(q, k, v, o, lse, do, dq, dk, dv, *cfg, ws, 2)
+            if timed:
+                e[3].record(stream)
+            ra.ringattn_bwd_phase(q, k, v, o, lse, do, dq, dk, dv, *cfg, ws, 4)
+            launches += 3
+        if fw is not None:
+            ra.blockwise_ffn(x, w1, w2, w3, y, fw.chunk, ffn_ws)
+            launches += 2 * (fw.T // fw.chunk)
+        if timed:
+            ev.setdefault("fwd", []).append((e[0], e[1]))
+            if aw.bwd:
+                ev.setdefault("bwd_main", []).append((e[2], e[3]))
+        return launches
+
+    for _ in range(args.warmup):
+        step()
+    if ra.ringattn_get_error() != 0:
+        raise RuntimeError("device status word set during warm-up")
+
+    clocks = ClockSampler(dev.index)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t_start, t_stop = event(), event()
+    t_start.record(stream)
+    launches = 0
+    for _ in range(args.steps):
+        launches += step(timed=True)
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    if ra.ringattn_get_error() != 0:
+        raise RuntimeError("device status word set during the timed region")
+    ms_total = t_start.elapsed_time(t_stop)
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+
+    flops_step = attn_step_flops(aw) + (ffn_flops(fw) if fw else 0.0)
+    value = flops_step * world / (ms_step * 1e-3) / 1e12
+    tokens_s = aw.B * aw.N * world / (ms_step * 1e-3)
+    pk = peaks()
+
+    # dominant kernel: the backward main loop when there is a backward
+    def mean_ms(pairs):
+        return sum(a.elapsed_time(b) for a, b in pairs) / len(pairs)
+
+    if aw.bwd:
+        kname, kms = "bwd_tc_kernel", mean_ms(ev["bwd_main"])
+        kflops = attn_fwd_flops(aw) * 2.5
+    else:
+        kname, kms = "fwd_tc_kernel", mean_ms(ev["fwd"])
+        kflops = attn_fwd_flops(aw)
+    achieved = kflops / (kms * 1e-3) / 1e12
+    src = os.path.join(ROOT, "exact_blockwise_long_b200", "csrc",
+                       "bwd_tc.cu" if kname.startswith("bwd") else "fwd_tc.cu")
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    tr = NCU_TRAFFIC.get((kname, args.workload))
+    traffic = tr["bytes"] if tr and tr["sha256"] == sha else None
+    roof = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": pk["bf16_sustained"],
+            "unit": "TFLOP/s", "frac": achieved / pk["bf16_sustained"], "traffic": traffic,
+            "peak_kind": f"bf16 dense, sustained ({pk['source']})",
+            "frac_of_burst": achieved / pk["bf16_burst"], "kernel_ms": kms,
+            "fwd_kernel_ms": mean_ms(ev["fwd"]),
+            "fwd_tflops": attn_fwd_flops(aw) / (mean_ms(ev["fwd"]) * 1e-3) / 1e12}
+
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": describe(aw, fw),
+            "tokens_per_s": tokens_s, "pct_of_bf16_peak": 100.0 * value / world / pk["bf16_sustained"],
+            "roofline": roof, "gpu_launches": launches, "clocks": clk}
+
+    # end to end through the public API: pinned host inputs in, results out
+    if not args.no_e2e:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        hdo = do.cpu().pin_memory() if aw.bwd else None
+        outs = [o, lse] + ([dq, dk, dv] if aw.bwd else [])
+        houts = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv) + ((hdo,) if aw.bwd else ()))
+        d2h = sum(t.numel() * t.element_size() for t in outs)
+        e2e_steps = max(3, min(args.steps, 10))
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a, b = event(), event()
+        a.record(stream)
+        for _ in range(e2e_steps):
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            if aw.bwd:
+                do.copy_(hdo, non_blocking=True)
+            ra.ringattn_fwd(q, k, v, o, lse, *cfg)
+            if aw.bwd:
+                ra.ringattn_bwd(q, k, v, o, lse, do, dq, dk, dv, *cfg, ws)
+            if fw is not None:
+                ra.blockwise_ffn(x, w1, w2, w3, y, fw.chunk, ffn_ws)
+            for h, d_ in zip(houts, outs):
+                h.copy_(d_, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b) / e2e_steps
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        line["e2e"] = {"value": flops_step * world / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
+                       "steps": e2e_steps}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if not args.no_cpu_baseline and world == 1:
+            dt, fl, desc, threads = oracle_sample(aw, fw, n_tokens=8192, min_seconds=10.0)
+            line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads,
+                                    "kind": "oracle", "sample": desc, "seconds": dt}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

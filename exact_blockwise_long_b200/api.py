@@ -102,6 +102,18 @@ def ringattn_bwd(q, k, v, out, lse, dout, dq, dk, dv, S, q_chunk, k_chunk, causa
     return dq, dk, dv
 
 
+def ringattn_bwd_phase(q, k, v, out, lse, dout, dq, dk, dv, S, q_chunk, k_chunk, causal, workspace, phase_mask,
+                       scale=0.0, stream=None):
+    """Run the selected phases of ringattn_bwd (bit 0 preprocess, 1 main, 2 dQ convert)."""
+    B, H, N, D = _bhnd(q)
+    nbytes = workspace.numel() * workspace.element_size()
+    call("ringattn_bwd_phase", _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), _dev(lse, "lse"),
+         _dev(dout, "dout"), _dev(dq, "dq"), _dev(dk, "dk"), _dev(dv, "dv"), B, H, N, D, _dtype(q),
+         int(S), int(q_chunk), int(k_chunk), int(bool(causal)), float(scale), _dev(workspace, "workspace"),
+         nbytes, int(phase_mask), _stream(stream))
+    return dq, dk, dv
+
+
 def blockwise_ffn_workspace_size(chunk, d_ff, dtype=torch.bfloat16) -> int:
     return int(lib().blockwise_ffn_workspace_size(int(chunk), int(d_ff), _DT[dtype]))
 

@@ -190,10 +190,11 @@ size_t ringattn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D) {
   return ((dq + 255) & ~(size_t)255) + 2 * ((dvec + 255) & ~(size_t)255);
 }
 
-int ringattn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
-                 const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N, int64_t D,
-                 int dtype, int S, int q_chunk, int k_chunk, int causal, float scale, void* workspace,
-                 size_t workspace_bytes, void* stream) {
+int ringattn_bwd_phase(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                       const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N, int64_t D,
+                       int dtype, int S, int q_chunk, int k_chunk, int causal, float scale, void* workspace,
+                       size_t workspace_bytes, int phase_mask, void* stream) {
+  if (phase_mask <= 0 || phase_mask > 7) return RA_ERR_ARG;
   int rc = check_attn(q, k, v, B, H, N, D, dtype, S, q_chunk, k_chunk, causal);
   if (rc == kEmpty) return dtype == RA_BF16 ? RA_OK : RA_ERR_UNSUPPORTED;
   if (rc != RA_OK) return rc;
@@ -205,7 +206,15 @@ int ringattn_bwd(const void* q, const void* k, const void* v, const void* out, c
   if (!workspace || workspace_bytes < ringattn_bwd_workspace_size(B, H, N, D)) return RA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return RA_ERR_ALIGN;
   AttnArgs a{q, k, v, B, H, N, D, dtype, S, q_chunk, k_chunk, causal, resolve_scale(scale, D)};
-  return launch_bwd_tc(a, out, lse, dout, dq, dk, dv, workspace, static_cast<cudaStream_t>(stream));
+  return launch_bwd_tc(a, out, lse, dout, dq, dk, dv, workspace, phase_mask, static_cast<cudaStream_t>(stream));
+}
+
+int ringattn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N, int64_t D,
+                 int dtype, int S, int q_chunk, int k_chunk, int causal, float scale, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+  return ringattn_bwd_phase(q, k, v, out, lse, dout, dq, dk, dv, B, H, N, D, dtype, S, q_chunk, k_chunk, causal,
+                            scale, workspace, workspace_bytes, 7, stream);
 }
 
 size_t blockwise_ffn_workspace_size(int64_t chunk, int64_t d_ff, int dtype) {

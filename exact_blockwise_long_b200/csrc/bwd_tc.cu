@@ -434,7 +434,7 @@ int sm_count() {
 
 template <int D>
 int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* dout, void* dq, void* dk, void* dv,
-             void* workspace, cudaStream_t stream) {
+             void* workspace, int phase_mask, cudaStream_t stream) {
   const int64_t rows = a.B * a.H * a.N;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* dq_acc = reinterpret_cast<float*>(ws);
@@ -444,7 +444,7 @@ int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* d
   float* lse2 = reinterpret_cast<float*>(ws + dq_bytes + vec_bytes);
   const int sms = sm_count();
 
-  {
+  if (phase_mask & 1) {
     const int64_t want = (rows + 7) / 8;
     const unsigned grid = (unsigned)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
     bwd_preprocess_kernel<D><<<grid, 256, 0, stream>>>((const __nv_bfloat16*)out, (const __nv_bfloat16*)dout, lse,
@@ -452,6 +452,7 @@ int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* d
     if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
   }
 
+  if (phase_mask & 2) {
   alignas(64) CUtensorMap tq, tk, tv, tdo;
   if (make_tmap_bf16_2d(&tq, a.q, D, rows, D * 2, 64, kT) != RA_OK) return RA_ERR_CUDA;
   if (make_tmap_bf16_2d(&tk, a.k, D, rows, D * 2, 64, kT) != RA_OK) return RA_ERR_CUDA;
@@ -477,8 +478,9 @@ int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* d
   if (set_smem_attr((const void*)kern, BLayout<D>::kBytes) != RA_OK) return RA_ERR_CUDA;
   kern<<<(unsigned)(p.BH * p.num_tiles), kThreads, BLayout<D>::kBytes, stream>>>(tq, tk, tv, tdo, p);
   if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
+  }
 
-  {
+  if (phase_mask & 4) {
     const int64_t n8 = rows * D / 8;
     const int64_t want = (n8 + 255) / 256;
     const unsigned grid = (unsigned)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
@@ -491,9 +493,9 @@ int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* d
 }  // namespace
 
 int launch_bwd_tc(const AttnArgs& a, const void* out, const float* lse, const void* dout, void* dq, void* dk,
-                  void* dv, void* workspace, cudaStream_t stream) {
-  if (a.D == 64) return launch_d<64>(a, out, lse, dout, dq, dk, dv, workspace, stream);
-  if (a.D == 128) return launch_d<128>(a, out, lse, dout, dq, dk, dv, workspace, stream);
+                  void* dv, void* workspace, int phase_mask, cudaStream_t stream) {
+  if (a.D == 64) return launch_d<64>(a, out, lse, dout, dq, dk, dv, workspace, phase_mask, stream);
+  if (a.D == 128) return launch_d<128>(a, out, lse, dout, dq, dk, dv, workspace, phase_mask, stream);
   return RA_ERR_UNSUPPORTED;
 }
 

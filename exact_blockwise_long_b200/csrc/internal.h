@@ -39,8 +39,9 @@ int launch_merge(float* o_a, float* lse_a, const float* o_b, const float* lse_b,
                  cudaStream_t stream);
 
 // Backward: preprocess, KV-stationary tcgen05 main loop, dQ conversion.
+// phase_mask: bit 0 preprocess, bit 1 main loop, bit 2 dQ conversion.
 int launch_bwd_tc(const AttnArgs& a, const void* out, const float* lse, const void* dout, void* dq, void* dk,
-                  void* dv, void* workspace, cudaStream_t stream);
+                  void* dv, void* workspace, int phase_mask, cudaStream_t stream);
 
 // Blockwise SwiGLU FFN on the tensor cores.
 int launch_ffn_tc(const void* x, const void* w1, const void* w2, const void* w3, void* y, int64_t T,

@@ -166,6 +166,24 @@ RA_API int ringattn_bwd(const void* q, const void* k, const void* v, const void*
                  int S, int q_chunk, int k_chunk, int causal, float scale,
                  void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * ringattn_bwd_phase -- ringattn_bwd split into its three launches, for
+ * callers that schedule or time them separately.  phase_mask (1..7) selects
+ * bit 0: preprocess (D_i, lse_i*log2(e), zero the dQ accumulator in
+ * workspace), bit 1: the tensor-core main loop (dK, dV written, dQ
+ * accumulated in workspace), bit 2: dq = bf16(scale * accumulator).  The
+ * phases must run in that order on the same workspace; mask 7 is
+ * ringattn_bwd.  Arguments and errors as ringattn_bwd, plus RA_ERR_ARG for
+ * a mask outside 1..7.
+ */
+RA_API int ringattn_bwd_phase(const void* q, const void* k, const void* v, const void* out,
+                              const float* lse, const void* dout,
+                              void* dq, void* dk, void* dv,
+                              int64_t B, int64_t H, int64_t N, int64_t D, int dtype,
+                              int S, int q_chunk, int k_chunk, int causal, float scale,
+                              void* workspace, size_t workspace_bytes, int phase_mask,
+                              void* stream);
+
 /* Bytes of device workspace blockwise_ffn needs for one chunk's hidden
  * activation h [chunk, d_ff] in `dtype`. */
 RA_API size_t blockwise_ffn_workspace_size(int64_t chunk, int64_t d_ff, int dtype);
