@@ -38,7 +38,16 @@ METRIC = "ring-attn fwd+bwd TFLOP/s & tokens/s on 1 B200; % of BF16 tensor peak"
 # DRAM traffic per launch of the dominant kernel, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
 # source it was taken on (sha256 of the source file).
-NCU_TRAFFIC = {}
+# Captured on 8 heads of the n32k_d128 workload and scaled x4 to its 32 heads
+# (heads are independent units; see profiles/*_n32k_d128_h8.md).
+NCU_TRAFFIC = {
+    ("bwd_tc_kernel", "n32k_d128"): {
+        "bytes": 4 * (1.981993e9 + 1.020117e9),
+        "sha256": "e06329c00d98f3e52db8c2e1a033de7de3074db543e82d5c8047b6c411731676"},
+    ("fwd_tc_kernel", "n32k_d128"): {
+        "bytes": 4 * (885.399040e6 + 49.013248e6),
+        "sha256": "26b9afff19374c15dd6c7df4a19c6b061c4c89d40db9dc13f8c0d13b00d4d2bc"},
+}
 
 
 def parse():
