@@ -13,6 +13,7 @@ from .api import (  # noqa: F401
     ringattn_merge,
     ringattn_bwd,
     ringattn_bwd_phase,
+    ringattn_bwd_noalloc,
     ringattn_bwd_workspace_size,
     blockwise_ffn,
     blockwise_ffn_workspace_size,
@@ -21,7 +22,7 @@ from .api import (  # noqa: F401
 )
 
 __all__ = [
-    "ringattn_fwd", "ringattn_fwd_step", "ringattn_merge", "ringattn_bwd", "ringattn_bwd_phase", "ringattn_bwd_workspace_size",
+    "ringattn_fwd", "ringattn_fwd_step", "ringattn_merge", "ringattn_bwd", "ringattn_bwd_phase", "ringattn_bwd_noalloc", "ringattn_bwd_workspace_size",
     "blockwise_ffn", "blockwise_ffn_workspace_size", "ringattn_get_error", "ringattn_selftest_timeout",
     "RA_BF16", "RA_F32", "RingAttnError", "lib",
 ]

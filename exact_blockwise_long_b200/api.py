@@ -114,6 +114,20 @@ def ringattn_bwd_phase(q, k, v, out, lse, dout, dq, dk, dv, S, q_chunk, k_chunk,
     return dq, dk, dv
 
 
+def ringattn_bwd_noalloc(q, k, v, out, lse, dout, dq, dk, dv, S, q_chunk, k_chunk, causal, scale=0.0, stream=None):
+    """ringattn_bwd without a workspace: the library's fixed static scratch is
+    used instead, for callers that cannot allocate device memory.  Calls must
+    not overlap on the GPU (they share that scratch)."""
+    B, H, N, D = _bhnd(q)
+    for t in (k, v, out, dout, dq, dk, dv):
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("attention tensors must share shape and dtype")
+    call("ringattn_bwd_noalloc", _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), _dev(lse, "lse"),
+         _dev(dout, "dout"), _dev(dq, "dq"), _dev(dk, "dk"), _dev(dv, "dv"), B, H, N, D, _dtype(q),
+         int(S), int(q_chunk), int(k_chunk), int(bool(causal)), float(scale), _stream(stream))
+    return dq, dk, dv
+
+
 def blockwise_ffn_workspace_size(chunk, d_ff, dtype=torch.bfloat16) -> int:
     return int(lib().blockwise_ffn_workspace_size(int(chunk), int(d_ff), _DT[dtype]))
 

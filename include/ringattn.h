@@ -184,6 +184,33 @@ RA_API int ringattn_bwd_phase(const void* q, const void* k, const void* v, const
                               void* workspace, size_t workspace_bytes, int phase_mask,
                               void* stream);
 
+/*
+ * ringattn_bwd_noalloc -- ringattn_bwd that allocates nothing and takes no
+ * workspace.  The paper has no counterpart; it serves callers that cannot
+ * allocate device memory when they run the backward (an allocator owned by
+ * another framework, a device-memory budget fixed at start-up, or a hot
+ * path where a cudaMalloc that may synchronise the device is not allowed).
+ *
+ * The scratch ringattn_bwd would take from `workspace` comes from one
+ * static device array of RINGATTN_NOALLOC_SCRATCH_BYTES (64 MiB) that every
+ * GPU which loads this library keeps until the process exits.  Problems
+ * whose ringattn_bwd_workspace_size() exceeds it return RA_ERR_WORKSPACE
+ * (with D = 128: B*H*N up to about 127 thousand rows, e.g. H=4, N=32768).
+ * The first call on a device looks up the array's device address; make that
+ * first call before any stream capture.  All calls share the one array and
+ * it keeps the last call's contents (each call re-clears what must start at
+ * zero), so calls that overlap on the GPU -- on different streams, or from
+ * different host threads -- race and corrupt each other's gradients:
+ * serialise them.  Arguments, results and other errors as ringattn_bwd.
+ */
+#define RINGATTN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+RA_API int ringattn_bwd_noalloc(const void* q, const void* k, const void* v, const void* out,
+                                const float* lse, const void* dout,
+                                void* dq, void* dk, void* dv,
+                                int64_t B, int64_t H, int64_t N, int64_t D, int dtype,
+                                int S, int q_chunk, int k_chunk, int causal, float scale,
+                                void* stream);
+
 /* Bytes of device workspace blockwise_ffn needs for one chunk's hidden
  * activation h [chunk, d_ff] in `dtype`. */
 RA_API size_t blockwise_ffn_workspace_size(int64_t chunk, int64_t d_ff, int dtype);
