@@ -1,0 +1,82 @@
+"""GPU parity of the blockwise SwiGLU feed-forward (tcgen05 GEMMs) against
+the fp64 oracle on the same seeded bf16 input bits.
+
+Tolerance (derived in the design doc): |y_gpu - y_ref| <= 2^-8 |y_ref| + 0.03.
+The relative part covers the final bf16 rounding of y (2^-9) with margin;
+the absolute part covers h rounded to bf16 before the down projection."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_blockwise_long_b200.synthetic import FFN_WORKLOADS, FFNWorkload, ffn_inputs, to_f64
+
+pytestmark = pytest.mark.gpu
+
+RTOL = 2.0 ** -8
+ATOL = 0.03
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from exact_blockwise_long_b200 import build
+    build.build()
+    import exact_blockwise_long_b200 as ra
+    ra.lib()
+    torch.cuda.set_device(0)
+
+
+def run_ffn(x, w1, w2, w3, chunk):
+    import exact_blockwise_long_b200 as ra
+    y = torch.empty_like(x)
+    ws = torch.empty(ra.blockwise_ffn_workspace_size(chunk, w1.shape[0]), device="cuda", dtype=torch.uint8)
+    ra.blockwise_ffn(x, w1, w2, w3, y, chunk, ws)
+    assert ra.ringattn_get_error() == 0
+    return y
+
+
+def within(got, ref):
+    err = np.abs(got - ref)
+    return bool(np.all(err <= RTOL * np.abs(ref) + ATOL)), float(err.max())
+
+
+@pytest.mark.parametrize("T,dm,dff,chunk", [(512, 256, 384, 128), (768, 128, 256, 256), (256, 512, 1024, 256)])
+def test_ffn_full_oracle(T, dm, dff, chunk):
+    w = FFNWorkload("t", T, dm, dff, chunk, 9, w_std=0.06)
+    x, w1, w2, w3 = ffn_inputs(w)
+    y = run_ffn(x, w1, w2, w3, chunk)
+    ref = oracle.blockwise_ffn(to_f64(x), to_f64(w1), to_f64(w2), to_f64(w3), chunk)
+    ok, err = within(to_f64(y), ref)
+    assert ok, err
+
+
+def test_ffn_zero_inputs_give_zero():
+    w = FFNWorkload("t", 256, 256, 384, 128, 10)
+    x, w1, w2, w3 = ffn_inputs(w)
+    assert torch.count_nonzero(run_ffn(torch.zeros_like(x), w1, w2, w3, 128)) == 0
+    assert torch.count_nonzero(run_ffn(x, w1, w2, torch.zeros_like(w3), 128)) == 0
+
+
+def test_ffn_chunking_does_not_change_rows():
+    w = FFNWorkload("t", 1024, 256, 512, 128, 11)
+    x, w1, w2, w3 = ffn_inputs(w)
+    a = run_ffn(x, w1, w2, w3, 128)
+    b = run_ffn(x, w1, w2, w3, 1024)
+    assert torch.equal(a, b)  # rows are independent: bit-identical
+
+
+def test_ffn_7b_shape_sampled_rows():
+    """The 7B layer's FFN shape (4096 -> 11008 -> 4096, 2048-token chunks)
+    on two chunks; 64 seeded rows checked against fp64."""
+    w = FFN_WORKLOADS["layer7b_ffn"]
+    x, w1, w2, w3 = ffn_inputs(w, T=4096)
+    y = run_ffn(x, w1, w2, w3, w.chunk)
+    rows = np.sort(np.random.default_rng(w.seed + 1000).choice(4096, 64, replace=False))
+    rows[0], rows[-1] = 0, 4095
+    idx = torch.as_tensor(rows, device="cuda")
+    ref = oracle.swiglu_ffn(to_f64(x[idx]), to_f64(w1), to_f64(w2), to_f64(w3))
+    ok, err = within(to_f64(y[idx]), ref)
+    assert ok, err
