@@ -89,6 +89,21 @@ def ffn_flops(f):
     return 6.0 * f.T * f.d_model * f.d_ff
 
 
+def max_over_ranks(x: float, dist=None, device=None) -> float:
+    """The largest value of x over all ranks (a no-op with one process)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank: float, world: int, ms_step: float) -> float:
+    """Weak scaling: every rank did flops_per_rank in (at most) ms_step."""
+    return flops_per_rank * world / (ms_step * 1e-3) / 1e12
+
+
 def describe(aw, fw):
     d = {"workload": f"{aw.name}: ring attention {'fwd+bwd' if aw.bwd else 'fwd'}, B={aw.B}, H={aw.H}, "
                      f"N={aw.N}, d={aw.D}, S={aw.S}, q_chunk={aw.q_chunk}, k_chunk={aw.k_chunk}, "
@@ -335,15 +350,11 @@ def main():
     clk = clocks.stop()
     if ra.ringattn_get_error() != 0:
         raise RuntimeError("device status word set during the timed region")
-    ms_total = t_start.elapsed_time(t_stop)
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(t_start.elapsed_time(t_stop), dist if world > 1 else None, dev)
     ms_step = ms_total / args.steps
 
     flops_step = attn_step_flops(aw) + (ffn_flops(fw) if fw else 0.0)
-    value = flops_step * world / (ms_step * 1e-3) / 1e12
+    value = whole_job_tflops(flops_step, world, ms_step)
     tokens_s = aw.B * aw.N * world / (ms_step * 1e-3)
     pk = peaks()
 
@@ -405,12 +416,8 @@ def main():
                 h.copy_(d_, non_blocking=True)
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b) / e2e_steps
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        line["e2e"] = {"value": flops_step * world / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, dist if world > 1 else None, dev)
+        line["e2e"] = {"value": whole_job_tflops(flops_step, world, e_ms), "unit": "TFLOP/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
                        "steps": e2e_steps}
 
