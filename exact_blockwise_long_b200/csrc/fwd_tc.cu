@@ -103,6 +103,149 @@ struct RingWalk {
   }
 };
 
+// ---------------------------------------------------------------------------
+// Softmax pieces shared by both kernels.  One thread owns one query row
+// (one TMEM lane) of a 128 x 128 score tile, so the row max and the row sum
+// never leave the thread; they are reduced over several independent partial
+// accumulators to keep the dependency chains short.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void load_scores(uint32_t tS, float (&s)[kBN]) {
+  uint32_t a[32], b[32], c[32], d[32];
+  tmem_ld32(tS, a);
+  tmem_ld32(tS + 32, b);
+  tmem_ld32(tS + 64, c);
+  tmem_ld32(tS + 96, d);
+  tmem_ld_wait();
+#pragma unroll
+  for (int x = 0; x < 32; ++x) {
+    s[x] = __uint_as_float(a[x]);
+    s[32 + x] = __uint_as_float(b[x]);
+    s[64 + x] = __uint_as_float(c[x]);
+    s[96 + x] = __uint_as_float(d[x]);
+  }
+}
+
+// Causal mask inside the diagonal tile: key c is in the future of row r.
+__device__ __forceinline__ void mask_future(float (&s)[kBN], int r) {
+#pragma unroll
+  for (int c = 0; c < kBN; ++c)
+    if (c > r) s[c] = -INFINITY;
+}
+
+__device__ __forceinline__ float row_max(const float (&s)[kBN]) {
+  float m[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m[k] = max3f(s[k], s[k + 8], s[k + 16]);
+#pragma unroll
+  for (int x = 24; x < 120; x += 16)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m[k] = max3f(m[k], s[x + k], s[x + 8 + k]);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m[k] = fmaxf(m[k], s[120 + k]);
+  return max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+}
+
+// P = 2^(s * scale * log2(e) - m) as bf16 pairs over the first 64 columns of
+// the tile's TMEM (P of keys 2c, 2c+1 in column c); returns the row sum of
+// the fp32 probabilities.  Masked scores are -inf and give exactly 0.
+__device__ __forceinline__ float exp_store(const float (&s)[kBN], uint32_t tS, float sl2, float m) {
+  const float2 k2 = make_float2(sl2, sl2), nm2 = make_float2(-m, -m);
+  float2 acc[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int x = 0; x < 32; ++x) {
+      const float2 t = fma2(make_float2(s[h * 64 + 2 * x], s[h * 64 + 2 * x + 1]), k2, nm2);
+      const float2 pr = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+      acc[x & 3] = add2(acc[x & 3], pr);
+      pk[x] = pack_bf16x2(pr.x, pr.y);
+    }
+    tmem_st32(tS + h * 32, pk);
+  }
+  const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
+  const float2 t = add2(a01, a23);
+  return t.x + t.y;
+}
+
+// Multiply this row of O (D fp32 columns in TMEM) by alpha.
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
+#pragma unroll
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t reg[32];
+    tmem_ld32(tO + cc * 32, reg);
+    tmem_ld_wait();
+#pragma unroll
+    for (int x = 0; x < 32; ++x) reg[x] = __float_as_uint(__uint_as_float(reg[x]) * alpha);
+    tmem_st32(tO + cc * 32, reg);
+  }
+}
+
+// Final O / l and LSE of one query row held by this thread (TMEM lane), or,
+// in ring-step mode, the exact merge of that row's normalised partial into
+// the fp32 running accumulators in HBM.  tO: TMEM address of the row's O.
+template <int D>
+__device__ __forceinline__ void store_row(uint32_t tO, float m_run, float l_run, int grow, const Params& p) {
+  const float lse_t = (m_run + __log2f(l_run)) * kLn2;
+  const float inv = 1.f / l_run;
+  if (p.step < 0) {
+    __nv_bfloat16* orow = p.out + (size_t)grow * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t reg[32];
+      tmem_ld32(tO + c * 32, reg);
+      tmem_ld_wait();
+      uint32_t pk[16];
+#pragma unroll
+      for (int x = 0; x < 16; ++x)
+        pk[x] = pack_bf16x2(__uint_as_float(reg[2 * x]) * inv, __uint_as_float(reg[2 * x + 1]) * inv);
+      uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+      for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+    }
+    p.lse[grow] = lse_t;
+  } else {
+    const float lse_a = p.lse_acc[grow];
+    float wa = 0.f, wb = 1.f, lse_new = lse_t;
+    if (lse_a != -INFINITY) {
+      const float mx2 = fmaxf(lse_a, lse_t);
+      const float ea = expf(lse_a - mx2), eb = expf(lse_t - mx2);
+      const float tot = ea + eb;
+      lse_new = mx2 + logf(tot);
+      wa = ea / tot;
+      wb = eb / tot;
+    }
+    float* arow = p.o_acc + (size_t)grow * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t reg[32];
+      tmem_ld32(tO + c * 32, reg);
+      tmem_ld_wait();
+      float4* dst = reinterpret_cast<float4*>(arow + c * 32);
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        float4 o4;
+        o4.x = __uint_as_float(reg[4 * x + 0]) * inv * wb;
+        o4.y = __uint_as_float(reg[4 * x + 1]) * inv * wb;
+        o4.z = __uint_as_float(reg[4 * x + 2]) * inv * wb;
+        o4.w = __uint_as_float(reg[4 * x + 3]) * inv * wb;
+        if (wa != 0.f) {
+          const float4 a4 = dst[x];
+          o4.x = fmaf(wa, a4.x, o4.x);
+          o4.y = fmaf(wa, a4.y, o4.y);
+          o4.z = fmaf(wa, a4.z, o4.z);
+          o4.w = fmaf(wa, a4.w, o4.w);
+        }
+        dst[x] = o4;
+      }
+    }
+    p.lse_acc[grow] = lse_new;
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -254,23 +397,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(&bar_sf[sb], (n >> 1) & 1, p.st, abort_flag))) return false;
       tc_fence_after();
       float s[kBN];
-#pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t reg[32];
-        tmem_ld32(tS + c * 32, reg);
-        tmem_ld_wait();
-#pragma unroll
-        for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(reg[x]);
-      }
-      if (diag) {
-#pragma unroll
-        for (int c = 0; c < kBN; ++c)
-          if (c > r) s[c] = -INFINITY;
-      }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
-      const float m_new = fmaxf(m_run, mx * sl2);
+      load_scores(tS, s);
+      if (diag) mask_future(s, r);
+      const float m_new = fmaxf(m_run, row_max(s) * sl2);
       if (n == 0) {
         m_run = m_new;
       } else if (__any_sync(0xffffffffu, m_new > m_run + kRescaleLog2)) {
@@ -281,31 +410,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const float alpha = ex2_approx(m_run - m_new);
         l_run *= alpha;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t reg[32];
-          tmem_ld32(tO + lane_off + c * 32, reg);
-          tmem_ld_wait();
-#pragma unroll
-          for (int x = 0; x < 32; ++x) reg[x] = __float_as_uint(__uint_as_float(reg[x]) * alpha);
-          tmem_st32(tO + lane_off + c * 32, reg);
-        }
+        rescale_o<D>(tO + lane_off, alpha);
         m_run = m_new;
       }
-      const float neg_m = -m_run;
-      float rowsum = 0.f;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const float p0 = ex2_approx(fmaf(s[h * 64 + 2 * x], sl2, neg_m));
-          const float p1 = ex2_approx(fmaf(s[h * 64 + 2 * x + 1], sl2, neg_m));
-          rowsum += p0 + p1;
-          pk[x] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(tS + h * 32, pk);
-      }
+      const float rowsum = exp_store(s, tS, sl2, m_run);
       tmem_st_wait();
       l_run += rowsum;
       tc_fence_before();
@@ -315,69 +423,289 @@ __global__ void __launch_bounds__(kThreads, 1)
     });
     if (ok && __all_sync(0xffffffffu, mbar_wait(bar_od, (n - 1) & 1, p.st, abort_flag))) {
       tc_fence_after();
-      const int grow = qrow0 + r;  // row of the [BH*N, D] view
-      const float lse_t = (m_run + __log2f(l_run)) * kLn2;
-      const float inv = 1.f / l_run;
-      if (p.step < 0) {
-        __nv_bfloat16* orow = p.out + (size_t)grow * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t reg[32];
-          tmem_ld32(tO + lane_off + c * 32, reg);
-          tmem_ld_wait();
-          uint32_t pk[16];
-#pragma unroll
-          for (int x = 0; x < 16; ++x)
-            pk[x] = pack_bf16x2(__uint_as_float(reg[2 * x]) * inv, __uint_as_float(reg[2 * x + 1]) * inv);
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
-        }
-        p.lse[grow] = lse_t;
-      } else {
-        // fused exact merge into the running fp32 accumulators in HBM
-        const float lse_a = p.lse_acc[grow];
-        float wa = 0.f, wb = 1.f, lse_new = lse_t;
-        if (lse_a != -INFINITY) {
-          const float mx2 = fmaxf(lse_a, lse_t);
-          const float ea = expf(lse_a - mx2), eb = expf(lse_t - mx2);
-          const float tot = ea + eb;
-          lse_new = mx2 + logf(tot);
-          wa = ea / tot;
-          wb = eb / tot;
-        }
-        float* arow = p.o_acc + (size_t)grow * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t reg[32];
-          tmem_ld32(tO + lane_off + c * 32, reg);
-          tmem_ld_wait();
-          float4* dst = reinterpret_cast<float4*>(arow + c * 32);
-#pragma unroll
-          for (int x = 0; x < 8; ++x) {
-            float4 o4;
-            o4.x = __uint_as_float(reg[4 * x + 0]) * inv * wb;
-            o4.y = __uint_as_float(reg[4 * x + 1]) * inv * wb;
-            o4.z = __uint_as_float(reg[4 * x + 2]) * inv * wb;
-            o4.w = __uint_as_float(reg[4 * x + 3]) * inv * wb;
-            if (wa != 0.f) {
-              const float4 a4 = dst[x];
-              o4.x = fmaf(wa, a4.x, o4.x);
-              o4.y = fmaf(wa, a4.y, o4.y);
-              o4.z = fmaf(wa, a4.z, o4.z);
-              o4.w = fmaf(wa, a4.w, o4.w);
-            }
-            dst[x] = o4;
-          }
-        }
-        p.lse_acc[grow] = lse_new;
-      }
+      store_row<D>(tO + lane_off, m_run, l_run, qrow0 + r, p);
     }
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Two query tiles per CTA (256 rows), used when the shard length is a
+// multiple of 256.  Two softmax warpgroups, one per 128-row tile, take turns
+// with the tensor core: while one warpgroup turns its scores into
+// probabilities the MMA warp runs the other tile's P V and Q K^T, so the
+// exponentials of one tile overlap the MMAs of the other.
+//   warps 0-3  softmax + epilogue of tile 0 (TMEM lanes 0-127)
+//   warps 4-7  softmax + epilogue of tile 1
+//   warp 8     TMEM allocator, then (one lane) TMA producer
+//   warp 9     MMA issuer (one lane); warps 10-11 idle
+// The softmax warpgroups take registers from the third warpgroup so each
+// softmax thread holds its row of 128 scores in registers.
+// Tensor memory: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [384,384+D);
+// P of each tile is written as bf16 over the first 64 columns of its S.
+// MMA issue order per key tile n: S0_n, PV1_{n-1}, S1_n, PV0_n.  A tile's
+// S_n is issued after its PV_{n-1}, so once a softmax warp sees S_n complete
+// the O it may rescale holds every earlier tile's P V already.
+// ---------------------------------------------------------------------------
+constexpr int kThreads2 = 384;
+// Register split: launched at kLaunchRegs per thread (384 x 168 = 64512);
+// the softmax warpgroups rise to kSoftmaxRegs, the producer/MMA warpgroup
+// drops to kOtherRegs: 256 x 200 + 128 x 104 = 64512.  Per sub-partition:
+// 2 x 32 x 200 + 32 x 104 = 16128 of 16384.  The host launches this kernel
+// only when the compiled register count equals kLaunchRegs.
+constexpr int kLaunchRegs = 168;
+constexpr uint32_t kSoftmaxRegs = 200;
+constexpr uint32_t kOtherRegs = 104;
+static_assert(256 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads2 * kLaunchRegs, "register split exceeds launch");
+
+template <int D>
+struct Layout2 {
+  static constexpr int kTileBytes = kBM * D * 2;
+  static constexpr int kSlabBytes = kBM * 128;
+  static constexpr int kQ = 0;  // Q0, Q1
+  static constexpr int kK = 2 * kTileBytes;
+  static constexpr int kV = kK + kKSt * kTileBytes;
+  static constexpr int kBar = kV + kVSt * kTileBytes;
+  static constexpr int kNumBars = 1 + 2 * kKSt + 2 * kVSt + 2 + 2 + 1;
+  static constexpr int kTmemSlot = kBar + kNumBars * 8;
+  static constexpr int kAbort = kTmemSlot + 4;
+  static constexpr int kBytes = kAbort + 4;
+  static constexpr int kAlloc = kBytes + 1024;  // slack for aligning the base to 1024
+};
+static_assert(Layout2<128>::kAlloc <= 232448, "forward tile set exceeds shared memory");
+
+// Key tiles met by a pair of query tiles (qt0, qt0 + 1) of one shard, in
+// ring order.  Under the causal mask the last key tile of the diagonal shard
+// (qt0 + 1) lies entirely in the future of tile 0, which skips it.
+struct PairWalk {
+  int ishard, S, tps, qt0, causal, step;
+  template <typename F>
+  __device__ __forceinline__ bool run(F&& body) const {
+    for (int t = 0; t < S; ++t) {
+      if (step >= 0 && t != step) continue;
+      int j = ishard - t;
+      if (j < 0) j += S;
+      if (causal && j > ishard) continue;
+      const int kt0 = j * tps;
+      const int kt1 = (causal && j == ishard) ? qt0 + 2 : kt0 + tps;
+      for (int kt = kt0; kt < kt1; ++kt)
+        if (!body(kt, !(causal && kt > qt0), causal && kt == qt0, causal && kt == qt0 + 1)) return false;
+    }
+    return true;
+  }
+  __device__ __forceinline__ int count() const {
+    int n = 0;
+    for (int t = 0; t < S; ++t) {
+      if (step >= 0 && t != step) continue;
+      int j = ishard - t;
+      if (j < 0) j += S;
+      if (causal && j > ishard) continue;
+      n += (causal && j == ishard) ? (qt0 + 2 - j * tps) : tps;
+    }
+    return n;
+  }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads2, 1)
+    fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const Params p) {
+  using LY = Layout2<D>;
+  extern __shared__ uint8_t smem_raw2[];
+  uint8_t* smem = smem_raw2 + ((1024 - (smem_u32(smem_raw2) & 1023)) & 1023);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int num_pairs = p.num_qtiles / 2;
+  const int pair = num_pairs - 1 - (int)(blockIdx.x / p.BH);  // heaviest causal pairs first
+  const int bh = (int)(blockIdx.x % p.BH);
+  const int qt0 = 2 * pair;
+  const int qrow0 = bh * p.N + qt0 * kBM;
+  PairWalk walk{(qt0 * kBM) / p.L, p.S, p.L / kBN, qt0, p.causal, p.step};
+  if (walk.count() == 0) return;  // step mode, causal pair skipped
+
+  uint8_t* sQ = smem + LY::kQ;
+  uint8_t* sK = smem + LY::kK;
+  uint8_t* sV = smem + LY::kV;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + LY::kBar);
+  uint64_t* bar_q = bars;
+  uint64_t* bar_kf = bar_q + 1;
+  uint64_t* bar_ke = bar_kf + kKSt;
+  uint64_t* bar_vf = bar_ke + kKSt;
+  uint64_t* bar_ve = bar_vf + kVSt;
+  uint64_t* bar_sf = bar_ve + kVSt;  // [2] S of tile t computed
+  uint64_t* bar_pf = bar_sf + 2;     // [2] P of tile t written
+  uint64_t* bar_done = bar_pf + 2;   // every MMA finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + LY::kTmemSlot);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LY::kAbort);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < kKSt; ++s) {
+      mbar_init(&bar_kf[s], 1);
+      mbar_init(&bar_ke[s], 1);
+    }
+    for (int s = 0; s < kVSt; ++s) {
+      mbar_init(&bar_vf[s], 1);
+      mbar_init(&bar_ve[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bar_sf[t], 1);
+      mbar_init(&bar_pf[t], 128);
+    }
+    mbar_init(bar_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= 8) {
+   regs_dec<kOtherRegs>();
+   if (warp == 8) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(bar_q, 2 * LY::kTileBytes);
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int s = 0; s < D / 64; ++s)
+          tma_load_2d(sQ + t * LY::kTileBytes + s * LY::kSlabBytes, &tmQ, bar_q, s * 64, qrow0 + t * kBM);
+      int n = 0;
+      walk.run([&](int kt, bool, bool, bool) {
+        const int krow = bh * p.N + kt * kBN;
+        const int ks = n % kKSt, vs = n % kVSt;
+        if (!mbar_wait(&bar_ke[ks], ((n / kKSt) & 1) ^ 1, p.st, abort_flag)) return false;
+        mbar_arrive_expect_tx(&bar_kf[ks], LY::kTileBytes);
+#pragma unroll
+        for (int s = 0; s < D / 64; ++s)
+          tma_load_2d(sK + ks * LY::kTileBytes + s * LY::kSlabBytes, &tmK, &bar_kf[ks], s * 64, krow);
+        if (!mbar_wait(&bar_ve[vs], ((n / kVSt) & 1) ^ 1, p.st, abort_flag)) return false;
+        mbar_arrive_expect_tx(&bar_vf[vs], LY::kTileBytes);
+#pragma unroll
+        for (int s = 0; s < D / 64; ++s)
+          tma_load_2d(sV + vs * LY::kTileBytes + s * LY::kSlabBytes, &tmV, &bar_vf[vs], s * 64, krow);
+        ++n;
+        return true;
+      });
+    }
+  } else if (warp == 9) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t idS = idesc_bf16_f32(kBM, kBN, false, false);
+      constexpr uint32_t idPV = idesc_bf16_f32(kBM, D, false, true);
+      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
+      int n = 0, prev_vs = 0;
+      int pv_cnt[2] = {0, 0};
+      auto issue_s = [&](int t, uint32_t kb) {
+        const uint32_t qb = q_base + t * LY::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * LY::kSlabBytes + (kk & 3) * 32;
+          mma_bf16_ss(tmem + t * 128, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idS,
+                      kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bar_sf[t]);
+      };
+      auto issue_pv = [&](int t, int vs) -> bool {
+        if (!mbar_wait(&bar_pf[t], pv_cnt[t] & 1, p.st, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t vb = v_base + vs * LY::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
+                      sdesc_sw128(vb + kk * 16 * 128, LY::kSlabBytes, 1024), idPV,
+                      (pv_cnt[t] > 0 || kk > 0) ? 1u : 0u);
+        ++pv_cnt[t];
+        return true;
+      };
+      bool ok = mbar_wait(bar_q, 0, p.st, abort_flag);
+      if (ok) {
+        ok = walk.run([&](int, bool do0, bool, bool) {
+          const int ks = n % kKSt, vs = n % kVSt;
+          if (!mbar_wait(&bar_kf[ks], (n / kKSt) & 1, p.st, abort_flag)) return false;
+          tc_fence_after();
+          const uint32_t kb = k_base + ks * LY::kTileBytes;
+          if (do0) issue_s(0, kb);
+          if (n > 0) {
+            if (!issue_pv(1, prev_vs)) return false;
+            mma_commit(&bar_ve[prev_vs]);
+          }
+          issue_s(1, kb);
+          mma_commit(&bar_ke[ks]);
+          if (!mbar_wait(&bar_vf[vs], (n / kVSt) & 1, p.st, abort_flag)) return false;
+          if (do0 && !issue_pv(0, vs)) return false;
+          prev_vs = vs;
+          ++n;
+          return true;
+        });
+        if (ok && n > 0 && issue_pv(1, prev_vs)) mma_commit(&bar_ve[prev_vs]);
+      }
+      mma_commit(bar_done);
+    }
+   }
+  } else {
+    regs_inc<kSoftmaxRegs>();
+    // ---------------- softmax / correction / epilogue of one tile ----------------
+    constexpr uint32_t FULL = 0xffffffffu;
+    const int tile = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + tile * 128 + lane_off;
+    const uint32_t tO = tmem + 256 + tile * 128 + lane_off;
+    const float sl2 = p.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;
+    int c = 0;
+    const bool ok = walk.run([&](int, bool do0, bool diag0, bool diag1) {
+      if (tile == 0 && !do0) return true;
+      const bool diag = tile ? diag1 : diag0;
+      if (!__all_sync(FULL, mbar_wait(&bar_sf[tile], c & 1, p.st, abort_flag))) return false;
+      tc_fence_after();
+      float s[kBN];
+      load_scores(tS, s);
+      if (diag) mask_future(s, r);
+      const float m_new = fmaxf(m_run, row_max(s) * sl2);
+      if (c == 0) {
+        m_run = m_new;
+      } else if (__any_sync(FULL, m_new > m_run + kRescaleLog2)) {
+        // this tile's S is complete, hence so is its previous P V: rescale O
+        const float alpha = ex2_approx(m_run - m_new);
+        l_run *= alpha;
+        rescale_o<D>(tO, alpha);
+        m_run = m_new;
+      }
+      const float rowsum = exp_store(s, tS, sl2, m_run);
+      tmem_st_wait();
+      l_run += rowsum;
+      tc_fence_before();
+      mbar_arrive(&bar_pf[tile]);
+      ++c;
+      return true;
+    });
+    if (ok && __all_sync(FULL, mbar_wait(bar_done, 0, p.st, abort_flag))) {
+      tc_fence_after();
+      store_row<D>(tO, m_run, l_run, qrow0 + tile * kBM + r, p);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -406,10 +734,23 @@ int launch_d(const AttnArgs& a, void* out, float* lse, float* o_acc, float* lse_
   p.scale_log2 = a.scale * 1.4426950408889634f;
   int rc = current_status(&p.st);
   if (rc != RA_OK) return rc;
-  auto kern = fwd_tc_kernel<D>;
-  if (set_smem_attr((const void*)kern, Layout<D>::kAlloc) != RA_OK) return RA_ERR_CUDA;
-  const unsigned grid = (unsigned)(p.BH * p.num_qtiles);
-  kern<<<grid, kThreads, Layout<D>::kAlloc, stream>>>(tq, tk, tv, p);
+  bool two_tiles = (p.L % (2 * kBM) == 0);
+  if (two_tiles) {
+    cudaFuncAttributes fa;
+    two_tiles = cudaFuncGetAttributes(&fa, (const void*)fwd_tc2_kernel<D>) == cudaSuccess &&
+                fa.numRegs == kLaunchRegs;
+  }
+  if (two_tiles) {
+    auto kern = fwd_tc2_kernel<D>;
+    if (set_smem_attr((const void*)kern, Layout2<D>::kAlloc) != RA_OK) return RA_ERR_CUDA;
+    const unsigned grid = (unsigned)(p.BH * (p.num_qtiles / 2));
+    kern<<<grid, kThreads2, Layout2<D>::kAlloc, stream>>>(tq, tk, tv, p);
+  } else {
+    auto kern = fwd_tc_kernel<D>;
+    if (set_smem_attr((const void*)kern, Layout<D>::kAlloc) != RA_OK) return RA_ERR_CUDA;
+    const unsigned grid = (unsigned)(p.BH * p.num_qtiles);
+    kern<<<grid, kThreads, Layout<D>::kAlloc, stream>>>(tq, tk, tv, p);
+  }
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
