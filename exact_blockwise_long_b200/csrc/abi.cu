@@ -62,6 +62,17 @@ int make_tmap_bf16_2d(void* tmap, const void* base, uint64_t inner, uint64_t row
   return r == CUDA_SUCCESS ? RA_OK : RA_ERR_CUDA;
 }
 
+int head_group(int per_head, int heads, double bytes_per_head, double budget_bytes) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int g_waves = (2 * sms + per_head - 1) / per_head;
+  const double g_fit = budget_bytes / (bytes_per_head > 1.0 ? bytes_per_head : 1.0);
+  int g = g_fit > (double)g_waves ? (g_fit > 1e6 ? 1000000 : (int)g_fit) : g_waves;
+  if (g < 1) g = 1;
+  if (g > heads) g = heads;
+  return g;
+}
+
 int set_smem_attr(const void* func, int bytes) {
   return cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
              ? RA_OK

@@ -63,6 +63,7 @@ struct BParams {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int BH, N, S, L, causal, num_tiles;
+  int group;  // heads per scheduling group
   float scale, scale_log2;
   DevStatus st;
 };
@@ -99,9 +100,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
-  // Work item: heaviest causal key tiles (smallest index) first.
-  const int kt = (int)(blockIdx.x / p.BH);
-  const int bh = (int)(blockIdx.x % p.BH);
+  // Work item: heads in small groups, so the CTAs in flight share a few
+  // heads' Q, dO and dQ accumulator in L2; the heaviest causal key tiles
+  // (smallest index) come first.
+  int bh, kt;
+  grouped_order((int)blockIdx.x, p.num_tiles, p.BH, p.group, bh, kt);
   const int krow0 = bh * p.N + kt * kT;
   const int tps = p.L / kT;
   RingWalkKV walk{(kt * kT) / p.L, p.S, tps, kt, p.causal};
@@ -470,6 +473,8 @@ int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* d
   p.L = (int)(a.N / a.S);
   p.causal = a.causal;
   p.num_tiles = (int)(a.N / kT);
+  // per head: Q, dO, K, V (bf16) and the fp32 dQ accumulator
+  p.group = head_group(p.num_tiles, p.BH, (double)a.N * D * (4 * 2 + 4), 100.0e6);
   p.scale = a.scale;
   p.scale_log2 = a.scale * kLog2e;
   int rc = current_status(&p.st);

@@ -248,6 +248,25 @@ __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
+// Grid order for attention work items
+// ---------------------------------------------------------------------------
+// Heads are taken in groups of `group` (the last group may be smaller); the
+// work items of a group are interleaved across its heads, heaviest tile
+// first.  Small groups keep the CTAs in flight on few heads (their K, V, Q,
+// dO and dQ stay in L2); the group size is chosen on the host so a group
+// still fills a couple of waves of SMs.  Returns (head, rank) where rank 0 is
+// the heaviest tile of the head.
+__device__ __forceinline__ void grouped_order(int block, int per_head, int heads, int group, int& head,
+                                              int& rank) {
+  const int g = block / (group * per_head);
+  const int in = block - g * group * per_head;
+  const int g0 = g * group;
+  const int gh = min(group, heads - g0);
+  rank = in / gh;
+  head = g0 + in % gh;
+}
+
+// ---------------------------------------------------------------------------
 // Arithmetic helpers
 // ---------------------------------------------------------------------------
 // Hardware base-2 exponential (MUFU.EX2).

@@ -69,6 +69,7 @@ struct Params {
   float* lse_acc;   // step mode: fp32 running lse
   int BH, N, S, L, causal, step;
   int num_qtiles;
+  int group;  // heads per scheduling group
   float scale_log2;
   DevStatus st;
 };
@@ -257,9 +258,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work item: heaviest causal query tiles are scheduled first.
-  const int qt = p.num_qtiles - 1 - (int)(blockIdx.x / p.BH);
-  const int bh = (int)(blockIdx.x % p.BH);
+  // Work item: heads in small groups, heaviest causal query tiles first.
+  int bh, rank;
+  grouped_order((int)blockIdx.x, p.num_qtiles, p.BH, p.group, bh, rank);
+  const int qt = p.num_qtiles - 1 - rank;
   const int q0 = qt * kBM;
   const int qrow0 = bh * p.N + q0;
   RingWalk walk{q0 / p.L, p.S, p.L / kBN, qt, p.causal, p.step};
@@ -522,9 +524,12 @@ __global__ void __launch_bounds__(kThreads2, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  // Heads in small groups (their K and V stay in L2), heaviest causal query
+  // pairs first.
   const int num_pairs = p.num_qtiles / 2;
-  const int pair = num_pairs - 1 - (int)(blockIdx.x / p.BH);  // heaviest causal pairs first
-  const int bh = (int)(blockIdx.x % p.BH);
+  int bh, rank;
+  grouped_order((int)blockIdx.x, num_pairs, p.BH, p.group, bh, rank);
+  const int pair = num_pairs - 1 - rank;
   const int qt0 = 2 * pair;
   const int qrow0 = bh * p.N + qt0 * kBM;
   PairWalk walk{(qt0 * kBM) / p.L, p.S, p.L / kBN, qt0, p.causal, p.step};
@@ -740,6 +745,8 @@ int launch_d(const AttnArgs& a, void* out, float* lse, float* o_acc, float* lse_
     two_tiles = cudaFuncGetAttributes(&fa, (const void*)fwd_tc2_kernel<D>) == cudaSuccess &&
                 fa.numRegs == kLaunchRegs;
   }
+  // per head the key/value tiles every query tile streams through
+  p.group = head_group(two_tiles ? p.num_qtiles / 2 : p.num_qtiles, p.BH, 2.0 * a.N * D * 2, 60.0e6);
   if (two_tiles) {
     auto kern = fwd_tc2_kernel<D>;
     if (set_smem_attr((const void*)kern, Layout2<D>::kAlloc) != RA_OK) return RA_ERR_CUDA;

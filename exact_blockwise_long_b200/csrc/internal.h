@@ -55,6 +55,11 @@ int launch_selftest_timeout(int timeout_us, cudaStream_t stream);
 int make_tmap_bf16_2d(void* tmap /* CUtensorMap* */, const void* base, uint64_t inner, uint64_t rows,
                       uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_rows);
 
+// Head-group size for grouped_order: as many heads as keep their working
+// set (bytes_per_head) within budget_bytes of the 126 MB L2, but enough that
+// a group holds two waves of work items; at least one, at most `heads`.
+int head_group(int per_head, int heads, double bytes_per_head, double budget_bytes);
+
 // Opt a kernel into more than 48 KB of dynamic shared memory.
 int set_smem_attr(const void* func, int bytes);
 
