@@ -40,14 +40,7 @@ METRIC = "ring-attn fwd+bwd TFLOP/s & tokens/s on 1 B200; % of BF16 tensor peak"
 # source it was taken on (sha256 of the source file).
 # Captured on 8 heads of the n32k_d128 workload and scaled x4 to its 32 heads
 # (heads are independent units; see profiles/*_n32k_d128_h8.md).
-NCU_TRAFFIC = {
-    ("bwd_tc_kernel", "n32k_d128"): {
-        "bytes": 4 * (1.981993e9 + 1.020117e9),
-        "sha256": "e06329c00d98f3e52db8c2e1a033de7de3074db543e82d5c8047b6c411731676"},
-    ("fwd_tc_kernel", "n32k_d128"): {
-        "bytes": 4 * (885.399040e6 + 49.013248e6),
-        "sha256": "26b9afff19374c15dd6c7df4a19c6b061c4c89d40db9dc13f8c0d13b00d4d2bc"},
-}
+NCU_TRAFFIC = {}
 
 
 def parse():
@@ -303,7 +296,7 @@ def main():
 
     def step(timed=False):
         if timed:
-            e = [event() for _ in range(4)]
+            e = [event() for _ in range(5)]
             e[0].record(stream)
         ra.ringattn_fwd(q, k, v, o, lse, *cfg)
         launches = 1
@@ -317,6 +310,8 @@ def main():
             if timed:
                 e[3].record(stream)
             ra.ringattn_bwd_phase(q, k, v, o, lse, do, dq, dk, dv, *cfg, ws, 4)
+            if timed:
+                e[4].record(stream)
             launches += 3
         if fw is not None:
             ra.blockwise_ffn(x, w1, w2, w3, y, fw.chunk, ffn_ws)
@@ -324,7 +319,8 @@ def main():
         if timed:
             ev.setdefault("fwd", []).append((e[0], e[1]))
             if aw.bwd:
-                ev.setdefault("bwd_main", []).append((e[2], e[3]))
+                ev.setdefault("bwd_kv", []).append((e[2], e[3]))
+                ev.setdefault("bwd_q", []).append((e[3], e[4]))
         return launches
 
     for _ in range(args.warmup):
@@ -362,15 +358,18 @@ def main():
     def mean_ms(pairs):
         return sum(a.elapsed_time(b) for a, b in pairs) / len(pairs)
 
+    # Algorithmic FLOPs per launch: the forward's two matmuls; the dK/dV
+    # kernel's four (S, dP, dV, dK), the dQ kernel's one (dQ; its S and dP
+    # are recomputation, not credited): 2 + 4 + 1 = 7 = 3.5 x the forward's 2.
+    fwd_fl = attn_fwd_flops(aw)
+    kernels = {"fwd_tc_kernel": (mean_ms(ev["fwd"]), fwd_fl, "fwd_tc.cu")}
     if aw.bwd:
-        kname, kms = "bwd_tc_kernel", mean_ms(ev["bwd_main"])
-        kflops = attn_fwd_flops(aw) * 2.5
-    else:
-        kname, kms = "fwd_tc_kernel", mean_ms(ev["fwd"])
-        kflops = attn_fwd_flops(aw)
+        kernels["bwd_kv_kernel"] = (mean_ms(ev["bwd_kv"]), 2.0 * fwd_fl, "bwd_tc.cu")
+        kernels["bwd_q_kernel"] = (mean_ms(ev["bwd_q"]), 0.5 * fwd_fl, "bwd_tc.cu")
+    kname = max(kernels, key=lambda k_: kernels[k_][0])
+    kms, kflops, ksrc = kernels[kname]
     achieved = kflops / (kms * 1e-3) / 1e12
-    src = os.path.join(ROOT, "exact_blockwise_long_b200", "csrc",
-                       "bwd_tc.cu" if kname.startswith("bwd") else "fwd_tc.cu")
+    src = os.path.join(ROOT, "exact_blockwise_long_b200", "csrc", ksrc)
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
     tr = NCU_TRAFFIC.get((kname, args.workload))
     traffic = tr["bytes"] if tr and tr["sha256"] == sha else None
@@ -378,8 +377,8 @@ def main():
             "unit": "TFLOP/s", "frac": achieved / pk["bf16_sustained"], "traffic": traffic,
             "peak_kind": f"bf16 dense, sustained ({pk['source']})",
             "frac_of_burst": achieved / pk["bf16_burst"], "kernel_ms": kms,
-            "fwd_kernel_ms": mean_ms(ev["fwd"]),
-            "fwd_tflops": attn_fwd_flops(aw) / (mean_ms(ev["fwd"]) * 1e-3) / 1e12}
+            "kernels": {k_: {"ms": v_[0], "algorithmic_tflops": v_[1] / (v_[0] * 1e-3) / 1e12}
+                        for k_, v_ in kernels.items()}}
 
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",

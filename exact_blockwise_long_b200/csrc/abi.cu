@@ -196,9 +196,8 @@ int ringattn_merge(float* o_a, float* lse_a, const float* o_b, const float* lse_
 
 size_t ringattn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D) {
   if (B <= 0 || H <= 0 || N <= 0 || D <= 0) return 0;  // empty problems need no workspace
-  const size_t dq = (size_t)B * H * N * D * sizeof(float);
   const size_t dvec = (size_t)B * H * N * sizeof(float);
-  return ((dq + 255) & ~(size_t)255) + 2 * ((dvec + 255) & ~(size_t)255);
+  return 2 * ((dvec + 255) & ~(size_t)255);
 }
 
 int ringattn_bwd_phase(const void* q, const void* k, const void* v, const void* out, const float* lse,

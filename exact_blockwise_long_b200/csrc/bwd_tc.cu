@@ -4,26 +4,29 @@
 // abstract) but print no backward algorithm; this is the plain chain rule
 // through the softmax, recomputing P from the forward's log-sum-exp:
 //   P_ij = exp(s_ij - lse_i) on visible pairs,  D_i = dO_i . O_i
-//   dV_j += sum_i P_ij dO_i           dS_ij = P_ij (dO_i . V_j - D_i)
-//   dK_j += scale sum_i dS_ij Q_i     dQ_i += scale sum_j dS_ij K_j
+//   dV_j = sum_i P_ij dO_i            dS_ij = P_ij (dO_i . V_j - D_i)
+//   dK_j = scale sum_i dS_ij Q_i      dQ_i = scale sum_j dS_ij K_j
 //
-// Ring order, turned around for the key side: each CTA keeps one 128-key
-// tile of KV shard j stationary (its dK, dV accumulate in tensor memory) and
-// the query shards pass by in ring order i = (j + t) mod S; under the causal
-// mask pairs i < j are skipped and the diagonal pair is masked in its tiles.
-// The pairs visited are exactly the forward's pairs.
+// Both sides of the ring: the key/value gradients keep a KV tile stationary
+// while the query shards pass by in ring order i = (j + t) mod S (the
+// forward's pairs, loop nest turned around); the query gradient keeps a
+// query tile stationary and visits the KV shards in ring order
+// j = (i - t) mod S, exactly like the forward.  Under the causal mask pairs
+// of shards in the future are skipped and the diagonal pair is masked inside
+// its tiles.  Each gradient accumulates in tensor memory and is written to
+// HBM once, so there are no atomics and the result is deterministic.
 //
 // Three launches:
-//   preprocess  D_i = dO_i . O_i, lse_i * log2(e), dQ accumulator <- 0
-//   main loop   per (key tile, query tile): 5 tcgen05 MMAs
-//                 S^T  = K Q^T        (TMEM cols [0,128))
-//                 dP^T = V dO^T       (TMEM cols [128,256))
-//                 dV  += P^T dO       (P^T bf16 in TMEM over S^T)
-//                 dK  += dS^T Q       (dS^T bf16 in TMEM over dP^T)
-//                 dQ   = dS K         (dS from shared memory, result over dP^T)
-//               dQ is drained from TMEM with fp32 vector reductions into the
-//               dQ accumulator in HBM.
-//   convert     dq = bf16(scale * dQ accumulator)
+//   preprocess  D_i = dO_i . O_i and lse_i * log2(e)             (HBM-bound)
+//   dK/dV       per (key tile, query tile) 4 tcgen05 MMAs:
+//                 S^T  = K Q^T    (TMEM [0,128))
+//                 dP^T = V dO^T   (TMEM [128,256))
+//                 dV  += P^T dO   (P^T bf16 over S^T, A operand from TMEM)
+//                 dK  += dS^T Q   (dS^T bf16 over dP^T, A operand from TMEM)
+//   dQ          per (query tile, key tile) 3 tcgen05 MMAs:
+//                 S    = Q K^T    (TMEM [0,128) / [128,256), double buffered)
+//                 dP   = dO V^T   (TMEM [256,384))
+//                 dQ  += dS K     (dS bf16 through shared memory)
 #include <math.h>
 
 #include "common.cuh"
@@ -32,43 +35,26 @@
 namespace ra {
 namespace {
 
-constexpr int kT = 128;        // keys per CTA (TMEM lanes) and queries per step
-constexpr int kQSt = 2;        // Q / dO stages
+constexpr int kT = 128;        // rows per tile (TMEM lanes)
+constexpr int kSt = 2;         // streamed-tile stages
 constexpr int kThreads = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kTmemCols = 512;
-
-template <int D>
-struct BLayout {
-  static constexpr int kTile = kT * D * 2;   // 128 rows x D bf16 (D/64 slabs of 16 KB)
-  static constexpr int kSlab = kT * 128;
-  static constexpr int kK = 0;
-  static constexpr int kV = kK + kTile;
-  static constexpr int kDS = kV + kTile;          // dS as an MN-major operand: 2 slabs [128 keys][64 queries]
-  static constexpr int kQ = kDS + kT * kT * 2;
-  static constexpr int kDO = kQ + kQSt * kTile;
-  static constexpr int kVec = kDO + kQSt * kTile;  // per stage: lse*log2e [128] and D [128] (fp32)
-  static constexpr int kBar = kVec + kQSt * 1024;
-  static constexpr int kNumBars = 1 + 2 * kQSt + 7;
-  static constexpr int kTmemSlot = kBar + kNumBars * 8;
-  static constexpr int kAbort = kTmemSlot + 4;
-  static constexpr int kBytes = kAbort + 4;
-};
-static_assert(BLayout<128>::kBytes <= 232448, "backward tile set exceeds shared memory");
+constexpr uint32_t FULL = 0xffffffffu;
 
 struct BParams {
-  const float* lse2;   // lse * log2(e)   [BH*N]
-  const float* dvec;   // D_i = dO_i . O_i [BH*N]
-  float* dq_acc;       // [BH*N, D] fp32
+  const float* lse2;   // lse * log2(e)    [BH*N]
+  const float* dvec;   // D_i = dO_i . O_i  [BH*N]
+  __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int BH, N, S, L, causal, num_tiles;
-  int group;  // heads per scheduling group
+  int group;           // heads per scheduling group
   float scale, scale_log2;
   DevStatus st;
 };
 
-// Query tiles a key tile meets, in ring order.
+// Query tiles a stationary key tile meets, in ring order (j + t) mod S.
 struct RingWalkKV {
   int jshard, S, tps, kt, causal;
   template <typename F>
@@ -78,60 +64,149 @@ struct RingWalkKV {
       if (i >= S) i -= S;
       if (causal && i < jshard) continue;
       const int qt0 = (causal && i == jshard) ? kt : i * tps;
-      const int qt1 = i * tps + tps;
-      for (int qt = qt0; qt < qt1; ++qt)
+      for (int qt = qt0; qt < i * tps + tps; ++qt)
         if (!body(qt, causal && qt == kt)) return false;
     }
     return true;
   }
+  __device__ __forceinline__ int count() const {
+    int n = 0;
+    for (int t = 0; t < S; ++t) {
+      int i = jshard + t;
+      if (i >= S) i -= S;
+      if (causal && i < jshard) continue;
+      n += (causal && i == jshard) ? (i * tps + tps - kt) : tps;
+    }
+    return n;
+  }
 };
 
+// Key tiles a stationary query tile meets, in ring order (i - t) mod S.
+struct RingWalkQ {
+  int ishard, S, tps, qt, causal;
+  template <typename F>
+  __device__ __forceinline__ bool run(F&& body) const {
+    for (int t = 0; t < S; ++t) {
+      int j = ishard - t;
+      if (j < 0) j += S;
+      if (causal && j > ishard) continue;
+      const int kt1 = (causal && j == ishard) ? qt + 1 : j * tps + tps;
+      for (int kt = j * tps; kt < kt1; ++kt)
+        if (!body(kt, causal && kt == qt)) return false;
+    }
+    return true;
+  }
+  __device__ __forceinline__ int count() const {
+    int n = 0;
+    for (int t = 0; t < S; ++t) {
+      int j = ishard - t;
+      if (j < 0) j += S;
+      if (causal && j > ishard) continue;
+      n += (causal && j == ishard) ? (qt + 1 - j * tps) : tps;
+    }
+    return n;
+  }
+};
+
+__device__ __forceinline__ void load_row128(uint32_t taddr, float (&s)[kT]) {
+  uint32_t a[32], b[32], c[32], d[32];
+  tmem_ld32(taddr, a);
+  tmem_ld32(taddr + 32, b);
+  tmem_ld32(taddr + 64, c);
+  tmem_ld32(taddr + 96, d);
+  tmem_ld_wait();
+#pragma unroll
+  for (int x = 0; x < 32; ++x) {
+    s[x] = __uint_as_float(a[x]);
+    s[32 + x] = __uint_as_float(b[x]);
+    s[64 + x] = __uint_as_float(c[x]);
+    s[96 + x] = __uint_as_float(d[x]);
+  }
+}
+
+// Store one TMEM row of D fp32 columns, times `mul`, as bf16 to global.
+template <int D>
+__device__ __forceinline__ void store_acc_row(uint32_t taddr, float mul, __nv_bfloat16* dst_row) {
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t reg[32];
+    tmem_ld32(taddr + c * 32, reg);
+    tmem_ld_wait();
+    uint32_t pk[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x)
+      pk[x] = pack_bf16x2(__uint_as_float(reg[2 * x]) * mul, __uint_as_float(reg[2 * x + 1]) * mul);
+    uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+    for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+  }
+}
+
+// ===========================================================================
+// dK, dV: key/value tile stationary
+// ===========================================================================
+template <int D>
+struct KVLayout {
+  static constexpr int kTile = kT * D * 2;  // 128 rows x D bf16 (D/64 slabs)
+  static constexpr int kSlab = kT * 128;
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + kTile;
+  static constexpr int kQ = kV + kTile;
+  static constexpr int kDO = kQ + kSt * kTile;
+  static constexpr int kVec = kDO + kSt * kTile;  // per stage: lse*log2e [128], D [128]
+  static constexpr int kBar = kVec + kSt * 1024;
+  static constexpr int kNumBars = 1 + 2 * kSt + 5;
+  static constexpr int kTmemSlot = kBar + kNumBars * 8;
+  static constexpr int kAbort = kTmemSlot + 4;
+  static constexpr int kBytes = kAbort + 4;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+static_assert(KVLayout<128>::kAlloc <= 232448, "dK/dV tile set exceeds shared memory");
+
+// Warp roles: warp 0 TMA producer (K, V once; Q, dO, lse, D per step),
+// warp 1 MMA issuer, warp 2 TMEM allocator, warps 4-7 one thread per key
+// row: P^T, dS^T, and the dK/dV epilogue.
+// MMA order per step n: dP_n, dV_n, S_{n+1}, dK_n (S_0 first); S_{n+1} is
+// issued as soon as dV_n has read P_n out of the S columns.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+    bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                   const BParams p) {
-  using LY = BLayout<D>;
-  extern __shared__ __align__(1024) uint8_t smem[];
+  using LY = KVLayout<D>;
+  extern __shared__ uint8_t smem_kv[];
+  uint8_t* smem = smem_kv + ((1024 - (smem_u32(smem_kv) & 1023)) & 1023);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  if (smem_u32(smem) & 1023) {  // the swizzled tiles need a 1024-byte aligned base
-    if (threadIdx.x == 0) atomicExch(p.st.word, (int)RA_ERR_ALIGN);
-    return;
-  }
 
-  // Work item: heads in small groups, so the CTAs in flight share a few
-  // heads' Q, dO and dQ accumulator in L2; the heaviest causal key tiles
-  // (smallest index) come first.
+  // heads in small groups; the heaviest causal key tiles (smallest index) first
   int bh, kt;
   grouped_order((int)blockIdx.x, p.num_tiles, p.BH, p.group, bh, kt);
   const int krow0 = bh * p.N + kt * kT;
   const int tps = p.L / kT;
-  RingWalkKV walk{(kt * kT) / p.L, p.S, tps, kt, p.causal};
+  const RingWalkKV walk{(kt * kT) / p.L, p.S, tps, kt, p.causal};
+  const int n_total = walk.count();
 
   uint8_t* sK = smem + LY::kK;
   uint8_t* sV = smem + LY::kV;
-  uint8_t* sDS = smem + LY::kDS;
   uint8_t* sQ = smem + LY::kQ;
   uint8_t* sDO = smem + LY::kDO;
   float* sVec = reinterpret_cast<float*>(smem + LY::kVec);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + LY::kBar);
   uint64_t* bar_kv = bars;
   uint64_t* bar_qf = bar_kv + 1;
-  uint64_t* bar_qe = bar_qf + kQSt;
-  uint64_t* bar_sf = bar_qe + kQSt;   // S^T computed
-  uint64_t* bar_dpf = bar_sf + 1;     // dP^T computed
-  uint64_t* bar_pr = bar_dpf + 1;     // P^T written to TMEM
-  uint64_t* bar_dsr = bar_pr + 1;     // dS^T written to TMEM and shared memory
-  uint64_t* bar_dqf = bar_dsr + 1;    // dQ computed
-  uint64_t* bar_dqe = bar_dqf + 1;    // dQ drained
-  uint64_t* bar_acc = bar_dqe + 1;    // dK, dV final
+  uint64_t* bar_qe = bar_qf + kSt;
+  uint64_t* bar_sf = bar_qe + kSt;   // S^T computed
+  uint64_t* bar_dpf = bar_sf + 1;    // dP^T computed
+  uint64_t* bar_pr = bar_dpf + 1;    // P^T written to TMEM
+  uint64_t* bar_dsr = bar_pr + 1;    // dS^T written to TMEM
+  uint64_t* bar_done = bar_dsr + 1;  // dK, dV final
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + LY::kTmemSlot);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LY::kAbort);
 
   if (threadIdx.x == 0) {
     mbar_init(bar_kv, 1);
-    for (int s = 0; s < kQSt; ++s) {
+    for (int s = 0; s < kSt; ++s) {
       mbar_init(&bar_qf[s], 1);
       mbar_init(&bar_qe[s], 1);
     }
@@ -139,9 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_dpf, 1);
     mbar_init(bar_pr, 128);
     mbar_init(bar_dsr, 128);
-    mbar_init(bar_dqf, 1);
-    mbar_init(bar_dqe, 128);
-    mbar_init(bar_acc, 1);
+    mbar_init(bar_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -157,7 +230,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer ----------------
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
@@ -170,9 +242,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int n = 0;
       walk.run([&](int qt, bool) {
-        const int st = n % kQSt;
+        const int st = n % kSt;
         const int qrow = bh * p.N + qt * kT;
-        if (!mbar_wait(&bar_qe[st], ((n / kQSt) & 1) ^ 1, p.st, abort_flag)) return false;
+        if (!mbar_wait(&bar_qe[st], ((n / kSt) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_qf[st], 2 * LY::kTile + 1024);
 #pragma unroll
         for (int s = 0; s < D / 64; ++s) {
@@ -187,91 +259,85 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------- MMA issuer ----------------
       constexpr uint32_t idSS = idesc_bf16_f32(kT, kT, false, false);  // K-major x K-major
       constexpr uint32_t idTS = idesc_bf16_f32(kT, D, false, true);    // TMEM A x MN-major B
-      constexpr uint32_t idDQ = idesc_bf16_f32(kT, D, true, true);     // MN-major A x MN-major B
-      const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV), ds_base = smem_u32(sDS);
+      const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV);
       const uint32_t q_base = smem_u32(sQ), do_base = smem_u32(sDO);
-      int n = 0;
-      bool ok = mbar_wait(bar_kv, 0, p.st, abort_flag);
+      auto issue_s = [&](int st) {
+        const uint32_t qb = q_base + st * LY::kTile;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * LY::kSlab + (kk & 3) * 32;
+          mma_bf16_ss(tS, sdesc_sw128(k_base + off, 16, 1024), sdesc_sw128(qb + off, 16, 1024), idSS,
+                      kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_sf);
+      };
+      bool ok = mbar_wait(bar_kv, 0, p.st, abort_flag) && mbar_wait(&bar_qf[0], 0, p.st, abort_flag);
       if (ok) {
-        ok = walk.run([&](int, bool) {
-          const int st = n % kQSt;
-          if (!mbar_wait(&bar_qf[st], (n / kQSt) & 1, p.st, abort_flag)) return false;
-          tc_fence_after();
-          const uint32_t qb = q_base + st * LY::kTile, dob = do_base + st * LY::kTile;
-          // S^T = K Q^T  (the S^T / P^T region was last read by dV of the previous step)
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * LY::kSlab + (kk & 3) * 32;
-            mma_bf16_ss(tS, sdesc_sw128(k_base + off, 16, 1024), sdesc_sw128(qb + off, 16, 1024), idSS,
-                        kk > 0 ? 1u : 0u);
-          }
-          mma_commit(bar_sf);
-          // dP^T = V dO^T, once the previous dQ has been drained from the same columns
-          if (n > 0 && !mbar_wait(bar_dqe, (n - 1) & 1, p.st, abort_flag)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * LY::kSlab + (kk & 3) * 32;
-            mma_bf16_ss(tDP, sdesc_sw128(v_base + off, 16, 1024), sdesc_sw128(dob + off, 16, 1024), idSS,
-                        kk > 0 ? 1u : 0u);
-          }
-          mma_commit(bar_dpf);
-          // dV += P^T dO
-          if (!mbar_wait(bar_pr, n & 1, p.st, abort_flag)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kT / 16; ++kk)
-            mma_bf16_ts(tDV, tS + kk * 8, sdesc_sw128(dob + kk * 2048, LY::kSlab, 1024), idTS,
-                        (n > 0 || kk > 0) ? 1u : 0u);
-          // dK += dS^T Q ; dQ = dS K
-          if (!mbar_wait(bar_dsr, n & 1, p.st, abort_flag)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kT / 16; ++kk)
-            mma_bf16_ts(tDK, tDP + kk * 8, sdesc_sw128(qb + kk * 2048, LY::kSlab, 1024), idTS,
-                        (n > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < kT / 16; ++kk)
-            mma_bf16_ss(tDP, sdesc_sw128(ds_base + kk * 2048, LY::kSlab, 1024),
-                        sdesc_sw128(k_base + kk * 2048, LY::kSlab, 1024), idDQ, kk > 0 ? 1u : 0u);
-          mma_commit(bar_dqf);
-          mma_commit(&bar_qe[st]);
-          ++n;
-          return true;
-        });
+        tc_fence_after();
+        issue_s(0);
       }
-      mma_commit(bar_acc);
+      for (int n = 0; ok && n < n_total; ++n) {
+        const int st = n % kSt;
+        const uint32_t qb = q_base + st * LY::kTile, dob = do_base + st * LY::kTile;
+        // dP^T = V dO^T (its columns were last read by dK of the previous step)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * LY::kSlab + (kk & 3) * 32;
+          mma_bf16_ss(tDP, sdesc_sw128(v_base + off, 16, 1024), sdesc_sw128(dob + off, 16, 1024), idSS,
+                      kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_dpf);
+        // dV += P^T dO
+        if (!(ok = mbar_wait(bar_pr, n & 1, p.st, abort_flag))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kT / 16; ++kk)
+          mma_bf16_ts(tDV, tS + kk * 8, sdesc_sw128(dob + kk * 2048, LY::kSlab, 1024), idTS,
+                      (n > 0 || kk > 0) ? 1u : 0u);
+        // S^T of the next query tile into the columns dV has just read
+        if (n + 1 < n_total) {
+          const int st1 = (n + 1) % kSt;
+          if (!(ok = mbar_wait(&bar_qf[st1], ((n + 1) / kSt) & 1, p.st, abort_flag))) break;
+          tc_fence_after();
+          issue_s(st1);
+        }
+        // dK += dS^T Q
+        if (!(ok = mbar_wait(bar_dsr, n & 1, p.st, abort_flag))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kT / 16; ++kk)
+          mma_bf16_ts(tDK, tDP + kk * 8, sdesc_sw128(qb + kk * 2048, LY::kSlab, 1024), idTS,
+                      (n > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bar_qe[st]);
+      }
+      mma_commit(bar_done);
     }
   } else if (warp >= 4) {
-    // ------- P^T, dS^T, dQ drain, dK/dV epilogue: one thread per key row -------
-    const int r = (warp - 4) * 32 + lane;
+    const int r = (warp - 4) * 32 + lane;  // key row = TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const float sl2 = p.scale_log2;
-    constexpr uint32_t FULL = 0xffffffffu;
+    const float2 sl22 = make_float2(p.scale_log2, p.scale_log2);
     int n = 0;
-    const bool ok = walk.run([&](int qt, bool diag) {
-      const int st = n % kQSt;
-      if (!__all_sync(FULL, mbar_wait(&bar_qf[st], (n / kQSt) & 1, p.st, abort_flag))) return false;
+    const bool ok = walk.run([&](int, bool diag) {
+      const int st = n % kSt;
+      if (!__all_sync(FULL, mbar_wait(&bar_qf[st], (n / kSt) & 1, p.st, abort_flag))) return false;
       if (!__all_sync(FULL, mbar_wait(bar_sf, n & 1, p.st, abort_flag))) return false;
       tc_fence_after();
       const float* lse2 = sVec + st * 256;
       const float* dvec = lse2 + 128;
       float P[kT];
+      load_row128(tS + lane_off, P);
 #pragma unroll
-      for (int c = 0; c < kT / 32; ++c) {
-        uint32_t reg[32];
-        tmem_ld32(tS + lane_off + c * 32, reg);
-        tmem_ld_wait();
-#pragma unroll
-        for (int x = 0; x < 32; ++x) P[c * 32 + x] = __uint_as_float(reg[x]);
+      for (int c = 0; c < kT; c += 2) {
+        const float2 t = fma2(make_float2(P[c], P[c + 1]), sl22, make_float2(-lse2[c], -lse2[c + 1]));
+        P[c] = ex2_approx(t.x);
+        P[c + 1] = ex2_approx(t.y);
       }
+      if (diag) {
 #pragma unroll
-      for (int c = 0; c < kT; ++c) {
-        const float pv = ex2_approx(fmaf(P[c], sl2, -lse2[c]));
-        P[c] = (diag && r > c) ? 0.f : pv;  // key r is in the future of query c
+        for (int c = 0; c < kT; ++c)
+          if (r > c) P[c] = 0.f;  // key r is in the future of query c
       }
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -286,10 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       if (!__all_sync(FULL, mbar_wait(bar_dpf, n & 1, p.st, abort_flag))) return false;
       tc_fence_after();
-      // dS^T = P^T (dP^T - D), 32 query columns at a time; bf16 to TMEM (over
-      // the dP^T columns already read) and to the MN-major shared operand.
-      const uint32_t row_sw = (uint32_t)(r & 7);
-      uint8_t* ds_row = sDS + (r >> 3) * 1024 + (r & 7) * 128;
+      // dS^T = P^T (dP^T - D), written as bf16 over the dP^T columns already read
 #pragma unroll
       for (int c = 0; c < kT / 32; ++c) {
         uint32_t reg[32];
@@ -298,67 +361,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int x = 0; x < 16; ++x) {
-          const int q0 = c * 32 + 2 * x;
-          const float d0 = P[q0] * (__uint_as_float(reg[2 * x]) - dvec[q0]);
-          const float d1 = P[q0 + 1] * (__uint_as_float(reg[2 * x + 1]) - dvec[q0 + 1]);
+          const int q = c * 32 + 2 * x;
+          const float d0 = P[q] * (__uint_as_float(reg[2 * x]) - dvec[q]);
+          const float d1 = P[q + 1] * (__uint_as_float(reg[2 * x + 1]) - dvec[q + 1]);
           pk[x] = pack_bf16x2(d0, d1);
         }
         tmem_st16(tDP + lane_off + c * 16, pk);
-        // queries [32c, 32c+32) -> slab c/2, 16-byte chunks (c%2)*4 .. +4
-        uint8_t* slab = ds_row + (c >> 1) * LY::kSlab;
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const uint32_t chunk = (uint32_t)((c & 1) * 4 + x);
-          *reinterpret_cast<uint4*>(slab + ((chunk ^ row_sw) << 4)) =
-              make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
-        }
       }
       tmem_st_wait();
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar_dsr);
-
-      // drain dQ (row r of this step's query tile) into the fp32 accumulator
-      if (!__all_sync(FULL, mbar_wait(bar_dqf, n & 1, p.st, abort_flag))) return false;
-      tc_fence_after();
-      float* dq_row = p.dq_acc + ((size_t)bh * p.N + (size_t)qt * kT + r) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t reg[32];
-        tmem_ld32(tDP + lane_off + c * 32, reg);
-        tmem_ld_wait();
-#pragma unroll
-        for (int x = 0; x < 8; ++x)
-          red_add_v4(dq_row + c * 32 + 4 * x, __uint_as_float(reg[4 * x]), __uint_as_float(reg[4 * x + 1]),
-                     __uint_as_float(reg[4 * x + 2]), __uint_as_float(reg[4 * x + 3]));
-      }
-      tc_fence_before();
-      mbar_arrive(bar_dqe);
       ++n;
       return true;
     });
-    if (ok && __all_sync(FULL, mbar_wait(bar_acc, 0, p.st, abort_flag))) {
+    if (ok && __all_sync(FULL, mbar_wait(bar_done, 0, p.st, abort_flag))) {
       tc_fence_after();
-      const size_t grow = (size_t)krow0 + r;
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t tacc = which ? tDV : tDK;
-        const float mul = which ? 1.f : p.scale;
-        __nv_bfloat16* dst_row = (which ? p.dv : p.dk) + grow * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t reg[32];
-          tmem_ld32(tacc + lane_off + c * 32, reg);
-          tmem_ld_wait();
-          uint32_t pk[16];
-#pragma unroll
-          for (int x = 0; x < 16; ++x)
-            pk[x] = pack_bf16x2(__uint_as_float(reg[2 * x]) * mul, __uint_as_float(reg[2 * x + 1]) * mul);
-          uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
-#pragma unroll
-          for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
-        }
-      }
+      store_acc_row<D>(tDK + lane_off, p.scale, p.dk + ((size_t)krow0 + r) * D);
+      store_acc_row<D>(tDV + lane_off, 1.f, p.dv + ((size_t)krow0 + r) * D);
     }
   }
 
@@ -370,14 +389,254 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// D_i = dO_i . O_i, lse_i * log2(e), and zero the dQ accumulator row.
-// One warp per row; HBM-bound.
+// ===========================================================================
+// dQ: query tile stationary
+// ===========================================================================
+template <int D>
+struct QLayout {
+  static constexpr int kTile = kT * D * 2;
+  static constexpr int kSlab = kT * 128;
+  static constexpr int kQ = 0;
+  static constexpr int kDO = kQ + kTile;
+  static constexpr int kK = kDO + kTile;
+  static constexpr int kV = kK + kSt * kTile;
+  static constexpr int kDS = kV + kSt * kTile;  // dS [128 queries][128 keys] bf16, K-major, 2 slabs
+  static constexpr int kBar = kDS + kT * kT * 2;
+  static constexpr int kNumBars = 1 + 4 * kSt + 2 + 4;
+  static constexpr int kTmemSlot = kBar + kNumBars * 8;
+  static constexpr int kAbort = kTmemSlot + 4;
+  static constexpr int kBytes = kAbort + 4;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+static_assert(QLayout<128>::kAlloc <= 232448, "dQ tile set exceeds shared memory");
+
+// Warp roles: warp 0 TMA producer (Q, dO once; K, V per step), warp 1 MMA
+// issuer, warp 2 TMEM allocator, warps 4-7 one thread per query row: P, dS
+// (to shared memory) and the dQ epilogue.
+// MMA order per step n: dP_n, S_{n+1}, dQ_n (S_0 first); S is double
+// buffered so the next scores are ready when a row's dS is done.
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                 const BParams p) {
+  using LY = QLayout<D>;
+  extern __shared__ uint8_t smem_q[];
+  uint8_t* smem = smem_q + ((1024 - (smem_u32(smem_q) & 1023)) & 1023);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // heads in small groups; the heaviest causal query tiles (largest index) first
+  int bh, rank;
+  grouped_order((int)blockIdx.x, p.num_tiles, p.BH, p.group, bh, rank);
+  const int qt = p.num_tiles - 1 - rank;
+  const int qrow0 = bh * p.N + qt * kT;
+  const int tps = p.L / kT;
+  const RingWalkQ walk{(qt * kT) / p.L, p.S, tps, qt, p.causal};
+  const int n_total = walk.count();
+
+  uint8_t* sQ = smem + LY::kQ;
+  uint8_t* sDO = smem + LY::kDO;
+  uint8_t* sK = smem + LY::kK;
+  uint8_t* sV = smem + LY::kV;
+  uint8_t* sDS = smem + LY::kDS;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + LY::kBar);
+  uint64_t* bar_qd = bars;
+  uint64_t* bar_kf = bar_qd + 1;
+  uint64_t* bar_ke = bar_kf + kSt;
+  uint64_t* bar_vf = bar_ke + kSt;
+  uint64_t* bar_ve = bar_vf + kSt;
+  uint64_t* bar_sf = bar_ve + kSt;   // [2] S buffer b computed
+  uint64_t* bar_dpf = bar_sf + 2;    // dP computed
+  uint64_t* bar_dsr = bar_dpf + 1;   // dS written to shared memory
+  uint64_t* bar_dsf = bar_dsr + 1;   // dS buffer free (previous dQ done)
+  uint64_t* bar_done = bar_dsf + 1;  // dQ final
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + LY::kTmemSlot);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LY::kAbort);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_qd, 1);
+    for (int s = 0; s < kSt; ++s) {
+      mbar_init(&bar_kf[s], 1);
+      mbar_init(&bar_ke[s], 1);
+      mbar_init(&bar_vf[s], 1);
+      mbar_init(&bar_ve[s], 1);
+    }
+    mbar_init(&bar_sf[0], 1);
+    mbar_init(&bar_sf[1], 1);
+    mbar_init(bar_dpf, 1);
+    mbar_init(bar_dsr, 128);
+    mbar_init(bar_dsf, 1);
+    mbar_init(bar_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tDP = tmem + 256, tDQ = tmem + 384;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+      mbar_arrive_expect_tx(bar_qd, 2 * LY::kTile);
+#pragma unroll
+      for (int s = 0; s < D / 64; ++s) {
+        tma_load_2d(sQ + s * LY::kSlab, &tmQ, bar_qd, s * 64, qrow0);
+        tma_load_2d(sDO + s * LY::kSlab, &tmDO, bar_qd, s * 64, qrow0);
+      }
+      int n = 0;
+      walk.run([&](int kt, bool) {
+        const int st = n % kSt;
+        const int krow = bh * p.N + kt * kT;
+        if (!mbar_wait(&bar_ke[st], ((n / kSt) & 1) ^ 1, p.st, abort_flag)) return false;
+        mbar_arrive_expect_tx(&bar_kf[st], LY::kTile);
+#pragma unroll
+        for (int s = 0; s < D / 64; ++s)
+          tma_load_2d(sK + st * LY::kTile + s * LY::kSlab, &tmK, &bar_kf[st], s * 64, krow);
+        if (!mbar_wait(&bar_ve[st], ((n / kSt) & 1) ^ 1, p.st, abort_flag)) return false;
+        mbar_arrive_expect_tx(&bar_vf[st], LY::kTile);
+#pragma unroll
+        for (int s = 0; s < D / 64; ++s)
+          tma_load_2d(sV + st * LY::kTile + s * LY::kSlab, &tmV, &bar_vf[st], s * 64, krow);
+        ++n;
+        return true;
+      });
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idSS = idesc_bf16_f32(kT, kT, false, false);  // K-major x K-major
+      constexpr uint32_t idDQ = idesc_bf16_f32(kT, D, false, true);    // K-major dS x MN-major K
+      const uint32_t q_base = smem_u32(sQ), do_base = smem_u32(sDO), ds_base = smem_u32(sDS);
+      const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV);
+      auto issue_s = [&](int n) -> bool {
+        const int st = n % kSt;
+        if (!mbar_wait(&bar_kf[st], (n / kSt) & 1, p.st, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t kb = k_base + st * LY::kTile;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * LY::kSlab + (kk & 3) * 32;
+          mma_bf16_ss(tmem + (n & 1) * 128, sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
+                      idSS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bar_sf[n & 1]);
+        return true;
+      };
+      bool ok = mbar_wait(bar_qd, 0, p.st, abort_flag) && issue_s(0);
+      for (int n = 0; ok && n < n_total; ++n) {
+        const int st = n % kSt;
+        // dP = dO V^T (its columns were last read for dS of the previous step)
+        if (!(ok = mbar_wait(&bar_vf[st], (n / kSt) & 1, p.st, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t vb = v_base + st * LY::kTile;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * LY::kSlab + (kk & 3) * 32;
+          mma_bf16_ss(tDP, sdesc_sw128(do_base + off, 16, 1024), sdesc_sw128(vb + off, 16, 1024), idSS,
+                      kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_dpf);
+        mma_commit(&bar_ve[st]);
+        // scores of the next key tile into the other S buffer
+        if (n + 1 < n_total && !(ok = issue_s(n + 1))) break;
+        // dQ += dS K
+        if (!(ok = mbar_wait(bar_dsr, n & 1, p.st, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t kb = k_base + st * LY::kTile;
+#pragma unroll
+        for (int kk = 0; kk < kT / 16; ++kk)
+          mma_bf16_ss(tDQ, sdesc_sw128(ds_base + (kk >> 2) * LY::kSlab + (kk & 3) * 32, 16, 1024),
+                      sdesc_sw128(kb + kk * 2048, LY::kSlab, 1024), idDQ, (n > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bar_ke[st]);
+        mma_commit(bar_dsf);
+      }
+      mma_commit(bar_done);
+    }
+  } else if (warp >= 4) {
+    const int r = (warp - 4) * 32 + lane;  // query row = TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const float nl2 = -p.lse2[qrow0 + r];
+    const float Dr = p.dvec[qrow0 + r];
+    const float2 sl22 = make_float2(p.scale_log2, p.scale_log2), nl22 = make_float2(nl2, nl2);
+    uint8_t* ds_row = sDS + (r >> 3) * 1024 + (r & 7) * 128;
+    const uint32_t row_sw = (uint32_t)(r & 7);
+    int n = 0;
+    const bool ok = walk.run([&](int, bool diag) {
+      if (!__all_sync(FULL, mbar_wait(&bar_sf[n & 1], (n >> 1) & 1, p.st, abort_flag))) return false;
+      tc_fence_after();
+      float P[kT];
+      load_row128(tmem + (n & 1) * 128 + lane_off, P);
+#pragma unroll
+      for (int c = 0; c < kT; c += 2) {
+        const float2 t = fma2(make_float2(P[c], P[c + 1]), sl22, nl22);
+        P[c] = ex2_approx(t.x);
+        P[c + 1] = ex2_approx(t.y);
+      }
+      if (diag) {
+#pragma unroll
+        for (int c = 0; c < kT; ++c)
+          if (c > r) P[c] = 0.f;  // key c is in the future of query r
+      }
+      if (!__all_sync(FULL, mbar_wait(bar_dpf, n & 1, p.st, abort_flag))) return false;
+      tc_fence_after();
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < kT / 32; ++c) {
+        uint32_t reg[32];
+        tmem_ld32(tDP + lane_off + c * 32, reg);
+        tmem_ld_wait();
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const int k = c * 32 + 2 * x;
+          pk[c * 16 + x] = pack_bf16x2(P[k] * (__uint_as_float(reg[2 * x]) - Dr),
+                                       P[k + 1] * (__uint_as_float(reg[2 * x + 1]) - Dr));
+        }
+      }
+      // the previous dQ MMA must have finished reading the dS buffer
+      if (n > 0 && !__all_sync(FULL, mbar_wait(bar_dsf, (n - 1) & 1, p.st, abort_flag))) return false;
+      // dS row r: keys [64 s, 64 s + 64) in slab s, 16-byte chunk c at c ^ (r & 7)
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        uint8_t* slab = ds_row + (c >> 3) * LY::kSlab;
+        const uint32_t chunk = (uint32_t)(c & 7);
+        *reinterpret_cast<uint4*>(slab + ((chunk ^ row_sw) << 4)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar_dsr);
+      ++n;
+      return true;
+    });
+    if (ok && __all_sync(FULL, mbar_wait(bar_done, 0, p.st, abort_flag))) {
+      tc_fence_after();
+      store_acc_row<D>(tDQ + lane_off, p.scale, p.dq + ((size_t)qrow0 + r) * D);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// D_i = dO_i . O_i and lse_i * log2(e); one warp per row; HBM-bound.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ out,
                                                              const __nv_bfloat16* __restrict__ dout,
                                                              const float* __restrict__ lse, float* __restrict__ dvec,
-                                                             float* __restrict__ lse2, float* __restrict__ dq_acc,
-                                                             int64_t rows) {
+                                                             float* __restrict__ lse2, int64_t rows) {
   constexpr int E = D / 32;  // elements per lane (2 or 4)
   const int lane = threadIdx.x & 31;
   const int64_t w0 = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -397,12 +656,10 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16
         acc = fmaf(fa.x, fb.x, acc);
         acc = fmaf(fa.y, fb.y, acc);
       }
-      *reinterpret_cast<float4*>(dq_acc + row * D + lane * E) = make_float4(0.f, 0.f, 0.f, 0.f);
     } else {
       const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(o));
       const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(g));
       acc = fmaf(fa.x, fb.x, fa.y * fb.y);
-      *reinterpret_cast<float2*>(dq_acc + row * D + lane * E) = make_float2(0.f, 0.f);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -410,22 +667,6 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16
       dvec[row] = acc;
       lse2[row] = lse[row] * kLog2e;
     }
-  }
-}
-
-// dq = bf16(scale * dq_acc), 8 elements per thread per step.
-__global__ void __launch_bounds__(256) bwd_convert_kernel(const float* __restrict__ acc,
-                                                          __nv_bfloat16* __restrict__ dq, float scale, int64_t n8) {
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride) {
-    const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
-    const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
-    uint4 o;
-    o.x = pack_bf16x2(a.x * scale, a.y * scale);
-    o.y = pack_bf16x2(a.z * scale, a.w * scale);
-    o.z = pack_bf16x2(b.x * scale, b.y * scale);
-    o.w = pack_bf16x2(b.z * scale, b.w * scale);
-    reinterpret_cast<uint4*>(dq)[i] = o;
   }
 }
 
@@ -440,22 +681,20 @@ int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* d
              void* workspace, int phase_mask, cudaStream_t stream) {
   const int64_t rows = a.B * a.H * a.N;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* dq_acc = reinterpret_cast<float*>(ws);
-  const size_t dq_bytes = ((size_t)rows * D * 4 + 255) & ~(size_t)255;
   const size_t vec_bytes = ((size_t)rows * 4 + 255) & ~(size_t)255;
-  float* dvec = reinterpret_cast<float*>(ws + dq_bytes);
-  float* lse2 = reinterpret_cast<float*>(ws + dq_bytes + vec_bytes);
-  const int sms = sm_count();
+  float* dvec = reinterpret_cast<float*>(ws);
+  float* lse2 = reinterpret_cast<float*>(ws + vec_bytes);
 
   if (phase_mask & 1) {
     const int64_t want = (rows + 7) / 8;
-    const unsigned grid = (unsigned)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
+    const int64_t cap = (int64_t)sm_count() * 16;
+    const unsigned grid = (unsigned)(want < cap ? want : cap);
     bwd_preprocess_kernel<D><<<grid, 256, 0, stream>>>((const __nv_bfloat16*)out, (const __nv_bfloat16*)dout, lse,
-                                                       dvec, lse2, dq_acc, rows);
+                                                       dvec, lse2, rows);
     if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
   }
+  if ((phase_mask & 6) == 0) return RA_OK;
 
-  if (phase_mask & 2) {
   alignas(64) CUtensorMap tq, tk, tv, tdo;
   if (make_tmap_bf16_2d(&tq, a.q, D, rows, D * 2, 64, kT) != RA_OK) return RA_ERR_CUDA;
   if (make_tmap_bf16_2d(&tk, a.k, D, rows, D * 2, 64, kT) != RA_OK) return RA_ERR_CUDA;
@@ -464,7 +703,7 @@ int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* d
   BParams p{};
   p.lse2 = lse2;
   p.dvec = dvec;
-  p.dq_acc = dq_acc;
+  p.dq = (__nv_bfloat16*)dq;
   p.dk = (__nv_bfloat16*)dk;
   p.dv = (__nv_bfloat16*)dv;
   p.BH = (int)(a.B * a.H);
@@ -473,23 +712,23 @@ int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* d
   p.L = (int)(a.N / a.S);
   p.causal = a.causal;
   p.num_tiles = (int)(a.N / kT);
-  // per head: Q, dO, K, V (bf16) and the fp32 dQ accumulator
-  p.group = head_group(p.num_tiles, p.BH, (double)a.N * D * (4 * 2 + 4), 100.0e6);
+  // per head: Q, dO, K, V (bf16) stream through L2
+  p.group = head_group(p.num_tiles, p.BH, (double)a.N * D * 4 * 2, 100.0e6);
   p.scale = a.scale;
   p.scale_log2 = a.scale * kLog2e;
   int rc = current_status(&p.st);
   if (rc != RA_OK) return rc;
-  auto kern = bwd_tc_kernel<D>;
-  if (set_smem_attr((const void*)kern, BLayout<D>::kBytes) != RA_OK) return RA_ERR_CUDA;
-  kern<<<(unsigned)(p.BH * p.num_tiles), kThreads, BLayout<D>::kBytes, stream>>>(tq, tk, tv, tdo, p);
-  if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
+  const unsigned grid = (unsigned)(p.BH * p.num_tiles);
+  if (phase_mask & 2) {
+    auto kern = bwd_kv_kernel<D>;
+    if (set_smem_attr((const void*)kern, KVLayout<D>::kAlloc) != RA_OK) return RA_ERR_CUDA;
+    kern<<<grid, kThreads, KVLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
+    if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
   }
-
   if (phase_mask & 4) {
-    const int64_t n8 = rows * D / 8;
-    const int64_t want = (n8 + 255) / 256;
-    const unsigned grid = (unsigned)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
-    bwd_convert_kernel<<<grid, 256, 0, stream>>>(dq_acc, (__nv_bfloat16*)dq, a.scale, n8);
+    auto kern = bwd_q_kernel<D>;
+    if (set_smem_attr((const void*)kern, QLayout<D>::kAlloc) != RA_OK) return RA_ERR_CUDA;
+    kern<<<grid, kThreads, QLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
     if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
   }
   return RA_OK;

@@ -136,9 +136,9 @@ RA_API int ringattn_fwd_step(const void* q, const void* k, const void* v,
 RA_API int ringattn_merge(float* o_a, float* lse_a, const float* o_b, const float* lse_b,
                    int64_t rows, int64_t D, void* stream);
 
-/* Bytes of device workspace ringattn_bwd needs: the fp32 dQ accumulator
- * [B,H,N,D] plus two fp32 row vectors [B,H,N] (D_i = dO_i . O_i and
- * lse_i * log2(e)), each region 256-byte aligned.  0 for empty problems. */
+/* Bytes of device workspace ringattn_bwd needs: two fp32 row vectors
+ * [B,H,N] (D_i = dO_i . O_i and lse_i * log2(e)), each region 256-byte
+ * aligned.  0 for empty problems. */
 RA_API size_t ringattn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D);
 
 /*
@@ -148,8 +148,11 @@ RA_API size_t ringattn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64
  *   dv_j = sum_i P_ij dout_i
  *   dS_ij = P_ij (dout_i . v_j - D_i)
  *   dq_i = scale sum_j dS_ij k_j ;  dk_j = scale sum_i dS_ij q_i
- * Each key/value shard stays put while the query shards pass by in ring
- * order i = (j + t) mod S (causal: pairs i < j skipped).
+ * dK and dV keep each key/value tile stationary while the query shards
+ * pass by in ring order i = (j + t) mod S; dQ keeps each query tile
+ * stationary and visits the KV shards in ring order j = (i - t) mod S
+ * (causal: pairs in the future skipped).  Every gradient accumulates on chip
+ * and is written once: no atomics, bit-reproducible.
  *
  *   q,k,v,out,dout [B,H,N,D] of `dtype` (out and lse from ringattn_fwd)
  *   lse            [B,H,N] fp32
@@ -169,12 +172,12 @@ RA_API int ringattn_bwd(const void* q, const void* k, const void* v, const void*
 /*
  * ringattn_bwd_phase -- ringattn_bwd split into its three launches, for
  * callers that schedule or time them separately.  phase_mask (1..7) selects
- * bit 0: preprocess (D_i, lse_i*log2(e), zero the dQ accumulator in
- * workspace), bit 1: the tensor-core main loop (dK, dV written, dQ
- * accumulated in workspace), bit 2: dq = bf16(scale * accumulator).  The
- * phases must run in that order on the same workspace; mask 7 is
- * ringattn_bwd.  Arguments and errors as ringattn_bwd, plus RA_ERR_ARG for
- * a mask outside 1..7.
+ * bit 0: preprocess (D_i and lse_i*log2(e) into workspace), bit 1: the
+ * key/value-stationary tensor-core loop (writes dk, dv), bit 2: the
+ * query-stationary tensor-core loop (writes dq).  Bits 1 and 2 read what bit
+ * 0 wrote into the same workspace and are independent of each other; mask 7
+ * is ringattn_bwd.  Arguments and errors as ringattn_bwd, plus RA_ERR_ARG
+ * for a mask outside 1..7.
  */
 RA_API int ringattn_bwd_phase(const void* q, const void* k, const void* v, const void* out,
                               const float* lse, const void* dout,
@@ -195,7 +198,7 @@ RA_API int ringattn_bwd_phase(const void* q, const void* k, const void* v, const
  * static device array of RINGATTN_NOALLOC_SCRATCH_BYTES (64 MiB) that every
  * GPU which loads this library keeps until the process exits.  Problems
  * whose ringattn_bwd_workspace_size() exceeds it return RA_ERR_WORKSPACE
- * (with D = 128: B*H*N up to about 127 thousand rows, e.g. H=4, N=32768).
+ * (B*H*N up to about 8.3 million rows, e.g. H=32, N=262144).
  * The first call on a device looks up the array's device address; make that
  * first call before any stream capture.  All calls share the one array and
  * it keeps the last call's contents (each call re-clears what must start at

@@ -89,7 +89,7 @@ def test_step_and_merge_argument_errors(L):
 
 def test_bwd_workspace_contract(L):
     ws = L.ringattn_bwd_workspace_size(1, 32, 32768, 128)
-    assert ws >= 32 * 32768 * 128 * 4 + 32 * 32768 * 4
+    assert ws >= 2 * 32 * 32768 * 4                  # D_i and lse*log2(e), fp32
     assert L.ringattn_bwd_workspace_size(0, 1, 1, 1) == 0
     b = L.ringattn_bwd
     ws = L.ringattn_bwd_workspace_size(1, 1, 1024, 128)

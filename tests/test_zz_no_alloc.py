@@ -66,7 +66,7 @@ def test_noalloc_matches_workspace_backward_twice(L, B, H, N, D, S, qc, kc, caus
 
 def test_noalloc_rejects_problems_beyond_its_scratch(L):
     limit = 64 << 20
-    B, H, N, D = 1, 8, 32768, 128          # needs about 136 MB of scratch
+    B, H, N, D = 4, 32, 131072, 128        # needs about 134 MB of scratch
     assert L.ringattn_bwd_workspace_size(B, H, N, D) > limit
     fake = [0x10000] * 9                   # never touched: the size check comes first
     rc = L.ringattn_bwd_noalloc(*fake, B, H, N, D, 0, 16, 512, 1024, 1, 0.0, None)
