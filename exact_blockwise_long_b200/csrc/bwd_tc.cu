@@ -26,7 +26,7 @@
 //   dQ          per (query tile, key tile) 3 tcgen05 MMAs:
 //                 S    = Q K^T    (TMEM [0,128) / [128,256), double buffered)
 //                 dP   = dO V^T   (TMEM [256,384))
-//                 dQ  += dS K     (dS bf16 through shared memory)
+//                 dQ  += dS K     (dS bf16 over S, A operand from TMEM)
 #include <math.h>
 
 #include "common.cuh"
@@ -37,7 +37,8 @@ namespace {
 
 constexpr int kT = 128;        // rows per tile (TMEM lanes)
 constexpr int kSt = 2;         // streamed-tile stages
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;   // 4 role warps + two element-wise warpgroups
+constexpr int kHalf = 64;      // score columns per element-wise warpgroup
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t FULL = 0xffffffffu;
@@ -124,11 +125,23 @@ __device__ __forceinline__ void load_row128(uint32_t taddr, float (&s)[kT]) {
   }
 }
 
-// Store one TMEM row of D fp32 columns, times `mul`, as bf16 to global.
-template <int D>
+__device__ __forceinline__ void load_row64(uint32_t taddr, float (&s)[kHalf]) {
+  uint32_t a[32], b[32];
+  tmem_ld32(taddr, a);
+  tmem_ld32(taddr + 32, b);
+  tmem_ld_wait();
+#pragma unroll
+  for (int x = 0; x < 32; ++x) {
+    s[x] = __uint_as_float(a[x]);
+    s[32 + x] = __uint_as_float(b[x]);
+  }
+}
+
+// Store W fp32 columns of one TMEM row, times `mul`, as bf16 to global.
+template <int W>
 __device__ __forceinline__ void store_acc_row(uint32_t taddr, float mul, __nv_bfloat16* dst_row) {
 #pragma unroll
-  for (int c = 0; c < D / 32; ++c) {
+  for (int c = 0; c < W / 32; ++c) {
     uint32_t reg[32];
     tmem_ld32(taddr + c * 32, reg);
     tmem_ld_wait();
@@ -164,8 +177,12 @@ struct KVLayout {
 static_assert(KVLayout<128>::kAlloc <= 232448, "dK/dV tile set exceeds shared memory");
 
 // Warp roles: warp 0 TMA producer (K, V once; Q, dO, lse, D per step),
-// warp 1 MMA issuer, warp 2 TMEM allocator, warps 4-7 one thread per key
-// row: P^T, dS^T, and the dK/dV epilogue.
+// warp 1 MMA issuer, warp 2 TMEM allocator, warps 4-7 and 8-11 one thread
+// per key row each, the first warpgroup on query columns [0,64), the second
+// on [64,128): P^T, dS^T and half of the dK/dV epilogue.  Each warpgroup
+// writes its bf16 P^T (dS^T) over the first 32 of the S^T (dP^T) columns it
+// has itself read, so the A operand of dV (dK) sits in columns [0,32) and
+// [64,96).
 // MMA order per step n: dP_n, dV_n, S_{n+1}, dK_n (S_0 first); S_{n+1} is
 // issued as soon as dV_n has read P_n out of the S columns.
 template <int D>
@@ -212,8 +229,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar_sf, 1);
     mbar_init(bar_dpf, 1);
-    mbar_init(bar_pr, 128);
-    mbar_init(bar_dsr, 128);
+    mbar_init(bar_pr, 2 * 128);
+    mbar_init(bar_dsr, 2 * 128);
     mbar_init(bar_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -263,6 +280,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idTS = idesc_bf16_f32(kT, D, false, true);    // TMEM A x MN-major B
       const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV);
       const uint32_t q_base = smem_u32(sQ), do_base = smem_u32(sDO);
+      // TMEM column of the bf16 A operand for queries [16 kk, 16 kk + 16)
+      auto a_col = [](int kk) -> uint32_t { return kk < 4 ? kk * 8 : 64 + (kk - 4) * 8; };
       auto issue_s = [&](int st) {
         const uint32_t qb = q_base + st * LY::kTile;
 #pragma unroll
@@ -294,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kT / 16; ++kk)
-          mma_bf16_ts(tDV, tS + kk * 8, sdesc_sw128(dob + kk * 2048, LY::kSlab, 1024), idTS,
+          mma_bf16_ts(tDV, tS + a_col(kk), sdesc_sw128(dob + kk * 2048, LY::kSlab, 1024), idTS,
                       (n > 0 || kk > 0) ? 1u : 0u);
         // S^T of the next query tile into the columns dV has just read
         if (n + 1 < n_total) {
@@ -308,15 +327,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kT / 16; ++kk)
-          mma_bf16_ts(tDK, tDP + kk * 8, sdesc_sw128(qb + kk * 2048, LY::kSlab, 1024), idTS,
+          mma_bf16_ts(tDK, tDP + a_col(kk), sdesc_sw128(qb + kk * 2048, LY::kSlab, 1024), idTS,
                       (n > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bar_qe[st]);
       }
       mma_commit(bar_done);
     }
   } else if (warp >= 4) {
-    const int r = (warp - 4) * 32 + lane;  // key row = TMEM lane
+    const int h = (warp >> 2) - 1;          // query columns [64 h, 64 h + 64)
+    const int r = (warp & 3) * 32 + lane;   // key row = TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t cS = tS + lane_off + h * kHalf, cDP = tDP + lane_off + h * kHalf;
     const float2 sl22 = make_float2(p.scale_log2, p.scale_log2);
     int n = 0;
     const bool ok = walk.run([&](int, bool diag) {
@@ -324,27 +345,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(FULL, mbar_wait(&bar_qf[st], (n / kSt) & 1, p.st, abort_flag))) return false;
       if (!__all_sync(FULL, mbar_wait(bar_sf, n & 1, p.st, abort_flag))) return false;
       tc_fence_after();
-      const float* lse2 = sVec + st * 256;
+      const float* lse2 = sVec + st * 256 + h * kHalf;
       const float* dvec = lse2 + 128;
-      float P[kT];
-      load_row128(tS + lane_off, P);
+      float P[kHalf];
+      load_row64(cS, P);
 #pragma unroll
-      for (int c = 0; c < kT; c += 2) {
+      for (int c = 0; c < kHalf; c += 2) {
         const float2 t = fma2(make_float2(P[c], P[c + 1]), sl22, make_float2(-lse2[c], -lse2[c + 1]));
         P[c] = ex2_approx(t.x);
         P[c + 1] = ex2_approx(t.y);
       }
       if (diag) {
 #pragma unroll
-        for (int c = 0; c < kT; ++c)
-          if (r > c) P[c] = 0.f;  // key r is in the future of query c
+        for (int c = 0; c < kHalf; ++c)
+          if (r > h * kHalf + c) P[c] = 0.f;  // key r is in the future of the query
       }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      {
         uint32_t pk[32];
 #pragma unroll
-        for (int x = 0; x < 32; ++x) pk[x] = pack_bf16x2(P[h * 64 + 2 * x], P[h * 64 + 2 * x + 1]);
-        tmem_st32(tS + lane_off + h * 32, pk);
+        for (int x = 0; x < 32; ++x) pk[x] = pack_bf16x2(P[2 * x], P[2 * x + 1]);
+        tmem_st32(cS, pk);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -352,21 +372,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       if (!__all_sync(FULL, mbar_wait(bar_dpf, n & 1, p.st, abort_flag))) return false;
       tc_fence_after();
-      // dS^T = P^T (dP^T - D), written as bf16 over the dP^T columns already read
-#pragma unroll
-      for (int c = 0; c < kT / 32; ++c) {
-        uint32_t reg[32];
-        tmem_ld32(tDP + lane_off + c * 32, reg);
+      // dS^T = P^T (dP^T - D) as bf16 over the first half of this group's dP^T columns
+      {
+        uint32_t a[32], b[32];
+        tmem_ld32(cDP, a);
+        tmem_ld32(cDP + 32, b);
         tmem_ld_wait();
-        uint32_t pk[16];
+        uint32_t pk[32];
 #pragma unroll
         for (int x = 0; x < 16; ++x) {
-          const int q = c * 32 + 2 * x;
-          const float d0 = P[q] * (__uint_as_float(reg[2 * x]) - dvec[q]);
-          const float d1 = P[q + 1] * (__uint_as_float(reg[2 * x + 1]) - dvec[q + 1]);
-          pk[x] = pack_bf16x2(d0, d1);
+          const int q = 2 * x;
+          pk[x] = pack_bf16x2(P[q] * (__uint_as_float(a[2 * x]) - dvec[q]),
+                              P[q + 1] * (__uint_as_float(a[2 * x + 1]) - dvec[q + 1]));
+          pk[16 + x] = pack_bf16x2(P[32 + q] * (__uint_as_float(b[2 * x]) - dvec[32 + q]),
+                                   P[33 + q] * (__uint_as_float(b[2 * x + 1]) - dvec[33 + q]));
         }
-        tmem_st16(tDP + lane_off + c * 16, pk);
+        tmem_st32(cDP, pk);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -376,8 +397,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     });
     if (ok && __all_sync(FULL, mbar_wait(bar_done, 0, p.st, abort_flag))) {
       tc_fence_after();
-      store_acc_row<D>(tDK + lane_off, p.scale, p.dk + ((size_t)krow0 + r) * D);
-      store_acc_row<D>(tDV + lane_off, 1.f, p.dv + ((size_t)krow0 + r) * D);
+      const size_t row = (size_t)krow0 + r;
+      store_acc_row<D / 2>(tDK + lane_off + h * (D / 2), p.scale, p.dk + row * D + h * (D / 2));
+      store_acc_row<D / 2>(tDV + lane_off + h * (D / 2), 1.f, p.dv + row * D + h * (D / 2));
     }
   }
 
@@ -392,6 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ===========================================================================
 // dQ: query tile stationary
 // ===========================================================================
+constexpr int kKStQ = 3;  // K stages of the dQ pass (K is held from S until dQ)
+
 template <int D>
 struct QLayout {
   static constexpr int kTile = kT * D * 2;
@@ -399,10 +423,9 @@ struct QLayout {
   static constexpr int kQ = 0;
   static constexpr int kDO = kQ + kTile;
   static constexpr int kK = kDO + kTile;
-  static constexpr int kV = kK + kSt * kTile;
-  static constexpr int kDS = kV + kSt * kTile;  // dS [128 queries][128 keys] bf16, K-major, 2 slabs
-  static constexpr int kBar = kDS + kT * kT * 2;
-  static constexpr int kNumBars = 1 + 4 * kSt + 2 + 4;
+  static constexpr int kV = kK + kKStQ * kTile;
+  static constexpr int kBar = kV + kSt * kTile;
+  static constexpr int kNumBars = 1 + 2 * kKStQ + 2 * kSt + 2 + 3;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4;
@@ -411,8 +434,11 @@ struct QLayout {
 static_assert(QLayout<128>::kAlloc <= 232448, "dQ tile set exceeds shared memory");
 
 // Warp roles: warp 0 TMA producer (Q, dO once; K, V per step), warp 1 MMA
-// issuer, warp 2 TMEM allocator, warps 4-7 one thread per query row: P, dS
-// (to shared memory) and the dQ epilogue.
+// issuer, warp 2 TMEM allocator, warps 4-7 and 8-11 one thread per query
+// row each, the first warpgroup on key columns [0,64), the second on
+// [64,128): P, dS and half of the dQ epilogue.  Each warpgroup writes its
+// bf16 dS over the first 32 of the S columns it has itself read, so the A
+// operand of dQ sits in columns [0,32) and [64,96) of that step's S buffer.
 // MMA order per step n: dP_n, S_{n+1}, dQ_n (S_0 first); S is double
 // buffered so the next scores are ready when a row's dS is done.
 template <int D>
@@ -439,34 +465,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sDO = smem + LY::kDO;
   uint8_t* sK = smem + LY::kK;
   uint8_t* sV = smem + LY::kV;
-  uint8_t* sDS = smem + LY::kDS;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + LY::kBar);
   uint64_t* bar_qd = bars;
   uint64_t* bar_kf = bar_qd + 1;
-  uint64_t* bar_ke = bar_kf + kSt;
-  uint64_t* bar_vf = bar_ke + kSt;
+  uint64_t* bar_ke = bar_kf + kKStQ;
+  uint64_t* bar_vf = bar_ke + kKStQ;
   uint64_t* bar_ve = bar_vf + kSt;
   uint64_t* bar_sf = bar_ve + kSt;   // [2] S buffer b computed
   uint64_t* bar_dpf = bar_sf + 2;    // dP computed
-  uint64_t* bar_dsr = bar_dpf + 1;   // dS written to shared memory
-  uint64_t* bar_dsf = bar_dsr + 1;   // dS buffer free (previous dQ done)
-  uint64_t* bar_done = bar_dsf + 1;  // dQ final
+  uint64_t* bar_dsr = bar_dpf + 1;   // dS written to TMEM
+  uint64_t* bar_done = bar_dsr + 1;  // dQ final
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + LY::kTmemSlot);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LY::kAbort);
 
   if (threadIdx.x == 0) {
     mbar_init(bar_qd, 1);
-    for (int s = 0; s < kSt; ++s) {
+    for (int s = 0; s < kKStQ; ++s) {
       mbar_init(&bar_kf[s], 1);
       mbar_init(&bar_ke[s], 1);
+    }
+    for (int s = 0; s < kSt; ++s) {
       mbar_init(&bar_vf[s], 1);
       mbar_init(&bar_ve[s], 1);
     }
     mbar_init(&bar_sf[0], 1);
     mbar_init(&bar_sf[1], 1);
     mbar_init(bar_dpf, 1);
-    mbar_init(bar_dsr, 128);
-    mbar_init(bar_dsf, 1);
+    mbar_init(bar_dsr, 2 * 128);
     mbar_init(bar_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -495,18 +520,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int n = 0;
       walk.run([&](int kt, bool) {
-        const int st = n % kSt;
+        const int ks = n % kKStQ, vs = n % kSt;
         const int krow = bh * p.N + kt * kT;
-        if (!mbar_wait(&bar_ke[st], ((n / kSt) & 1) ^ 1, p.st, abort_flag)) return false;
-        mbar_arrive_expect_tx(&bar_kf[st], LY::kTile);
+        if (!mbar_wait(&bar_ke[ks], ((n / kKStQ) & 1) ^ 1, p.st, abort_flag)) return false;
+        mbar_arrive_expect_tx(&bar_kf[ks], LY::kTile);
 #pragma unroll
         for (int s = 0; s < D / 64; ++s)
-          tma_load_2d(sK + st * LY::kTile + s * LY::kSlab, &tmK, &bar_kf[st], s * 64, krow);
-        if (!mbar_wait(&bar_ve[st], ((n / kSt) & 1) ^ 1, p.st, abort_flag)) return false;
-        mbar_arrive_expect_tx(&bar_vf[st], LY::kTile);
+          tma_load_2d(sK + ks * LY::kTile + s * LY::kSlab, &tmK, &bar_kf[ks], s * 64, krow);
+        if (!mbar_wait(&bar_ve[vs], ((n / kSt) & 1) ^ 1, p.st, abort_flag)) return false;
+        mbar_arrive_expect_tx(&bar_vf[vs], LY::kTile);
 #pragma unroll
         for (int s = 0; s < D / 64; ++s)
-          tma_load_2d(sV + st * LY::kTile + s * LY::kSlab, &tmV, &bar_vf[st], s * 64, krow);
+          tma_load_2d(sV + vs * LY::kTile + s * LY::kSlab, &tmV, &bar_vf[vs], s * 64, krow);
         ++n;
         return true;
       });
@@ -514,14 +539,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idSS = idesc_bf16_f32(kT, kT, false, false);  // K-major x K-major
-      constexpr uint32_t idDQ = idesc_bf16_f32(kT, D, false, true);    // K-major dS x MN-major K
-      const uint32_t q_base = smem_u32(sQ), do_base = smem_u32(sDO), ds_base = smem_u32(sDS);
+      constexpr uint32_t idDQ = idesc_bf16_f32(kT, D, false, true);    // TMEM dS x MN-major K
+      const uint32_t q_base = smem_u32(sQ), do_base = smem_u32(sDO);
       const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV);
+      auto a_col = [](int kk) -> uint32_t { return kk < 4 ? kk * 8 : 64 + (kk - 4) * 8; };
       auto issue_s = [&](int n) -> bool {
-        const int st = n % kSt;
-        if (!mbar_wait(&bar_kf[st], (n / kSt) & 1, p.st, abort_flag)) return false;
+        const int ks = n % kKStQ;
+        if (!mbar_wait(&bar_kf[ks], (n / kKStQ) & 1, p.st, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t kb = k_base + st * LY::kTile;
+        const uint32_t kb = k_base + ks * LY::kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * LY::kSlab + (kk & 3) * 32;
@@ -533,11 +559,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       bool ok = mbar_wait(bar_qd, 0, p.st, abort_flag) && issue_s(0);
       for (int n = 0; ok && n < n_total; ++n) {
-        const int st = n % kSt;
+        const int ks = n % kKStQ, vs = n % kSt;
         // dP = dO V^T (its columns were last read for dS of the previous step)
-        if (!(ok = mbar_wait(&bar_vf[st], (n / kSt) & 1, p.st, abort_flag))) break;
+        if (!(ok = mbar_wait(&bar_vf[vs], (n / kSt) & 1, p.st, abort_flag))) break;
         tc_fence_after();
-        const uint32_t vb = v_base + st * LY::kTile;
+        const uint32_t vb = v_base + vs * LY::kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * LY::kSlab + (kk & 3) * 32;
@@ -545,73 +571,65 @@ __global__ void __launch_bounds__(kThreads, 1)
                       kk > 0 ? 1u : 0u);
         }
         mma_commit(bar_dpf);
-        mma_commit(&bar_ve[st]);
+        mma_commit(&bar_ve[vs]);
         // scores of the next key tile into the other S buffer
         if (n + 1 < n_total && !(ok = issue_s(n + 1))) break;
-        // dQ += dS K
+        // dQ += dS K, dS read from this step's S buffer
         if (!(ok = mbar_wait(bar_dsr, n & 1, p.st, abort_flag))) break;
         tc_fence_after();
-        const uint32_t kb = k_base + st * LY::kTile;
+        const uint32_t kb = k_base + ks * LY::kTile;
+        const uint32_t tds = tmem + (n & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < kT / 16; ++kk)
-          mma_bf16_ss(tDQ, sdesc_sw128(ds_base + (kk >> 2) * LY::kSlab + (kk & 3) * 32, 16, 1024),
-                      sdesc_sw128(kb + kk * 2048, LY::kSlab, 1024), idDQ, (n > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bar_ke[st]);
-        mma_commit(bar_dsf);
+          mma_bf16_ts(tDQ, tds + a_col(kk), sdesc_sw128(kb + kk * 2048, LY::kSlab, 1024), idDQ,
+                      (n > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bar_ke[ks]);
       }
       mma_commit(bar_done);
     }
   } else if (warp >= 4) {
-    const int r = (warp - 4) * 32 + lane;  // query row = TMEM lane
+    const int h = (warp >> 2) - 1;          // key columns [64 h, 64 h + 64)
+    const int r = (warp & 3) * 32 + lane;   // query row = TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const float nl2 = -p.lse2[qrow0 + r];
     const float Dr = p.dvec[qrow0 + r];
     const float2 sl22 = make_float2(p.scale_log2, p.scale_log2), nl22 = make_float2(nl2, nl2);
-    uint8_t* ds_row = sDS + (r >> 3) * 1024 + (r & 7) * 128;
-    const uint32_t row_sw = (uint32_t)(r & 7);
     int n = 0;
     const bool ok = walk.run([&](int, bool diag) {
       if (!__all_sync(FULL, mbar_wait(&bar_sf[n & 1], (n >> 1) & 1, p.st, abort_flag))) return false;
       tc_fence_after();
-      float P[kT];
-      load_row128(tmem + (n & 1) * 128 + lane_off, P);
+      const uint32_t cS = tmem + (n & 1) * 128 + lane_off + h * kHalf;
+      float P[kHalf];
+      load_row64(cS, P);
 #pragma unroll
-      for (int c = 0; c < kT; c += 2) {
+      for (int c = 0; c < kHalf; c += 2) {
         const float2 t = fma2(make_float2(P[c], P[c + 1]), sl22, nl22);
         P[c] = ex2_approx(t.x);
         P[c + 1] = ex2_approx(t.y);
       }
       if (diag) {
 #pragma unroll
-        for (int c = 0; c < kT; ++c)
-          if (c > r) P[c] = 0.f;  // key c is in the future of query r
+        for (int c = 0; c < kHalf; ++c)
+          if (h * kHalf + c > r) P[c] = 0.f;  // key in the future of query r
       }
       if (!__all_sync(FULL, mbar_wait(bar_dpf, n & 1, p.st, abort_flag))) return false;
       tc_fence_after();
-      uint32_t pk[64];
-#pragma unroll
-      for (int c = 0; c < kT / 32; ++c) {
-        uint32_t reg[32];
-        tmem_ld32(tDP + lane_off + c * 32, reg);
+      {
+        uint32_t a[32], b[32];
+        tmem_ld32(tDP + lane_off + h * kHalf, a);
+        tmem_ld32(tDP + lane_off + h * kHalf + 32, b);
         tmem_ld_wait();
+        uint32_t pk[32];
 #pragma unroll
         for (int x = 0; x < 16; ++x) {
-          const int k = c * 32 + 2 * x;
-          pk[c * 16 + x] = pack_bf16x2(P[k] * (__uint_as_float(reg[2 * x]) - Dr),
-                                       P[k + 1] * (__uint_as_float(reg[2 * x + 1]) - Dr));
+          pk[x] = pack_bf16x2(P[2 * x] * (__uint_as_float(a[2 * x]) - Dr),
+                              P[2 * x + 1] * (__uint_as_float(a[2 * x + 1]) - Dr));
+          pk[16 + x] = pack_bf16x2(P[32 + 2 * x] * (__uint_as_float(b[2 * x]) - Dr),
+                                   P[33 + 2 * x] * (__uint_as_float(b[2 * x + 1]) - Dr));
         }
+        tmem_st32(cS, pk);  // bf16 dS over this group's first 32 S columns (already read)
       }
-      // the previous dQ MMA must have finished reading the dS buffer
-      if (n > 0 && !__all_sync(FULL, mbar_wait(bar_dsf, (n - 1) & 1, p.st, abort_flag))) return false;
-      // dS row r: keys [64 s, 64 s + 64) in slab s, 16-byte chunk c at c ^ (r & 7)
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        uint8_t* slab = ds_row + (c >> 3) * LY::kSlab;
-        const uint32_t chunk = (uint32_t)(c & 7);
-        *reinterpret_cast<uint4*>(slab + ((chunk ^ row_sw) << 4)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      }
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_dsr);
       ++n;
@@ -619,7 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     });
     if (ok && __all_sync(FULL, mbar_wait(bar_done, 0, p.st, abort_flag))) {
       tc_fence_after();
-      store_acc_row<D>(tDQ + lane_off, p.scale, p.dq + ((size_t)qrow0 + r) * D);
+      store_acc_row<D / 2>(tDQ + lane_off + h * (D / 2), p.scale, p.dq + ((size_t)qrow0 + r) * D + h * (D / 2));
     }
   }
 
