@@ -40,7 +40,17 @@ METRIC = "ring-attn fwd+bwd TFLOP/s & tokens/s on 1 B200; % of BF16 tensor peak"
 # source it was taken on (sha256 of the source file).
 # Captured on 8 heads of the n32k_d128 workload and scaled x4 to its 32 heads
 # (heads are independent units; see profiles/*_n32k_d128_h8.md).
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    ("bwd_kv_kernel", "n32k_d128"): {
+        "bytes": 4 * (272.112128e6 + 107.426816e6),
+        "sha256": "1e5d1c805c75bc9da5373177b94fe9ffc8ed319fd715584d09866ecbff829fda"},
+    ("bwd_q_kernel", "n32k_d128"): {
+        "bytes": 4 * (271.273472e6 + 51.107840e6),
+        "sha256": "1e5d1c805c75bc9da5373177b94fe9ffc8ed319fd715584d09866ecbff829fda"},
+    ("fwd_tc_kernel", "n32k_d128"): {
+        "bytes": 4 * (202.958592e6 + 49.582848e6),
+        "sha256": "e9db5aae1017ae8e993d973016b04ffacdea9fd4f4df0e639cd340068e47deb0"},
+}
 
 
 def parse():
