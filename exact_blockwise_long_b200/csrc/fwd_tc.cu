@@ -458,12 +458,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr int kThreads2 = 384;
 // Register split: launched at kLaunchRegs per thread (384 x 168 = 64512);
 // the softmax warpgroups rise to kSoftmaxRegs, the producer/MMA warpgroup
-// drops to kOtherRegs: 256 x 200 + 128 x 104 = 64512.  Per sub-partition:
-// 2 x 32 x 200 + 32 x 104 = 16128 of 16384.  The host launches this kernel
+// drops to kOtherRegs: 256 x 208 + 128 x 88 = 64512.  Per sub-partition:
+// 2 x 32 x 208 + 32 x 88 = 16128 of 16384.  The host launches this kernel
 // only when the compiled register count equals kLaunchRegs.
 constexpr int kLaunchRegs = 168;
-constexpr uint32_t kSoftmaxRegs = 200;
-constexpr uint32_t kOtherRegs = 104;
+constexpr uint32_t kSoftmaxRegs = 208;
+constexpr uint32_t kOtherRegs = 88;
 static_assert(256 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads2 * kLaunchRegs, "register split exceeds launch");
 
 template <int D>
