@@ -55,14 +55,14 @@ def test_bwd_full_oracle(B, H, N, D, S, qc, kc, causal):
     assert max(errs) <= TOL_BF16_GRAD, errs
 
 
-def test_bwd_repeatable_within_atomics_noise():
-    """dK, dV are written once per key tile (deterministic); dQ sums fp32
-    atomics, so only its last bits may change between runs."""
+def test_bwd_bit_reproducible():
+    """Every gradient accumulates on chip and is written once (no atomics):
+    repeated runs give identical bits."""
     q, k, v, do = small_attention_inputs(1, 2, 1024, 128, 5)
     a = run_bwd(q, k, v, do, 4, 128, 128, True)
-    b = run_bwd(q, k, v, do, 4, 128, 128, True)
-    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
-    assert (a[0].float() - b[0].float()).abs().max().item() <= 1e-2
+    for _ in range(3):
+        b = run_bwd(q, k, v, do, 4, 128, 128, True)
+        assert all(torch.equal(x, y) for x, y in zip(a, b))
 
 
 @pytest.mark.parametrize("name", ["n8k_d64_causal", "n8k_d64_full", "n32k_d128"])
@@ -94,3 +94,64 @@ def test_workload_bwd_sampled(name):
         kidx = torch.as_tensor(keys, device="cuda")
         assert max_abs(to_f64(dk[b, h][kidx]), gk) <= TOL_BF16_GRAD
         assert max_abs(to_f64(dv[b, h][kidx]), gv) <= TOL_BF16_GRAD
+
+
+@pytest.mark.slow
+def test_layer7b_attention_fwd_bwd_sampled():
+    """The 7B layer's attention at full size (N=131072, 32 heads x 128, S=32,
+    chunks 2048): 256 sampled forward rows and dq rows, and dk/dv on 64 key
+    rows of the last shard of two heads (under the causal mask those rows
+    need only the last shard's queries, so the fp64 check stays cheap)."""
+    from helpers import TOL_BF16_LSE, TOL_BF16_O, check_rows
+    w = WORKLOADS["layer7b_attn"]
+    q, k, v, do = attention_inputs(w)
+    o, lse = run_fwd(q, k, v, w.S, w.q_chunk, w.k_chunk, w.causal)
+    rows = sample_rows(w.B, w.H, w.N, 256, w.seed)
+    e_o, e_l = check_rows(q, k, v, o, lse, rows, w.causal)
+    assert e_o <= TOL_BF16_O and e_l <= TOL_BF16_LSE, (e_o, e_l)
+    import exact_blockwise_long_b200 as ra
+    B, H, N, D = q.shape
+    ws = torch.empty(ra.ringattn_bwd_workspace_size(B, H, N, D), device="cuda", dtype=torch.uint8)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ra.ringattn_bwd(q, k, v, o, lse, do, dq, dk, dv, w.S, w.q_chunk, w.k_chunk, w.causal, ws)
+    assert ra.ringattn_get_error() == 0
+    err_q = 0.0
+    for b, h in sorted({(int(b), int(h)) for b, h, _ in rows})[:8]:
+        sel = rows[(rows[:, 0] == b) & (rows[:, 1] == h)]
+        local = np.stack([np.zeros(len(sel), np.int64), np.zeros(len(sel), np.int64), sel[:, 2]], 1)
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        ref = oracle.attention_backward_query_rows(to_f64(q[sl]), to_f64(k[sl]), to_f64(v[sl]), to_f64(do[sl]),
+                                                   local, w.causal)
+        got = to_f64(dq[b, h][torch.as_tensor(sel[:, 2], device="cuda")])
+        err_q = max(err_q, max_abs(got, ref))
+    assert err_q <= TOL_BF16_GRAD, err_q
+    L = w.N // w.S
+    rng = np.random.default_rng(w.seed + 3000)
+    for b, h in [(0, 3), (0, 30)]:
+        keys = np.sort(rng.choice(np.arange(w.N - L, w.N), 64, replace=False))
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        gk, gv = oracle.attention_backward_key_rows(to_f64(q[sl]), to_f64(k[sl]), to_f64(v[sl]), to_f64(do[sl]),
+                                                    0, 0, keys, w.causal)
+        kidx = torch.as_tensor(keys, device="cuda")
+        assert max_abs(to_f64(dk[b, h][kidx]), gk) <= TOL_BF16_GRAD
+        assert max_abs(to_f64(dv[b, h][kidx]), gv) <= TOL_BF16_GRAD
+
+
+@pytest.mark.slow
+def test_layer7b_ffn_full_size_sampled():
+    """The 7B layer's feed-forward over all N=131072 tokens in 2048-token
+    chunks; 64 seeded rows checked against fp64 (bound as in test_ffn_gpu)."""
+    import exact_blockwise_long_b200 as ra
+    from exact_blockwise_long_b200.synthetic import FFN_WORKLOADS, ffn_inputs
+    w = FFN_WORKLOADS["layer7b_ffn"]
+    x, w1, w2, w3 = ffn_inputs(w)
+    y = torch.empty_like(x)
+    ws = torch.empty(ra.blockwise_ffn_workspace_size(w.chunk, w.d_ff), device="cuda", dtype=torch.uint8)
+    ra.blockwise_ffn(x, w1, w2, w3, y, w.chunk, ws)
+    assert ra.ringattn_get_error() == 0
+    rows = np.sort(np.random.default_rng(w.seed + 1000).choice(w.T, 64, replace=False))
+    rows[0], rows[-1] = 0, w.T - 1
+    idx = torch.as_tensor(rows, device="cuda")
+    ref = oracle.swiglu_ffn(to_f64(x[idx]), to_f64(w1), to_f64(w2), to_f64(w3))
+    err = np.abs(to_f64(y[idx]) - ref)
+    assert np.all(err <= 2.0 ** -8 * np.abs(ref) + 0.03), float(err.max())
