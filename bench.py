@@ -59,7 +59,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="n32k_d128",
-                    choices=["n32k_d128", "n8k_d64_causal", "n8k_d64_full", "layer7b", "n1m_d128"])
+                    choices=["n32k_d128", "n8k_d64_causal", "n8k_d64_full", "layer7b", "n1m_d128",
+                             "n32k_d128_gqa8"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -109,7 +110,8 @@ def whole_job_tflops(flops_per_rank: float, world: int, ms_step: float) -> float
 
 def describe(aw, fw):
     d = {"workload": f"{aw.name}: ring attention {'fwd+bwd' if aw.bwd else 'fwd'}, B={aw.B}, H={aw.H}, "
-                     f"N={aw.N}, d={aw.D}, S={aw.S}, q_chunk={aw.q_chunk}, k_chunk={aw.k_chunk}, "
+                     + (f"Hkv={aw.kv_heads}, " if aw.kv_heads != aw.H else "")
+                     + f"N={aw.N}, d={aw.D}, S={aw.S}, q_chunk={aw.q_chunk}, k_chunk={aw.k_chunk}, "
                      f"{'causal' if aw.causal else 'non-causal'}"
                      + (f"; blockwise SwiGLU FFN {fw.d_model}->{fw.d_ff}->{fw.d_model}, chunk {fw.chunk}"
                         if fw else ""),
@@ -298,6 +300,19 @@ def main():
         ffn_ws = torch.empty(ra.blockwise_ffn_workspace_size(fw.chunk, fw.d_ff), device=dev, dtype=torch.uint8)
     stream = torch.cuda.current_stream()
     cfg = (aw.S, aw.q_chunk, aw.k_chunk, aw.causal)
+    gqa = aw.kv_heads != aw.H
+
+    def fwd_call(qq, kk, vv, oo, ll):
+        if gqa:
+            ra.ringattn_fwd_gqa(qq, kk, vv, oo, ll, *cfg)
+        else:
+            ra.ringattn_fwd(qq, kk, vv, oo, ll, *cfg)
+
+    def bwd_call(qq, kk, vv, oo, ll, dd, gq, gk, gv):
+        if gqa:
+            ra.ringattn_bwd_gqa(qq, kk, vv, oo, ll, dd, gq, gk, gv, *cfg, ws)
+        else:
+            ra.ringattn_bwd(qq, kk, vv, oo, ll, dd, gq, gk, gv, *cfg, ws)
 
     ev = {}
 
@@ -308,11 +323,17 @@ def main():
         if timed:
             e = [event() for _ in range(5)]
             e[0].record(stream)
-        ra.ringattn_fwd(q, k, v, o, lse, *cfg)
+        fwd_call(q, k, v, o, lse)
         launches = 1
         if timed:
             e[1].record(stream)
-        if aw.bwd:
+        if aw.bwd and gqa:
+            bwd_call(q, k, v, o, lse, do, dq, dk, dv)
+            if timed:
+                e[2].record(stream)
+                e[4].record(stream)
+            launches += 3
+        elif aw.bwd:
             ra.ringattn_bwd_phase(q, k, v, o, lse, do, dq, dk, dv, *cfg, ws, 1)
             if timed:
                 e[2].record(stream)
@@ -328,7 +349,9 @@ def main():
             launches += 2 * (fw.T // fw.chunk)
         if timed:
             ev.setdefault("fwd", []).append((e[0], e[1]))
-            if aw.bwd:
+            if aw.bwd and gqa:
+                ev.setdefault("bwd", []).append((e[1], e[4]))
+            elif aw.bwd:
                 ev.setdefault("bwd_kv", []).append((e[2], e[3]))
                 ev.setdefault("bwd_q", []).append((e[3], e[4]))
         return launches
@@ -374,7 +397,10 @@ def main():
     fwd_fl = attn_fwd_flops(aw)
     fwd_name = "fwd_tc2_kernel" if (aw.N // aw.S) % 256 == 0 else "fwd_tc_kernel"
     kernels = {fwd_name: (mean_ms(ev["fwd"]), fwd_fl, "fwd_tc.cu")}
-    if aw.bwd:
+    if aw.bwd and gqa:
+        # one call: preprocess + dK/dV + dQ launches, timed together
+        kernels["bwd_kv_kernel+bwd_q_kernel"] = (mean_ms(ev["bwd"]), 2.5 * fwd_fl, "bwd_tc.cu")
+    elif aw.bwd:
         kernels["bwd_kv_kernel"] = (mean_ms(ev["bwd_kv"]), 2.0 * fwd_fl, "bwd_tc.cu")
         kernels["bwd_q_kernel"] = (mean_ms(ev["bwd_q"]), 0.5 * fwd_fl, "bwd_tc.cu")
     kname = max(kernels, key=lambda k_: kernels[k_][0])
@@ -434,9 +460,9 @@ def main():
                 stream.wait_event(copied[bi])  # step j-2's results have been read back
             qq, kk, vv = ins[bi][0], ins[bi][1], ins[bi][2]
             oo, ll = outs[bi][0], outs[bi][1]
-            ra.ringattn_fwd(qq, kk, vv, oo, ll, *cfg)
+            fwd_call(qq, kk, vv, oo, ll)
             if aw.bwd:
-                ra.ringattn_bwd(qq, kk, vv, oo, ll, ins[bi][3], outs[bi][2], outs[bi][3], outs[bi][4], *cfg, ws)
+                bwd_call(qq, kk, vv, oo, ll, ins[bi][3], outs[bi][2], outs[bi][3], outs[bi][4])
             if fw is not None:
                 ra.blockwise_ffn(ins[bi][-1], w1, w2, w3, outs[bi][-1], fw.chunk, ffn_ws)
             done[bi].record(stream)

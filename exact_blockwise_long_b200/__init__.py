@@ -9,6 +9,8 @@ kernels.  PyTorch is used for device memory and streams only.
 from ._lib import RA_BF16, RA_F32, RingAttnError, lib  # noqa: F401
 from .api import (  # noqa: F401
     ringattn_fwd,
+    ringattn_fwd_gqa,
+    ringattn_bwd_gqa,
     ringattn_fwd_step,
     ringattn_merge,
     ringattn_bwd,
@@ -22,7 +24,7 @@ from .api import (  # noqa: F401
 )
 
 __all__ = [
-    "ringattn_fwd", "ringattn_fwd_step", "ringattn_merge", "ringattn_bwd", "ringattn_bwd_phase", "ringattn_bwd_noalloc", "ringattn_bwd_workspace_size",
+    "ringattn_fwd", "ringattn_fwd_gqa", "ringattn_bwd_gqa", "ringattn_fwd_step", "ringattn_merge", "ringattn_bwd", "ringattn_bwd_phase", "ringattn_bwd_noalloc", "ringattn_bwd_workspace_size",
     "blockwise_ffn", "blockwise_ffn_workspace_size", "ringattn_get_error", "ringattn_selftest_timeout",
     "RA_BF16", "RA_F32", "RingAttnError", "lib",
 ]

@@ -32,6 +32,9 @@ SIGNATURES = {
     "ringattn_version": (_I, []),
     "ringattn_status_string": (ctypes.c_char_p, [_I]),
     "ringattn_fwd": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _F, _P]),
+    "ringattn_fwd_gqa": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _F, _P]),
+    "ringattn_bwd_gqa": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I,
+                              _F, _P, _SZ, _P]),
     "ringattn_fwd_step": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _F, _I, _P]),
     "ringattn_merge": (_I, [_P, _P, _P, _P, _I64, _I64, _P]),
     "ringattn_bwd_workspace_size": (_SZ, [_I64, _I64, _I64, _I64]),

@@ -54,6 +54,42 @@ def ringattn_fwd(q, k, v, out, lse, S, q_chunk, k_chunk, causal, scale=0.0, stre
     return out, lse
 
 
+def ringattn_fwd_gqa(q, k, v, out, lse, S, q_chunk, k_chunk, causal, scale=0.0, stream=None):
+    """ringattn_fwd with grouped key/value heads: k, v are [B, Hkv, N, D]."""
+    B, H, N, D = _bhnd(q)
+    Hkv = int(k.shape[1])
+    if tuple(k.shape) != (B, Hkv, N, D) or k.shape != v.shape or out.shape != q.shape:
+        raise ValueError("q, out are [B, H, N, D]; k, v are [B, Hkv, N, D]")
+    for t in (k, v, out):
+        if t.dtype != q.dtype:
+            raise ValueError("q, k, v, out must share dtype")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N):
+        raise ValueError("lse must be float32 [B, H, N]")
+    call("ringattn_fwd_gqa", _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), _dev(lse, "lse"),
+         B, H, Hkv, N, D, _dtype(q), int(S), int(q_chunk), int(k_chunk), int(bool(causal)), float(scale),
+         _stream(stream))
+    return out, lse
+
+
+def ringattn_bwd_gqa(q, k, v, out, lse, dout, dq, dk, dv, S, q_chunk, k_chunk, causal, workspace,
+                     scale=0.0, stream=None):
+    """ringattn_bwd with grouped key/value heads: k, v, dk, dv are [B, Hkv, N, D]."""
+    B, H, N, D = _bhnd(q)
+    Hkv = int(k.shape[1])
+    for t in (out, dout, dq):
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("q, out, dout, dq must share shape and dtype")
+    for t in (v, dk, dv):
+        if t.shape != k.shape or t.dtype != q.dtype:
+            raise ValueError("k, v, dk, dv must share shape [B, Hkv, N, D] and dtype")
+    nbytes = workspace.numel() * workspace.element_size()
+    call("ringattn_bwd_gqa", _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), _dev(lse, "lse"),
+         _dev(dout, "dout"), _dev(dq, "dq"), _dev(dk, "dk"), _dev(dv, "dv"), B, H, Hkv, N, D, _dtype(q),
+         int(S), int(q_chunk), int(k_chunk), int(bool(causal)), float(scale), _dev(workspace, "workspace"),
+         nbytes, _stream(stream))
+    return dq, dk, dv
+
+
 def ringattn_fwd_step(q, k, v, o_acc, lse_acc, S, q_chunk, k_chunk, causal, t, scale=0.0, stream=None):
     """Merge ring step t of (q, k, v) into the fp32 accumulators (o_acc, lse_acc)."""
     B, H, N, D = _bhnd(q)

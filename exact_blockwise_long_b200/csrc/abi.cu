@@ -158,12 +158,19 @@ const char* ringattn_status_string(int status) {
 int ringattn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t H,
                  int64_t N, int64_t D, int dtype, int S, int q_chunk, int k_chunk, int causal, float scale,
                  void* stream) {
+  return ringattn_fwd_gqa(q, k, v, out, lse, B, H, H, N, D, dtype, S, q_chunk, k_chunk, causal, scale, stream);
+}
+
+int ringattn_fwd_gqa(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t H,
+                     int64_t Hkv, int64_t N, int64_t D, int dtype, int S, int q_chunk, int k_chunk, int causal,
+                     float scale, void* stream) {
+  if (Hkv < 0 || (Hkv == 0 && H != 0) || (Hkv > 0 && H % Hkv != 0)) return RA_ERR_ARG;
   int rc = check_attn(q, k, v, B, H, N, D, dtype, S, q_chunk, k_chunk, causal);
   if (rc == kEmpty) return RA_OK;
   if (rc != RA_OK) return rc;
   if (!out || !lse) return RA_ERR_ARG;
   if (!aligned16(out) || !aligned16(lse)) return RA_ERR_ALIGN;
-  AttnArgs a{q, k, v, B, H, N, D, dtype, S, q_chunk, k_chunk, causal, resolve_scale(scale, D)};
+  AttnArgs a{q, k, v, B, H, N, D, dtype, S, q_chunk, k_chunk, causal, resolve_scale(scale, D), Hkv};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == RA_F32) return launch_fwd_simt(a, out, lse, nullptr, nullptr, -1, st);
   return launch_fwd_tc(a, out, lse, nullptr, nullptr, -1, st);
@@ -172,13 +179,14 @@ int ringattn_fwd(const void* q, const void* k, const void* v, void* out, float* 
 int ringattn_fwd_step(const void* q, const void* k, const void* v, float* o_acc, float* lse_acc, int64_t B,
                       int64_t H, int64_t N, int64_t D, int dtype, int S, int q_chunk, int k_chunk, int causal,
                       float scale, int t, void* stream) {
+  const int64_t Hkv = H;
   if (t < 0 || t >= S) return RA_ERR_ARG;
   int rc = check_attn(q, k, v, B, H, N, D, dtype, S, q_chunk, k_chunk, causal);
   if (rc == kEmpty) return RA_OK;
   if (rc != RA_OK) return rc;
   if (!o_acc || !lse_acc) return RA_ERR_ARG;
   if (!aligned16(o_acc) || !aligned16(lse_acc)) return RA_ERR_ALIGN;
-  AttnArgs a{q, k, v, B, H, N, D, dtype, S, q_chunk, k_chunk, causal, resolve_scale(scale, D)};
+  AttnArgs a{q, k, v, B, H, N, D, dtype, S, q_chunk, k_chunk, causal, resolve_scale(scale, D), Hkv};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == RA_F32) return launch_fwd_simt(a, nullptr, nullptr, o_acc, lse_acc, t, st);
   return launch_fwd_tc(a, nullptr, nullptr, o_acc, lse_acc, t, st);
@@ -200,11 +208,13 @@ size_t ringattn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D) {
   return 2 * ((dvec + 255) & ~(size_t)255);
 }
 
-int ringattn_bwd_phase(const void* q, const void* k, const void* v, const void* out, const float* lse,
-                       const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N, int64_t D,
-                       int dtype, int S, int q_chunk, int k_chunk, int causal, float scale, void* workspace,
-                       size_t workspace_bytes, int phase_mask, void* stream) {
+namespace {
+int bwd_impl(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+             void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t D, int dtype, int S,
+             int q_chunk, int k_chunk, int causal, float scale, void* workspace, size_t workspace_bytes,
+             int phase_mask, void* stream) {
   if (phase_mask <= 0 || phase_mask > 7) return RA_ERR_ARG;
+  if (Hkv < 0 || (Hkv == 0 && H != 0) || (Hkv > 0 && H % Hkv != 0)) return RA_ERR_ARG;
   int rc = check_attn(q, k, v, B, H, N, D, dtype, S, q_chunk, k_chunk, causal);
   if (rc == kEmpty) return dtype == RA_BF16 ? RA_OK : RA_ERR_UNSUPPORTED;
   if (rc != RA_OK) return rc;
@@ -215,8 +225,25 @@ int ringattn_bwd_phase(const void* q, const void* k, const void* v, const void* 
   if (dtype != RA_BF16) return RA_ERR_UNSUPPORTED;
   if (!workspace || workspace_bytes < ringattn_bwd_workspace_size(B, H, N, D)) return RA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return RA_ERR_ALIGN;
-  AttnArgs a{q, k, v, B, H, N, D, dtype, S, q_chunk, k_chunk, causal, resolve_scale(scale, D)};
+  AttnArgs a{q, k, v, B, H, N, D, dtype, S, q_chunk, k_chunk, causal, resolve_scale(scale, D), Hkv};
   return launch_bwd_tc(a, out, lse, dout, dq, dk, dv, workspace, phase_mask, static_cast<cudaStream_t>(stream));
+}
+}  // namespace
+
+int ringattn_bwd_phase(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                       const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N, int64_t D,
+                       int dtype, int S, int q_chunk, int k_chunk, int causal, float scale, void* workspace,
+                       size_t workspace_bytes, int phase_mask, void* stream) {
+  return bwd_impl(q, k, v, out, lse, dout, dq, dk, dv, B, H, H, N, D, dtype, S, q_chunk, k_chunk, causal, scale,
+                  workspace, workspace_bytes, phase_mask, stream);
+}
+
+int ringattn_bwd_gqa(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                     const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t Hkv, int64_t N,
+                     int64_t D, int dtype, int S, int q_chunk, int k_chunk, int causal, float scale,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_impl(q, k, v, out, lse, dout, dq, dk, dv, B, H, Hkv, N, D, dtype, S, q_chunk, k_chunk, causal, scale,
+                  workspace, workspace_bytes, 7, stream);
 }
 
 int ringattn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,

@@ -50,23 +50,29 @@ struct BParams {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int BH, N, S, L, causal, num_tiles;
+  int H, G;            // query heads; query heads per key/value head
+  int BHkv;            // batch x key/value heads
   int group;           // heads per scheduling group
   float scale, scale_log2;
   DevStatus st;
 };
 
-// Query tiles a stationary key tile meets, in ring order (j + t) mod S.
+// Query tiles a stationary key tile meets, in ring order (j + t) mod S, for
+// each of the G query heads (flat indices qbh0 .. qbh0 + G - 1) that share
+// its key/value head.
 struct RingWalkKV {
-  int jshard, S, tps, kt, causal;
+  int jshard, S, tps, kt, causal, qbh0, G;
   template <typename F>
   __device__ __forceinline__ bool run(F&& body) const {
-    for (int t = 0; t < S; ++t) {
-      int i = jshard + t;
-      if (i >= S) i -= S;
-      if (causal && i < jshard) continue;
-      const int qt0 = (causal && i == jshard) ? kt : i * tps;
-      for (int qt = qt0; qt < i * tps + tps; ++qt)
-        if (!body(qt, causal && qt == kt)) return false;
+    for (int g = 0; g < G; ++g) {
+      for (int t = 0; t < S; ++t) {
+        int i = jshard + t;
+        if (i >= S) i -= S;
+        if (causal && i < jshard) continue;
+        const int qt0 = (causal && i == jshard) ? kt : i * tps;
+        for (int qt = qt0; qt < i * tps + tps; ++qt)
+          if (!body(qbh0 + g, qt, causal && qt == kt)) return false;
+      }
     }
     return true;
   }
@@ -78,7 +84,7 @@ struct RingWalkKV {
       if (causal && i < jshard) continue;
       n += (causal && i == jshard) ? (i * tps + tps - kt) : tps;
     }
-    return n;
+    return n * G;
   }
 };
 
@@ -108,22 +114,6 @@ struct RingWalkQ {
     return n;
   }
 };
-
-__device__ __forceinline__ void load_row128(uint32_t taddr, float (&s)[kT]) {
-  uint32_t a[32], b[32], c[32], d[32];
-  tmem_ld32(taddr, a);
-  tmem_ld32(taddr + 32, b);
-  tmem_ld32(taddr + 64, c);
-  tmem_ld32(taddr + 96, d);
-  tmem_ld_wait();
-#pragma unroll
-  for (int x = 0; x < 32; ++x) {
-    s[x] = __uint_as_float(a[x]);
-    s[32 + x] = __uint_as_float(b[x]);
-    s[64 + x] = __uint_as_float(c[x]);
-    s[96 + x] = __uint_as_float(d[x]);
-  }
-}
 
 __device__ __forceinline__ void load_row64(uint32_t taddr, float (&s)[kHalf]) {
   uint32_t a[32], b[32];
@@ -196,12 +186,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // heads in small groups; the heaviest causal key tiles (smallest index) first
-  int bh, kt;
-  grouped_order((int)blockIdx.x, p.num_tiles, p.BH, p.group, bh, kt);
-  const int krow0 = bh * p.N + kt * kT;
+  // key/value heads in small groups; the heaviest causal key tiles (smallest
+  // index) first
+  int kvbh, kt;
+  grouped_order((int)blockIdx.x, p.num_tiles, p.BHkv, p.group, kvbh, kt);
+  const int krow0 = kvbh * p.N + kt * kT;
   const int tps = p.L / kT;
-  const RingWalkKV walk{(kt * kT) / p.L, p.S, tps, kt, p.causal};
+  const int Hkv = p.H / p.G;
+  const int qbh0 = (kvbh / Hkv) * p.H + (kvbh % Hkv) * p.G;  // first query head of the group
+  const RingWalkKV walk{(kt * kT) / p.L, p.S, tps, kt, p.causal, qbh0, p.G};
   const int n_total = walk.count();
 
   uint8_t* sK = smem + LY::kK;
@@ -258,9 +251,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(sV + s * LY::kSlab, &tmV, bar_kv, s * 64, krow0);
       }
       int n = 0;
-      walk.run([&](int qt, bool) {
+      walk.run([&](int qbh, int qt, bool) {
         const int st = n % kSt;
-        const int qrow = bh * p.N + qt * kT;
+        const int qrow = qbh * p.N + qt * kT;
         if (!mbar_wait(&bar_qe[st], ((n / kSt) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_qf[st], 2 * LY::kTile + 1024);
 #pragma unroll
@@ -340,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t cS = tS + lane_off + h * kHalf, cDP = tDP + lane_off + h * kHalf;
     const float2 sl22 = make_float2(p.scale_log2, p.scale_log2);
     int n = 0;
-    const bool ok = walk.run([&](int, bool diag) {
+    const bool ok = walk.run([&](int, int, bool diag) {
       const int st = n % kSt;
       if (!__all_sync(FULL, mbar_wait(&bar_qf[st], (n / kSt) & 1, p.st, abort_flag))) return false;
       if (!__all_sync(FULL, mbar_wait(bar_sf, n & 1, p.st, abort_flag))) return false;
@@ -521,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int n = 0;
       walk.run([&](int kt, bool) {
         const int ks = n % kKStQ, vs = n % kSt;
-        const int krow = bh * p.N + kt * kT;
+        const int krow = kv_head_of(bh, p.H, p.G) * p.N + kt * kT;
         if (!mbar_wait(&bar_ke[ks], ((n / kKStQ) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_kf[ks], LY::kTile);
 #pragma unroll
@@ -714,9 +707,10 @@ int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* d
   if ((phase_mask & 6) == 0) return RA_OK;
 
   alignas(64) CUtensorMap tq, tk, tv, tdo;
+  const int64_t kv_rows = a.B * a.Hkv * a.N;
   if (make_tmap_bf16_2d(&tq, a.q, D, rows, D * 2, 64, kT) != RA_OK) return RA_ERR_CUDA;
-  if (make_tmap_bf16_2d(&tk, a.k, D, rows, D * 2, 64, kT) != RA_OK) return RA_ERR_CUDA;
-  if (make_tmap_bf16_2d(&tv, a.v, D, rows, D * 2, 64, kT) != RA_OK) return RA_ERR_CUDA;
+  if (make_tmap_bf16_2d(&tk, a.k, D, kv_rows, D * 2, 64, kT) != RA_OK) return RA_ERR_CUDA;
+  if (make_tmap_bf16_2d(&tv, a.v, D, kv_rows, D * 2, 64, kT) != RA_OK) return RA_ERR_CUDA;
   if (make_tmap_bf16_2d(&tdo, dout, D, rows, D * 2, 64, kT) != RA_OK) return RA_ERR_CUDA;
   BParams p{};
   p.lse2 = lse2;
@@ -725,28 +719,32 @@ int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* d
   p.dk = (__nv_bfloat16*)dk;
   p.dv = (__nv_bfloat16*)dv;
   p.BH = (int)(a.B * a.H);
+  p.H = (int)a.H;
+  p.G = (int)(a.H / a.Hkv);
+  p.BHkv = (int)(a.B * a.Hkv);
   p.N = (int)a.N;
   p.S = a.S;
   p.L = (int)(a.N / a.S);
   p.causal = a.causal;
   p.num_tiles = (int)(a.N / kT);
-  // per head: Q, dO, K, V (bf16) stream through L2
-  p.group = head_group(p.num_tiles, p.BH, (double)a.N * D * 4 * 2, 100.0e6);
   p.scale = a.scale;
   p.scale_log2 = a.scale * kLog2e;
   int rc = current_status(&p.st);
   if (rc != RA_OK) return rc;
-  const unsigned grid = (unsigned)(p.BH * p.num_tiles);
   if (phase_mask & 2) {
+    // per key/value head: K, V and its query heads' Q, dO stream through L2
+    p.group = head_group(p.num_tiles, p.BHkv, (double)a.N * D * 2 * (2 + 2 * p.G), 100.0e6);
     auto kern = bwd_kv_kernel<D>;
     if (set_smem_attr((const void*)kern, KVLayout<D>::kAlloc) != RA_OK) return RA_ERR_CUDA;
-    kern<<<grid, kThreads, KVLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
+    kern<<<(unsigned)(p.BHkv * p.num_tiles), kThreads, KVLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
     if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
   }
   if (phase_mask & 4) {
+    // per query head: Q, dO, K, V (bf16) stream through L2
+    p.group = head_group(p.num_tiles, p.BH, (double)a.N * D * 4 * 2, 100.0e6);
     auto kern = bwd_q_kernel<D>;
     if (set_smem_attr((const void*)kern, QLayout<D>::kAlloc) != RA_OK) return RA_ERR_CUDA;
-    kern<<<grid, kThreads, QLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
+    kern<<<(unsigned)(p.BH * p.num_tiles), kThreads, QLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
     if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
   }
   return RA_OK;

@@ -266,6 +266,12 @@ __device__ __forceinline__ void grouped_order(int block, int per_head, int heads
   head = g0 + in % gh;
 }
 
+// Flat (batch, key/value head) index of flat (batch, query head) bh when
+// groups of G = H / Hkv query heads share one key/value head.
+__device__ __forceinline__ int kv_head_of(int bh, int H, int G) {
+  return (bh / H) * (H / G) + (bh % H) / G;
+}
+
 // ---------------------------------------------------------------------------
 // Arithmetic helpers
 // ---------------------------------------------------------------------------

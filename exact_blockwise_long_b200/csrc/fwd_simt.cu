@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(const T* __restrict_
                                                             const T* __restrict__ v, T* __restrict__ out,
                                                             float* __restrict__ lse, float* __restrict__ o_acc,
                                                             float* __restrict__ lse_acc, int N, int S,
-                                                            int causal, float scale, int step) {
+                                                            int causal, float scale, int step, int H, int G) {
   constexpr int DP = D / kTPR;
   extern __shared__ float smem_f[];
   float* sK = smem_f;             // [kBK][D]
@@ -72,6 +72,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(const T* __restrict_
   const int ishard = q0 / L;
   const int row = q0 + r;
   const size_t head = (size_t)bh * N * D;
+  const size_t kv_head = (size_t)((bh / H) * (H / G) + (bh % H) / G) * N * D;
 
   float qr[DP];
 #pragma unroll
@@ -99,7 +100,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(const T* __restrict_
     for (int kt = kbeg; kt < kend; kt += kBK) {
       __syncthreads();
       for (int e = tid; e < kBK * D; e += kThreads) {
-        const size_t g = head + (size_t)kt * D + e;
+        const size_t g = kv_head + (size_t)kt * D + e;
         sK[e] = to_f32(k[g]);
         sV[e] = to_f32(v[g]);
       }
@@ -182,12 +183,14 @@ int launch_typed(const AttnArgs& a, void* out, float* lse, float* o_acc, float* 
     auto kern = fwd_simt_kernel<D, T, false>;
     if (set_smem_attr((const void*)kern, smem) != RA_OK) return RA_ERR_CUDA;
     kern<<<grid, kThreads, smem, stream>>>((const T*)a.q, (const T*)a.k, (const T*)a.v, (T*)out, lse, nullptr,
-                                           nullptr, (int)a.N, a.S, a.causal, a.scale, 0);
+                                           nullptr, (int)a.N, a.S, a.causal, a.scale, 0, (int)a.H,
+                                           (int)(a.H / a.Hkv));
   } else {
     auto kern = fwd_simt_kernel<D, T, true>;
     if (set_smem_attr((const void*)kern, smem) != RA_OK) return RA_ERR_CUDA;
     kern<<<grid, kThreads, smem, stream>>>((const T*)a.q, (const T*)a.k, (const T*)a.v, nullptr, nullptr,
-                                           o_acc, lse_acc, (int)a.N, a.S, a.causal, a.scale, step);
+                                           o_acc, lse_acc, (int)a.N, a.S, a.causal, a.scale, step, (int)a.H,
+                                           (int)(a.H / a.Hkv));
   }
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }

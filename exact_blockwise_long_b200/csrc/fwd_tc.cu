@@ -68,6 +68,7 @@ struct Params {
   float* o_acc;     // step mode: fp32 running output
   float* lse_acc;   // step mode: fp32 running lse
   int BH, N, S, L, causal, step;
+  int H, G;  // query heads; query heads per key/value head
   int num_qtiles;
   int group;  // heads per scheduling group
   float scale_log2;
@@ -322,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < D / 64; ++s) tma_load_2d(sQ + s * LY::kSlabBytes, &tmQ, bar_q, s * 64, qrow0);
       int n = 0;
       walk.run([&](int kt, bool) {
-        const int krow = bh * p.N + kt * kBN;
+        const int krow = kv_head_of(bh, p.H, p.G) * p.N + kt * kBN;
         const int ks = n % kKSt, vs = n % kVSt;
         if (!mbar_wait(&bar_ke[ks], ((n / kKSt) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_kf[ks], LY::kTileBytes);
@@ -593,7 +594,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
           tma_load_2d(sQ + t * LY::kTileBytes + s * LY::kSlabBytes, &tmQ, bar_q, s * 64, qrow0 + t * kBM);
       int n = 0;
       walk.run([&](int kt, bool, bool, bool) {
-        const int krow = bh * p.N + kt * kBN;
+        const int krow = kv_head_of(bh, p.H, p.G) * p.N + kt * kBN;
         const int ks = n % kKSt, vs = n % kVSt;
         if (!mbar_wait(&bar_ke[ks], ((n / kKSt) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_kf[ks], LY::kTileBytes);
@@ -721,15 +722,18 @@ int launch_d(const AttnArgs& a, void* out, float* lse, float* o_acc, float* lse_
              cudaStream_t stream) {
   alignas(64) CUtensorMap tq, tk, tv;
   const uint64_t rows = (uint64_t)(a.B * a.H * a.N);
+  const uint64_t kv_rows = (uint64_t)(a.B * a.Hkv * a.N);
   if (make_tmap_bf16_2d(&tq, a.q, D, rows, D * 2, 64, kBM) != RA_OK) return RA_ERR_CUDA;
-  if (make_tmap_bf16_2d(&tk, a.k, D, rows, D * 2, 64, kBN) != RA_OK) return RA_ERR_CUDA;
-  if (make_tmap_bf16_2d(&tv, a.v, D, rows, D * 2, 64, kBN) != RA_OK) return RA_ERR_CUDA;
+  if (make_tmap_bf16_2d(&tk, a.k, D, kv_rows, D * 2, 64, kBN) != RA_OK) return RA_ERR_CUDA;
+  if (make_tmap_bf16_2d(&tv, a.v, D, kv_rows, D * 2, 64, kBN) != RA_OK) return RA_ERR_CUDA;
   Params p{};
   p.out = (__nv_bfloat16*)out;
   p.lse = lse;
   p.o_acc = o_acc;
   p.lse_acc = lse_acc;
   p.BH = (int)(a.B * a.H);
+  p.H = (int)a.H;
+  p.G = (int)(a.H / a.Hkv);
   p.N = (int)a.N;
   p.S = a.S;
   p.L = (int)(a.N / a.S);

@@ -23,6 +23,7 @@ struct AttnArgs {
   int dtype;
   int S, q_chunk, k_chunk, causal;
   float scale;  // already resolved (> 0)
+  int64_t Hkv;  // key/value heads; query head h reads key/value head h / (H / Hkv)
 };
 
 // Exact fp32 CUDA-core ring forward (whole ring, or one step merged into

@@ -35,6 +35,11 @@ class AttnWorkload:
     dtype: torch.dtype = torch.bfloat16
     k_scale: float = 1.0
     bwd: bool = True
+    Hkv: int = 0  # key/value heads (grouped-query attention); 0 means H
+
+    @property
+    def kv_heads(self) -> int:
+        return self.Hkv or self.H
 
 
 @dataclass(frozen=True)
@@ -61,6 +66,9 @@ WORKLOADS = {
     "layer7b_attn": AttnWorkload("layer7b_attn", 1, 32, 131072, 128, 32, 2048, 2048, True, 3),
     # million-token causal forward: S=64, q_chunk 1024, k_chunk 4096
     "n1m_d128": AttnWorkload("n1m_d128", 1, 32, 1048576, 128, 64, 1024, 4096, True, 4, bwd=False),
+    # the 32k workload with grouped key/value heads: 8 KV heads for 32 query heads
+    "n32k_d128_gqa8": AttnWorkload("n32k_d128_gqa8", 1, 32, 32768, 128, 16, 512, 1024, True, 5, k_scale=2.0,
+                                   Hkv=8),
 }
 
 FFN_WORKLOADS = {
@@ -85,18 +93,19 @@ def _draw(shape, g, device, scale, dtype):
 def attention_inputs(w: AttnWorkload, device="cuda", with_dout: bool | None = None):
     """q, k, v (and dO when the workload has a backward) as [B,H,N,D] tensors."""
     shape = (w.B, w.H, w.N, w.D)
+    kv_shape = (w.B, w.kv_heads, w.N, w.D)
     g = _gen(device, w.seed)
     q = _draw(shape, g, device, 1.0, w.dtype)
-    k = _draw(shape, g, device, w.k_scale, w.dtype)
-    v = _draw(shape, g, device, 1.0, w.dtype)
+    k = _draw(kv_shape, g, device, w.k_scale, w.dtype)
+    v = _draw(kv_shape, g, device, 1.0, w.dtype)
     want_do = w.bwd if with_dout is None else with_dout
     do = _draw(shape, g, device, 1.0, w.dtype) if want_do else None
     return q, k, v, do
 
 
-def small_attention_inputs(B, H, N, D, seed, dtype=torch.bfloat16, device="cuda", k_scale=1.0):
+def small_attention_inputs(B, H, N, D, seed, dtype=torch.bfloat16, device="cuda", k_scale=1.0, Hkv=0):
     """q, k, v, dO for ad-hoc test shapes (same recipe as the workloads)."""
-    w = AttnWorkload("adhoc", B, H, N, D, 1, N, N, True, seed, dtype, k_scale)
+    w = AttnWorkload("adhoc", B, H, N, D, 1, N, N, True, seed, dtype, k_scale, Hkv=Hkv)
     return attention_inputs(w, device, with_dout=True)
 
 

@@ -103,6 +103,18 @@ RA_API int ringattn_fwd(const void* q, const void* k, const void* v, void* out, 
                  void* stream);
 
 /*
+ * ringattn_fwd_gqa -- ringattn_fwd with grouped key/value heads (GQA; MQA
+ * when Hkv == 1): query head h attends with key/value head h / (H / Hkv).
+ * q, out [B,H,N,D]; k, v [B,Hkv,N,D]; lse [B,H,N].  H % Hkv == 0.  Fewer
+ * key/value heads mean fewer bytes per ring step.  Other arguments and
+ * errors as ringattn_fwd; ringattn_fwd is this call with Hkv = H.
+ */
+RA_API int ringattn_fwd_gqa(const void* q, const void* k, const void* v, void* out, float* lse,
+                            int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t D, int dtype,
+                            int S, int q_chunk, int k_chunk, int causal, float scale,
+                            void* stream);
+
+/*
  * ringattn_fwd_step -- one ring step t with a fused merge into running
  * fp32 accumulators (the per-step building block of a multi-device ring).
  *
@@ -168,6 +180,19 @@ RA_API int ringattn_bwd(const void* q, const void* k, const void* v, const void*
                  int64_t B, int64_t H, int64_t N, int64_t D, int dtype,
                  int S, int q_chunk, int k_chunk, int causal, float scale,
                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * ringattn_bwd_gqa -- ringattn_bwd with grouped key/value heads: k, v, dk,
+ * dv are [B,Hkv,N,D]; dk and dv of a key/value head sum the contributions of
+ * all H / Hkv query heads that share it (accumulated on chip, one write).
+ * Other arguments as ringattn_bwd (same workspace size, computed with H).
+ */
+RA_API int ringattn_bwd_gqa(const void* q, const void* k, const void* v, const void* out,
+                            const float* lse, const void* dout,
+                            void* dq, void* dk, void* dv,
+                            int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t D, int dtype,
+                            int S, int q_chunk, int k_chunk, int causal, float scale,
+                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * ringattn_bwd_phase -- ringattn_bwd split into its three launches, for

@@ -30,6 +30,10 @@ Parity status per function (what pins it is in ``tests/test_oracle.py``):
                                  forms, brute force, scipy softmax/logsumexp)
 * ``attention_backward``         pinned (central finite differences, shift and
                                  homogeneity invariants)
+* ``attention_forward_gqa`` / ``attention_backward_gqa``
+                                 pinned (one key/value head per query head
+                                 reduces to the pinned plain functions; MQA
+                                 closed form; finite differences)
 * ``ring_blockwise_forward``     pinned (equals the full matrix for every S
                                  and chunk size, order invariant)
 * ``lse_merge``                  pinned (closed form of two-part softmax,
@@ -47,6 +51,8 @@ Parity status per function (what pins it is in ``tests/test_oracle.py``):
 from .attention import (  # noqa: F401
     attention_forward,
     attention_backward,
+    attention_forward_gqa,
+    attention_backward_gqa,
     ring_blockwise_forward,
     ring_blockwise_step,
     lse_merge,

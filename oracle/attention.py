@@ -113,6 +113,55 @@ def attention_backward(q, k, v, do, causal: bool, scale=None):
 
 
 # ---------------------------------------------------------------------------
+# Grouped key/value heads (GQA; MQA when there is one key/value head).
+# ---------------------------------------------------------------------------
+
+def attention_forward_gqa(q, k, v, causal: bool, scale=None):
+    """Attention where query head h reads key/value head h // (H // Hkv).
+
+    q: [B,H,N,d]; k, v: [B,Hkv,N,d] with H % Hkv == 0.  Each query head is
+    plain softmax attention against its group's keys and values.
+    Returns (o [B,H,N,d], lse [B,H,N]).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H = q.shape[:2]
+    G = H // k.shape[1]
+    o = np.empty(q.shape[:3] + (v.shape[3],))
+    lse = np.empty(q.shape[:3])
+    for b in range(B):
+        for h in range(H):
+            hk = h // G
+            ob, lb = attention_forward(q[b:b + 1, h:h + 1], k[b:b + 1, hk:hk + 1], v[b:b + 1, hk:hk + 1],
+                                       causal, scale)
+            o[b, h], lse[b, h] = ob[0, 0], lb[0, 0]
+    return o, lse
+
+
+def attention_backward_gqa(q, k, v, do, causal: bool, scale=None):
+    """Gradient of sum(do * o) for attention_forward_gqa.
+
+    dq of each query head as in the plain case; dk and dv of a key/value
+    head are the sums over the query heads that read it (chain rule through
+    the shared operand).  Returns (dq [B,H,N,d], dk, dv [B,Hkv,N,d]).
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, H = q.shape[:2]
+    G = H // k.shape[1]
+    dq = np.empty_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(H):
+            hk = h // G
+            gq, gk, gv = attention_backward(q[b:b + 1, h:h + 1], k[b:b + 1, hk:hk + 1], v[b:b + 1, hk:hk + 1],
+                                            do[b:b + 1, h:h + 1], causal, scale)
+            dq[b, h] = gq[0, 0]
+            dk[b, hk] += gk[0, 0]
+            dv[b, hk] += gv[0, 0]
+    return dq, dk, dv
+
+
+# ---------------------------------------------------------------------------
 # Sampled rows: the same definition restricted to chosen rows.
 # ---------------------------------------------------------------------------
 

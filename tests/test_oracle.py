@@ -404,3 +404,52 @@ def test_ffn_zero_cases_and_chunking():
 def test_silu_matches_expit():
     z = np.linspace(-40, 40, 1001)
     np.testing.assert_allclose(oracle.silu(z), z * scipy.special.expit(z), rtol=1e-14, atol=1e-300)
+
+
+# ---------------------------------------------------------------------------
+# Grouped key/value heads
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_with_one_query_head_per_kv_head_is_plain(causal):
+    B, H, N, d = 2, 3, 20, 8
+    q, k, v, do = (_rand((B, H, N, d), 50 + i) for i in range(4))
+    o1, l1 = oracle.attention_forward_gqa(q, k, v, causal)
+    o2, l2 = oracle.attention_forward(q, k, v, causal)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+    g1 = oracle.attention_backward_gqa(q, k, v, do, causal)
+    g2 = oracle.attention_backward(q, k, v, do, causal)
+    for a, b in zip(g1, g2):
+        np.testing.assert_allclose(a, b, atol=1e-14)
+
+
+def test_mqa_zero_queries_give_the_shared_mean():
+    B, H, N, d = 1, 4, 15, 6
+    q = np.zeros((B, H, N, d))
+    k, v = _rand((B, 1, N, d), 60), _rand((B, 1, N, d), 61)
+    o, lse = oracle.attention_forward_gqa(q, k, v, causal=False)
+    np.testing.assert_allclose(o, np.broadcast_to(v.mean(axis=2, keepdims=True), o.shape), atol=1e-13)
+    np.testing.assert_allclose(lse, np.log(N), atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_backward_finite_differences(causal):
+    """dk, dv of a shared key/value head collect every query head's pull."""
+    B, H, Hkv, N, d = 1, 4, 2, 6, 3
+    q, do = _rand((B, H, N, d), 62), _rand((B, H, N, d), 63)
+    k, v = _rand((B, Hkv, N, d), 64), _rand((B, Hkv, N, d), 65)
+    dq, dk, dv = oracle.attention_backward_gqa(q, k, v, do, causal)
+
+    def loss(k_, v_):
+        return float((oracle.attention_forward_gqa(q, k_, v_, causal)[0] * do).sum())
+
+    eps = 1e-6
+    for x, g, is_k in ((k, dk, True), (v, dv, False)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            num[idx] = ((loss(xp, v) - loss(xm, v)) if is_k else (loss(k, xp) - loss(k, xm))) / (2 * eps)
+        assert np.abs(num - g).max() / max(1.0, np.abs(g).max()) < 1e-6
