@@ -60,7 +60,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="n32k_d128",
                     choices=["n32k_d128", "n8k_d64_causal", "n8k_d64_full", "layer7b", "n1m_d128",
-                             "n32k_d128_gqa8"])
+                             "n32k_d128_gqa8", "decode_n128k"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -254,6 +254,54 @@ def run_reference(args):
 # the native arm
 # ---------------------------------------------------------------------------
 
+def run_decode(args, ra, dev, rank, world, dist):
+    """One decode step (new token per head against the sharded cache) per
+    bench step; HBM-bound, so the roofline is bandwidth."""
+    import torch
+    from dataclasses import replace
+    from exact_blockwise_long_b200.synthetic import DECODE_WORKLOADS, decode_inputs
+    w = DECODE_WORKLOADS[args.workload]
+    q, k, v = decode_inputs(replace(w, seed=w.seed + 1000 * rank), device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H), device=dev, dtype=torch.float32)
+    ws = torch.empty(ra.ringattn_decode_workspace_size(w.B, w.H, w.N, w.D, w.S, w.k_chunk), device=dev,
+                     dtype=torch.uint8)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        ra.ringattn_decode(q, k, v, out, lse, w.S, w.k_chunk, ws)
+    clocks = ClockSampler(dev.index)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        ra.ringattn_decode(q, k, v, out, lse, w.S, w.k_chunk, ws)
+    b.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if ra.ringattn_get_error() != 0:
+        raise RuntimeError("device status word set during the timed region")
+    ms = max_over_ranks(a.elapsed_time(b) / args.steps, dist if world > 1 else None, dev)
+    flops = 4.0 * w.B * w.H * w.N * w.D
+    cache_bytes = 2.0 * w.B * w.Hkv * w.N * w.D * 2
+    pk = peaks()
+    gbs = cache_bytes / (ms * 1e-3) / 1e9
+    return {"metric": METRIC, "value": whole_job_tflops(flops, world, ms), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{w.name}: decode, one new token per head against a cache of N={w.N} in "
+                                   f"S={w.S} shards, B={w.B}, H={w.H}, Hkv={w.Hkv}, d={w.D}, k_chunk={w.k_chunk}",
+                       "l2": "cache larger than L2 (no flush between steps)"},
+            "tokens_per_s": w.B * world / (ms * 1e-3),
+            "roofline": {"bound": "hbm", "kernel": "decode_partial_kernel+decode_merge_kernel",
+                         "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                         "traffic": None, "peak_kind": f"HBM copy ({pk['source']})"},
+            "gpu_launches": 2 * args.steps, "clocks": clk}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -281,6 +329,15 @@ def main():
     import exact_blockwise_long_b200 as ra
     from dataclasses import replace
     from exact_blockwise_long_b200.synthetic import attention_inputs, ffn_inputs
+
+    if args.workload.startswith("decode"):
+        line = run_decode(args, ra, dev, rank, world, dist)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return 0
 
     aw, fw = workload(args.workload)
     if args.heads:

@@ -44,6 +44,8 @@ SIGNATURES = {
                                 _F, _P, _SZ, _I, _P]),
     "ringattn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I,
                                   _F, _P]),
+    "ringattn_decode_workspace_size": (_SZ, [_I64, _I64, _I64, _I64, _I, _I]),
+    "ringattn_decode": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I, _I, _I, _F, _P, _SZ, _P]),
     "blockwise_ffn_workspace_size": (_SZ, [_I64, _I64, _I]),
     "blockwise_ffn": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I, _P, _SZ, _P]),
     "ringattn_get_error": (_I, [_P]),

@@ -164,6 +164,27 @@ def ringattn_bwd_noalloc(q, k, v, out, lse, dout, dq, dk, dv, S, q_chunk, k_chun
     return dq, dk, dv
 
 
+def ringattn_decode_workspace_size(B, H, N, D, S, k_chunk) -> int:
+    return int(lib().ringattn_decode_workspace_size(int(B), int(H), int(N), int(D), int(S), int(k_chunk)))
+
+
+def ringattn_decode(q, k, v, out, lse, S, k_chunk, workspace, scale=0.0, stream=None):
+    """out, lse <- one query token per (batch, head) against the [B, Hkv, N, D] cache."""
+    if q.dim() != 3 or k.dim() != 4:
+        raise ValueError("q, out are [B, H, D]; k, v are [B, Hkv, N, D]")
+    B, H, D = (int(x) for x in q.shape)
+    Hkv, N = int(k.shape[1]), int(k.shape[2])
+    if tuple(k.shape) != (B, Hkv, N, D) or v.shape != k.shape or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H):
+        raise ValueError("lse must be float32 [B, H]")
+    nbytes = workspace.numel() * workspace.element_size()
+    call("ringattn_decode", _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), _dev(lse, "lse"),
+         B, H, Hkv, N, D, _dtype(q), int(S), int(k_chunk), float(scale), _dev(workspace, "workspace"), nbytes,
+         _stream(stream))
+    return out, lse
+
+
 def blockwise_ffn_workspace_size(chunk, d_ff, dtype=torch.bfloat16) -> int:
     return int(lib().blockwise_ffn_workspace_size(int(chunk), int(d_ff), _DT[dtype]))
 

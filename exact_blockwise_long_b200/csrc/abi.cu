@@ -254,6 +254,34 @@ int ringattn_bwd(const void* q, const void* k, const void* v, const void* out, c
                             scale, workspace, workspace_bytes, 7, stream);
 }
 
+size_t ringattn_decode_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D, int S, int k_chunk) {
+  if (B <= 0 || H <= 0 || N <= 0 || D <= 0 || S <= 0 || k_chunk <= 0) return 0;
+  const size_t splits = (size_t)decode_splits(N, S, k_chunk);
+  const size_t lse_bytes = ((size_t)B * H * splits * 4 + 255) & ~(size_t)255;
+  return lse_bytes + (size_t)B * H * splits * D * 4;
+}
+
+int ringattn_decode(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t H,
+                    int64_t Hkv, int64_t N, int64_t D, int dtype, int S, int k_chunk, float scale, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  if (B < 0 || H < 0 || N < 0 || Hkv <= 0 || S <= 0 || k_chunk <= 0) return RA_ERR_ARG;
+  if (dtype != RA_BF16 && dtype != RA_F32) return RA_ERR_DTYPE;
+  if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
+  if (H % Hkv) return RA_ERR_ARG;
+  if (B == 0 || H == 0 || N == 0) return RA_OK;
+  if (!q || !k || !v || !out || !lse) return RA_ERR_ARG;
+  if (k_chunk % 128) return RA_ERR_SHAPE;
+  if (dtype != RA_BF16) return RA_ERR_UNSUPPORTED;
+  const int64_t G = H / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return RA_ERR_UNSUPPORTED;
+  if (B * Hkv * N > (int64_t)INT32_MAX) return RA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse)) return RA_ERR_ALIGN;
+  if (!workspace || workspace_bytes < ringattn_decode_workspace_size(B, H, N, D, S, k_chunk)) return RA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return RA_ERR_ALIGN;
+  return launch_decode(q, k, v, out, lse, B, H, Hkv, N, D, S, k_chunk, resolve_scale(scale, D), workspace,
+                       static_cast<cudaStream_t>(stream));
+}
+
 size_t blockwise_ffn_workspace_size(int64_t chunk, int64_t d_ff, int dtype) {
   if (chunk <= 0 || d_ff <= 0) return 0;
   const size_t el = (dtype == RA_F32) ? 4 : 2;

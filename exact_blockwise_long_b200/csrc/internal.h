@@ -48,6 +48,13 @@ int launch_bwd_tc(const AttnArgs& a, const void* out, const float* lse, const vo
 int launch_ffn_tc(const void* x, const void* w1, const void* w2, const void* w3, void* y, int64_t T,
                   int64_t d_model, int64_t d_ff, int64_t chunk, void* workspace, cudaStream_t stream);
 
+// Decode: splits of the key/value cache (S shards of ceil(N/S) keys, each
+// cut into pieces of at most k_chunk keys) and the launch.
+int decode_splits(int64_t N, int S, int k_chunk);
+int launch_decode(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t H,
+                  int64_t Hkv, int64_t N, int64_t D, int S, int k_chunk, float scale, void* workspace,
+                  cudaStream_t stream);
+
 int launch_selftest_timeout(int timeout_us, cudaStream_t stream);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point.

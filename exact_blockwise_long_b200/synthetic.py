@@ -77,6 +77,26 @@ FFN_WORKLOADS = {
 }
 
 
+@dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    B: int
+    H: int
+    Hkv: int
+    N: int
+    D: int
+    S: int
+    k_chunk: int
+    seed: int
+
+
+DECODE_WORKLOADS = {
+    # one decode step after a ring prefill of 131072 tokens (S=32) for a batch of 8,
+    # 32 query heads sharing 8 key/value heads of 128
+    "decode_n128k": DecodeWorkload("decode_n128k", 8, 32, 8, 131072, 128, 32, 1024, 6),
+}
+
+
 def _gen(device, seed: int) -> torch.Generator:
     g = torch.Generator(device=device)
     g.manual_seed(int(seed))
@@ -107,6 +127,15 @@ def small_attention_inputs(B, H, N, D, seed, dtype=torch.bfloat16, device="cuda"
     """q, k, v, dO for ad-hoc test shapes (same recipe as the workloads)."""
     w = AttnWorkload("adhoc", B, H, N, D, 1, N, N, True, seed, dtype, k_scale, Hkv=Hkv)
     return attention_inputs(w, device, with_dout=True)
+
+
+def decode_inputs(w: DecodeWorkload, device="cuda"):
+    """q [B,H,D] (one new token per head), k, v [B,Hkv,N,D] (the cache)."""
+    g = _gen(device, w.seed)
+    q = _draw((w.B, w.H, w.D), g, device, 1.0, torch.bfloat16)
+    k = _draw((w.B, w.Hkv, w.N, w.D), g, device, 1.0, torch.bfloat16)
+    v = _draw((w.B, w.Hkv, w.N, w.D), g, device, 1.0, torch.bfloat16)
+    return q, k, v
 
 
 def ffn_inputs(w: FFNWorkload, device="cuda", T: int | None = None):

@@ -239,6 +239,36 @@ RA_API int ringattn_bwd_noalloc(const void* q, const void* k, const void* v, con
                                 int S, int q_chunk, int k_chunk, int causal, float scale,
                                 void* stream);
 
+/* Bytes of device workspace ringattn_decode needs: an fp32 partial output
+ * and log-sum-exp per (batch, head, split). */
+RA_API size_t ringattn_decode_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D, int S, int k_chunk);
+
+/*
+ * ringattn_decode -- one new query token per (batch, head) against a key/
+ * value cache of N tokens held as S ring shards (inference after a ring
+ * prefill; paper abstract: training and inference).
+ *
+ *   out_bh = sum_j exp(s_j - lse_bh) v_j,  s_j = scale q_bh . k_j over all
+ *   N cached keys (the new token sees the whole cache), with key/value head
+ *   h / (H / Hkv) for query head h.
+ * Each shard of ceil(N/S) keys is cut into pieces of k_chunk keys; every
+ * piece yields an exact normalised partial and the partials are combined
+ * with the exact log-sum-exp merge (darcstar note, DarcStar commentary,
+ * paragraph one), so the result does not depend on S or k_chunk beyond
+ * fp32 rounding.
+ *
+ *   q, out   [B,H,D] bf16        k, v  [B,Hkv,N,D] bf16 (contiguous)
+ *   lse      [B,H] fp32 natural log
+ *   k_chunk  multiple of 128;  H / Hkv in {1,2,4,8,16};  D 64 or 128
+ *   workspace ringattn_decode_workspace_size() bytes, 16-byte aligned
+ * Errors: RA_ERR_ARG, RA_ERR_SHAPE, RA_ERR_DTYPE, RA_ERR_ALIGN,
+ * RA_ERR_UNSUPPORTED (fp32 or another group size), RA_ERR_WORKSPACE.
+ */
+RA_API int ringattn_decode(const void* q, const void* k, const void* v, void* out, float* lse,
+                           int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t D, int dtype,
+                           int S, int k_chunk, float scale,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of device workspace blockwise_ffn needs for one chunk's hidden
  * activation h [chunk, d_ff] in `dtype`. */
 RA_API size_t blockwise_ffn_workspace_size(int64_t chunk, int64_t d_ff, int dtype);

@@ -34,6 +34,8 @@ Parity status per function (what pins it is in ``tests/test_oracle.py``):
                                  pinned (one key/value head per query head
                                  reduces to the pinned plain functions; MQA
                                  closed form; finite differences)
+* ``attention_decode``           pinned (the last row of causal attention
+                                 over the same keys; q = 0 closed form)
 * ``ring_blockwise_forward``     pinned (equals the full matrix for every S
                                  and chunk size, order invariant)
 * ``lse_merge``                  pinned (closed form of two-part softmax,
@@ -53,6 +55,7 @@ from .attention import (  # noqa: F401
     attention_backward,
     attention_forward_gqa,
     attention_backward_gqa,
+    attention_decode,
     ring_blockwise_forward,
     ring_blockwise_step,
     lse_merge,

@@ -161,6 +161,30 @@ def attention_backward_gqa(q, k, v, do, causal: bool, scale=None):
     return dq, dk, dv
 
 
+def attention_decode(q, k, v, scale=None):
+    """One new query token per (batch, head) against a cache of N keys.
+
+    q: [B,H,d]; k, v: [B,Hkv,N,d]; query head h reads key/value head
+    h // (H // Hkv).  The new token sees every cached key.
+    Returns (o [B,H,d], lse [B,H]).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, d = q.shape
+    G = H // k.shape[1]
+    sc = _scale(d, scale)
+    o = np.empty((B, H, v.shape[3]))
+    lse = np.empty((B, H))
+    for b in range(B):
+        for h in range(H):
+            s = sc * (k[b, h // G] @ q[b, h])
+            m = s.max()
+            e = np.exp(s - m)
+            den = e.sum()
+            o[b, h] = (e / den) @ v[b, h // G]
+            lse[b, h] = m + np.log(den)
+    return o, lse
+
+
 # ---------------------------------------------------------------------------
 # Sampled rows: the same definition restricted to chosen rows.
 # ---------------------------------------------------------------------------

@@ -453,3 +453,23 @@ def test_gqa_backward_finite_differences(causal):
             xm[idx] -= eps
             num[idx] = ((loss(xp, v) - loss(xm, v)) if is_k else (loss(k, xp) - loss(k, xm))) / (2 * eps)
         assert np.abs(num - g).max() / max(1.0, np.abs(g).max()) < 1e-6
+
+
+def test_decode_is_the_last_causal_row():
+    """A decode query at position N-1 equals row N-1 of causal attention over
+    the same keys (reduction to the pinned full-matrix definition)."""
+    B, H, Hkv, N, d = 2, 4, 2, 19, 8
+    qfull = _rand((B, H, N, d), 70)
+    k, v = _rand((B, Hkv, N, d), 71), _rand((B, Hkv, N, d), 72)
+    o_full, l_full = oracle.attention_forward_gqa(qfull, k, v, causal=True)
+    o, lse = oracle.attention_decode(qfull[:, :, N - 1], k, v)
+    np.testing.assert_allclose(o, o_full[:, :, N - 1], atol=1e-13)
+    np.testing.assert_allclose(lse, l_full[:, :, N - 1], atol=1e-13)
+
+
+def test_decode_zero_query_gives_mean():
+    B, H, N, d = 1, 2, 30, 4
+    k, v = _rand((B, 1, N, d), 73), _rand((B, 1, N, d), 74)
+    o, lse = oracle.attention_decode(np.zeros((B, H, d)), k, v)
+    np.testing.assert_allclose(o, np.broadcast_to(v.mean(axis=2), o.shape), atol=1e-13)
+    np.testing.assert_allclose(lse, np.log(N), atol=1e-13)
