@@ -27,55 +27,67 @@
 namespace ra {
 namespace {
 
-constexpr int kKeys = 128;        // keys per tile
-constexpr int kThreads = 128;     // one thread per key (scores) / per column (P V)
+constexpr int kKeys = 64;         // keys per tile
+constexpr int kThreads = 256;
 constexpr int kStages = 3;
-constexpr int kMaxG = 16;         // query heads per key/value head handled by one CTA
+constexpr int kQuarters = kThreads / kKeys;  // partial dots per key in the score phase
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int D>
+template <int D, int G>
 struct DLayout {
   static constexpr int kTile = kKeys * D * 2;
   static constexpr int kSlab = kKeys * 128;
   static constexpr int kK = 0;
   static constexpr int kV = kK + kStages * kTile;
-  static constexpr int kQ = kV + kStages * kTile;       // fp32 [kMaxG][D]
-  static constexpr int kP = kQ + kMaxG * D * 4;          // fp32 [kMaxG][kKeys]
-  static constexpr int kRed = kP + kMaxG * kKeys * 4;    // fp32 [4 warps][kMaxG]
-  static constexpr int kBar = kRed + 4 * kMaxG * 4;
-  static constexpr int kBytes = kBar + 2 * kStages * 8 + 8;
+  static constexpr int kQ = kV + kStages * kTile;            // fp32 [G][D]
+  static constexpr int kS = kQ + G * D * 4;                  // fp32 [quarters][G][kKeys] partial scores
+  static constexpr int kP = kS + kQuarters * G * kKeys * 4;  // fp32 [G][kKeys]
+  static constexpr int kRed = kP + G * kKeys * 4;            // fp32 [2][2 warps][G]
+  static constexpr int kBar = kRed + 4 * G * 4;
+  static constexpr int kBytes = kBar + kStages * 8 + 8;
   static constexpr int kAlloc = kBytes + 1024;
 };
+static_assert(DLayout<128, 16>::kAlloc <= 232448, "decode tile set exceeds shared memory");
 
 struct DParams {
   const __nv_bfloat16* q;  // [B*H, D]
   float* part_o;           // [B*H, splits, D]
   float* part_lse;         // [B*H, splits]
   int H, G, N, splits, chunk;
-  int L, pieces;  // shard length, pieces per shard
+  int L, pieces;           // shard length, pieces per shard
   float scale_log2;
   DevStatus st;
 };
 
-// swizzled element (row, col) of a [rows][D] bf16 tile loaded as 64-column
+// swizzled element (row, col) of a [kKeys][D] bf16 tile loaded as 64-column
 // slabs with the 128-byte swizzle
-template <int D>
 __device__ __forceinline__ const __nv_bfloat16* tile_at(const uint8_t* tile, int row, int col) {
   const int slab = col >> 6, c = col & 63;
   const int chunk = (c >> 3) ^ (row & 7);
   return reinterpret_cast<const __nv_bfloat16*>(tile + slab * (kKeys * 128) + row * 128 + chunk * 16) + (c & 7);
 }
 
+// Threads: scores -- thread t takes key t % 64 over head dimensions
+// [D/4 (t / 64), +D/4) for every query head of the group (four partial dots
+// per key, summed through shared memory); softmax -- threads 0..63, one key
+// each, block max and block sum per query head; P V -- thread t takes the
+// column pair 2 (t % (D/2)) over its share of the tile's keys, with packed
+// f32x2 multiply-adds; the key shares are summed once, at the end.
 template <int D, int G>
 __global__ void __launch_bounds__(kThreads) decode_partial_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                   const __grid_constant__ CUtensorMap tmV,
                                                                   const DParams p) {
-  using LY = DLayout<D>;
+  using LY = DLayout<D, G>;
+  constexpr int kDimQ = D / kQuarters;         // head dimensions per partial dot
+  constexpr int kPairs = D / 2;                // column pairs
+  constexpr int kShares = kThreads / kPairs;   // key shares in P V
+  constexpr int kPerShare = kKeys / kShares;
   extern __shared__ uint8_t smem_d[];
   uint8_t* smem = smem_d + ((1024 - (smem_u32(smem_d) & 1023)) & 1023);
   uint8_t* sK = smem + LY::kK;
   uint8_t* sV = smem + LY::kV;
   float* sQ = reinterpret_cast<float*>(smem + LY::kQ);
+  float* sS = reinterpret_cast<float*>(smem + LY::kS);
   float* sP = reinterpret_cast<float*>(smem + LY::kP);
   float* sRed = reinterpret_cast<float*>(smem + LY::kRed);
   uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + LY::kBar);
@@ -117,88 +129,117 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(const __grid_c
     for (int t = 0; t < min(kStages - 1, ntiles); ++t) load(t);
   }
 
-  float m[G], l[G], acc[G];  // running max (log2 units), denominator, O[g][tid]
+  const int skey = tid % kKeys, quarter = tid / kKeys;    // score role
+  const int pair = tid % kPairs, share = tid / kPairs;    // P V role
+  float m[G], l[G];                                       // running max (log2 units) and denominator
+  float2 acc[G];                                          // O[g][2 pair, 2 pair + 1] over this key share
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     m[g] = -INFINITY;
     l[g] = 0.f;
-    acc[g] = 0.f;
+    acc[g] = make_float2(0.f, 0.f);
   }
   bool ok = true;
   for (int t = 0; t < ntiles; ++t) {
     const int s = t % kStages;
-    // the stage refilled next was last read in tile t - 1; every thread has
-    // passed the barrier at the end of that tile
+    // the stage refilled here was last read in tile t - 1, which every
+    // thread has left (barrier at the end of each tile)
     if (tid == 0 && t + kStages - 1 < ntiles) load(t + kStages - 1);
     ok = __syncthreads_and(mbar_wait(&bar_full[s], (t / kStages) & 1, p.st, abort_flag));
     if (!ok) break;
     const uint8_t* tK = sK + s * LY::kTile;
     const uint8_t* tV = sV + s * LY::kTile;
-    const int key = k0 + t * kKeys + tid;
-    // scores: one key per thread, every query head of the group
-    float sc[G];
+    {
+      float2 sc[G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) sc[g] = 0.f;
-#pragma unroll 4
-    for (int c = 0; c < D; c += 8) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(tile_at<D>(tK, tid, c));
-      const __nv_bfloat162* kv = reinterpret_cast<const __nv_bfloat162*>(&raw);
+      for (int g = 0; g < G; ++g) sc[g] = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 kf = __bfloat1622float2(kv[e]);
+      for (int c = quarter * kDimQ; c < quarter * kDimQ + kDimQ; c += 8) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(tile_at(tK, skey, c));
+        const __nv_bfloat162* kv = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
-        for (int g = 0; g < G; ++g)
-          sc[g] = fmaf(kf.x, sQ[g * D + c + 2 * e], fmaf(kf.y, sQ[g * D + c + 2 * e + 1], sc[g]));
+        for (int e = 0; e < 4; ++e) {
+          const float2 kf = __bfloat1622float2(kv[e]);
+#pragma unroll
+          for (int g = 0; g < G; ++g)
+            sc[g] = fma2(kf, *reinterpret_cast<const float2*>(&sQ[g * D + c + 2 * e]), sc[g]);
+        }
       }
+#pragma unroll
+      for (int g = 0; g < G; ++g) sS[(quarter * G + g) * kKeys + skey] = sc[g].x + sc[g].y;
     }
-    // tile max per query head: warp shuffle, then across the four warps
+    __syncthreads();
+    // softmax pieces: one key per thread of the first two warps
+    float sv[G];
+    if (tid < kKeys) {
+      const bool live = (k0 + t * kKeys + tid) < k1;
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float x = (key < k1) ? sc[g] * p.scale_log2 : -INFINITY;
-      sc[g] = x;
+      for (int g = 0; g < G; ++g) {
+        float x = (sS[g * kKeys + tid] + sS[(G + g) * kKeys + tid]) +
+                  (sS[(2 * G + g) * kKeys + tid] + sS[(3 * G + g) * kKeys + tid]);
+        x = live ? x * p.scale_log2 : -INFINITY;
+        sv[g] = x;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-      if (lane == 0) sRed[warp * kMaxG + g] = x;
+        for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+        if (lane == 0) sRed[warp * G + g] = x;
+      }
     }
     __syncthreads();
     float alpha[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      const float mt = fmaxf(fmaxf(sRed[g], sRed[kMaxG + g]), fmaxf(sRed[2 * kMaxG + g], sRed[3 * kMaxG + g]));
-      const float mn = fmaxf(m[g], mt);
+      const float mn = fmaxf(m[g], fmaxf(sRed[g], sRed[G + g]));
       alpha[g] = (m[g] == -INFINITY) ? 0.f : ex2_approx(m[g] - mn);
       m[g] = mn;
-      sP[g * kKeys + tid] = ex2_approx(sc[g] - mn);  // 0 for keys past the end
     }
-    __syncthreads();
-    // P V: one output column per thread; the denominator from the same P
+    if (tid < kKeys) {
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      acc[g] *= alpha[g];
-      l[g] *= alpha[g];
-    }
-    const int col = tid;
-    if (col < D) {
-#pragma unroll 4
-      for (int k = 0; k < kKeys; ++k) {
-        const float vv = __bfloat162float(*tile_at<D>(tV, k, col));
+      for (int g = 0; g < G; ++g) {
+        const float pv = ex2_approx(sv[g] - m[g]);  // 0 for keys past the end
+        sP[g * kKeys + tid] = pv;
+        float x = pv;
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float pk = sP[g * kKeys + k];
-          acc[g] = fmaf(pk, vv, acc[g]);
-          l[g] += pk;
-        }
+        for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        if (lane == 0) sRed[(2 + warp) * G + g] = x;
       }
     }
-    __syncthreads();  // this tile's stage and P are free
-  }
-  if (!ok || tid >= D) return;
+    __syncthreads();
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
+    for (int g = 0; g < G; ++g) {
+      l[g] = l[g] * alpha[g] + (sRed[2 * G + g] + sRed[3 * G + g]);
+      acc[g].x *= alpha[g];
+      acc[g].y *= alpha[g];
+    }
+    // P V over this thread's key share for its column pair
+#pragma unroll
+    for (int kk = 0; kk < kPerShare; ++kk) {
+      const int k = share * kPerShare + kk;
+      const float2 vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(tile_at(tV, k, 2 * pair)));
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float pk = sP[g * kKeys + k];
+        acc[g] = fma2(vf, make_float2(pk, pk), acc[g]);
+      }
+    }
+    __syncthreads();  // this tile's stage, partial scores and P are free
+  }
+  if (!ok) return;
+  // sum the key shares (in the key/value stages, all consumed by now) and
+  // write the partials
+  float* sO = reinterpret_cast<float*>(sK);  // [kShares][G][D]
+  static_assert(kShares * G * D * 4 <= 2 * kStages * LY::kTile, "key-share sums exceed the stages");
+#pragma unroll
+  for (int g = 0; g < G; ++g) *reinterpret_cast<float2*>(&sO[(share * G + g) * D + 2 * pair]) = acc[g];
+  __syncthreads();
+  for (int i = tid; i < G * D; i += kThreads) {
+    const int g = i / D, c = i % D;
+    float o = 0.f;
+#pragma unroll
+    for (int sh = 0; sh < kShares; ++sh) o += sO[(sh * G + g) * D + c];
     const size_t prow = (size_t)(qbh0 + g) * p.splits + split;
     const bool empty = (l[g] == 0.f);
-    p.part_o[prow * D + tid] = empty ? 0.f : acc[g] / l[g];
-    if (tid == 0) p.part_lse[prow] = empty ? -INFINITY : (m[g] + __log2f(l[g])) * 0.6931471805599453f;
+    p.part_o[prow * D + c] = empty ? 0.f : o / l[g];
+    if (c == 0) p.part_lse[prow] = empty ? -INFINITY : (m[g] + __log2f(l[g])) * 0.6931471805599453f;
   }
 }
 
@@ -234,8 +275,8 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const float* __restri
 template <int D, int G>
 int launch_partial(const CUtensorMap& tk, const CUtensorMap& tv, const DParams& p, int grid, cudaStream_t stream) {
   auto kern = decode_partial_kernel<D, G>;
-  if (set_smem_attr((const void*)kern, DLayout<D>::kAlloc) != RA_OK) return RA_ERR_CUDA;
-  kern<<<grid, kThreads, DLayout<D>::kAlloc, stream>>>(tk, tv, p);
+  if (set_smem_attr((const void*)kern, DLayout<D, G>::kAlloc) != RA_OK) return RA_ERR_CUDA;
+  kern<<<grid, kThreads, DLayout<D, G>::kAlloc, stream>>>(tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
