@@ -11,9 +11,9 @@
 //
 // Two launches:
 //   partial  one CTA per (batch, key/value head, split of C keys): the
-//            key/value tiles stream through shared memory by TMA (three
-//            stages, 128-byte swizzle); scores use one thread per key, P V
-//            one thread per output column; all G query heads that share the
+//            key/value tiles (64 keys) stream through shared memory by TMA
+//            (two stages, 128-byte swizzle; shared memory sized to the group
+//            so three CTAs share an SM); all G query heads that share the
 //            key/value head are served from the same tile (the cache is read
 //            once per key/value head).  Writes (o_s, lse_s) in fp32.
 //   merge    one warp per (batch, head): exact merge over the splits,
@@ -29,7 +29,7 @@ namespace {
 
 constexpr int kKeys = 64;         // keys per tile
 constexpr int kThreads = 256;
-constexpr int kStages = 3;
+constexpr int kStages = 2;
 constexpr int kQuarters = kThreads / kKeys;  // partial dots per key in the score phase
 constexpr float kLog2e = 1.4426950408889634f;
 
