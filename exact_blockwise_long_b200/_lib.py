@@ -48,6 +48,8 @@ SIGNATURES = {
     "ringattn_decode": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I, _I, _I, _F, _P, _SZ, _P]),
     "blockwise_ffn_workspace_size": (_SZ, [_I64, _I64, _I]),
     "blockwise_ffn": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I, _P, _SZ, _P]),
+    "blockwise_ffn_bwd_workspace_size": (_SZ, [_I64, _I64, _I]),
+    "blockwise_ffn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I, _P, _SZ, _P]),
     "ringattn_get_error": (_I, [_P]),
     "ringattn_selftest_timeout": (_I, [_I, _P]),
 }

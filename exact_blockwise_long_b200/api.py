@@ -203,6 +203,26 @@ def blockwise_ffn(x, w1, w2, w3, y, chunk, workspace, stream=None):
     return y
 
 
+def blockwise_ffn_bwd_workspace_size(chunk, d_ff, dtype=torch.bfloat16) -> int:
+    return int(lib().blockwise_ffn_bwd_workspace_size(int(chunk), int(d_ff), _DT[dtype]))
+
+
+def blockwise_ffn_bwd(x, w1, w2, w3, dy, dx, dw1, dw2, dw3, chunk, workspace, stream=None):
+    """dx (bf16), dw1, dw2, dw3 (fp32) <- gradient of sum(dy * y) through blockwise_ffn."""
+    T, d_model = (int(s) for s in x.shape)
+    d_ff = int(w1.shape[0])
+    if dy.shape != x.shape or dx.shape != x.shape:
+        raise ValueError("x, dy, dx are [T, d_model]")
+    for t, shp in ((dw1, (d_ff, d_model)), (dw3, (d_ff, d_model)), (dw2, (d_model, d_ff))):
+        if t.dtype != torch.float32 or tuple(t.shape) != shp:
+            raise ValueError("weight gradients are float32 in the weights' shapes")
+    nbytes = workspace.numel() * workspace.element_size()
+    call("blockwise_ffn_bwd", _dev(x, "x"), _dev(w1, "w1"), _dev(w2, "w2"), _dev(w3, "w3"), _dev(dy, "dy"),
+         _dev(dx, "dx"), _dev(dw1, "dw1"), _dev(dw2, "dw2"), _dev(dw3, "dw3"), T, d_model, d_ff, int(chunk),
+         _dtype(x), _dev(workspace, "workspace"), nbytes, _stream(stream))
+    return dx, dw1, dw2, dw3
+
+
 def ringattn_get_error(stream=None) -> int:
     """Synchronise the stream; return and clear the device status word."""
     return int(lib().ringattn_get_error(_stream(stream)))

@@ -303,6 +303,36 @@ int blockwise_ffn(const void* x, const void* w1, const void* w2, const void* w3,
   return launch_ffn_tc(x, w1, w2, w3, y, T, d_model, d_ff, chunk, workspace, static_cast<cudaStream_t>(stream));
 }
 
+size_t blockwise_ffn_bwd_workspace_size(int64_t chunk, int64_t d_ff, int dtype) {
+  if (chunk <= 0 || d_ff <= 0 || dtype != RA_BF16) return 0;
+  return ffn_bwd_workspace_bytes(chunk, d_ff);
+}
+
+int blockwise_ffn_bwd(const void* x, const void* w1, const void* w2, const void* w3, const void* dy, void* dx,
+                      float* dw1, float* dw2, float* dw3, int64_t T, int64_t d_model, int64_t d_ff, int64_t chunk,
+                      int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  if (T < 0 || d_model <= 0 || d_ff <= 0 || chunk <= 0) return RA_ERR_ARG;
+  if (dtype != RA_BF16 && dtype != RA_F32) return RA_ERR_DTYPE;
+  if (dtype != RA_BF16) return RA_ERR_UNSUPPORTED;
+  if (!w1 || !w2 || !w3 || !dw1 || !dw2 || !dw3) return RA_ERR_ARG;
+  if (T > 0 && (!x || !dy || !dx)) return RA_ERR_ARG;  // token buffers may be null when there are no tokens
+  if (T % chunk || chunk % 128 || d_model % 128 || d_ff % 128) return RA_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(w1) || !aligned16(w2) || !aligned16(w3) || !aligned16(dy) || !aligned16(dx) ||
+      !aligned16(dw1) || !aligned16(dw2) || !aligned16(dw3))
+    return RA_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T == 0) {  // no tokens: the weight gradients are zero
+    const size_t wbytes = (size_t)d_ff * d_model * sizeof(float);
+    if (cudaMemsetAsync(dw1, 0, wbytes, st) != cudaSuccess || cudaMemsetAsync(dw2, 0, wbytes, st) != cudaSuccess ||
+        cudaMemsetAsync(dw3, 0, wbytes, st) != cudaSuccess)
+      return RA_ERR_CUDA;
+    return RA_OK;
+  }
+  if (!workspace || workspace_bytes < blockwise_ffn_bwd_workspace_size(chunk, d_ff, dtype)) return RA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return RA_ERR_ALIGN;
+  return launch_ffn_bwd_tc(x, w1, w2, w3, dy, dx, dw1, dw2, dw3, T, d_model, d_ff, chunk, workspace, st);
+}
+
 int ringattn_get_error(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return RA_ERR_CUDA;

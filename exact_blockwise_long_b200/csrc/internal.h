@@ -55,6 +55,12 @@ int launch_decode(const void* q, const void* k, const void* v, void* out, float*
                   int64_t Hkv, int64_t N, int64_t D, int S, int k_chunk, float scale, void* workspace,
                   cudaStream_t stream);
 
+// Blockwise SwiGLU FFN backward: workspace (dg, du, h of one chunk) and launch.
+size_t ffn_bwd_workspace_bytes(int64_t chunk, int64_t d_ff);
+int launch_ffn_bwd_tc(const void* x, const void* w1, const void* w2, const void* w3, const void* dy, void* dx,
+                      float* dw1, float* dw2, float* dw3, int64_t T, int64_t d_model, int64_t d_ff, int64_t chunk,
+                      void* workspace, cudaStream_t stream);
+
 int launch_selftest_timeout(int timeout_us, cudaStream_t stream);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point.

@@ -7,7 +7,7 @@ upcasts those bf16 values exactly to float64).
 
 Recipe (per workload): a torch.Generator on the target device seeded with
 the workload seed draws float32 standard normals in the order q, k, v, dO
-(then x, w1, w3, w2 for the feed-forward), each scaled as the workload says
+(then x, w1, w3, w2 and, for its backward, dy for the feed-forward), each scaled as the workload says
 (k by 2 for the sharpened 32k workload, weights by 0.02), then rounded to the
 compute dtype with round-to-nearest-even.
 """
@@ -138,14 +138,17 @@ def decode_inputs(w: DecodeWorkload, device="cuda"):
     return q, k, v
 
 
-def ffn_inputs(w: FFNWorkload, device="cuda", T: int | None = None):
-    """x [T, d_model], w1 [d_ff, d_model], w3 [d_ff, d_model], w2 [d_model, d_ff]."""
+def ffn_inputs(w: FFNWorkload, device="cuda", T: int | None = None, with_dy: bool = False):
+    """x [T, d_model], w1 [d_ff, d_model], w3 [d_ff, d_model], w2 [d_model, d_ff]
+    (and, with with_dy, the output gradient dy [T, d_model], drawn last)."""
     T = w.T if T is None else T
     g = _gen(device, w.seed)
     x = _draw((T, w.d_model), g, device, 1.0, w.dtype)
     w1 = _draw((w.d_ff, w.d_model), g, device, w.w_std, w.dtype)
     w3 = _draw((w.d_ff, w.d_model), g, device, w.w_std, w.dtype)
     w2 = _draw((w.d_model, w.d_ff), g, device, w.w_std, w.dtype)
+    if with_dy:
+        return x, w1, w2, w3, _draw((T, w.d_model), g, device, 1.0, w.dtype)
     return x, w1, w2, w3
 
 

@@ -290,6 +290,35 @@ RA_API int blockwise_ffn(const void* x, const void* w1, const void* w2, const vo
                   int64_t T, int64_t d_model, int64_t d_ff, int64_t chunk, int dtype,
                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* Bytes of device workspace blockwise_ffn_bwd needs: one chunk's dg, du and
+ * h, each [chunk, d_ff] bf16. */
+RA_API size_t blockwise_ffn_bwd_workspace_size(int64_t chunk, int64_t d_ff, int dtype);
+
+/*
+ * blockwise_ffn_bwd -- gradient of sum(dy * y) for blockwise_ffn, chunk by
+ * chunk (paper abstract: blockwise feed-forward, used for training).  With
+ * g = x w1^T, u = x w3^T, s = 1/(1+e^-g), h = g s u:
+ *   dh = dy w2;  du = dh * g s;  dg = dh * u * s (1 + g (1 - s))
+ *   dx = dg w1 + du w3;  dw1 = sum dg^T x;  dw3 = sum du^T x;
+ *   dw2 = sum dy^T h   (sums over all T tokens)
+ * Each chunk recomputes its g and u; only one chunk's dg, du, h exist at a
+ * time (in workspace).
+ *
+ *   x, dy [T, d_model] bf16;  w1, w3 [d_ff, d_model];  w2 [d_model, d_ff]
+ *   dx  [T, d_model] bf16 written
+ *   dw1, dw3 [d_ff, d_model] fp32 and dw2 [d_model, d_ff] fp32, written
+ *   (summed over the chunks in fp32)
+ *   T % chunk == 0; chunk, d_model, d_ff multiples of 128.  T == 0 zeroes
+ *   the weight gradients (x, dy, dx may then be null).
+ * Only RA_BF16 is implemented.  Errors: RA_ERR_ARG (null pointer, negative
+ * size), RA_ERR_SHAPE, RA_ERR_ALIGN (any pointer not 16-byte aligned),
+ * RA_ERR_WORKSPACE, RA_ERR_UNSUPPORTED (RA_F32), RA_ERR_CUDA.
+ */
+RA_API int blockwise_ffn_bwd(const void* x, const void* w1, const void* w2, const void* w3, const void* dy,
+                             void* dx, float* dw1, float* dw2, float* dw3,
+                             int64_t T, int64_t d_model, int64_t d_ff, int64_t chunk, int dtype,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
 /*
  * ringattn_get_error -- synchronise `stream`, return the device status word
  * of the current device (RA_OK or RA_ERR_TIMEOUT) and clear it.  Also

@@ -48,6 +48,12 @@ Parity status per function (what pins it is in ``tests/test_oracle.py``):
 * ``swiglu_ffn`` / ``blockwise_ffn``
                                  pinned (zero inputs, chunk invariance,
                                  explicit loop, scipy expit)
+* ``swiglu_ffn_backward`` / ``blockwise_ffn_backward``
+                                 pinned (central finite differences of
+                                 sum(dy * y), zero-weight closed forms, chunk
+                                 invariance, linearity in dy)
+* ``swiglu_ffn_backward_terms``  error-bound helper (sums of |term|), pinned
+                                 by dominating |gradient| element-wise
 """
 
 from .attention import (  # noqa: F401
@@ -66,4 +72,12 @@ from .attention import (  # noqa: F401
     ring_visit_order,
     ring_visit_order_bwd,
 )
-from .ffn import swiglu_ffn, blockwise_ffn, silu  # noqa: F401
+from .ffn import (  # noqa: F401
+    swiglu_ffn,
+    blockwise_ffn,
+    silu,
+    sigmoid,
+    swiglu_ffn_backward,
+    blockwise_ffn_backward,
+    swiglu_ffn_backward_terms,
+)

@@ -406,6 +406,88 @@ def test_silu_matches_expit():
     np.testing.assert_allclose(oracle.silu(z), z * scipy.special.expit(z), rtol=1e-14, atol=1e-300)
 
 
+def _ffn_case(T=5, dm=4, dff=6, seed=60, wscale=0.7):
+    x = _rand((T, dm), seed)
+    w1, w3 = _rand((dff, dm), seed + 1, wscale), _rand((dff, dm), seed + 2, wscale)
+    w2 = _rand((dm, dff), seed + 3, wscale)
+    dy = _rand((T, dm), seed + 4)
+    return x, w1, w2, w3, dy
+
+
+def test_ffn_backward_finite_differences():
+    """Every entry of dx, dw1, dw2, dw3 against a central difference of
+    sum(dy * y), y from the pinned forward."""
+    x, w1, w2, w3, dy = _ffn_case()
+    grads = oracle.swiglu_ffn_backward(x, w1, w2, w3, dy)
+    args = [x, w1, w2, w3]
+    eps = 1e-6
+    for which, gi in zip((0, 1, 2, 3), grads):
+        fd = np.empty_like(args[which])
+        for idx in np.ndindex(*args[which].shape):
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[which][idx] += eps
+            minus[which][idx] -= eps
+            fd[idx] = (np.sum(dy * oracle.swiglu_ffn(*plus)) - np.sum(dy * oracle.swiglu_ffn(*minus))) / (2 * eps)
+        np.testing.assert_allclose(gi, fd, rtol=1e-7, atol=1e-8)
+
+
+def test_ffn_backward_zero_weight_closed_forms():
+    x, w1, w2, w3, dy = _ffn_case(seed=70)
+    # no up projection: h = 0, so only dw3 can be non-zero
+    dx, dw1, dw2, dw3 = oracle.swiglu_ffn_backward(x, w1, w2, np.zeros_like(w3), dy)
+    assert np.all(dx == 0) and np.all(dw1 == 0) and np.all(dw2 == 0) and np.abs(dw3).max() > 0.1
+    # no down projection: dh = 0, so only dw2 can be non-zero
+    dx, dw1, dw2, dw3 = oracle.swiglu_ffn_backward(x, w1, np.zeros_like(w2), w3, dy)
+    assert np.all(dx == 0) and np.all(dw1 == 0) and np.all(dw3 == 0) and np.abs(dw2).max() > 0.1
+    # zero input: g = u = h = 0 and every gradient vanishes (silu(0) = 0)
+    for gr in oracle.swiglu_ffn_backward(np.zeros_like(x), w1, w2, w3, dy):
+        assert np.all(gr == 0)
+    # one token, one hidden unit, one feature: scalar calculus by hand
+    # y = silu(a x) (b x) c; dy/dx = c b (silu(a x) + a x silu'(a x)) with
+    # silu'(z) = expit(z) (1 + z (1 - expit(z)))
+    a, b, c, xv = 0.8, -1.3, 0.6, 0.9
+    z = a * xv
+    sp = scipy.special.expit(z) * (1 + z * (1 - scipy.special.expit(z)))
+    dx, dw1, dw2, dw3 = oracle.swiglu_ffn_backward(np.array([[xv]]), np.array([[a]]), np.array([[c]]),
+                                                   np.array([[b]]), np.array([[1.0]]))
+    silu_z = z * scipy.special.expit(z)
+    assert math.isclose(dx[0, 0], c * b * (silu_z + a * xv * sp), rel_tol=1e-13)
+    assert math.isclose(dw1[0, 0], c * b * xv * xv * sp, rel_tol=1e-13)
+    assert math.isclose(dw2[0, 0], silu_z * b * xv, rel_tol=1e-13)
+    assert math.isclose(dw3[0, 0], c * silu_z * xv, rel_tol=1e-13)
+
+
+def test_ffn_backward_chunking_and_linearity():
+    x, w1, w2, w3, dy = _ffn_case(T=24, dm=5, dff=7, seed=80)
+    ref = oracle.swiglu_ffn_backward(x, w1, w2, w3, dy)
+    for c in (1, 2, 3, 4, 6, 8, 12, 24):
+        for a, b in zip(oracle.blockwise_ffn_backward(x, w1, w2, w3, dy, c), ref):
+            np.testing.assert_allclose(a, b, atol=1e-12)
+    dy2 = _rand(dy.shape, 81)
+    g2 = oracle.swiglu_ffn_backward(x, w1, w2, w3, dy2)
+    g12 = oracle.swiglu_ffn_backward(x, w1, w2, w3, 2.0 * dy - 3.0 * dy2)
+    for a, b, c in zip(g12, ref, g2):
+        np.testing.assert_allclose(a, 2.0 * b - 3.0 * c, atol=1e-12)
+    # hidden units are independent: a subset of them has exactly the weight
+    # gradients of those units in the full layer
+    units = np.array([0, 3, 6])
+    _, s1, s2, s3 = oracle.swiglu_ffn_backward(x, w1[units], w2[:, units], w3[units], dy)
+    np.testing.assert_allclose(s1, ref[1][units], atol=1e-12)
+    np.testing.assert_allclose(s2, ref[2][:, units], atol=1e-12)
+    np.testing.assert_allclose(s3, ref[3][units], atol=1e-12)
+
+
+def test_ffn_backward_terms_bound_gradients():
+    x, w1, w2, w3, dy = _ffn_case(T=9, dm=5, dff=7, seed=90)
+    for gr, tm in zip(oracle.swiglu_ffn_backward(x, w1, w2, w3, dy), oracle.swiglu_ffn_backward_terms(x, w1, w2, w3, dy)):
+        assert np.all(np.abs(gr) <= tm + 1e-12) and np.all(tm > 0)
+    # all inputs positive: every term is positive and the bound is attained
+    pos = [np.abs(a) for a in (x, w1, w2, w3, dy)]
+    for gr, tm in zip(oracle.swiglu_ffn_backward(*pos), oracle.swiglu_ffn_backward_terms(*pos)):
+        np.testing.assert_allclose(gr, tm, rtol=1e-13)
+
+
 # ---------------------------------------------------------------------------
 # Grouped key/value heads
 # ---------------------------------------------------------------------------
