@@ -90,7 +90,9 @@ def attn_step_flops(w):
 
 
 def ffn_flops(f):
-    return 6.0 * f.T * f.d_model * f.d_ff
+    """Forward (three GEMMs) plus backward (dh, dx from dg and du, dw1, dw3,
+    dw2: six GEMMs; the backward's recomputation of g and u is not counted)."""
+    return 18.0 * f.T * f.d_model * f.d_ff
 
 
 def max_over_ranks(x: float, dist=None, device=None) -> float:
@@ -113,7 +115,7 @@ def describe(aw, fw):
                      + (f"Hkv={aw.kv_heads}, " if aw.kv_heads != aw.H else "")
                      + f"N={aw.N}, d={aw.D}, S={aw.S}, q_chunk={aw.q_chunk}, k_chunk={aw.k_chunk}, "
                      f"{'causal' if aw.causal else 'non-causal'}"
-                     + (f"; blockwise SwiGLU FFN {fw.d_model}->{fw.d_ff}->{fw.d_model}, chunk {fw.chunk}"
+                     + (f"; blockwise SwiGLU FFN {fw.d_model}->{fw.d_ff}->{fw.d_model} fwd+bwd, chunk {fw.chunk}"
                         if fw else ""),
          "B": aw.B, "H": aw.H, "seq_len": aw.N, "head_dim": aw.D, "shards": aw.S,
          "q_chunk": aw.q_chunk, "k_chunk": aw.k_chunk, "causal": aw.causal,
@@ -216,6 +218,17 @@ def oracle_sample(aw, fw, n_tokens=4096, min_seconds=0.0, max_heads=32):
     flops = attn_step_flops(small) * heads
     desc = (f"fp64 oracle (numpy) {'forward+backward' if aw.bwd else 'forward'} of {heads} head(s) cut to "
             f"their first {n} tokens, same workload recipe; causal FLOPs counted once")
+    if fw is not None:
+        from exact_blockwise_long_b200.synthetic import ffn_inputs
+        tf = 256
+        x, w1, w2, w3, dy = (to_f64(t) for t in ffn_inputs(replace(fw, chunk=tf), device="cpu", T=tf,
+                                                          with_dy=True))
+        t0 = time.perf_counter()
+        oracle.blockwise_ffn(x, w1, w2, w3, tf)
+        oracle.blockwise_ffn_backward(x, w1, w2, w3, dy, tf)
+        dt += time.perf_counter() - t0
+        flops += ffn_flops(replace(fw, T=tf))
+        desc += f"; plus the SwiGLU FFN forward+backward of {tf} tokens at the layer's full width"
     try:
         from threadpoolctl import threadpool_info
         threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
@@ -352,9 +365,13 @@ def main():
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         ws = torch.empty(ra.ringattn_bwd_workspace_size(B, H, N, D), device=dev, dtype=torch.uint8)
     if fw is not None:
-        x, w1, w2, w3 = ffn_inputs(replace(fw, seed=fw.seed + 1000 * rank), device=dev)
-        y = torch.empty_like(x)
+        x, w1, w2, w3, dy = ffn_inputs(replace(fw, seed=fw.seed + 1000 * rank), device=dev, with_dy=True)
+        y, dx = torch.empty_like(x), torch.empty_like(x)
+        dw1, dw3 = (torch.empty(w1.shape, device=dev, dtype=torch.float32) for _ in range(2))
+        dw2 = torch.empty(w2.shape, device=dev, dtype=torch.float32)
         ffn_ws = torch.empty(ra.blockwise_ffn_workspace_size(fw.chunk, fw.d_ff), device=dev, dtype=torch.uint8)
+        ffn_bws = torch.empty(ra.blockwise_ffn_bwd_workspace_size(fw.chunk, fw.d_ff), device=dev,
+                              dtype=torch.uint8)
     stream = torch.cuda.current_stream()
     cfg = (aw.S, aw.q_chunk, aw.k_chunk, aw.causal)
     gqa = aw.kv_heads != aw.H
@@ -378,7 +395,7 @@ def main():
 
     def step(timed=False):
         if timed:
-            e = [event() for _ in range(5)]
+            e = [event() for _ in range(7)]
             e[0].record(stream)
         fwd_call(q, k, v, o, lse)
         launches = 1
@@ -402,8 +419,14 @@ def main():
                 e[4].record(stream)
             launches += 3
         if fw is not None:
+            if timed:
+                e[5].record(stream)
             ra.blockwise_ffn(x, w1, w2, w3, y, fw.chunk, ffn_ws)
-            launches += 2 * (fw.T // fw.chunk)
+            ra.blockwise_ffn_bwd(x, w1, w2, w3, dy, dx, dw1, dw2, dw3, fw.chunk, ffn_bws)
+            launches += 6 * (fw.T // fw.chunk)  # forward: 2 per chunk, backward: 4 per chunk
+            if timed:
+                e[6].record(stream)
+                ev.setdefault("ffn", []).append((e[5], e[6]))
         if timed:
             ev.setdefault("fwd", []).append((e[0], e[1]))
             if aw.bwd and gqa:
@@ -461,6 +484,9 @@ def main():
         kernels["bwd_kv_kernel"] = (mean_ms(ev["bwd_kv"]), 2.0 * fwd_fl, "bwd_tc.cu")
         kernels["bwd_q_kernel"] = (mean_ms(ev["bwd_q"]), 0.5 * fwd_fl, "bwd_tc.cu")
     kname = max(kernels, key=lambda k_: kernels[k_][0])
+    if fw is not None:
+        # the feed-forward's forward and backward GEMMs, timed together
+        kernels["ffn_tc_kernel+ffn_bwd_gemm_kernel"] = (mean_ms(ev["ffn"]), ffn_flops(fw), "ffn_bwd_tc.cu")
     kms, kflops, ksrc = kernels[kname]
     achieved = kflops / (kms * 1e-3) / 1e12
     src = os.path.join(ROOT, "exact_blockwise_long_b200", "csrc", ksrc)
@@ -485,8 +511,8 @@ def main():
     # let step j+1's host-to-device copy and step j-1's device-to-host copy
     # run on their own streams while step j computes.
     if not args.no_e2e:
-        in0 = [q, k, v] + ([do] if aw.bwd else []) + ([x] if fw is not None else [])
-        out0 = [o, lse] + ([dq, dk, dv] if aw.bwd else []) + ([y] if fw is not None else [])
+        in0 = [q, k, v] + ([do] if aw.bwd else []) + ([x, dy] if fw is not None else [])
+        out0 = [o, lse] + ([dq, dk, dv] if aw.bwd else []) + ([y, dx, dw1, dw2, dw3] if fw is not None else [])
         hin = [t.cpu().pin_memory() for t in in0]
         hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in out0]
         ins = [in0, [torch.empty_like(t) for t in in0]]
@@ -521,7 +547,9 @@ def main():
             if aw.bwd:
                 bwd_call(qq, kk, vv, oo, ll, ins[bi][3], outs[bi][2], outs[bi][3], outs[bi][4])
             if fw is not None:
-                ra.blockwise_ffn(ins[bi][-1], w1, w2, w3, outs[bi][-1], fw.chunk, ffn_ws)
+                xx, gy = ins[bi][-2], ins[bi][-1]
+                ra.blockwise_ffn(xx, w1, w2, w3, outs[bi][-5], fw.chunk, ffn_ws)
+                ra.blockwise_ffn_bwd(xx, w1, w2, w3, gy, *outs[bi][-4:], fw.chunk, ffn_bws)
             done[bi].record(stream)
             s_out.wait_event(done[bi])
             with torch.cuda.stream(s_out):

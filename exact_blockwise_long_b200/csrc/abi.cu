@@ -38,8 +38,26 @@ int current_status(DevStatus* out) {
   return RA_OK;
 }
 
+namespace {
+int make_tmap_2d(void* tmap, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t rows,
+                 uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_rows);
+}
+
 int make_tmap_bf16_2d(void* tmap, const void* base, uint64_t inner, uint64_t rows, uint64_t row_pitch_bytes,
                       uint32_t box_inner, uint32_t box_rows) {
+  return make_tmap_2d(tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, inner, rows, row_pitch_bytes, box_inner,
+                      box_rows);
+}
+
+int make_tmap_f32_2d(void* tmap, const void* base, uint64_t inner, uint64_t rows, uint64_t row_pitch_bytes,
+                     uint32_t box_inner, uint32_t box_rows) {
+  return make_tmap_2d(tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, inner, rows, row_pitch_bytes, box_inner,
+                      box_rows);
+}
+
+namespace {
+int make_tmap_2d(void* tmap, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t rows,
+                 uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_rows) {
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_encode) {
@@ -55,12 +73,13 @@ int make_tmap_bf16_2d(void* tmap, const void* base, uint64_t inner, uint64_t row
   cuuint64_t strides[1] = {row_pitch_bytes};
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = g_encode(reinterpret_cast<CUtensorMap*>(tmap), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+  CUresult r = g_encode(reinterpret_cast<CUtensorMap*>(tmap), dt, 2,
                         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? RA_OK : RA_ERR_CUDA;
 }
+}  // namespace
 
 int head_group(int per_head, int heads, double bytes_per_head, double budget_bytes) {
   int dev = 0, sms = 148;

@@ -19,7 +19,10 @@
 //   kDw2        dw2 = dy^T h
 // Operands are K-major (rows of the activations, [out, in] weight rows) or
 // MN-major (an operand used transposed); both come in by TMA with the
-// 128-byte swizzle, 16 KB per 128 x 64 tile.
+// 128-byte swizzle, 16 KB per 128 x 64 tile.  Results leave by TMA too:
+// bf16 tiles as stores, fp32 weight gradients as a store on the first chunk
+// and an element-wise TMA add on the later ones (one add per element per
+// launch, in stream order, so the sums are deterministic).
 #include <math.h>
 
 #include "common.cuh"
@@ -74,13 +77,11 @@ struct BLay {
 };
 
 struct BGParams {
-  __nv_bfloat16* out_bf16[3];  // kSwiGLUBwd: dg, du, h; kDx: dx
-  float* out_f32[2];           // kDw13: dw1, dw3; kDw2: dw2
-  int ldo;                     // output row pitch (elements)
-  int accumulate;              // weight gradients: add to the fp32 output (0 on the first chunk)
-  int a_off[2], b_off[3];      // K-major: first row; MN-major: first K index
-  int kblocks;                 // 64-deep K steps
-  int kb_split;                // kDx: K step where (dg, w1) hand over to (du, w3)
+  int out_row;            // first output row of this launch (dx: the chunk's first token)
+  int accumulate;         // weight gradients: add into the fp32 output (0 on the first chunk)
+  int a_off[2], b_off[3]; // K-major: first row; MN-major: first K index
+  int kblocks;            // 64-deep K steps
+  int kb_split;           // kDx: K step where (dg, w1) hand over to (du, w3)
   int m_tiles;
   DevStatus st;
 };
@@ -107,7 +108,9 @@ template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     ffn_bwd_gemm_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tA1,
                         const __grid_constant__ CUtensorMap tB0, const __grid_constant__ CUtensorMap tB1,
-                        const __grid_constant__ CUtensorMap tB2, const BGParams p) {
+                        const __grid_constant__ CUtensorMap tB2, const __grid_constant__ CUtensorMap tO0,
+                        const __grid_constant__ CUtensorMap tO1, const __grid_constant__ CUtensorMap tO2,
+                        const BGParams p) {
   using C = BCfg<MODE>;
   using LY = BLay<MODE>;
   extern __shared__ uint8_t smem_fb[];
@@ -200,12 +203,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(bar_done);
     }
   } else if (warp >= 4) {
+    // Epilogue: accumulator rows -> 128-byte-swizzled staging boxes in the
+    // (now idle) pipeline buffers -> TMA stores (or TMA adds for the fp32
+    // weight gradients after the first chunk).  One 16 KB box holds 128 rows
+    // x 128 bytes: 64 bf16 or 32 fp32 columns.
     const int r = (warp - 4) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    if (__all_sync(0xffffffffu, mbar_wait(bar_done, 0, p.st, abort_flag))) {
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, p.st, abort_flag));
+    if (ok) {
       tc_fence_after();
-      const size_t row = (size_t)(mt * kBM + r);
-      const size_t col0 = (size_t)nt * kBN;
+      const uint32_t row_base = smem_u32(smem) + (uint32_t)r * 128;
+      const uint32_t sw = (uint32_t)(r & 7);
 #pragma unroll 1
       for (int c = 0; c < kBN / 32; ++c) {
         if constexpr (MODE == kSwiGLUBwd) {
@@ -235,9 +243,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int o = 0; o < 3; ++o) {
             const uint32_t* src = o == 0 ? pg : (o == 1 ? pu : ph);
-            uint4* dst = reinterpret_cast<uint4*>(p.out_bf16[o] + row * p.ldo + col0 + c * 32);
+            const uint32_t box = row_base + (uint32_t)(o * 2 + (c >> 1)) * kTile;
 #pragma unroll
-            for (int x = 0; x < 4; ++x) dst[x] = make_uint4(src[4 * x], src[4 * x + 1], src[4 * x + 2], src[4 * x + 3]);
+            for (int x = 0; x < 4; ++x) {
+              const uint32_t unit = (uint32_t)((c & 1) * 4 + x);
+              st_shared_v4(box + ((unit ^ sw) << 4), src[4 * x], src[4 * x + 1], src[4 * x + 2], src[4 * x + 3]);
+            }
           }
         } else if constexpr (MODE == kDx) {
           uint32_t a[32];
@@ -246,32 +257,54 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int x = 0; x < 16; ++x) pk[x] = pack_bf16x2(__uint_as_float(a[2 * x]), __uint_as_float(a[2 * x + 1]));
-          uint4* dst = reinterpret_cast<uint4*>(p.out_bf16[0] + row * p.ldo + col0 + c * 32);
+          const uint32_t box = row_base + (uint32_t)(c >> 1) * kTile;
 #pragma unroll
-          for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+          for (int x = 0; x < 4; ++x) {
+            const uint32_t unit = (uint32_t)((c & 1) * 4 + x);
+            st_shared_v4(box + ((unit ^ sw) << 4), pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+          }
         } else {
 #pragma unroll
           for (int o = 0; o < C::nAcc; ++o) {
             uint32_t a[32];
             tmem_ld32(tmem + lane_off + o * kBN + c * 32, a);
             tmem_ld_wait();
-            float4* dst = reinterpret_cast<float4*>(p.out_f32[o] + row * p.ldo + col0 + c * 32);
+            const uint32_t box = row_base + (uint32_t)(o * 4 + c) * kTile;
 #pragma unroll
-            for (int x = 0; x < 8; ++x) {
-              float4 v = make_float4(__uint_as_float(a[4 * x]), __uint_as_float(a[4 * x + 1]),
-                                     __uint_as_float(a[4 * x + 2]), __uint_as_float(a[4 * x + 3]));
-              if (p.accumulate) {
-                const float4 old = dst[x];
-                v.x += old.x;
-                v.y += old.y;
-                v.z += old.z;
-                v.w += old.w;
-              }
-              dst[x] = v;
-            }
+            for (int x = 0; x < 8; ++x)
+              st_shared_v4(box + (((uint32_t)x ^ sw) << 4), a[4 * x], a[4 * x + 1], a[4 * x + 2], a[4 * x + 3]);
           }
         }
       }
+      fence_proxy_async_smem();
+    }
+    named_bar_sync(1, 128);
+    if (threadIdx.x == 128 && ok) {
+      const uint8_t* stage = smem;
+      const int y = p.out_row + mt * kBM;
+      if constexpr (MODE == kSwiGLUBwd || MODE == kDx) {
+        constexpr int nOut = MODE == kSwiGLUBwd ? 3 : 1;
+#pragma unroll
+        for (int o = 0; o < nOut; ++o) {
+          const CUtensorMap* m = o == 0 ? &tO0 : (o == 1 ? &tO1 : &tO2);
+          tma_store_2d(m, stage + (o * 2) * kTile, nt * kBN, y);
+          tma_store_2d(m, stage + (o * 2 + 1) * kTile, nt * kBN + 64, y);
+        }
+      } else {
+#pragma unroll
+        for (int o = 0; o < C::nAcc; ++o) {
+          const CUtensorMap* m = o == 0 ? &tO0 : &tO1;
+#pragma unroll
+          for (int c = 0; c < kBN / 32; ++c) {
+            if (p.accumulate)
+              tma_add_2d(m, stage + (o * 4 + c) * kTile, nt * kBN + c * 32, y);
+            else
+              tma_store_2d(m, stage + (o * 4 + c) * kTile, nt * kBN + c * 32, y);
+          }
+        }
+      }
+      bulk_commit_group();
+      bulk_wait_read_all();
     }
   }
 
@@ -284,11 +317,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int MODE>
-int launch_mode(const CUtensorMap* maps[5], const BGParams& p, int grid, cudaStream_t stream) {
+int launch_mode(const CUtensorMap* maps[8], const BGParams& p, int grid, cudaStream_t stream) {
   static_assert(BLay<MODE>::kAlloc <= 232448, "FFN backward stages exceed shared memory");
+  // the epilogue's staging boxes live in the pipeline buffers
+  constexpr int kStaging = MODE == kSwiGLUBwd ? 6 : (MODE == kDx ? 2 : 4 * BCfg<MODE>::nAcc);
+  static_assert(kStaging * kTile <= BLay<MODE>::kBar, "epilogue staging exceeds the pipeline buffers");
   auto kern = ffn_bwd_gemm_kernel<MODE>;
   if (set_smem_attr((const void*)kern, BLay<MODE>::kAlloc) != RA_OK) return RA_ERR_CUDA;
-  kern<<<grid, kThreads, BLay<MODE>::kAlloc, stream>>>(*maps[0], *maps[1], *maps[2], *maps[3], *maps[4], p);
+  kern<<<grid, kThreads, BLay<MODE>::kAlloc, stream>>>(*maps[0], *maps[1], *maps[2], *maps[3], *maps[4], *maps[5],
+                                                       *maps[6], *maps[7], p);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
@@ -310,7 +347,13 @@ int launch_ffn_bwd_tc(const void* x, const void* w1, const void* w2, const void*
   // K-major maps (box 64 K x 128 rows) and MN-major maps (box 64 MN x 64 K)
   alignas(64) CUtensorMap x_k, dy_k, w1_k, w3_k, dg_k, du_k;       // K-major
   alignas(64) CUtensorMap w2_m, w1_m, w3_m, x_m, dg_m, du_m, dy_m, h_m;  // MN-major
+  alignas(64) CUtensorMap h_o, dx_o, dw1_o, dw3_o, dw2_o;               // output boxes
   int ok = RA_OK;
+  ok |= make_tmap_bf16_2d(&h_o, h, d_ff, chunk, d_ff * 2, 64, 128);
+  ok |= make_tmap_bf16_2d(&dx_o, dx, d_model, T, d_model * 2, 64, 128);
+  ok |= make_tmap_f32_2d(&dw1_o, dw1, d_model, d_ff, d_model * 4, 32, 128);
+  ok |= make_tmap_f32_2d(&dw3_o, dw3, d_model, d_ff, d_model * 4, 32, 128);
+  ok |= make_tmap_f32_2d(&dw2_o, dw2, d_ff, d_model, d_ff * 4, 32, 128);
   ok |= make_tmap_bf16_2d(&x_k, x, d_model, T, d_model * 2, 64, 128);
   ok |= make_tmap_bf16_2d(&dy_k, dy, d_model, T, d_model * 2, 64, 128);
   ok |= make_tmap_bf16_2d(&w1_k, w1, d_model, d_ff, d_model * 2, 64, 128);
@@ -331,52 +374,42 @@ int launch_ffn_bwd_tc(const void* x, const void* w1, const void* w2, const void*
     const int c = (int)c0;
     {  // g, u, dh -> dg, du, h
       BGParams p{};
-      p.out_bf16[0] = dg;
-      p.out_bf16[1] = du;
-      p.out_bf16[2] = h;
-      p.ldo = df;
       p.a_off[0] = c;
       p.a_off[1] = c;
       p.kblocks = dm / kBK;
       p.m_tiles = ch / kBM;
       p.st = st;
-      const CUtensorMap* maps[5] = {&x_k, &dy_k, &w1_k, &w3_k, &w2_m};
+      const CUtensorMap* maps[8] = {&x_k, &dy_k, &w1_k, &w3_k, &w2_m, &dg_k, &du_k, &h_o};
       if ((rc = launch_mode<kSwiGLUBwd>(maps, p, (ch / kBM) * (df / kBN), stream)) != RA_OK) return rc;
     }
     {  // dx = dg w1 + du w3
       BGParams p{};
-      p.out_bf16[0] = static_cast<__nv_bfloat16*>(dx) + c0 * d_model;
-      p.ldo = dm;
+      p.out_row = c;
       p.kblocks = 2 * (df / kBK);
       p.kb_split = df / kBK;
       p.m_tiles = ch / kBM;
       p.st = st;
-      const CUtensorMap* maps[5] = {&dg_k, &du_k, &w1_m, &w3_m, &w3_m};
+      const CUtensorMap* maps[8] = {&dg_k, &du_k, &w1_m, &w3_m, &w3_m, &dx_o, &dx_o, &dx_o};
       if ((rc = launch_mode<kDx>(maps, p, (ch / kBM) * (dm / kBN), stream)) != RA_OK) return rc;
     }
     {  // dw1, dw3 (+)= dg^T x, du^T x
       BGParams p{};
-      p.out_f32[0] = dw1;
-      p.out_f32[1] = dw3;
-      p.ldo = dm;
       p.accumulate = c0 > 0;
       p.b_off[0] = c;
       p.kblocks = ch / kBK;
       p.m_tiles = df / kBM;
       p.st = st;
-      const CUtensorMap* maps[5] = {&dg_m, &du_m, &x_m, &x_m, &x_m};
+      const CUtensorMap* maps[8] = {&dg_m, &du_m, &x_m, &x_m, &x_m, &dw1_o, &dw3_o, &dw3_o};
       if ((rc = launch_mode<kDw13>(maps, p, (df / kBM) * (dm / kBN), stream)) != RA_OK) return rc;
     }
     {  // dw2 (+)= dy^T h
       BGParams p{};
-      p.out_f32[0] = dw2;
-      p.ldo = df;
       p.accumulate = c0 > 0;
       p.a_off[0] = c;
       p.kblocks = ch / kBK;
       p.m_tiles = dm / kBM;
       p.st = st;
-      const CUtensorMap* maps[5] = {&dy_m, &dy_m, &h_m, &h_m, &h_m};
+      const CUtensorMap* maps[8] = {&dy_m, &dy_m, &h_m, &h_m, &h_m, &dw2_o, &dw2_o, &dw2_o};
       if ((rc = launch_mode<kDw2>(maps, p, (dm / kBM) * (df / kBN), stream)) != RA_OK) return rc;
     }
   }

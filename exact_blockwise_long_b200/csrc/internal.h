@@ -69,6 +69,10 @@ int launch_selftest_timeout(int timeout_us, cudaStream_t stream);
 int make_tmap_bf16_2d(void* tmap /* CUtensorMap* */, const void* base, uint64_t inner, uint64_t rows,
                       uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_rows);
 
+// The same for a 2-D fp32 map (box inner extent at most 32 elements).
+int make_tmap_f32_2d(void* tmap /* CUtensorMap* */, const void* base, uint64_t inner, uint64_t rows,
+                     uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_rows);
+
 // Head-group size for grouped_order: as many heads as keep their working
 // set (bytes_per_head) within budget_bytes of the 126 MB L2, but enough that
 // a group holds two waves of work items; at least one, at most `heads`.
