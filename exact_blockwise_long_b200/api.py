@@ -223,6 +223,54 @@ def blockwise_ffn_bwd(x, w1, w2, w3, dy, dx, dw1, dw2, dw3, chunk, workspace, st
     return dx, dw1, dw2, dw3
 
 
+def blockwise_layer_saved_size(B, N, H, D) -> int:
+    return int(lib().blockwise_layer_saved_size(int(B), int(N), int(H), int(D)))
+
+
+def blockwise_layer_fwd_workspace_size(ffn_chunk, d_ff) -> int:
+    return int(lib().blockwise_layer_fwd_workspace_size(int(ffn_chunk), int(d_ff)))
+
+
+def blockwise_layer_bwd_workspace_size(B, N, H, D, d_ff, ffn_chunk) -> int:
+    return int(lib().blockwise_layer_bwd_workspace_size(int(B), int(N), int(H), int(D), int(d_ff), int(ffn_chunk)))
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
+def blockwise_layer_fwd(x, weights, y, saved, B, N, H, D, S, q_chunk, k_chunk, causal, ffn_chunk, workspace,
+                        eps=1e-5, stream=None):
+    """y <- the blockwise transformer layer of x ([B*N, H*D] bf16); `saved`
+    receives the activations the backward reads.  `weights` is the tuple
+    (g_attn, wq, wk, wv, wo, g_ffn, w1, w2, w3)."""
+    g_attn, wq, wk, wv, wo, g_ffn, w1, w2, w3 = weights
+    d_ff = int(w1.shape[0])
+    names = ("g_attn", "wq", "wk", "wv", "wo", "g_ffn", "w1", "w2", "w3")
+    call("blockwise_layer_fwd", _dev(x, "x"), *[_dev(t, n) for t, n in zip(weights, names)], _dev(y, "y"),
+         _dev(saved, "saved"), _nbytes(saved), int(B), int(N), int(H), int(D), d_ff, int(S), int(q_chunk),
+         int(k_chunk), int(bool(causal)), int(ffn_chunk), float(eps), _dev(workspace, "workspace"),
+         _nbytes(workspace), _stream(stream))
+    return y
+
+
+def blockwise_layer_bwd(x, weights, saved, dy, dx, grads, B, N, H, D, S, q_chunk, k_chunk, causal, ffn_chunk,
+                        workspace, stream=None):
+    """dx (bf16) and the fp32 parameter gradients `grads` = (dg_attn, dwq,
+    dwk, dwv, dwo, dg_ffn, dw1, dw2, dw3) of sum(dy * layer(x))."""
+    names = ("g_attn", "wq", "wk", "wv", "wo", "g_ffn", "w1", "w2", "w3")
+    for t, w in zip(grads, weights):
+        if t.dtype != torch.float32 or tuple(t.shape) != tuple(w.shape):
+            raise ValueError("parameter gradients are float32 in the parameters' shapes")
+    d_ff = int(weights[6].shape[0])
+    call("blockwise_layer_bwd", _dev(x, "x"), *[_dev(t, n) for t, n in zip(weights, names)],
+         _dev(saved, "saved"), _nbytes(saved), _dev(dy, "dy"), _dev(dx, "dx"),
+         *[_dev(t, "d" + n) for t, n in zip(grads, names)], int(B), int(N), int(H), int(D), d_ff, int(S),
+         int(q_chunk), int(k_chunk), int(bool(causal)), int(ffn_chunk), _dev(workspace, "workspace"),
+         _nbytes(workspace), _stream(stream))
+    return dx, grads
+
+
 def ringattn_get_error(stream=None) -> int:
     """Synchronise the stream; return and clear the device status word."""
     return int(lib().ringattn_get_error(_stream(stream)))

@@ -48,6 +48,7 @@ struct GLayout {
 
 struct GParams {
   __nv_bfloat16* out;   // [M rows of this launch, ldo]
+  const __nv_bfloat16* res;  // kDown: residual added to y (same layout as out), or null
   int a_row0;           // first row of A in its tensor map
   int ldo;              // output row pitch (elements)
   int K;                // reduction length
@@ -159,8 +160,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else {
           tmem_ld_wait();
+          if (p.res) {  // y = residual + h w2^T, rounded once
+            const uint4* rr = reinterpret_cast<const uint4*>(p.res + (size_t)(mt * kBM + r) * p.ldo +
+                                                             (size_t)nt * BN + c * 32);
 #pragma unroll
-          for (int x = 0; x < 16; ++x) pk[x] = pack_bf16x2(__uint_as_float(g[2 * x]), __uint_as_float(g[2 * x + 1]));
+            for (int x = 0; x < 4; ++x) {
+              const uint4 q = rr[x];
+              const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int i = 8 * x + 2 * e;
+                pk[4 * x + e] = pack_bf16x2(__uint_as_float(g[i]) + __uint_as_float(w[e] << 16),
+                                            __uint_as_float(g[i + 1]) + __uint_as_float(w[e] & 0xffff0000u));
+              }
+            }
+          } else {
+#pragma unroll
+            for (int x = 0; x < 16; ++x)
+              pk[x] = pack_bf16x2(__uint_as_float(g[2 * x]), __uint_as_float(g[2 * x + 1]));
+          }
         }
         uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
@@ -179,11 +197,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int MODE, int BN>
 int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1, __nv_bfloat16* out,
-                int a_row0, int ldo, int M, int N, int K, const DevStatus& st, cudaStream_t stream) {
+                int a_row0, int ldo, int M, int N, int K, const DevStatus& st, cudaStream_t stream,
+                const __nv_bfloat16* res = nullptr) {
   using LY = GLayout<MODE, BN>;
   static_assert(LY::kBytes <= 232448, "GEMM stages exceed shared memory");
   GParams p{};
   p.out = out;
+  p.res = res;
   p.a_row0 = a_row0;
   p.ldo = ldo;
   p.K = K;
@@ -199,7 +219,8 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap
 }  // namespace
 
 int launch_ffn_tc(const void* x, const void* w1, const void* w2, const void* w3, void* y, int64_t T,
-                  int64_t d_model, int64_t d_ff, int64_t chunk, void* workspace, cudaStream_t stream) {
+                  int64_t d_model, int64_t d_ff, int64_t chunk, void* workspace, cudaStream_t stream,
+                  const void* residual) {
   constexpr int kBNUp = 128;    // per weight: two 128-column accumulators
   constexpr int kBNDown = 128;
   if (d_ff % kBNUp || d_model % kBNDown || d_model % kBK || d_ff % kBK || chunk % kBM) return RA_ERR_SHAPE;
@@ -219,8 +240,10 @@ int launch_ffn_tc(const void* x, const void* w1, const void* w2, const void* w3,
     rc = launch_gemm<kGateUp, kBNUp>(tx, tw1, tw3, h, (int)c0, (int)d_ff, (int)chunk, (int)d_ff, (int)d_model, st,
                                      stream);
     if (rc != RA_OK) return rc;
+    const __nv_bfloat16* res =
+        residual ? static_cast<const __nv_bfloat16*>(residual) + c0 * d_model : nullptr;
     rc = launch_gemm<kDown, kBNDown>(th, tw2, tw2, yb + c0 * d_model, 0, (int)d_model, (int)chunk, (int)d_model,
-                                     (int)d_ff, st, stream);
+                                     (int)d_ff, st, stream, res);
     if (rc != RA_OK) return rc;
   }
   return RA_OK;

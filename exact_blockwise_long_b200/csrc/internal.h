@@ -45,8 +45,10 @@ int launch_bwd_tc(const AttnArgs& a, const void* out, const float* lse, const vo
                   void* dv, void* workspace, int phase_mask, cudaStream_t stream);
 
 // Blockwise SwiGLU FFN on the tensor cores.
+// residual: optional bf16 [T, d_model] added to y before its rounding.
 int launch_ffn_tc(const void* x, const void* w1, const void* w2, const void* w3, void* y, int64_t T,
-                  int64_t d_model, int64_t d_ff, int64_t chunk, void* workspace, cudaStream_t stream);
+                  int64_t d_model, int64_t d_ff, int64_t chunk, void* workspace, cudaStream_t stream,
+                  const void* residual = nullptr);
 
 // Decode: splits of the key/value cache (S shards of ceil(N/S) keys, each
 // cut into pieces of at most k_chunk keys) and the launch.
@@ -60,6 +62,46 @@ size_t ffn_bwd_workspace_bytes(int64_t chunk, int64_t d_ff);
 int launch_ffn_bwd_tc(const void* x, const void* w1, const void* w2, const void* w3, const void* dy, void* dx,
                       float* dw1, float* dw2, float* dw3, int64_t T, int64_t d_model, int64_t d_ff, int64_t chunk,
                       void* workspace, cudaStream_t stream);
+
+// Generic bf16 GEMM (csrc/gemm_tc.cu): D[M,N] = sum_s A_s[M,K_s] B_s[N,K_s]^T.
+// An operand is a logical row-major bf16 matrix [rows, cols]: K-major
+// (rows index M or N, cols index K) or MN-major (rows index K, cols index M
+// or N).  With hs_ntok > 0 the logical [batch*hs_ntok, hs_heads*hs_d] matrix
+// is stored head-split as [batch, hs_heads, hs_ntok, hs_d].  (r0, c0) is the
+// operand's origin inside the logical matrix.
+struct GemmOperand {
+  const void* ptr;
+  int64_t rows, cols;
+  int mn_major;
+  int64_t hs_ntok, hs_heads, hs_d;
+  int64_t r0, c0;
+};
+struct GemmSeg {
+  GemmOperand a, b;
+  int64_t K;
+};
+struct GemmOut {
+  void* ptr;                        // [M, N] (bf16: plain or head-split; fp32: plain)
+  int f32;                          // fp32 output (else bf16)
+  int add;                          // fp32: add into the existing values
+  int64_t hs_ntok, hs_heads, hs_d;  // bf16 head-split output
+  const void* residual;             // bf16 [M, N] added before rounding (bf16 output), or null
+};
+// M % 128 == 0, N % 256 == 0, K_s % 64 == 0; splits 1 or 2 (2: fp32 output
+// only, K split across two CTAs that each add onto a zeroed output).
+int launch_gemm_tc(const GemmSeg* segs, int nseg, int64_t M, int64_t N, const GemmOut& out, int splits,
+                   cudaStream_t stream);
+
+// RMS normalisation (csrc/rmsnorm.cu) of rows of d_model bf16 values
+// (d_model = 256 * {1,2,4,8,16}): out = x * rstd * g, rstd = (mean(x^2) + eps)^-1/2.
+int launch_rmsnorm_fwd(const void* x, const void* g, void* out, float* rstd, int64_t T, int64_t d_model, float eps,
+                       cudaStream_t stream);
+// dx = dres + rstd (g*dxn - xhat mean(g*dxn*xhat)), xhat = x rstd (dres may be null);
+// dg = sum over rows of dxn * xhat (fp32), through `partial` scratch of
+// rmsnorm_dg_partial_floats(T, d_model) floats.
+int launch_rmsnorm_bwd(const void* x, const void* g, const float* rstd, const void* dxn, const void* dres, void* dx,
+                       float* dg, float* partial, int64_t T, int64_t d_model, cudaStream_t stream);
+size_t rmsnorm_dg_partial_floats(int64_t T, int64_t d_model);
 
 int launch_selftest_timeout(int timeout_us, cudaStream_t stream);
 

@@ -97,6 +97,39 @@ DECODE_WORKLOADS = {
 }
 
 
+@dataclass(frozen=True)
+class LayerWorkload:
+    name: str
+    B: int
+    N: int
+    H: int
+    D: int
+    d_ff: int
+    S: int
+    q_chunk: int
+    k_chunk: int
+    ffn_chunk: int
+    seed: int
+    causal: bool = True
+    w_std: float = 0.02
+    eps: float = 1e-5
+
+    @property
+    def d_model(self) -> int:
+        return self.H * self.D
+
+    @property
+    def T(self) -> int:
+        return self.B * self.N
+
+
+LAYER_WORKLOADS = {
+    # the whole 7B-shaped layer (norms, projections, ring attention, SwiGLU FFN)
+    # over N=131072 tokens, forward and backward
+    "layer7b_full": LayerWorkload("layer7b_full", 1, 131072, 32, 128, 11008, 32, 2048, 2048, 2048, 3),
+}
+
+
 def _gen(device, seed: int) -> torch.Generator:
     g = torch.Generator(device=device)
     g.manual_seed(int(seed))
@@ -170,3 +203,21 @@ def sample_rows(B: int, H: int, N: int, n: int, seed: int, include_ends: bool = 
 def to_f64(t: torch.Tensor) -> np.ndarray:
     """Exact upcast of a (bf16 / fp32) tensor to a float64 numpy array."""
     return t.detach().to("cpu", torch.float32).numpy().astype(np.float64)
+
+
+def layer_inputs(w: LayerWorkload, device="cuda"):
+    """x [T, d_model]; params (g_attn, wq, wk, wv, wo, g_ffn, w1, w2, w3);
+    dy [T, d_model].  Drawn in the order x, g_attn, wq, wk, wv, wo, g_ffn,
+    w1, w3, w2, dy; norm gains are 1 + 0.1 z, weights w_std z."""
+    g = _gen(device, w.seed)
+    dm, dff = w.d_model, w.d_ff
+    x = _draw((w.T, dm), g, device, 1.0, torch.bfloat16)
+    g_attn = (1.0 + 0.1 * torch.randn(dm, generator=g, device=device)).to(torch.bfloat16)
+    wq, wk, wv, wo = (_draw((dm, dm), g, device, w.w_std, torch.bfloat16) for _ in range(4))
+    g_ffn = (1.0 + 0.1 * torch.randn(dm, generator=g, device=device)).to(torch.bfloat16)
+    w1 = _draw((dff, dm), g, device, w.w_std, torch.bfloat16)
+    w3 = _draw((dff, dm), g, device, w.w_std, torch.bfloat16)
+    w2 = _draw((dm, dff), g, device, w.w_std, torch.bfloat16)
+    dy = _draw((w.T, dm), g, device, 1.0, torch.bfloat16)
+    return x, (g_attn, wq, wk, wv, wo, g_ffn, w1, w2, w3), dy
+

@@ -319,6 +319,47 @@ RA_API int blockwise_ffn_bwd(const void* x, const void* w1, const void* w2, cons
                              int64_t T, int64_t d_model, int64_t d_ff, int64_t chunk, int dtype,
                              void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * One blockwise transformer layer (paper abstract: self-attention and the
+ * feed-forward both computed blockwise, for training).  Pre-norm decoder
+ * layer, no biases, no rotary embedding:
+ *   xn  = x * rstd(x) * g_attn,          rstd(z) = (mean(z^2) + eps)^-1/2
+ *   q, k, v = xn wq^T, xn wk^T, xn wv^T  (heads split: [B, H, N, D])
+ *   o   = ring attention(q, k, v)        (scale 1/sqrt(D), S shards, chunks)
+ *   x2  = x + o wo^T
+ *   xn2 = x2 * rstd(x2) * g_ffn
+ *   y   = x2 + (silu(xn2 w1^T) * (xn2 w3^T)) w2^T   (in ffn_chunk-token chunks)
+ *
+ *   x, y, dy, dx   [B*N, H*D] bf16 (token t = b*N + n)
+ *   g_attn, g_ffn  [H*D] bf16;  wq, wk, wv, wo [H*D, H*D] bf16 ([out, in])
+ *   w1, w3 [d_ff, H*D], w2 [H*D, d_ff] bf16
+ *   saved: blockwise_layer_saved_size bytes, written by the forward (xn, q,
+ *     k, v, o, x2, xn2, lse, both rstd) and read by the backward
+ *   gradients: dx bf16; dg_attn, dg_ffn [H*D] fp32; dwq, dwk, dwv, dwo,
+ *     dw1, dw2, dw3 fp32 in the weights' shapes (written, not accumulated)
+ * Rules: D in {64, 128}; H*D in {256, 512, 1024, 2048, 4096}; N % 128 == 0;
+ * the attention's shard and chunk rules (N % S, shard % chunk, chunks
+ * multiples of 128); (B*N) % ffn_chunk == 0, ffn_chunk and d_ff multiples
+ * of 128; every pointer 16-byte aligned.  Errors: RA_ERR_ARG, RA_ERR_SHAPE,
+ * RA_ERR_UNSUPPORTED, RA_ERR_ALIGN, RA_ERR_WORKSPACE, RA_ERR_CUDA.
+ * ------------------------------------------------------------------------- */
+RA_API size_t blockwise_layer_saved_size(int64_t B, int64_t N, int64_t H, int64_t D);
+RA_API size_t blockwise_layer_fwd_workspace_size(int64_t ffn_chunk, int64_t d_ff);
+RA_API size_t blockwise_layer_bwd_workspace_size(int64_t B, int64_t N, int64_t H, int64_t D, int64_t d_ff,
+                                                 int64_t ffn_chunk);
+RA_API int blockwise_layer_fwd(const void* x, const void* g_attn, const void* wq, const void* wk, const void* wv,
+                               const void* wo, const void* g_ffn, const void* w1, const void* w2, const void* w3,
+                               void* y, void* saved, size_t saved_bytes, int64_t B, int64_t N, int64_t H,
+                               int64_t D, int64_t d_ff, int S, int q_chunk, int k_chunk, int causal, int ffn_chunk,
+                               float eps, void* workspace, size_t workspace_bytes, void* stream);
+RA_API int blockwise_layer_bwd(const void* x, const void* g_attn, const void* wq, const void* wk, const void* wv,
+                               const void* wo, const void* g_ffn, const void* w1, const void* w2, const void* w3,
+                               const void* saved, size_t saved_bytes, const void* dy, void* dx, float* dg_attn,
+                               float* dwq, float* dwk, float* dwv, float* dwo, float* dg_ffn, float* dw1,
+                               float* dw2, float* dw3, int64_t B, int64_t N, int64_t H, int64_t D, int64_t d_ff,
+                               int S, int q_chunk, int k_chunk, int causal, int ffn_chunk, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
 /*
  * ringattn_get_error -- synchronise `stream`, return the device status word
  * of the current device (RA_OK or RA_ERR_TIMEOUT) and clear it.  Also

@@ -54,6 +54,13 @@ Parity status per function (what pins it is in ``tests/test_oracle.py``):
                                  invariance, linearity in dy)
 * ``swiglu_ffn_backward_terms``  error-bound helper (sums of |term|), pinned
                                  by dominating |gradient| element-wise
+* ``rmsnorm`` / ``rmsnorm_backward``
+                                 pinned (unit mean square with g = 1, scale
+                                 invariance, constant rows, finite differences)
+* ``layer_forward`` / ``layer_backward``
+                                 pinned (central finite differences of every
+                                 parameter and input; wo = w2 = 0 closed form;
+                                 causal locality and batch independence)
 """
 
 from .attention import (  # noqa: F401
@@ -80,4 +87,11 @@ from .ffn import (  # noqa: F401
     swiglu_ffn_backward,
     blockwise_ffn_backward,
     swiglu_ffn_backward_terms,
+)
+from .layer import (  # noqa: F401
+    PARAM_NAMES,
+    layer_backward,
+    layer_forward,
+    rmsnorm,
+    rmsnorm_backward,
 )

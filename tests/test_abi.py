@@ -42,7 +42,7 @@ def test_only_declared_symbols_are_exported():
     import subprocess
     from exact_blockwise_long_b200 import _lib
     out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True).stdout
-    ours = {ln.split()[-1] for ln in out.splitlines() if " T " in ln and ("ringattn" in ln or "ffn" in ln)}
+    ours = {ln.split()[-1] for ln in out.splitlines() if " T " in ln and ("ringattn" in ln or "blockwise" in ln)}
     assert ours == set(declared_symbols())
 
 

@@ -555,3 +555,101 @@ def test_decode_zero_query_gives_mean():
     o, lse = oracle.attention_decode(np.zeros((B, H, d)), k, v)
     np.testing.assert_allclose(o, np.broadcast_to(v.mean(axis=2), o.shape), atol=1e-13)
     np.testing.assert_allclose(lse, np.log(N), atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# RMS normalisation and the whole layer
+# ---------------------------------------------------------------------------
+
+def test_rmsnorm_closed_forms_and_gradient():
+    x = _rand((6, 8), 300)
+    y, r = oracle.rmsnorm(x, np.ones(8), 0.0)
+    np.testing.assert_allclose(np.mean(y * y, axis=1), 1.0, rtol=1e-14)  # unit mean square
+    y2, _ = oracle.rmsnorm(3.7 * x, np.ones(8), 0.0)
+    np.testing.assert_allclose(y2, y, rtol=1e-13)                         # scale invariance
+    c, eps = 0.3, 0.01
+    yc, _ = oracle.rmsnorm(np.full((1, 8), c), np.arange(8.0), eps)       # constant row
+    np.testing.assert_allclose(yc[0], c / math.sqrt(c * c + eps) * np.arange(8.0), rtol=1e-14)
+    g = _rand(8, 301) + 1.0
+    dout = _rand((6, 8), 302)
+    dx, dg = oracle.rmsnorm_backward(x, g, dout, 1e-3)
+    e = 1e-6
+    for idx in np.ndindex(*x.shape):
+        xp, xm = x.copy(), x.copy()
+        xp[idx] += e
+        xm[idx] -= e
+        fd = (np.sum(dout * oracle.rmsnorm(xp, g, 1e-3)[0]) - np.sum(dout * oracle.rmsnorm(xm, g, 1e-3)[0])) / (2 * e)
+        assert abs(fd - dx[idx]) <= 1e-7 * (1 + abs(fd))
+    for j in range(8):
+        gp, gm = g.copy(), g.copy()
+        gp[j] += e
+        gm[j] -= e
+        fd = (np.sum(dout * oracle.rmsnorm(x, gp, 1e-3)[0]) - np.sum(dout * oracle.rmsnorm(x, gm, 1e-3)[0])) / (2 * e)
+        assert abs(fd - dg[j]) <= 1e-7 * (1 + abs(fd))
+
+
+def _layer_case(B=1, N=4, H=2, D=2, dff=3, seed=400, wscale=0.6):
+    dm = H * D
+    x = _rand((B * N, dm), seed)
+    params = [1.0 + 0.2 * _rand(dm, seed + 1)] + [_rand((dm, dm), seed + 2 + i, wscale) for i in range(4)] + \
+             [1.0 + 0.2 * _rand(dm, seed + 6), _rand((dff, dm), seed + 7, wscale), _rand((dm, dff), seed + 8, wscale),
+              _rand((dff, dm), seed + 9, wscale)]
+    dy = _rand((B * N, dm), seed + 10)
+    return x, params, dy
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_layer_backward_finite_differences(causal):
+    """Every entry of dx and of all nine parameter gradients against a central
+    difference of sum(dy * y) (two sequences, two heads)."""
+    B, N, H, D = 2, 4, 2, 2
+    x, params, dy = _layer_case(B, N, H, D)
+    eps_n = 1e-3
+    dx, grads = oracle.layer_backward(x, params, dy, B, N, H, D, causal, eps_n)
+
+    def loss(xx, pp):
+        return np.sum(dy * oracle.layer_forward(xx, pp, B, N, H, D, causal, eps_n)[0])
+
+    e = 1e-6
+    for idx in np.ndindex(*x.shape):
+        xp, xm = x.copy(), x.copy()
+        xp[idx] += e
+        xm[idx] -= e
+        fd = (loss(xp, params) - loss(xm, params)) / (2 * e)
+        assert abs(fd - dx[idx]) <= 1e-6 * (1 + abs(fd)), ("x", idx)
+    for pi, gr in enumerate(grads):
+        for idx in np.ndindex(*params[pi].shape):
+            pp = [p.copy() for p in params]
+            pm = [p.copy() for p in params]
+            pp[pi][idx] += e
+            pm[pi][idx] -= e
+            fd = (loss(x, pp) - loss(x, pm)) / (2 * e)
+            assert abs(fd - gr[idx]) <= 1e-6 * (1 + abs(fd)), (oracle.PARAM_NAMES[pi], idx)
+
+
+def test_layer_zero_output_projections_is_identity():
+    """wo = 0 and w2 = 0 switch both branches off: y = x and dx = dy."""
+    B, N, H, D = 1, 6, 2, 2
+    x, params, dy = _layer_case(B, N, H, D, seed=420)
+    params[4] = np.zeros_like(params[4])
+    params[7] = np.zeros_like(params[7])
+    y, _ = oracle.layer_forward(x, params, B, N, H, D)
+    assert np.array_equal(y, x)
+    dx, grads = oracle.layer_backward(x, params, dy, B, N, H, D)
+    np.testing.assert_allclose(dx, dy, atol=1e-15)
+    assert np.abs(grads[4]).max() > 0.01 and np.abs(grads[7]).max() > 0.01  # dwo, dw2 still flow
+    for i in (0, 1, 2, 3, 5, 6, 8):
+        assert np.all(grads[i] == 0), oracle.PARAM_NAMES[i]
+
+
+def test_layer_causal_locality_and_batch_independence():
+    B, N, H, D = 2, 6, 2, 2
+    x, params, _ = _layer_case(B, N, H, D, seed=440)
+    y, _ = oracle.layer_forward(x, params, B, N, H, D, causal=True)
+    xp = x.copy()
+    xp[4:6] += 5.0                   # later tokens of sequence 0
+    yp, _ = oracle.layer_forward(xp, params, B, N, H, D, causal=True)
+    np.testing.assert_allclose(yp[:4], y[:4], atol=1e-13)
+    np.testing.assert_allclose(yp[6:], y[6:], atol=1e-13)   # the other sequence
+    assert np.abs(yp[4:6] - y[4:6]).max() > 0.1
+
