@@ -59,12 +59,13 @@ def parse():
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="n32k_d128",
-                    choices=["n32k_d128", "n8k_d64_causal", "n8k_d64_full", "layer7b", "n1m_d128",
-                             "n32k_d128_gqa8", "decode_n128k"])
+                    choices=["n32k_d128", "n8k_d64_causal", "n8k_d64_full", "layer7b", "layer7b_full",
+                             "n1m_d128", "n32k_d128_gqa8", "decode_n128k"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (smaller profiling cases)")
+    ap.add_argument("--tokens", type=int, default=0, help="override the sequence length of layer7b_full")
     return ap.parse_args()
 
 
@@ -242,12 +243,28 @@ def run_reference(args):
     if rank != 0:
         return 0
     from dataclasses import replace
-    aw, fw = workload(args.workload)
-    if args.heads:
-        aw = replace(aw, H=args.heads)
+    if args.workload.startswith("decode"):
+        from exact_blockwise_long_b200.synthetic import DECODE_WORKLOADS
+        dw = DECODE_WORKLOADS[args.workload]
+        sampler = lambda: decode_oracle_sample(dw)  # noqa: E731
+        config = {"workload": f"{dw.name}: decode, one new token per head against a cache of N={dw.N}, B={dw.B}, "
+                              f"H={dw.H}, Hkv={dw.Hkv}, d={dw.D}"}
+    elif args.workload == "layer7b_full":
+        from exact_blockwise_long_b200.synthetic import LAYER_WORKLOADS
+        lw = LAYER_WORKLOADS[args.workload]
+        aw = fw = None
+        sampler = lambda: layer_oracle_sample(lw)  # noqa: E731
+        config = {"workload": f"{lw.name}: one blockwise transformer layer fwd+bwd, N={lw.N}, H={lw.H}, "
+                              f"d={lw.D}, d_ff={lw.d_ff}, S={lw.S}"}
+    else:
+        aw, fw = workload(args.workload)
+        if args.heads:
+            aw = replace(aw, H=args.heads)
+        sampler = lambda: oracle_sample(aw, fw)  # noqa: E731
+        config = describe(aw, fw)
     times, flops, desc, threads = [], 0.0, "", 1
     for i in range(args.warmup + args.steps):
-        dt, flops, desc, threads = oracle_sample(aw, fw)
+        dt, flops, desc, threads = sampler()
         if i >= args.warmup:
             times.append(dt)
     t = sum(times) / len(times)
@@ -255,7 +272,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": describe(aw, fw),
+            "config": config,
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": desc + f"; {args.steps} timed samples"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -315,6 +332,225 @@ def run_decode(args, ra, dev, rank, world, dist):
             "gpu_launches": 2 * args.steps, "clocks": clk}
 
 
+def layer_flops(w):
+    """Algorithmic FLOPs of one layer step (forward + backward):
+    projections 8 T dm^2 forward and 16 T dm^2 backward (dO, dWo, dxn from
+    three weights, dWq/dWk/dWv); attention 3.5 x its causal forward; the
+    feed-forward 18 T dm d_ff (forward 6, backward 12).  RMS norms are not
+    counted."""
+    from exact_blockwise_long_b200.synthetic import AttnWorkload
+    aw = AttnWorkload("x", w.B, w.H, w.N, w.D, w.S, w.q_chunk, w.k_chunk, w.causal, 0)
+    proj = 24.0 * w.T * w.d_model * w.d_model
+    ffn = 18.0 * w.T * w.d_model * w.d_ff
+    return proj, attn_fwd_flops(aw), ffn
+
+
+def layer_oracle_sample(w, tokens=1024):
+    """The fp64 oracle layer (forward, then backward) on `tokens` tokens of
+    one sequence at the layer's full widths.  Returns (seconds, FLOPs, desc, threads)."""
+    import oracle
+    from dataclasses import replace
+    from exact_blockwise_long_b200.synthetic import layer_inputs, to_f64
+    small = replace(w, B=1, N=tokens, S=1, q_chunk=tokens, k_chunk=tokens, ffn_chunk=tokens)
+    x, params, dy = layer_inputs(small, device="cpu")
+    xf, pf, dyf = to_f64(x), [to_f64(p_) for p_ in params], to_f64(dy)
+    t0 = time.perf_counter()
+    oracle.layer_forward(xf, pf, 1, tokens, w.H, w.D, w.causal, w.eps)
+    oracle.layer_backward(xf, pf, dyf, 1, tokens, w.H, w.D, w.causal, w.eps)
+    dt = time.perf_counter() - t0
+    proj, af, ffn = layer_flops(small)
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    desc = (f"fp64 oracle (numpy) layer forward+backward of one {tokens}-token sequence at the layer's widths "
+            f"(H={w.H}, d={w.D}, d_ff={w.d_ff}), same recipe; causal FLOPs counted once")
+    return dt, proj + 3.5 * af + ffn, desc, threads
+
+
+def decode_oracle_sample(w, min_seconds=2.0):
+    """The fp64 oracle decode on whole (batch, key/value head) groups of the
+    workload's cache, adding groups until min_seconds of CPU time.
+    Returns (seconds, FLOPs, desc, threads)."""
+    import oracle
+    from dataclasses import replace
+    from exact_blockwise_long_b200.synthetic import decode_inputs, to_f64
+    G = w.H // w.Hkv
+    dt, groups = 0.0, 0
+    while groups == 0 or (dt < min_seconds and groups < w.B * w.Hkv):
+        q, k, v = decode_inputs(replace(w, B=1, H=G, Hkv=1, seed=w.seed + 7919 * groups), device="cpu")
+        q, k, v = to_f64(q), to_f64(k), to_f64(v)
+        t0 = time.perf_counter()
+        oracle.attention_decode(q, k, v)
+        dt += time.perf_counter() - t0
+        groups += 1
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    desc = f"fp64 oracle (numpy) decode of {groups} (batch, key/value head) group(s) of {G} query heads, N={w.N}"
+    return dt, 4.0 * G * w.N * w.D * groups, desc, threads
+
+
+def run_layer(args, ra, dev, rank, world, dist):
+    """One training step of the whole blockwise layer: blockwise_layer_fwd then
+    blockwise_layer_bwd, with per-step events from the library's marks."""
+    import torch
+    from dataclasses import replace
+    from exact_blockwise_long_b200.synthetic import LAYER_WORKLOADS, layer_inputs
+    w = LAYER_WORKLOADS[args.workload]
+    if args.tokens:
+        w = replace(w, N=args.tokens)
+    x, params, dy = layer_inputs(replace(w, seed=w.seed + 1000 * rank), device=dev)
+    saved = torch.empty(ra.blockwise_layer_saved_size(w.B, w.N, w.H, w.D), device=dev, dtype=torch.uint8)
+    fws = torch.empty(ra.blockwise_layer_fwd_workspace_size(w.ffn_chunk, w.d_ff), device=dev, dtype=torch.uint8)
+    bws = torch.empty(ra.blockwise_layer_bwd_workspace_size(w.B, w.N, w.H, w.D, w.d_ff, w.ffn_chunk), device=dev,
+                      dtype=torch.uint8)
+    y, dx = torch.empty_like(x), torch.empty_like(x)
+    grads = tuple(torch.empty(p_.shape, device=dev, dtype=torch.float32) for p_ in params)
+    stream = torch.cuda.current_stream()
+    dims = (w.B, w.N, w.H, w.D, w.S, w.q_chunk, w.k_chunk, w.causal, w.ffn_chunk)
+    n_chunks = w.T // w.ffn_chunk
+    launches_per_step = (7 + 2 * n_chunks) + (4 * n_chunks + 3 + 1 + 1 + 3 + 1 + 3 + 3)
+
+    def event():
+        return torch.cuda.Event(enable_timing=True)
+
+    spans = []
+
+    def step(xx, gy, yy, gx, gr, timed=False):
+        fm = [event() for _ in range(6)] if timed else None
+        bm = [event() for _ in range(10)] if timed else None
+        if timed:
+            s0 = event()
+            s0.record(stream)
+        ra.blockwise_layer_fwd(xx, params, yy, saved, *dims, fws, eps=w.eps, marks=fm)
+        ra.blockwise_layer_bwd(xx, params, saved, gy, gx, gr, *dims, bws, marks=bm)
+        if timed:
+            spans.append((s0, fm, bm))
+
+    for _ in range(args.warmup):
+        step(x, dy, y, dx, grads)
+    torch.cuda.synchronize()
+    if ra.ringattn_get_error() != 0:
+        raise RuntimeError("device status word set during warm-up")
+    clocks = ClockSampler(dev.index)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    a, b = event(), event()
+    a.record(stream)
+    for _ in range(args.steps):
+        step(x, dy, y, dx, grads, timed=True)
+    b.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    if ra.ringattn_get_error() != 0:
+        raise RuntimeError("device status word set during the timed region")
+    ms = max_over_ranks(a.elapsed_time(b) / args.steps, dist if world > 1 else None, dev)
+    proj, af, ffn = layer_flops(w)
+    flops = proj + 3.5 * af + ffn
+    value = whole_job_tflops(flops, world, ms)
+
+    def avg(fn):
+        return sum(fn(s0, fm, bm) for s0, fm, bm in spans) / len(spans)
+
+    kernels = {
+        "fwd_tc2_kernel": (avg(lambda s0, fm, bm: fm[1].elapsed_time(fm[2])), af, "fwd_tc.cu"),
+        "bwd_kv_kernel": (avg(lambda s0, fm, bm: bm[4].elapsed_time(bm[5])), 2.0 * af, "bwd_tc.cu"),
+        "bwd_q_kernel": (avg(lambda s0, fm, bm: bm[5].elapsed_time(bm[6])), 0.5 * af, "bwd_tc.cu"),
+        "gemm_kernel": (avg(lambda s0, fm, bm: fm[0].elapsed_time(fm[1]) + fm[2].elapsed_time(fm[3]) +
+                            bm[1].elapsed_time(bm[3]) + bm[6].elapsed_time(bm[8])), proj, "gemm_tc.cu"),
+        "ffn_tc_kernel+ffn_bwd_gemm_kernel": (avg(lambda s0, fm, bm: fm[4].elapsed_time(fm[5]) +
+                                                  fm[5].elapsed_time(bm[0])), ffn, "ffn_bwd_tc.cu"),
+    }
+    kname = max(kernels, key=lambda k_: kernels[k_][0])
+    kms, kflops, ksrc = kernels[kname]
+    pk = peaks()
+    achieved = kflops / (kms * 1e-3) / 1e12
+    src = os.path.join(ROOT, "exact_blockwise_long_b200", "csrc", ksrc)
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    tr = NCU_TRAFFIC.get((kname, args.workload))
+    roof = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": pk["bf16_sustained"],
+            "unit": "TFLOP/s", "frac": achieved / pk["bf16_sustained"],
+            "traffic": tr["bytes"] if tr and tr["sha256"] == sha else None,
+            "peak_kind": f"bf16 dense, sustained ({pk['source']})", "frac_of_burst": achieved / pk["bf16_burst"],
+            "kernel_ms": kms,
+            "kernels": {k_: {"ms": v_[0], "algorithmic_tflops": v_[1] / (v_[0] * 1e-3) / 1e12}
+                        for k_, v_ in kernels.items()}}
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{w.name}: one blockwise transformer layer fwd+bwd (RMS norms, q/k/v/o "
+                                   f"projections, ring attention, SwiGLU FFN), B={w.B}, N={w.N}, H={w.H}, d={w.D}, "
+                                   f"d_ff={w.d_ff}, S={w.S}, q_chunk={w.q_chunk}, k_chunk={w.k_chunk}, "
+                                   f"ffn_chunk={w.ffn_chunk}, {'causal' if w.causal else 'non-causal'}",
+                       "B": w.B, "seq_len": w.N, "H": w.H, "head_dim": w.D, "d_ff": w.d_ff, "shards": w.S,
+                       "l2": "inputs larger than L2 (no flush between steps)"},
+            "tokens_per_s": w.T * world / (ms * 1e-3), "pct_of_bf16_peak": 100.0 * value / world / pk["bf16_sustained"],
+            "roofline": roof, "gpu_launches": launches_per_step * args.steps, "clocks": clk}
+
+    if not args.no_e2e:
+        # end to end: x and dy in from pinned host memory, y, dx and the nine
+        # parameter gradients back, on copy streams overlapped with compute
+        hin = [t.cpu().pin_memory() for t in (x, dy)]
+        outs0 = [y, dx] + list(grads)
+        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs0]
+        ins = [[x, dy], [torch.empty_like(x), torch.empty_like(dy)]]
+        outs = [outs0, [torch.empty_like(t) for t in outs0]]
+        h2d = sum(t.numel() * t.element_size() for t in hin)
+        d2h = sum(t.numel() * t.element_size() for t in hout)
+        e2e_steps = max(3, min(args.steps, 5))
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        in_ready, done, copied = [event(), event()], [event(), event()], [event(), event()]
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        ea, eb = event(), event()
+        ea.record(stream)
+        s_in.wait_event(ea)
+        for j in range(e2e_steps):
+            bi = j % 2
+            if j >= 2:
+                s_in.wait_event(done[bi])
+            with torch.cuda.stream(s_in):
+                for h_, d_ in zip(hin, ins[bi]):
+                    d_.copy_(h_, non_blocking=True)
+            in_ready[bi].record(s_in)
+            stream.wait_event(in_ready[bi])
+            if j >= 2:
+                stream.wait_event(copied[bi])
+            o_ = outs[bi]
+            step(ins[bi][0], ins[bi][1], o_[0], o_[1], tuple(o_[2:]))
+            done[bi].record(stream)
+            s_out.wait_event(done[bi])
+            with torch.cuda.stream(s_out):
+                for h_, d_ in zip(hout, outs[bi]):
+                    h_.copy_(d_, non_blocking=True)
+            copied[bi].record(s_out)
+        stream.wait_event(copied[(e2e_steps - 1) % 2])
+        stream.wait_event(copied[(e2e_steps - 2) % 2])
+        eb.record(stream)
+        torch.cuda.synchronize()
+        if ra.ringattn_get_error() != 0:
+            raise RuntimeError("device status word set during the end-to-end run")
+        e_ms = max_over_ranks(ea.elapsed_time(eb) / e2e_steps, dist if world > 1 else None, dev)
+        line["e2e"] = {"value": whole_job_tflops(flops, world, e_ms), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h, "ms_per_step": e_ms, "steps": e2e_steps,
+                       "copies": "pinned host, overlapped with compute on two copy streams"}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, fl, desc, threads = layer_oracle_sample(w)
+        line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                "sample": desc, "seconds": dt}
+    return line
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -343,8 +579,9 @@ def main():
     from dataclasses import replace
     from exact_blockwise_long_b200.synthetic import attention_inputs, ffn_inputs
 
-    if args.workload.startswith("decode"):
-        line = run_decode(args, ra, dev, rank, world, dist)
+    if args.workload.startswith("decode") or args.workload == "layer7b_full":
+        runner = run_decode if args.workload.startswith("decode") else run_layer
+        line = runner(args, ra, dev, rank, world, dist)
         if world > 1:
             dist.barrier()
             dist.destroy_process_group()

@@ -54,9 +54,9 @@ SIGNATURES = {
     "blockwise_layer_fwd_workspace_size": (_SZ, [_I64, _I64]),
     "blockwise_layer_bwd_workspace_size": (_SZ, [_I64, _I64, _I64, _I64, _I64, _I64]),
     "blockwise_layer_fwd": (_I, [_P] * 12 + [_SZ, _I64, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _F, _P, _SZ,
-                                             _P]),
+                                             _P, _P]),
     "blockwise_layer_bwd": (_I, [_P] * 11 + [_SZ] + [_P] * 11 + [_I64, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I,
-                                                                  _P, _SZ, _P]),
+                                                                  _P, _SZ, _P, _P]),
     "ringattn_get_error": (_I, [_P]),
     "ringattn_selftest_timeout": (_I, [_I, _P]),
 }

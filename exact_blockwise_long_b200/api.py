@@ -8,6 +8,8 @@ point of the same name on the current CUDA stream, and raises
 
 from __future__ import annotations
 
+import ctypes
+
 import torch
 
 from ._lib import RA_BF16, RA_F32, call, lib
@@ -239,8 +241,19 @@ def _nbytes(t):
     return t.numel() * t.element_size()
 
 
+def _marks(events):
+    """ctypes array of raw cudaEvent_t handles (recorded once so they exist), or None."""
+    if not events:
+        return None
+    for e in events:
+        if e.cuda_event == 0:
+            e.record()
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    return arr
+
+
 def blockwise_layer_fwd(x, weights, y, saved, B, N, H, D, S, q_chunk, k_chunk, causal, ffn_chunk, workspace,
-                        eps=1e-5, stream=None):
+                        eps=1e-5, stream=None, marks=None):
     """y <- the blockwise transformer layer of x ([B*N, H*D] bf16); `saved`
     receives the activations the backward reads.  `weights` is the tuple
     (g_attn, wq, wk, wv, wo, g_ffn, w1, w2, w3)."""
@@ -250,12 +263,12 @@ def blockwise_layer_fwd(x, weights, y, saved, B, N, H, D, S, q_chunk, k_chunk, c
     call("blockwise_layer_fwd", _dev(x, "x"), *[_dev(t, n) for t, n in zip(weights, names)], _dev(y, "y"),
          _dev(saved, "saved"), _nbytes(saved), int(B), int(N), int(H), int(D), d_ff, int(S), int(q_chunk),
          int(k_chunk), int(bool(causal)), int(ffn_chunk), float(eps), _dev(workspace, "workspace"),
-         _nbytes(workspace), _stream(stream))
+         _nbytes(workspace), _marks(marks), _stream(stream))
     return y
 
 
 def blockwise_layer_bwd(x, weights, saved, dy, dx, grads, B, N, H, D, S, q_chunk, k_chunk, causal, ffn_chunk,
-                        workspace, stream=None):
+                        workspace, stream=None, marks=None):
     """dx (bf16) and the fp32 parameter gradients `grads` = (dg_attn, dwq,
     dwk, dwv, dwo, dg_ffn, dw1, dw2, dw3) of sum(dy * layer(x))."""
     names = ("g_attn", "wq", "wk", "wv", "wo", "g_ffn", "w1", "w2", "w3")
@@ -267,7 +280,7 @@ def blockwise_layer_bwd(x, weights, saved, dy, dx, grads, B, N, H, D, S, q_chunk
          _dev(saved, "saved"), _nbytes(saved), _dev(dy, "dy"), _dev(dx, "dx"),
          *[_dev(t, "d" + n) for t, n in zip(grads, names)], int(B), int(N), int(H), int(D), d_ff, int(S),
          int(q_chunk), int(k_chunk), int(bool(causal)), int(ffn_chunk), _dev(workspace, "workspace"),
-         _nbytes(workspace), _stream(stream))
+         _nbytes(workspace), _marks(marks), _stream(stream))
     return dx, grads
 
 

@@ -96,6 +96,13 @@ GemmOut bf16_out(void* p, const void* residual = nullptr) { return GemmOut{p, 0,
 GemmOut bf16_split_out(void* p, int64_t N, int64_t H, int64_t D) { return GemmOut{p, 0, 0, N, H, D, nullptr}; }
 GemmOut f32_out(float* p) { return GemmOut{p, 1, 0, 0, 0, 0, nullptr}; }
 
+// Optional per-step timing marks: event i is recorded on the stream after
+// step i (null array or null entries are skipped).
+int mark(void* const* marks, int i, cudaStream_t st) {
+  if (!marks || !marks[i]) return RA_OK;
+  return cudaEventRecord(static_cast<cudaEvent_t>(marks[i]), st) == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
 size_t bwd_ws_bytes(int64_t B, int64_t N, int64_t H, int64_t D, int64_t d_ff, int64_t ffn_chunk) {
   const size_t T = (size_t)B * N, dm = (size_t)(H * D), act = T * dm * 2;
   size_t attn = (size_t)B * H * N * 4;
@@ -128,7 +135,7 @@ int blockwise_layer_fwd(const void* x, const void* g_attn, const void* wq, const
                         const void* wo, const void* g_ffn, const void* w1, const void* w2, const void* w3, void* y,
                         void* saved, size_t saved_size, int64_t B, int64_t N, int64_t H, int64_t D, int64_t d_ff,
                         int S, int q_chunk, int k_chunk, int causal, int ffn_chunk, float eps, void* workspace,
-                        size_t workspace_bytes, void* stream) {
+                        size_t workspace_bytes, void* const* marks, void* stream) {
   int rc = check_layer(B, N, H, D, d_ff, S, q_chunk, k_chunk, ffn_chunk, causal);
   if (rc != RA_OK) return rc;
   if (!(eps > 0.f)) return RA_ERR_ARG;
@@ -143,21 +150,28 @@ int blockwise_layer_fwd(const void* x, const void* g_attn, const void* wq, const
   const int64_t T = B * N, dm = H * D;
   Saved s = carve_saved(saved, B, N, H, D);
 
+  // steps (marks): 0 norm, 1 q/k/v projections, 2 attention, 3 output projection, 4 norm, 5 feed-forward
   if ((rc = launch_rmsnorm_fwd(x, g_attn, s.xn, s.rstd1, T, dm, eps, st)) != RA_OK) return rc;
+  if ((rc = mark(marks, 0, st)) != RA_OK) return rc;
   const void* w_qkv[3] = {wq, wk, wv};
   __nv_bfloat16* d_qkv[3] = {s.q, s.k, s.v};
   for (int i = 0; i < 3; ++i) {
     GemmSeg g{plain(s.xn, T, dm, 0), plain(w_qkv[i], dm, dm, 0), dm};
     if ((rc = launch_gemm_tc(&g, 1, T, dm, bf16_split_out(d_qkv[i], N, H, D), 1, st)) != RA_OK) return rc;
   }
+  if ((rc = mark(marks, 1, st)) != RA_OK) return rc;
   AttnArgs a{s.q, s.k, s.v, B, H, N, D, RA_BF16, S, q_chunk, k_chunk, causal, 1.0f / sqrtf((float)D), H};
   if ((rc = launch_fwd_tc(a, s.o, s.lse, nullptr, nullptr, -1, st)) != RA_OK) return rc;
+  if ((rc = mark(marks, 2, st)) != RA_OK) return rc;
   {
     GemmSeg g{split(s.o, T, dm, 0, N, H, D), plain(wo, dm, dm, 0), dm};
     if ((rc = launch_gemm_tc(&g, 1, T, dm, bf16_out(s.x2, x), 1, st)) != RA_OK) return rc;
   }
+  if ((rc = mark(marks, 3, st)) != RA_OK) return rc;
   if ((rc = launch_rmsnorm_fwd(s.x2, g_ffn, s.xn2, s.rstd2, T, dm, eps, st)) != RA_OK) return rc;
-  return launch_ffn_tc(s.xn2, w1, w2, w3, y, T, dm, d_ff, ffn_chunk, workspace, st, s.x2);
+  if ((rc = mark(marks, 4, st)) != RA_OK) return rc;
+  if ((rc = launch_ffn_tc(s.xn2, w1, w2, w3, y, T, dm, d_ff, ffn_chunk, workspace, st, s.x2)) != RA_OK) return rc;
+  return mark(marks, 5, st);
 }
 
 int blockwise_layer_bwd(const void* x, const void* g_attn, const void* wq, const void* wk, const void* wv,
@@ -165,7 +179,8 @@ int blockwise_layer_bwd(const void* x, const void* g_attn, const void* wq, const
                         const void* saved, size_t saved_size, const void* dy, void* dx, float* dg_attn, float* dwq,
                         float* dwk, float* dwv, float* dwo, float* dg_ffn, float* dw1, float* dw2, float* dw3,
                         int64_t B, int64_t N, int64_t H, int64_t D, int64_t d_ff, int S, int q_chunk, int k_chunk,
-                        int causal, int ffn_chunk, void* workspace, size_t workspace_bytes, void* stream) {
+                        int causal, int ffn_chunk, void* workspace, size_t workspace_bytes, void* const* marks,
+                        void* stream) {
   int rc = check_layer(B, N, H, D, d_ff, S, q_chunk, k_chunk, ffn_chunk, causal);
   if (rc != RA_OK) return rc;
   const void* ptrs[] = {x,   g_attn, wq,  wk,  wv,     wo,  g_ffn, w1,  w2,  w3,       saved,
@@ -192,22 +207,31 @@ int blockwise_layer_bwd(const void* x, const void* g_attn, const void* wq, const
   void* ws_ffn = c.take<uint8_t>(ffn_bwd_workspace_bytes(ffn_chunk, d_ff));
   float* partial = c.take<float>(rmsnorm_dg_partial_floats(T, dm) * 4);
 
+  // steps (marks): 0 feed-forward, 1 norm, 2 dO, 3 dWo, 4-6 attention (preprocess, dK/dV pass, dQ pass),
+  // 7 dxn, 8 dWq/dWk/dWv, 9 norm
   // feed-forward half: y = x2 + ffn(xn2)
   if ((rc = launch_ffn_bwd_tc(s.xn2, w1, w2, w3, dy, dxn2, dw1, dw2, dw3, T, dm, d_ff, ffn_chunk, ws_ffn, st)) !=
       RA_OK)
     return rc;
+  if ((rc = mark(marks, 0, st)) != RA_OK) return rc;
   if ((rc = launch_rmsnorm_bwd(s.x2, g_ffn, s.rstd2, dxn2, dy, dx2, dg_ffn, partial, T, dm, st)) != RA_OK) return rc;
+  if ((rc = mark(marks, 1, st)) != RA_OK) return rc;
   // attention half: x2 = x + o Wo^T
   {
     GemmSeg g{plain(dx2, T, dm, 0), plain(wo, dm, dm, 1), dm};  // dO = dx2 Wo
     if ((rc = launch_gemm_tc(&g, 1, T, dm, bf16_split_out(dO, N, H, D), 1, st)) != RA_OK) return rc;
   }
+  if ((rc = mark(marks, 2, st)) != RA_OK) return rc;
   {
     GemmSeg g{plain(dx2, T, dm, 1), split(s.o, T, dm, 1, N, H, D), T};  // dWo = dx2^T o
     if ((rc = launch_gemm_tc(&g, 1, dm, dm, f32_out(dwo), 1, st)) != RA_OK) return rc;
   }
+  if ((rc = mark(marks, 3, st)) != RA_OK) return rc;
   AttnArgs a{s.q, s.k, s.v, B, H, N, D, RA_BF16, S, q_chunk, k_chunk, causal, 1.0f / sqrtf((float)D), H};
-  if ((rc = launch_bwd_tc(a, s.o, s.lse, dO, dq, dk, dv, ws_attn, 7, st)) != RA_OK) return rc;
+  for (int ph = 0; ph < 3; ++ph) {
+    if ((rc = launch_bwd_tc(a, s.o, s.lse, dO, dq, dk, dv, ws_attn, 1 << ph, st)) != RA_OK) return rc;
+    if ((rc = mark(marks, 4 + ph, st)) != RA_OK) return rc;
+  }
   {
     // dxn = dq Wq + dk Wk + dv Wv (one accumulation over three K ranges)
     GemmSeg g[3] = {{split(dq, T, dm, 0, N, H, D), plain(wq, dm, dm, 1), dm},
@@ -215,13 +239,16 @@ int blockwise_layer_bwd(const void* x, const void* g_attn, const void* wq, const
                     {split(dv, T, dm, 0, N, H, D), plain(wv, dm, dm, 1), dm}};
     if ((rc = launch_gemm_tc(g, 3, T, dm, bf16_out(dxn), 1, st)) != RA_OK) return rc;
   }
+  if ((rc = mark(marks, 7, st)) != RA_OK) return rc;
   const __nv_bfloat16* gq[3] = {dq, dk, dv};
   float* gw[3] = {dwq, dwk, dwv};
   for (int i = 0; i < 3; ++i) {
     GemmSeg g{split(gq[i], T, dm, 1, N, H, D), plain(s.xn, T, dm, 1), T};  // dW = d(q|k|v)^T xn
     if ((rc = launch_gemm_tc(&g, 1, dm, dm, f32_out(gw[i]), 1, st)) != RA_OK) return rc;
   }
-  return launch_rmsnorm_bwd(x, g_attn, s.rstd1, dxn, dx2, dx, dg_attn, partial, T, dm, st);
+  if ((rc = mark(marks, 8, st)) != RA_OK) return rc;
+  if ((rc = launch_rmsnorm_bwd(x, g_attn, s.rstd1, dxn, dx2, dx, dg_attn, partial, T, dm, st)) != RA_OK) return rc;
+  return mark(marks, 9, st);
 }
 
 }  // extern "C"

@@ -342,6 +342,11 @@ RA_API int blockwise_ffn_bwd(const void* x, const void* w1, const void* w2, cons
  * multiples of 128); (B*N) % ffn_chunk == 0, ffn_chunk and d_ff multiples
  * of 128; every pointer 16-byte aligned.  Errors: RA_ERR_ARG, RA_ERR_SHAPE,
  * RA_ERR_UNSUPPORTED, RA_ERR_ALIGN, RA_ERR_WORKSPACE, RA_ERR_CUDA.
+ * marks: optional array of cudaEvent_t (null, or null entries, to skip);
+ * entry i is recorded on `stream` after step i -- forward: 0 norm, 1 q/k/v
+ * projections, 2 attention, 3 output projection, 4 norm, 5 feed-forward;
+ * backward: 0 feed-forward, 1 norm, 2 dO, 3 dWo, 4 attention preprocess,
+ * 5 dK/dV pass, 6 dQ pass, 7 dxn, 8 dWq/dWk/dWv, 9 norm.
  * ------------------------------------------------------------------------- */
 RA_API size_t blockwise_layer_saved_size(int64_t B, int64_t N, int64_t H, int64_t D);
 RA_API size_t blockwise_layer_fwd_workspace_size(int64_t ffn_chunk, int64_t d_ff);
@@ -351,14 +356,15 @@ RA_API int blockwise_layer_fwd(const void* x, const void* g_attn, const void* wq
                                const void* wo, const void* g_ffn, const void* w1, const void* w2, const void* w3,
                                void* y, void* saved, size_t saved_bytes, int64_t B, int64_t N, int64_t H,
                                int64_t D, int64_t d_ff, int S, int q_chunk, int k_chunk, int causal, int ffn_chunk,
-                               float eps, void* workspace, size_t workspace_bytes, void* stream);
+                               float eps, void* workspace, size_t workspace_bytes, void* const* marks,
+                               void* stream);
 RA_API int blockwise_layer_bwd(const void* x, const void* g_attn, const void* wq, const void* wk, const void* wv,
                                const void* wo, const void* g_ffn, const void* w1, const void* w2, const void* w3,
                                const void* saved, size_t saved_bytes, const void* dy, void* dx, float* dg_attn,
                                float* dwq, float* dwk, float* dwv, float* dwo, float* dg_ffn, float* dw1,
                                float* dw2, float* dw3, int64_t B, int64_t N, int64_t H, int64_t D, int64_t d_ff,
                                int S, int q_chunk, int k_chunk, int causal, int ffn_chunk, void* workspace,
-                               size_t workspace_bytes, void* stream);
+                               size_t workspace_bytes, void* const* marks, void* stream);
 
 /*
  * ringattn_get_error -- synchronise `stream`, return the device status word
