@@ -401,8 +401,8 @@ def run_layer(args, ra, dev, rank, world, dist):
     from dataclasses import replace
     from exact_blockwise_long_b200.synthetic import LAYER_WORKLOADS, layer_inputs
     w = LAYER_WORKLOADS[args.workload]
-    if args.tokens:
-        w = replace(w, N=args.tokens)
+    if args.tokens:  # a shorter sequence with the same shard length (smaller profiling cases)
+        w = replace(w, N=args.tokens, S=max(1, args.tokens // (w.N // w.S)))
     x, params, dy = layer_inputs(replace(w, seed=w.seed + 1000 * rank), device=dev)
     saved = torch.empty(ra.blockwise_layer_saved_size(w.B, w.N, w.H, w.D), device=dev, dtype=torch.uint8)
     fws = torch.empty(ra.blockwise_layer_fwd_workspace_size(w.ffn_chunk, w.d_ff), device=dev, dtype=torch.uint8)

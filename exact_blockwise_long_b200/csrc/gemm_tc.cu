@@ -14,7 +14,8 @@
 // coordinates are remapped per box, so no transpose kernel exists.
 //
 // One CTA computes one 128 x 256 output tile (tcgen05 M=128, N=256, fp32 in
-// 256 TMEM columns) over a 4-stage TMA ring of 64-deep K slabs.  Epilogues:
+// 256 TMEM columns) over a 4-stage TMA ring of 64-deep K slabs (3 stages
+// when a residual tile is prefetched).  Epilogues:
 // bf16 (optionally + a bf16 residual tile) or fp32 (store, or element-wise
 // TMA add onto a zeroed output when the K range is split across two CTAs;
 // two addends onto zero commute exactly, so the result is deterministic).
@@ -26,16 +27,26 @@ namespace ra {
 namespace {
 
 constexpr int kBM = 128, kBN = 256, kBK = 64;
-constexpr int kStages = 4;
 constexpr int kThreads = 256;
 constexpr int kATile = kBM * kBK * 2;  // 16 KB
 constexpr int kBTile = kBN * kBK * 2;  // 32 KB
 constexpr int kStage = kATile + kBTile;
-constexpr int kBarOff = kStages * kStage;
-constexpr int kTmemSlot = kBarOff + (2 * kStages + 2) * 8;
-constexpr int kAbortOff = kTmemSlot + 4;
-constexpr int kSmemBytes = kAbortOff + 4 + 1024;
 constexpr int kBox = 16384;  // one epilogue staging box: 128 rows x 128 bytes
+
+// Shared-memory layout per epilogue: a 4-stage ring; with a residual, a
+// 3-stage ring plus the residual tile (prefetched at the start, then
+// overwritten in place by the output tile).
+template <int EPI>
+struct GLay {
+  static constexpr int kStages = EPI == 1 ? 3 : 4;
+  static constexpr int kResOff = kStages * kStage;
+  static constexpr int kBarOff = kResOff + (EPI == 1 ? 4 * kBox : 0);
+  static constexpr int kTmemSlot = kBarOff + (2 * kStages + 2) * 8;
+  static constexpr int kAbortOff = kTmemSlot + 4;
+  static constexpr int kSmemBytes = kAbortOff + 4 + 1024;
+  static_assert(kSmemBytes <= 232448, "GEMM stages exceed shared memory");
+  static_assert(EPI != 2 || 8 * kBox <= kResOff, "fp32 staging exceeds the pipeline buffers");
+};
 
 struct OpGeo {
   int hs;                  // head-split storage
@@ -47,7 +58,8 @@ struct GemmParams {
   OpGeo a[3], b[3];
   int seg_end[3];          // cumulative K steps at the end of each segment
   OpGeo out;               // output (bf16 only may be head-split)
-  int m_tiles;
+  int m_tiles, n_tiles;
+  int n_fast;              // raster: consecutive CTAs share the A tile (n fastest) or the B tile
   int kb_per_split;        // K steps per blockIdx.y
   int kb_total;
   int f32_add;             // fp32 output: TMA add instead of store
@@ -101,22 +113,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const __grid_constant__ CUtensorMap tB1, const __grid_constant__ CUtensorMap tB2,
                 const __grid_constant__ CUtensorMap tOut, const __grid_constant__ CUtensorMap tRes,
                 const GemmParams p) {
+  using LY = GLay<EPI>;
+  constexpr int kStages = LY::kStages;
   extern __shared__ uint8_t smem_g[];
   uint8_t* smem = smem_g + ((1024 - (smem_u32(smem_g) & 1023)) & 1023);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int mt = (int)(blockIdx.x % p.m_tiles);
-  const int nt = (int)(blockIdx.x / p.m_tiles);
+  const int mt = p.n_fast ? (int)(blockIdx.x / p.n_tiles) : (int)(blockIdx.x % p.m_tiles);
+  const int nt = p.n_fast ? (int)(blockIdx.x % p.n_tiles) : (int)(blockIdx.x / p.m_tiles);
   const int kb0 = (int)blockIdx.y * p.kb_per_split;
   const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + LY::kBarOff);
   uint64_t* bar_full = bars;
   uint64_t* bar_empty = bars + kStages;
   uint64_t* bar_done = bars + 2 * kStages;
   uint64_t* bar_res = bars + 2 * kStages + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTmemSlot);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kAbortOff);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + LY::kTmemSlot);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LY::kAbortOff);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -139,6 +153,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
+      if (EPI == 1 && p.has_residual) {  // residual tile [128 rows x 256 cols], needed only by the epilogue
+        mbar_arrive_expect_tx(bar_res, 4 * kBox);
+        for (int j = 0; j < 4; ++j)
+          tma_load_2d(smem + LY::kResOff + j * kBox, &tRes, bar_res, nt * kBN + j * 64, mt * kBM);
+      }
       for (int kb = kb0; kb < kb1; ++kb) {
         const int i = kb - kb0;
         const int s = i % kStages;
@@ -175,18 +194,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // buffers -> TMA store / add
     const int r = (warp - 4) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t row_base = smem_u32(smem) + (uint32_t)r * 128;
+    // output boxes: the drained pipeline buffers, or the residual tile in place
+    const uint32_t stage_base = smem_u32(smem) + (EPI == 1 ? LY::kResOff : 0);
+    const uint32_t row_base = stage_base + (uint32_t)r * 128;
     const uint32_t sw = (uint32_t)(r & 7);
     int ox, oy;
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, p.st, abort_flag));
-    if (EPI == 1 && p.has_residual) {
-      // residual tile [128 rows x 256 cols] into boxes 0-3 (the pipeline is drained)
-      if (threadIdx.x == 128 && ok) {
-        mbar_arrive_expect_tx(bar_res, 4 * kBox);
-        for (int j = 0; j < 4; ++j) tma_load_2d(smem + j * kBox, &tRes, bar_res, nt * kBN + j * 64, mt * kBM);
-      }
-      ok = __all_sync(0xffffffffu, ok && mbar_wait(bar_res, 0, p.st, abort_flag));
-    }
+    if (EPI == 1 && p.has_residual) ok = __all_sync(0xffffffffu, ok && mbar_wait(bar_res, 0, p.st, abort_flag));
     if (ok) {
       tc_fence_after();
 #pragma unroll 1
@@ -233,18 +247,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     named_bar_sync(1, 128);
     if (threadIdx.x == 128 && ok) {
+      const uint8_t* stage = smem + (EPI == 1 ? LY::kResOff : 0);
       if constexpr (EPI == 2) {
         for (int c = 0; c < kBN / 32; ++c) {
           op_coord(p.out, mt * kBM, nt * kBN + c * 32, ox, oy);
           if (p.f32_add)
-            tma_add_2d(&tOut, smem + c * kBox, ox, oy);
+            tma_add_2d(&tOut, stage + c * kBox, ox, oy);
           else
-            tma_store_2d(&tOut, smem + c * kBox, ox, oy);
+            tma_store_2d(&tOut, stage + c * kBox, ox, oy);
         }
       } else {
         for (int j = 0; j < 4; ++j) {
           op_coord(p.out, mt * kBM, nt * kBN + j * 64, ox, oy);
-          tma_store_2d(&tOut, smem + j * kBox, ox, oy);
+          tma_store_2d(&tOut, stage + j * kBox, ox, oy);
         }
       }
       bulk_commit_group();
@@ -283,6 +298,7 @@ int operand_map(CUtensorMap* m, const GemmOperand& o, bool mn_major) {
 
 template <bool A_MN, bool B_MN, int EPI>
 int launch_typed(const CUtensorMap* maps, const GemmParams& p, dim3 grid, cudaStream_t stream) {
+  constexpr int kSmemBytes = GLay<EPI>::kSmemBytes;
   auto kern = gemm_kernel<A_MN, B_MN, EPI>;
   if (set_smem_attr((const void*)kern, kSmemBytes) != RA_OK) return RA_ERR_CUDA;
   kern<<<grid, kThreads, kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6],
@@ -290,8 +306,6 @@ int launch_typed(const CUtensorMap* maps, const GemmParams& p, dim3 grid, cudaSt
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
-static_assert(kSmemBytes <= 232448, "GEMM stages exceed shared memory");
-static_assert(8 * kBox <= kBarOff, "fp32 staging exceeds the pipeline buffers");
 
 }  // namespace
 
@@ -319,6 +333,11 @@ int launch_gemm_tc(const GemmSeg* segs, int nseg, int64_t M, int64_t N, const Ge
   if (out.f32 && out.hs_ntok > 0) return RA_ERR_UNSUPPORTED;
   p.out = geo_of(GemmOperand{out.ptr, M, N, 0, out.hs_ntok, out.hs_heads, out.hs_d, 0, 0});
   p.m_tiles = (int)(M / kBM);
+  p.n_tiles = (int)(N / kBN);
+  // Concurrent CTAs should share the larger operand's tiles: with M >= N the
+  // A rows (activations) are re-read from L2 by the n tiles running together
+  // and the smaller B stays L2-resident.
+  p.n_fast = M >= N;
   p.kb_total = kb;
   if (kb < splits) return RA_ERR_SHAPE;  // every split needs at least one K step
   p.kb_per_split = (kb + splits - 1) / splits;

@@ -96,6 +96,14 @@ GemmOut bf16_out(void* p, const void* residual = nullptr) { return GemmOut{p, 0,
 GemmOut bf16_split_out(void* p, int64_t N, int64_t H, int64_t D) { return GemmOut{p, 0, 0, N, H, D, nullptr}; }
 GemmOut f32_out(float* p) { return GemmOut{p, 1, 0, 0, 0, 0, nullptr}; }
 
+// Weight gradients [dm, dm] have few output tiles and a long K (all tokens):
+// split K in two (two fp32 adds onto a zeroed output commute exactly) when
+// the tiles alone would leave SMs idle in the last wave.
+int wgrad_splits(int64_t dm, int64_t T) {
+  const int64_t tiles = (dm / 128) * (dm / 256);
+  return (tiles < 4 * 148 && T >= 1024) ? 2 : 1;
+}
+
 // Optional per-step timing marks: event i is recorded on the stream after
 // step i (null array or null entries are skipped).
 int mark(void* const* marks, int i, cudaStream_t st) {
@@ -224,7 +232,7 @@ int blockwise_layer_bwd(const void* x, const void* g_attn, const void* wq, const
   if ((rc = mark(marks, 2, st)) != RA_OK) return rc;
   {
     GemmSeg g{plain(dx2, T, dm, 1), split(s.o, T, dm, 1, N, H, D), T};  // dWo = dx2^T o
-    if ((rc = launch_gemm_tc(&g, 1, dm, dm, f32_out(dwo), 1, st)) != RA_OK) return rc;
+    if ((rc = launch_gemm_tc(&g, 1, dm, dm, f32_out(dwo), wgrad_splits(dm, T), st)) != RA_OK) return rc;
   }
   if ((rc = mark(marks, 3, st)) != RA_OK) return rc;
   AttnArgs a{s.q, s.k, s.v, B, H, N, D, RA_BF16, S, q_chunk, k_chunk, causal, 1.0f / sqrtf((float)D), H};
@@ -244,7 +252,7 @@ int blockwise_layer_bwd(const void* x, const void* g_attn, const void* wq, const
   float* gw[3] = {dwq, dwk, dwv};
   for (int i = 0; i < 3; ++i) {
     GemmSeg g{split(gq[i], T, dm, 1, N, H, D), plain(s.xn, T, dm, 1), T};  // dW = d(q|k|v)^T xn
-    if ((rc = launch_gemm_tc(&g, 1, dm, dm, f32_out(gw[i]), 1, st)) != RA_OK) return rc;
+    if ((rc = launch_gemm_tc(&g, 1, dm, dm, f32_out(gw[i]), wgrad_splits(dm, T), st)) != RA_OK) return rc;
   }
   if ((rc = mark(marks, 8, st)) != RA_OK) return rc;
   if ((rc = launch_rmsnorm_bwd(x, g_attn, s.rstd1, dxn, dx2, dx, dg_attn, partial, T, dm, st)) != RA_OK) return rc;
