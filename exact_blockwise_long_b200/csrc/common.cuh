@@ -362,6 +362,32 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
   return d;
 }
 
+// 2^x for two values on the FMA and integer pipes instead of the MUFU (valid
+// for x <= 64; softmax arguments are <= 8).  Range reduction: x = j + f with
+// j = round-to-nearest(x), |f| <= 1/2, taken by adding 1.5 * 2^23 (the sum's
+// low mantissa bits are then j).  2^f comes from the cubic
+// 1 + f (c1 + f (c2 + f c3)), a minimax fit of relative error on [-1/2, 1/2]
+// made for this kernel (Lawson-reweighted least squares; max relative error
+// 1.02e-4, exact at f = 0).  2^j is applied by adding j to the exponent
+// field: the sum's bit pattern shifted left by 23 is j << 23 modulo 2^32.
+// x is clamped at -127 first, so the exponent field never wraps: the result
+// is then 0 or a denormal (masked scores, -inf, give exactly 0).
+constexpr float kEx2C1 = 0.69328284f, kEx2C2 = 0.24220967f, kEx2C3 = 0.0550084f;
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -127.f);
+  x.y = fmaxf(x.y, -127.f);
+  const float2 jm = add2(x, make_float2(kShift, kShift));
+  const float2 j = add2(jm, make_float2(-kShift, -kShift));
+  const float2 f = add2(x, make_float2(-j.x, -j.y));
+  float2 p = fma2(make_float2(kEx2C3, kEx2C3), f, make_float2(kEx2C2, kEx2C2));
+  p = fma2(p, f, make_float2(kEx2C1, kEx2C1));
+  p = fma2(p, f, make_float2(1.f, 1.f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(jm.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(jm.y) << 23)));
+}
+
+
 // Two floats to a packed bf16x2 (round to nearest even); lo in bits 0-15.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;

@@ -150,6 +150,11 @@ __device__ __forceinline__ float row_max(const float (&s)[kBN]) {
 // P = 2^(s * scale * log2(e) - m) as bf16 pairs over the first 64 columns of
 // the tile's TMEM (P of keys 2c, 2c+1 in column c); returns the row sum of
 // the fp32 probabilities.  Masked scores are -inf and give exactly 0.
+// One pair in kEx2PolyEvery is computed by ex2_poly2 on the FMA/integer
+// pipes, the rest by the MUFU: each 128 x 128 tile needs as many MUFU cycles
+// for its exponentials as tensor cycles for its two matmuls, so moving part
+// of them off the MUFU shortens the softmax's critical path.
+constexpr int kEx2PolyEvery = 4;
 __device__ __forceinline__ float exp_store(const float (&s)[kBN], uint32_t tS, float sl2, float m) {
   const float2 k2 = make_float2(sl2, sl2), nm2 = make_float2(-m, -m);
   float2 acc[4];
@@ -161,7 +166,8 @@ __device__ __forceinline__ float exp_store(const float (&s)[kBN], uint32_t tS, f
 #pragma unroll
     for (int x = 0; x < 32; ++x) {
       const float2 t = fma2(make_float2(s[h * 64 + 2 * x], s[h * 64 + 2 * x + 1]), k2, nm2);
-      const float2 pr = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+      const float2 pr = (x % kEx2PolyEvery == kEx2PolyEvery - 1) ? ex2_poly2(t)
+                                                                : make_float2(ex2_approx(t.x), ex2_approx(t.y));
       acc[x & 3] = add2(acc[x & 3], pr);
       pk[x] = pack_bf16x2(pr.x, pr.y);
     }
