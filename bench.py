@@ -413,7 +413,9 @@ def run_layer(args, ra, dev, rank, world, dist):
     stream = torch.cuda.current_stream()
     dims = (w.B, w.N, w.H, w.D, w.S, w.q_chunk, w.k_chunk, w.causal, w.ffn_chunk)
     n_chunks = w.T // w.ffn_chunk
-    launches_per_step = (7 + 2 * n_chunks) + (4 * n_chunks + 3 + 1 + 1 + 3 + 1 + 3 + 3)
+    # forward: norm, 3 projections, attention, o projection, norm, 2 GEMMs per FFN chunk;
+    # backward: 6 GEMMs per FFN chunk, norm (3), dO, dWo, attention (3), dxn, 3 dW, norm (3)
+    launches_per_step = (7 + 2 * n_chunks) + (6 * n_chunks + 3 + 1 + 1 + 3 + 1 + 3 + 3)
 
     def event():
         return torch.cuda.Event(enable_timing=True)
@@ -660,7 +662,7 @@ def main():
                 e[5].record(stream)
             ra.blockwise_ffn(x, w1, w2, w3, y, fw.chunk, ffn_ws)
             ra.blockwise_ffn_bwd(x, w1, w2, w3, dy, dx, dw1, dw2, dw3, fw.chunk, ffn_bws)
-            launches += 6 * (fw.T // fw.chunk)  # forward: 2 per chunk, backward: 4 per chunk
+            launches += 8 * (fw.T // fw.chunk)  # forward: 2 GEMMs per chunk, backward: 6 per chunk
             if timed:
                 e[6].record(stream)
                 ev.setdefault("ffn", []).append((e[5], e[6]))

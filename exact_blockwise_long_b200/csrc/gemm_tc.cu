@@ -1,8 +1,7 @@
-// bf16 GEMM on the sm_100a tensor cores for the projections of the blockwise
-// transformer layer ("Ring Attention with Blockwise Transformers", abstract:
-// the layer -- attention and feed-forward -- is computed blockwise; the
-// query/key/value and output projections around the attention are plain
-// per-token matmuls).
+// bf16 GEMM engine on the sm_100a tensor cores for the blockwise transformer
+// layer ("Ring Attention with Blockwise Transformers", abstract: the layer --
+// attention and feed-forward -- is computed blockwise; the projections around
+// the attention and the feed-forward's matmuls are plain per-token GEMMs).
 //
 //   D[M, N] = sum over up to three segments s of A_s[M, K_s] . B_s[N, K_s]^T
 //
@@ -11,15 +10,26 @@
 // (logical rows index K, columns index M or N: an operand used transposed).
 // A logical [tokens, heads*d] matrix may be stored head-split as
 // [batch, heads, tokens per sequence, d] (the attention layout): the load
-// coordinates are remapped per box, so no transpose kernel exists.
+// and store coordinates are remapped per box, so no transpose kernel exists.
 //
-// One CTA computes one 128 x 256 output tile (tcgen05 M=128, N=256, fp32 in
-// 256 TMEM columns) over a 4-stage TMA ring of 64-deep K slabs (3 stages
-// when a residual tile is prefetched).  Epilogues:
-// bf16 (optionally + a bf16 residual tile) or fp32 (store, or element-wise
-// TMA add onto a zeroed output when the K range is split across two CTAs;
-// two addends onto zero commute exactly, so the result is deterministic).
+// One CTA computes one 128 x 256 accumulator tile (tcgen05 M=128, N=256,
+// fp32 in 256 TMEM columns) over a TMA ring of 64-deep K slabs.  Epilogues
+// (results leave through 128-byte-swizzled staging boxes and TMA stores):
+//   kEpiBf16       bf16 tile
+//   kEpiBf16Res    bf16 tile + a bf16 residual tile (prefetched at start)
+//   kEpiF32        fp32 tile, stored or element-wise TMA-added (the K range
+//                  may be split across two CTAs adding onto a zeroed output:
+//                  two addends onto zero commute exactly, so it stays
+//                  deterministic)
+//   kEpiSwiGLU     B is stacked: rows 0-127 from w1, 128-255 from w3 (the same
+//                  hidden units), so the accumulator holds g | u and the tile
+//                  leaves as h = silu(g) * u  [128 x 128]
+//   kEpiSwiGLUBwd  the same g | u, plus a prefetched fp32 dh tile:
+//                  dg = dh u s (1 + g (1 - s)), du = dh g s, h = g s u,
+//                  s = 1 / (1 + e^-g)  (three bf16 tiles)
 // Warp roles: 0 TMA producer, 1 MMA issuer, 2 TMEM allocator, 4-7 epilogue.
+#include <math.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -31,21 +41,22 @@ constexpr int kThreads = 256;
 constexpr int kATile = kBM * kBK * 2;  // 16 KB
 constexpr int kBTile = kBN * kBK * 2;  // 32 KB
 constexpr int kStage = kATile + kBTile;
-constexpr int kBox = 16384;  // one epilogue staging box: 128 rows x 128 bytes
+constexpr int kBox = 16384;  // one staging box: 128 rows x 128 bytes
 
-// Shared-memory layout per epilogue: a 4-stage ring; with a residual, a
-// 3-stage ring plus the residual tile (prefetched at the start, then
-// overwritten in place by the output tile).
+// Shared memory per epilogue: a 4-stage ring; with an auxiliary input tile
+// (residual, dh) a 3-stage ring plus that tile (64 KB).
 template <int EPI>
 struct GLay {
-  static constexpr int kStages = EPI == 1 ? 3 : 4;
-  static constexpr int kResOff = kStages * kStage;
-  static constexpr int kBarOff = kResOff + (EPI == 1 ? 4 * kBox : 0);
+  static constexpr bool kAux = EPI == kEpiBf16Res || EPI == kEpiSwiGLUBwd;
+  static constexpr int kStages = kAux ? 3 : 4;
+  static constexpr int kAuxOff = kStages * kStage;
+  static constexpr int kBarOff = kAuxOff + (kAux ? 4 * kBox : 0);
   static constexpr int kTmemSlot = kBarOff + (2 * kStages + 2) * 8;
   static constexpr int kAbortOff = kTmemSlot + 4;
   static constexpr int kSmemBytes = kAbortOff + 4 + 1024;
   static_assert(kSmemBytes <= 232448, "GEMM stages exceed shared memory");
-  static_assert(EPI != 2 || 8 * kBox <= kResOff, "fp32 staging exceeds the pipeline buffers");
+  static_assert(EPI != kEpiF32 || 8 * kBox <= kAuxOff, "fp32 staging exceeds the pipeline buffers");
+  static_assert(EPI != kEpiSwiGLUBwd || 6 * kBox <= kAuxOff, "staging exceeds the pipeline buffers");
 };
 
 struct OpGeo {
@@ -54,16 +65,23 @@ struct OpGeo {
   int r0, c0;              // origin of the operand in its logical matrix
 };
 
+struct GemmMaps {
+  CUtensorMap a[3], b[3];  // per segment (b[1] is the stacked half for the SwiGLU epilogues)
+  CUtensorMap out[3];      // outputs
+  CUtensorMap aux;         // residual (bf16) or dh (fp32)
+};
+
 struct GemmParams {
   OpGeo a[3], b[3];
   int seg_end[3];          // cumulative K steps at the end of each segment
-  OpGeo out;               // output (bf16 only may be head-split)
+  OpGeo out;               // output geometry (bf16 only may be head-split)
   int m_tiles, n_tiles;
   int n_fast;              // raster: consecutive CTAs share the A tile (n fastest) or the B tile
   int kb_per_split;        // K steps per blockIdx.y
   int kb_total;
   int f32_add;             // fp32 output: TMA add instead of store
-  int has_residual;
+  int has_aux;
+  int n_valid;             // output columns; boxes of a half-full last tile past it are not stored
   DevStatus st;
 };
 
@@ -106,15 +124,23 @@ __device__ __forceinline__ uint64_t tile_desc(uint32_t tile, int kk) {
   return MN ? sdesc_sw128(tile + kk * 2048, 8192, 1024) : sdesc_sw128(tile + kk * 32, 16, 1024);
 }
 
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 q;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(q.x), "=r"(q.y), "=r"(q.z), "=r"(q.w) : "r"(addr));
+  return q;
+}
+
+// eight floats -> four packed bf16 pairs -> one swizzled 16-byte unit
+__device__ __forceinline__ void st_unit_bf16(uint32_t row_base_box, uint32_t unit, uint32_t sw, const float* v) {
+  st_shared_v4(row_base_box + ((unit ^ sw) << 4), pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+               pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+}
+
 template <bool A_MN, bool B_MN, int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tA1,
-                const __grid_constant__ CUtensorMap tA2, const __grid_constant__ CUtensorMap tB0,
-                const __grid_constant__ CUtensorMap tB1, const __grid_constant__ CUtensorMap tB2,
-                const __grid_constant__ CUtensorMap tOut, const __grid_constant__ CUtensorMap tRes,
-                const GemmParams p) {
+__global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   using LY = GLay<EPI>;
   constexpr int kStages = LY::kStages;
+  constexpr bool kSwi = EPI == kEpiSwiGLU || EPI == kEpiSwiGLUBwd;
   extern __shared__ uint8_t smem_g[];
   uint8_t* smem = smem_g + ((1024 - (smem_u32(smem_g) & 1023)) & 1023);
   const int warp = threadIdx.x >> 5;
@@ -123,12 +149,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nt = p.n_fast ? (int)(blockIdx.x % p.n_tiles) : (int)(blockIdx.x / p.m_tiles);
   const int kb0 = (int)blockIdx.y * p.kb_per_split;
   const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
+  // output columns per tile: 128 for the SwiGLU epilogues (g | u halves), else 256
+  constexpr int kOutN = kSwi ? 128 : kBN;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + LY::kBarOff);
   uint64_t* bar_full = bars;
   uint64_t* bar_empty = bars + kStages;
   uint64_t* bar_done = bars + 2 * kStages;
-  uint64_t* bar_res = bars + 2 * kStages + 1;
+  uint64_t* bar_aux = bars + 2 * kStages + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + LY::kTmemSlot);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LY::kAbortOff);
 
@@ -138,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar_empty[s], 1);
     }
     mbar_init(bar_done, 1);
-    mbar_init(bar_res, 1);
+    mbar_init(bar_aux, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -153,10 +181,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      if (EPI == 1 && p.has_residual) {  // residual tile [128 rows x 256 cols], needed only by the epilogue
-        mbar_arrive_expect_tx(bar_res, 4 * kBox);
-        for (int j = 0; j < 4; ++j)
-          tma_load_2d(smem + LY::kResOff + j * kBox, &tRes, bar_res, nt * kBN + j * 64, mt * kBM);
+      if (LY::kAux && p.has_aux) {  // the epilogue's input tile, fetched while the main loop runs
+        mbar_arrive_expect_tx(bar_aux, 4 * kBox);
+        for (int j = 0; j < 4; ++j) {
+          // residual: 4 x 64 bf16 columns; dh: 4 x 32 fp32 columns
+          const int x = EPI == kEpiBf16Res ? nt * kBN + j * 64 : nt * 128 + j * 32;
+          tma_load_2d(smem + LY::kAuxOff + j * kBox, &maps.aux, bar_aux, x, mt * kBM);
+        }
       }
       for (int kb = kb0; kb < kb1; ++kb) {
         const int i = kb - kb0;
@@ -164,12 +195,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&bar_empty[s], ((i / kStages) & 1) ^ 1, p.st, abort_flag)) break;
         const int seg = (kb >= p.seg_end[0]) + (kb >= p.seg_end[1]);
         const int k = kb - (seg ? p.seg_end[seg - 1] : 0);
-        const CUtensorMap* ma = seg == 0 ? &tA0 : (seg == 1 ? &tA1 : &tA2);
-        const CUtensorMap* mb = seg == 0 ? &tB0 : (seg == 1 ? &tB1 : &tB2);
         uint8_t* st = smem + s * kStage;
         mbar_arrive_expect_tx(&bar_full[s], kStage);
-        load_tile<A_MN, kBM>(st, ma, &bar_full[s], p.a[seg], mt * kBM, k);
-        load_tile<B_MN, kBN>(st + kATile, mb, &bar_full[s], p.b[seg], nt * kBN, k);
+        load_tile<A_MN, kBM>(st, &maps.a[seg], &bar_full[s], p.a[seg], mt * kBM, k);
+        if constexpr (kSwi) {  // 128 rows of w1, then the same 128 rows of w3
+          load_tile<false, 128>(st + kATile, &maps.b[0], &bar_full[s], p.b[0], nt * 128, k);
+          load_tile<false, 128>(st + kATile + 16384, &maps.b[1], &bar_full[s], p.b[1], nt * 128, k);
+        } else {
+          load_tile<B_MN, kBN>(st + kATile, &maps.b[seg], &bar_full[s], p.b[seg], nt * kBN, k);
+        }
       }
     }
   } else if (warp == 1) {
@@ -190,42 +224,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(bar_done);
     }
   } else if (warp >= 4) {
-    // accumulator rows -> swizzled 16 KB staging boxes in the idle pipeline
-    // buffers -> TMA store / add
+    // accumulator rows -> swizzled staging boxes -> TMA stores / adds.
+    // Staging: the drained pipeline buffers, or for kEpiBf16Res the residual
+    // tile itself (each thread overwrites only what it has read).
     const int r = (warp - 4) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    // output boxes: the drained pipeline buffers, or the residual tile in place
-    const uint32_t stage_base = smem_u32(smem) + (EPI == 1 ? LY::kResOff : 0);
+    const uint32_t stage_base = smem_u32(smem) + (EPI == kEpiBf16Res ? LY::kAuxOff : 0);
     const uint32_t row_base = stage_base + (uint32_t)r * 128;
+    const uint32_t aux_row = smem_u32(smem) + LY::kAuxOff + (uint32_t)r * 128;
     const uint32_t sw = (uint32_t)(r & 7);
-    int ox, oy;
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, p.st, abort_flag));
-    if (EPI == 1 && p.has_residual) ok = __all_sync(0xffffffffu, ok && mbar_wait(bar_res, 0, p.st, abort_flag));
+    if (LY::kAux && p.has_aux) ok = __all_sync(0xffffffffu, ok && mbar_wait(bar_aux, 0, p.st, abort_flag));
     if (ok) {
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t a[32];
-        tmem_ld32(tmem + lane_off + c * 32, a);
-        tmem_ld_wait();
-        if constexpr (EPI == 2) {
+      for (int c = 0; c < kOutN / 32; ++c) {
+        if constexpr (EPI == kEpiF32) {
+          uint32_t a[32];
+          tmem_ld32(tmem + lane_off + c * 32, a);
+          tmem_ld_wait();
           const uint32_t box = row_base + (uint32_t)c * kBox;
 #pragma unroll
           for (int x = 0; x < 8; ++x)
             st_shared_v4(box + (((uint32_t)x ^ sw) << 4), a[4 * x], a[4 * x + 1], a[4 * x + 2], a[4 * x + 3]);
-        } else {
+        } else if constexpr (EPI == kEpiBf16 || EPI == kEpiBf16Res) {
+          uint32_t a[32];
+          tmem_ld32(tmem + lane_off + c * 32, a);
+          tmem_ld_wait();
           const uint32_t box = row_base + (uint32_t)(c >> 1) * kBox;
           float v[32];
 #pragma unroll
           for (int x = 0; x < 32; ++x) v[x] = __uint_as_float(a[x]);
-          if (EPI == 1 && p.has_residual) {
+          if (EPI == kEpiBf16Res && p.has_aux) {
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
               const uint32_t unit = (uint32_t)((c & 1) * 4 + x);
-              uint4 q;
-              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                           : "=r"(q.x), "=r"(q.y), "=r"(q.z), "=r"(q.w)
-                           : "r"(box + ((unit ^ sw) << 4)));
+              const uint4 q = ld_shared_v4(box + ((unit ^ sw) << 4));
               const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
@@ -235,11 +269,48 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
 #pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            const uint32_t unit = (uint32_t)((c & 1) * 4 + x);
-            st_shared_v4(box + ((unit ^ sw) << 4), pack_bf16x2(v[8 * x], v[8 * x + 1]),
-                         pack_bf16x2(v[8 * x + 2], v[8 * x + 3]), pack_bf16x2(v[8 * x + 4], v[8 * x + 5]),
-                         pack_bf16x2(v[8 * x + 6], v[8 * x + 7]));
+          for (int x = 0; x < 4; ++x) st_unit_bf16(box, (uint32_t)((c & 1) * 4 + x), sw, v + 8 * x);
+        } else {
+          uint32_t g[32], u[32];
+          tmem_ld32(tmem + lane_off + c * 32, g);
+          tmem_ld32(tmem + lane_off + 128 + c * 32, u);
+          tmem_ld_wait();
+          if constexpr (EPI == kEpiSwiGLU) {
+            float h[32];
+#pragma unroll
+            for (int x = 0; x < 32; ++x) {
+              const float gg = __uint_as_float(g[x]);
+              h[x] = gg / (1.f + __expf(-gg)) * __uint_as_float(u[x]);
+            }
+            const uint32_t box = row_base + (uint32_t)(c >> 1) * kBox;
+#pragma unroll
+            for (int x = 0; x < 4; ++x) st_unit_bf16(box, (uint32_t)((c & 1) * 4 + x), sw, h + 8 * x);
+          } else {
+            // dh: fp32 box c of the prefetched tile (32 columns, 8 swizzled units)
+            float dg[32], du[32], h[32];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+              const uint4 q = ld_shared_v4(aux_row + (uint32_t)c * kBox + (((uint32_t)x ^ sw) << 4));
+              const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int i = 4 * x + e;
+                const float gg = __uint_as_float(g[i]), uu = __uint_as_float(u[i]);
+                const float d = __uint_as_float(w[e]);
+                const float sg = 1.f / (1.f + __expf(-gg));
+                const float si = gg * sg;
+                h[i] = si * uu;
+                du[i] = d * si;
+                dg[i] = d * uu * (sg * (1.f + gg * (1.f - sg)));
+              }
+            }
+#pragma unroll
+            for (int o = 0; o < 3; ++o) {
+              const float* src = o == 0 ? dg : (o == 1 ? du : h);
+              const uint32_t box = row_base + (uint32_t)(o * 2 + (c >> 1)) * kBox;
+#pragma unroll
+              for (int x = 0; x < 4; ++x) st_unit_bf16(box, (uint32_t)((c & 1) * 4 + x), sw, src + 8 * x);
+            }
           }
         }
       }
@@ -247,20 +318,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     named_bar_sync(1, 128);
     if (threadIdx.x == 128 && ok) {
-      const uint8_t* stage = smem + (EPI == 1 ? LY::kResOff : 0);
-      if constexpr (EPI == 2) {
+      const uint8_t* stage = smem + (EPI == kEpiBf16Res ? LY::kAuxOff : 0);
+      int ox, oy;
+      if constexpr (EPI == kEpiF32) {
         for (int c = 0; c < kBN / 32; ++c) {
+          if (nt * kBN + c * 32 >= p.n_valid) break;
           op_coord(p.out, mt * kBM, nt * kBN + c * 32, ox, oy);
           if (p.f32_add)
-            tma_add_2d(&tOut, stage + c * kBox, ox, oy);
+            tma_add_2d(&maps.out[0], stage + c * kBox, ox, oy);
           else
-            tma_store_2d(&tOut, stage + c * kBox, ox, oy);
+            tma_store_2d(&maps.out[0], stage + c * kBox, ox, oy);
         }
       } else {
-        for (int j = 0; j < 4; ++j) {
-          op_coord(p.out, mt * kBM, nt * kBN + j * 64, ox, oy);
-          tma_store_2d(&tOut, stage + j * kBox, ox, oy);
-        }
+        constexpr int kOuts = EPI == kEpiSwiGLUBwd ? 3 : 1;
+        for (int o = 0; o < kOuts; ++o)
+          for (int j = 0; j < kOutN / 64; ++j) {
+            if (nt * kOutN + j * 64 >= p.n_valid) break;
+            op_coord(p.out, mt * kBM, nt * kOutN + j * 64, ox, oy);
+            tma_store_2d(&maps.out[o], stage + (o * (kOutN / 64) + j) * kBox, ox, oy);
+          }
       }
       bulk_commit_group();
       bulk_wait_read_all();
@@ -297,22 +373,29 @@ int operand_map(CUtensorMap* m, const GemmOperand& o, bool mn_major) {
 }
 
 template <bool A_MN, bool B_MN, int EPI>
-int launch_typed(const CUtensorMap* maps, const GemmParams& p, dim3 grid, cudaStream_t stream) {
+int launch_typed(const GemmMaps& maps, const GemmParams& p, dim3 grid, cudaStream_t stream) {
   constexpr int kSmemBytes = GLay<EPI>::kSmemBytes;
   auto kern = gemm_kernel<A_MN, B_MN, EPI>;
   if (set_smem_attr((const void*)kern, kSmemBytes) != RA_OK) return RA_ERR_CUDA;
-  kern<<<grid, kThreads, kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6],
-                                               maps[7], p);
+  kern<<<grid, kThreads, kSmemBytes, stream>>>(maps, p);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
-
 
 }  // namespace
 
 int launch_gemm_tc(const GemmSeg* segs, int nseg, int64_t M, int64_t N, const GemmOut& out, int splits,
                    cudaStream_t stream) {
-  if (nseg < 1 || nseg > 3 || M <= 0 || N <= 0 || M % kBM || N % kBN) return RA_ERR_SHAPE;
-  if (splits < 1 || splits > 2 || (splits > 1 && (!out.f32 || out.add))) return RA_ERR_ARG;
+  const int epi = out.epi;
+  const bool swi = epi == kEpiSwiGLU || epi == kEpiSwiGLUBwd;
+  const int tile_n = swi ? 128 : kBN;
+  if (epi < kEpiBf16 || epi > kEpiSwiGLUBwd) return RA_ERR_ARG;
+  if (nseg < 1 || nseg > 3 || (swi && nseg != 2) || M <= 0 || N <= 0 || M % kBM || N % 128) return RA_ERR_SHAPE;
+  // a half-full last N tile relies on TMA zero fill and clipping, which a
+  // head-split (remapped) box does not have
+  if (!swi && N % kBN && (out.hs_ntok > 0 || segs[0].b.hs_ntok > 0)) return RA_ERR_SHAPE;
+  if (splits < 1 || splits > 2 || (splits > 1 && (epi != kEpiF32 || out.add))) return RA_ERR_ARG;
+  if ((epi == kEpiBf16Res || epi == kEpiSwiGLUBwd) && !out.aux) return RA_ERR_ARG;
+  if (epi == kEpiSwiGLUBwd && (!out.ptr2 || !out.ptr3)) return RA_ERR_ARG;
   const bool a_mn = segs[0].a.mn_major != 0, b_mn = segs[0].b.mn_major != 0;
   if (M > INT32_MAX / 2 || N > INT32_MAX / 2) return RA_ERR_UNSUPPORTED;
   GemmParams p{};
@@ -326,14 +409,16 @@ int launch_gemm_tc(const GemmSeg* segs, int nseg, int64_t M, int64_t N, const Ge
         if (o->hs_ntok > 0 && (o->hs_ntok % 128 || o->hs_d % 64 || o->rows % o->hs_ntok)) return RA_ERR_SHAPE;
       p.a[s] = geo_of(g.a);
       p.b[s] = geo_of(g.b);
-      kb += (int)(g.K / kBK);
+      // the SwiGLU epilogues stack segment 1's B under segment 0's; K runs once
+      if (!(swi && s == 1)) kb += (int)(g.K / kBK);
     }
     p.seg_end[s] = kb;
   }
-  if (out.f32 && out.hs_ntok > 0) return RA_ERR_UNSUPPORTED;
+  if (swi && (b_mn || a_mn || segs[1].K != segs[0].K)) return RA_ERR_ARG;
+  if (epi == kEpiF32 && out.hs_ntok > 0) return RA_ERR_UNSUPPORTED;
   p.out = geo_of(GemmOperand{out.ptr, M, N, 0, out.hs_ntok, out.hs_heads, out.hs_d, 0, 0});
   p.m_tiles = (int)(M / kBM);
-  p.n_tiles = (int)(N / kBN);
+  p.n_tiles = (int)((N + tile_n - 1) / tile_n);
   // Concurrent CTAs should share the larger operand's tiles: with M >= N the
   // A rows (activations) are re-read from L2 by the n tiles running together
   // and the smaller B stays L2-resident.
@@ -341,43 +426,56 @@ int launch_gemm_tc(const GemmSeg* segs, int nseg, int64_t M, int64_t N, const Ge
   p.kb_total = kb;
   if (kb < splits) return RA_ERR_SHAPE;  // every split needs at least one K step
   p.kb_per_split = (kb + splits - 1) / splits;
-  p.f32_add = out.f32 && (out.add || splits > 1);
-  p.has_residual = out.residual != nullptr;
+  p.f32_add = epi == kEpiF32 && (out.add || splits > 1);
+  p.has_aux = out.aux != nullptr;
+  p.n_valid = (int)N;
   int rc = current_status(&p.st);
   if (rc != RA_OK) return rc;
 
-  alignas(64) CUtensorMap maps[8];
+  alignas(64) GemmMaps maps;
   int ok = RA_OK;
   for (int s = 0; s < 3; ++s) {
     const GemmSeg& g = segs[s < nseg ? s : 0];
-    ok |= operand_map(&maps[s], g.a, a_mn);
-    ok |= operand_map(&maps[3 + s], g.b, b_mn);
+    ok |= operand_map(&maps.a[s], g.a, a_mn);
+    ok |= operand_map(&maps.b[s], g.b, b_mn);
   }
-  if (out.f32) {
-    ok |= make_tmap_f32_2d(&maps[6], out.ptr, (uint64_t)N, (uint64_t)M, (uint64_t)N * 4, 32, 128);
-  } else {
-    GemmOperand o{out.ptr, M, N, 0, out.hs_ntok, out.hs_heads, out.hs_d, 0, 0};
-    ok |= operand_map(&maps[6], o, false);
+  void* outs[3] = {out.ptr, out.ptr2 ? out.ptr2 : out.ptr, out.ptr3 ? out.ptr3 : out.ptr};
+  for (int o = 0; o < 3; ++o) {
+    if (epi == kEpiF32) {
+      ok |= make_tmap_f32_2d(&maps.out[o], outs[o], (uint64_t)N, (uint64_t)M, (uint64_t)N * 4, 32, 128);
+    } else {
+      GemmOperand og{outs[o], M, N, 0, out.hs_ntok, out.hs_heads, out.hs_d, 0, 0};
+      ok |= operand_map(&maps.out[o], og, false);
+    }
   }
-  if (out.residual)
-    ok |= make_tmap_bf16_2d(&maps[7], out.residual, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2, 64, 128);
+  if (epi == kEpiBf16Res)
+    ok |= make_tmap_bf16_2d(&maps.aux, out.aux, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2, 64, 128);
+  else if (epi == kEpiSwiGLUBwd)
+    ok |= make_tmap_f32_2d(&maps.aux, out.aux, (uint64_t)N, (uint64_t)M, (uint64_t)N * 4, 32, 128);
   else
-    maps[7] = maps[6];
+    maps.aux = maps.out[0];
   if (ok != RA_OK) return RA_ERR_CUDA;
-  if (out.f32 && splits > 1 && !out.add) {
+  if (epi == kEpiF32 && splits > 1) {
     if (cudaMemsetAsync(out.ptr, 0, (size_t)M * N * 4, stream) != cudaSuccess) return RA_ERR_CUDA;
   }
-  const dim3 grid((unsigned)((M / kBM) * (N / kBN)), (unsigned)splits);
-  if (out.f32) {
-    if (a_mn && b_mn) return launch_typed<true, true, 2>(maps, p, grid, stream);
-    return RA_ERR_UNSUPPORTED;
+  const dim3 grid((unsigned)(p.m_tiles * p.n_tiles), (unsigned)splits);
+  switch (epi) {
+    case kEpiF32:
+      if (a_mn && b_mn) return launch_typed<true, true, kEpiF32>(maps, p, grid, stream);
+      if (!a_mn && b_mn) return launch_typed<false, true, kEpiF32>(maps, p, grid, stream);
+      return RA_ERR_UNSUPPORTED;
+    case kEpiBf16Res:
+      if (!a_mn && !b_mn) return launch_typed<false, false, kEpiBf16Res>(maps, p, grid, stream);
+      return RA_ERR_UNSUPPORTED;
+    case kEpiSwiGLU:
+      return launch_typed<false, false, kEpiSwiGLU>(maps, p, grid, stream);
+    case kEpiSwiGLUBwd:
+      return launch_typed<false, false, kEpiSwiGLUBwd>(maps, p, grid, stream);
+    default:
+      if (!a_mn && !b_mn) return launch_typed<false, false, kEpiBf16>(maps, p, grid, stream);
+      if (!a_mn && b_mn) return launch_typed<false, true, kEpiBf16>(maps, p, grid, stream);
+      return RA_ERR_UNSUPPORTED;
   }
-  if (!a_mn && !b_mn) {
-    if (out.residual) return launch_typed<false, false, 1>(maps, p, grid, stream);
-    return launch_typed<false, false, 0>(maps, p, grid, stream);
-  }
-  if (!a_mn && b_mn) return launch_typed<false, true, 0>(maps, p, grid, stream);
-  return RA_ERR_UNSUPPORTED;
 }
 
 }  // namespace ra

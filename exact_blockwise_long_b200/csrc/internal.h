@@ -80,14 +80,21 @@ struct GemmSeg {
   GemmOperand a, b;
   int64_t K;
 };
+// Epilogues of launch_gemm_tc (see csrc/gemm_tc.cu).
+enum GemmEpi { kEpiBf16 = 0, kEpiBf16Res = 1, kEpiF32 = 2, kEpiSwiGLU = 3, kEpiSwiGLUBwd = 4 };
 struct GemmOut {
   void* ptr;                        // [M, N] (bf16: plain or head-split; fp32: plain)
-  int f32;                          // fp32 output (else bf16)
-  int add;                          // fp32: add into the existing values
+  int epi;                          // GemmEpi
+  int add;                          // kEpiF32: add into the existing values
   int64_t hs_ntok, hs_heads, hs_d;  // bf16 head-split output
-  const void* residual;             // bf16 [M, N] added before rounding (bf16 output), or null
+  const void* aux;                  // kEpiBf16Res: bf16 residual [M, N]; kEpiSwiGLUBwd: fp32 dh [M, N]
+  void* ptr2;                       // kEpiSwiGLUBwd: du (ptr: dg)
+  void* ptr3;                       // kEpiSwiGLUBwd: h
 };
-// M % 128 == 0, N % 256 == 0, K_s % 64 == 0; splits 1 or 2 (2: fp32 output
+// M % 128 == 0, K_s % 64 == 0, N % 128 == 0 (N % 256 == 0 with head-split
+// output or B); the last N tile may be half full (TMA fills and clips).
+// kEpiSwiGLU / kEpiSwiGLUBwd: two segments with the same A and K, B_0 = w1,
+// B_1 = w3 (K-major), N = d_ff (output width).  splits 1 or 2 (2: kEpiF32
 // only, K split across two CTAs that each add onto a zeroed output).
 int launch_gemm_tc(const GemmSeg* segs, int nseg, int64_t M, int64_t N, const GemmOut& out, int splits,
                    cudaStream_t stream);

@@ -92,9 +92,13 @@ GemmOperand plain(const void* p, int64_t rows, int64_t cols, int mn) {
 GemmOperand split(const void* p, int64_t rows, int64_t cols, int mn, int64_t N, int64_t H, int64_t D) {
   return GemmOperand{p, rows, cols, mn, N, H, D, 0, 0};
 }
-GemmOut bf16_out(void* p, const void* residual = nullptr) { return GemmOut{p, 0, 0, 0, 0, 0, residual}; }
-GemmOut bf16_split_out(void* p, int64_t N, int64_t H, int64_t D) { return GemmOut{p, 0, 0, N, H, D, nullptr}; }
-GemmOut f32_out(float* p) { return GemmOut{p, 1, 0, 0, 0, 0, nullptr}; }
+GemmOut bf16_out(void* p, const void* residual = nullptr) {
+  return GemmOut{p, residual ? kEpiBf16Res : kEpiBf16, 0, 0, 0, 0, residual, nullptr, nullptr};
+}
+GemmOut bf16_split_out(void* p, int64_t N, int64_t H, int64_t D) {
+  return GemmOut{p, kEpiBf16, 0, N, H, D, nullptr, nullptr, nullptr};
+}
+GemmOut f32_out(float* p) { return GemmOut{p, kEpiF32, 0, 0, 0, 0, nullptr, nullptr, nullptr}; }
 
 // Weight gradients [dm, dm] have few output tiles and a long K (all tokens):
 // split K in two (two fp32 adds onto a zeroed output commute exactly) when

@@ -290,8 +290,8 @@ RA_API int blockwise_ffn(const void* x, const void* w1, const void* w2, const vo
                   int64_t T, int64_t d_model, int64_t d_ff, int64_t chunk, int dtype,
                   void* workspace, size_t workspace_bytes, void* stream);
 
-/* Bytes of device workspace blockwise_ffn_bwd needs: one chunk's dg, du and
- * h, each [chunk, d_ff] bf16. */
+/* Bytes of device workspace blockwise_ffn_bwd needs: one chunk's dh
+ * [chunk, d_ff] fp32 and dg, du, h [chunk, d_ff] bf16. */
 RA_API size_t blockwise_ffn_bwd_workspace_size(int64_t chunk, int64_t d_ff, int dtype);
 
 /*
