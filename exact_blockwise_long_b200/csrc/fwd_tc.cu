@@ -154,8 +154,12 @@ __device__ __forceinline__ float row_max(const float (&s)[kBN]) {
 // pipes, the rest by the MUFU: each 128 x 128 tile needs as many MUFU cycles
 // for its exponentials as tensor cycles for its two matmuls, so moving part
 // of them off the MUFU shortens the softmax's critical path.
+// With bar_half, the first half of P (keys 0-63) is published on it as soon
+// as it is in TMEM, so the P V matmul over those keys can start while the
+// second half is computed.
 constexpr int kEx2PolyEvery = 4;
-__device__ __forceinline__ float exp_store(const float (&s)[kBN], uint32_t tS, float sl2, float m) {
+__device__ __forceinline__ float exp_store(const float (&s)[kBN], uint32_t tS, float sl2, float m,
+                                           uint64_t* bar_half = nullptr) {
   const float2 k2 = make_float2(sl2, sl2), nm2 = make_float2(-m, -m);
   float2 acc[4];
 #pragma unroll
@@ -172,6 +176,11 @@ __device__ __forceinline__ float exp_store(const float (&s)[kBN], uint32_t tS, f
       pk[x] = pack_bf16x2(pr.x, pr.y);
     }
     tmem_st32(tS + h * 32, pk);
+    if (h == 0 && bar_half) {
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_half);
+    }
   }
   const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
   const float2 t = add2(a01, a23);
@@ -481,7 +490,7 @@ struct Layout2 {
   static constexpr int kK = 2 * kTileBytes;
   static constexpr int kV = kK + kKSt * kTileBytes;
   static constexpr int kBar = kV + kVSt * kTileBytes;
-  static constexpr int kNumBars = 1 + 2 * kKSt + 2 * kVSt + 2 + 2 + 1;
+  static constexpr int kNumBars = 1 + 2 * kKSt + 2 * kVSt + 2 + 2 + 2 + 1;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4;
@@ -553,7 +562,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
   uint64_t* bar_ve = bar_vf + kVSt;
   uint64_t* bar_sf = bar_ve + kVSt;  // [2] S of tile t computed
   uint64_t* bar_pf = bar_sf + 2;     // [2] P of tile t written
-  uint64_t* bar_done = bar_pf + 2;   // every MMA finished
+  uint64_t* bar_ph = bar_pf + 2;     // [2] first half of P (keys 0-63) of tile t written
+  uint64_t* bar_done = bar_ph + 2;   // every MMA finished
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + LY::kTmemSlot);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LY::kAbort);
 
@@ -570,6 +580,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bar_sf[t], 1);
       mbar_init(&bar_pf[t], 128);
+      mbar_init(&bar_ph[t], 128);
     }
     mbar_init(bar_done, 1);
     *abort_flag = 0;
@@ -635,14 +646,17 @@ __global__ void __launch_bounds__(kThreads2, 1)
         mma_commit(&bar_sf[t]);
       };
       auto issue_pv = [&](int t, int vs) -> bool {
-        if (!mbar_wait(&bar_pf[t], pv_cnt[t] & 1, p.st, abort_flag)) return false;
-        tc_fence_after();
         const uint32_t vb = v_base + vs * LY::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
-                      sdesc_sw128(vb + kk * 16 * 128, LY::kSlabBytes, 1024), idPV,
-                      (pv_cnt[t] > 0 || kk > 0) ? 1u : 0u);
+        for (int half = 0; half < 2; ++half) {  // keys 0-63 as soon as their P is in TMEM, then 64-127
+          if (!mbar_wait(half ? &bar_pf[t] : &bar_ph[t], pv_cnt[t] & 1, p.st, abort_flag)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = half * (kBN / 32); kk < (half + 1) * (kBN / 32); ++kk)
+            mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
+                        sdesc_sw128(vb + kk * 16 * 128, LY::kSlabBytes, 1024), idPV,
+                        (pv_cnt[t] > 0 || kk > 0) ? 1u : 0u);
+        }
         ++pv_cnt[t];
         return true;
       };
@@ -701,7 +715,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
         rescale_o<D>(tO, alpha);
         m_run = m_new;
       }
-      const float rowsum = exp_store(s, tS, sl2, m_run);
+      const float rowsum = exp_store(s, tS, sl2, m_run, &bar_ph[tile]);
       tmem_st_wait();
       l_run += rowsum;
       tc_fence_before();
