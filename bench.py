@@ -467,10 +467,11 @@ def run_layer(args, ra, dev, rank, world, dist):
         "fwd_tc2_kernel": (avg(lambda s0, fm, bm: fm[1].elapsed_time(fm[2])), af, "fwd_tc.cu"),
         "bwd_kv_kernel": (avg(lambda s0, fm, bm: bm[4].elapsed_time(bm[5])), 2.0 * af, "bwd_tc.cu"),
         "bwd_q_kernel": (avg(lambda s0, fm, bm: bm[5].elapsed_time(bm[6])), 0.5 * af, "bwd_tc.cu"),
-        "gemm_kernel": (avg(lambda s0, fm, bm: fm[0].elapsed_time(fm[1]) + fm[2].elapsed_time(fm[3]) +
-                            bm[1].elapsed_time(bm[3]) + bm[6].elapsed_time(bm[8])), proj, "gemm_tc.cu"),
-        "ffn_tc_kernel+ffn_bwd_gemm_kernel": (avg(lambda s0, fm, bm: fm[4].elapsed_time(fm[5]) +
-                                                  fm[5].elapsed_time(bm[0])), ffn, "ffn_bwd_tc.cu"),
+        "gemm_kernel[projections]": (avg(lambda s0, fm, bm: fm[0].elapsed_time(fm[1]) + fm[2].elapsed_time(fm[3]) +
+                                         bm[1].elapsed_time(bm[3]) + bm[6].elapsed_time(bm[8])), proj,
+                                     "gemm_tc.cu"),
+        "gemm_kernel[ffn fwd+bwd]": (avg(lambda s0, fm, bm: fm[4].elapsed_time(fm[5]) +
+                                         fm[5].elapsed_time(bm[0])), ffn, "gemm_tc.cu"),
     }
     kname = max(kernels, key=lambda k_: kernels[k_][0])
     kms, kflops, ksrc = kernels[kname]
@@ -725,7 +726,7 @@ def main():
     kname = max(kernels, key=lambda k_: kernels[k_][0])
     if fw is not None:
         # the feed-forward's forward and backward GEMMs, timed together
-        kernels["ffn_tc_kernel+ffn_bwd_gemm_kernel"] = (mean_ms(ev["ffn"]), ffn_flops(fw), "ffn_bwd_tc.cu")
+        kernels["gemm_kernel[ffn fwd+bwd]"] = (mean_ms(ev["ffn"]), ffn_flops(fw), "gemm_tc.cu")
     kms, kflops, ksrc = kernels[kname]
     achieved = kflops / (kms * 1e-3) / 1e12
     src = os.path.join(ROOT, "exact_blockwise_long_b200", "csrc", ksrc)

@@ -13,10 +13,12 @@
 // and store coordinates are remapped per box, so no transpose kernel exists.
 //
 // One CTA computes one 128 x 256 accumulator tile (tcgen05 M=128, N=256,
-// fp32 in 256 TMEM columns) over a TMA ring of 64-deep K slabs.  Epilogues
+// fp32 in 256 TMEM columns) over a 4-stage TMA ring of 64-deep K slabs; the
+// residual or dh rows an epilogue needs are loaded into the epilogue warps'
+// registers while the main loop runs.  Epilogues
 // (results leave through 128-byte-swizzled staging boxes and TMA stores):
 //   kEpiBf16       bf16 tile
-//   kEpiBf16Res    bf16 tile + a bf16 residual tile (prefetched at start)
+//   kEpiBf16Res    bf16 tile + a bf16 residual tile
 //   kEpiF32        fp32 tile, stored or element-wise TMA-added (the K range
 //                  may be split across two CTAs adding onto a zeroed output:
 //                  two addends onto zero commute exactly, so it stays
@@ -24,7 +26,7 @@
 //   kEpiSwiGLU     B is stacked: rows 0-127 from w1, 128-255 from w3 (the same
 //                  hidden units), so the accumulator holds g | u and the tile
 //                  leaves as h = silu(g) * u  [128 x 128]
-//   kEpiSwiGLUBwd  the same g | u, plus a prefetched fp32 dh tile:
+//   kEpiSwiGLUBwd  the same g | u, plus an fp32 dh tile:
 //                  dg = dh u s (1 + g (1 - s)), du = dh g s, h = g s u,
 //                  s = 1 / (1 + e^-g)  (three bf16 tiles)
 // Warp roles: 0 TMA producer, 1 MMA issuer, 2 TMEM allocator, 4-7 epilogue.
@@ -43,20 +45,19 @@ constexpr int kBTile = kBN * kBK * 2;  // 32 KB
 constexpr int kStage = kATile + kBTile;
 constexpr int kBox = 16384;  // one staging box: 128 rows x 128 bytes
 
-// Shared memory per epilogue: a 4-stage ring; with an auxiliary input tile
-// (residual, dh) a 3-stage ring plus that tile (64 KB).
+// Shared memory: a 4-stage ring, reused as the epilogue's staging boxes once
+// the main loop has drained.  The epilogues' auxiliary inputs (residual, dh)
+// are read into the epilogue warps' registers while the main loop runs.
 template <int EPI>
 struct GLay {
-  static constexpr bool kAux = EPI == kEpiBf16Res || EPI == kEpiSwiGLUBwd;
-  static constexpr int kStages = kAux ? 3 : 4;
-  static constexpr int kAuxOff = kStages * kStage;
-  static constexpr int kBarOff = kAuxOff + (kAux ? 4 * kBox : 0);
-  static constexpr int kTmemSlot = kBarOff + (2 * kStages + 2) * 8;
+  static constexpr int kStages = 4;
+  static constexpr int kBarOff = kStages * kStage;
+  static constexpr int kTmemSlot = kBarOff + (2 * kStages + 1) * 8;
   static constexpr int kAbortOff = kTmemSlot + 4;
   static constexpr int kSmemBytes = kAbortOff + 4 + 1024;
   static_assert(kSmemBytes <= 232448, "GEMM stages exceed shared memory");
-  static_assert(EPI != kEpiF32 || 8 * kBox <= kAuxOff, "fp32 staging exceeds the pipeline buffers");
-  static_assert(EPI != kEpiSwiGLUBwd || 6 * kBox <= kAuxOff, "staging exceeds the pipeline buffers");
+  static_assert(EPI != kEpiF32 || 8 * kBox <= kBarOff, "fp32 staging exceeds the pipeline buffers");
+  static_assert(EPI != kEpiSwiGLUBwd || 6 * kBox <= kBarOff, "staging exceeds the pipeline buffers");
 };
 
 struct OpGeo {
@@ -68,7 +69,6 @@ struct OpGeo {
 struct GemmMaps {
   CUtensorMap a[3], b[3];  // per segment (b[1] is the stacked half for the SwiGLU epilogues)
   CUtensorMap out[3];      // outputs
-  CUtensorMap aux;         // residual (bf16) or dh (fp32)
 };
 
 struct GemmParams {
@@ -80,7 +80,8 @@ struct GemmParams {
   int kb_per_split;        // K steps per blockIdx.y
   int kb_total;
   int f32_add;             // fp32 output: TMA add instead of store
-  int has_aux;
+  const void* aux;         // kEpiBf16Res: bf16 residual [M, N]; kEpiSwiGLUBwd: fp32 dh [M, N]
+  int aux_ld;              // its row pitch (elements)
   int n_valid;             // output columns; boxes of a half-full last tile past it are not stored
   DevStatus st;
 };
@@ -156,7 +157,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   uint64_t* bar_full = bars;
   uint64_t* bar_empty = bars + kStages;
   uint64_t* bar_done = bars + 2 * kStages;
-  uint64_t* bar_aux = bars + 2 * kStages + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + LY::kTmemSlot);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LY::kAbortOff);
 
@@ -166,7 +166,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       mbar_init(&bar_empty[s], 1);
     }
     mbar_init(bar_done, 1);
-    mbar_init(bar_aux, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -181,14 +180,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
 
   if (warp == 0) {
     if (lane == 0) {
-      if (LY::kAux && p.has_aux) {  // the epilogue's input tile, fetched while the main loop runs
-        mbar_arrive_expect_tx(bar_aux, 4 * kBox);
-        for (int j = 0; j < 4; ++j) {
-          // residual: 4 x 64 bf16 columns; dh: 4 x 32 fp32 columns
-          const int x = EPI == kEpiBf16Res ? nt * kBN + j * 64 : nt * 128 + j * 32;
-          tma_load_2d(smem + LY::kAuxOff + j * kBox, &maps.aux, bar_aux, x, mt * kBM);
-        }
-      }
       for (int kb = kb0; kb < kb1; ++kb) {
         const int i = kb - kb0;
         const int s = i % kStages;
@@ -224,20 +215,35 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       mma_commit(bar_done);
     }
   } else if (warp >= 4) {
-    // accumulator rows -> swizzled staging boxes -> TMA stores / adds.
-    // Staging: the drained pipeline buffers, or for kEpiBf16Res the residual
-    // tile itself (each thread overwrites only what it has read).
+    // accumulator rows -> swizzled staging boxes in the drained pipeline
+    // buffers -> TMA stores / adds
     const int r = (warp - 4) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t stage_base = smem_u32(smem) + (EPI == kEpiBf16Res ? LY::kAuxOff : 0);
-    const uint32_t row_base = stage_base + (uint32_t)r * 128;
-    const uint32_t aux_row = smem_u32(smem) + LY::kAuxOff + (uint32_t)r * 128;
+    const uint32_t row_base = smem_u32(smem) + (uint32_t)r * 128;
     const uint32_t sw = (uint32_t)(r & 7);
-    bool ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, p.st, abort_flag));
-    if (LY::kAux && p.has_aux) ok = __all_sync(0xffffffffu, ok && mbar_wait(bar_aux, 0, p.st, abort_flag));
+    // the auxiliary row slice of this thread (residual: 256 bf16; dh: 128
+    // fp32), loaded while the main loop runs
+    constexpr bool kAux = EPI == kEpiBf16Res || EPI == kEpiSwiGLUBwd;
+    uint4 auxv[kAux ? 32 : 1];
+    if constexpr (kAux) {
+      const size_t row = (size_t)(mt * kBM + r);
+      if constexpr (EPI == kEpiBf16Res) {
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.aux) +
+                                                          row * p.aux_ld + (size_t)nt * kBN);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          auxv[j] = (nt * kBN + j * 8 < p.n_valid) ? __ldg(src + j) : make_uint4(0, 0, 0, 0);
+      } else {
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(p.aux) + row * p.aux_ld +
+                                                          (size_t)nt * 128);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) auxv[j] = __ldg(src + j);
+      }
+    }
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, p.st, abort_flag));
     if (ok) {
       tc_fence_after();
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < kOutN / 32; ++c) {
         if constexpr (EPI == kEpiF32) {
           uint32_t a[32];
@@ -255,11 +261,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           float v[32];
 #pragma unroll
           for (int x = 0; x < 32; ++x) v[x] = __uint_as_float(a[x]);
-          if (EPI == kEpiBf16Res && p.has_aux) {
+          if constexpr (EPI == kEpiBf16Res) {
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
-              const uint32_t unit = (uint32_t)((c & 1) * 4 + x);
-              const uint4 q = ld_shared_v4(box + ((unit ^ sw) << 4));
+              const uint4 q = auxv[c * 4 + x];
               const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
@@ -286,30 +291,26 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
 #pragma unroll
             for (int x = 0; x < 4; ++x) st_unit_bf16(box, (uint32_t)((c & 1) * 4 + x), sw, h + 8 * x);
           } else {
-            // dh: fp32 box c of the prefetched tile (32 columns, 8 swizzled units)
-            float dg[32], du[32], h[32];
+            // eight columns at a time: dh from the registers, dg, du, h to staging
 #pragma unroll
-            for (int x = 0; x < 8; ++x) {
-              const uint4 q = ld_shared_v4(aux_row + (uint32_t)c * kBox + (((uint32_t)x ^ sw) << 4));
-              const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+            for (int x = 0; x < 4; ++x) {
+              float dg[8], du[8], h[8];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int i = 4 * x + e;
-                const float gg = __uint_as_float(g[i]), uu = __uint_as_float(u[i]);
-                const float d = __uint_as_float(w[e]);
+              for (int e = 0; e < 8; ++e) {
+                const int i = 8 * x + e;
+                const uint4 q = auxv[c * 8 + i / 4];
+                const uint32_t w = (i & 3) == 0 ? q.x : ((i & 3) == 1 ? q.y : ((i & 3) == 2 ? q.z : q.w));
+                const float gg = __uint_as_float(g[i]), uu = __uint_as_float(u[i]), d = __uint_as_float(w);
                 const float sg = 1.f / (1.f + __expf(-gg));
                 const float si = gg * sg;
-                h[i] = si * uu;
-                du[i] = d * si;
-                dg[i] = d * uu * (sg * (1.f + gg * (1.f - sg)));
+                h[e] = si * uu;
+                du[e] = d * si;
+                dg[e] = d * uu * (sg * (1.f + gg * (1.f - sg)));
               }
-            }
-#pragma unroll
-            for (int o = 0; o < 3; ++o) {
-              const float* src = o == 0 ? dg : (o == 1 ? du : h);
-              const uint32_t box = row_base + (uint32_t)(o * 2 + (c >> 1)) * kBox;
-#pragma unroll
-              for (int x = 0; x < 4; ++x) st_unit_bf16(box, (uint32_t)((c & 1) * 4 + x), sw, src + 8 * x);
+              const uint32_t unit = (uint32_t)((c & 1) * 4 + x);
+              st_unit_bf16(row_base + (uint32_t)(0 * 2 + (c >> 1)) * kBox, unit, sw, dg);
+              st_unit_bf16(row_base + (uint32_t)(1 * 2 + (c >> 1)) * kBox, unit, sw, du);
+              st_unit_bf16(row_base + (uint32_t)(2 * 2 + (c >> 1)) * kBox, unit, sw, h);
             }
           }
         }
@@ -318,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     }
     named_bar_sync(1, 128);
     if (threadIdx.x == 128 && ok) {
-      const uint8_t* stage = smem + (EPI == kEpiBf16Res ? LY::kAuxOff : 0);
+      const uint8_t* stage = smem;
       int ox, oy;
       if constexpr (EPI == kEpiF32) {
         for (int c = 0; c < kBN / 32; ++c) {
@@ -427,7 +428,8 @@ int launch_gemm_tc(const GemmSeg* segs, int nseg, int64_t M, int64_t N, const Ge
   if (kb < splits) return RA_ERR_SHAPE;  // every split needs at least one K step
   p.kb_per_split = (kb + splits - 1) / splits;
   p.f32_add = epi == kEpiF32 && (out.add || splits > 1);
-  p.has_aux = out.aux != nullptr;
+  p.aux = out.aux;
+  p.aux_ld = (int)N;
   p.n_valid = (int)N;
   int rc = current_status(&p.st);
   if (rc != RA_OK) return rc;
@@ -448,12 +450,6 @@ int launch_gemm_tc(const GemmSeg* segs, int nseg, int64_t M, int64_t N, const Ge
       ok |= operand_map(&maps.out[o], og, false);
     }
   }
-  if (epi == kEpiBf16Res)
-    ok |= make_tmap_bf16_2d(&maps.aux, out.aux, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2, 64, 128);
-  else if (epi == kEpiSwiGLUBwd)
-    ok |= make_tmap_f32_2d(&maps.aux, out.aux, (uint64_t)N, (uint64_t)M, (uint64_t)N * 4, 32, 128);
-  else
-    maps.aux = maps.out[0];
   if (ok != RA_OK) return RA_ERR_CUDA;
   if (epi == kEpiF32 && splits > 1) {
     if (cudaMemsetAsync(out.ptr, 0, (size_t)M * N * 4, stream) != cudaSuccess) return RA_ERR_CUDA;
