@@ -57,6 +57,8 @@ SIGNATURES = {
                                              _P, _P]),
     "blockwise_layer_bwd": (_I, [_P] * 11 + [_SZ] + [_P] * 11 + [_I64, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I,
                                                                   _P, _SZ, _P, _P]),
+    "ringattn_accumulate": (_I, [_P, _P, _I64, _I, _P]),
+    "ringattn_cast": (_I, [_P, _P, _I64, _I, _P]),
     "ringattn_get_error": (_I, [_P]),
     "ringattn_selftest_timeout": (_I, [_I, _P]),
 }

@@ -284,6 +284,22 @@ def blockwise_layer_bwd(x, weights, saved, dy, dx, grads, B, N, H, D, S, q_chunk
     return dx, grads
 
 
+def ringattn_accumulate(acc, x, stream=None):
+    """acc (fp32) += x (bf16 or fp32), element-wise over the whole tensors."""
+    if acc.dtype != torch.float32 or acc.numel() != x.numel():
+        raise ValueError("acc must be float32 with as many elements as x")
+    call("ringattn_accumulate", _dev(acc, "acc"), _dev(x, "x"), acc.numel(), _dtype(x), _stream(stream))
+    return acc
+
+
+def ringattn_cast(x, out, stream=None):
+    """out (bf16 or fp32) <- x (fp32), rounded to nearest even."""
+    if x.dtype != torch.float32 or x.numel() != out.numel():
+        raise ValueError("x must be float32 with as many elements as out")
+    call("ringattn_cast", _dev(x, "x"), _dev(out, "out"), x.numel(), _dtype(out), _stream(stream))
+    return out
+
+
 def ringattn_get_error(stream=None) -> int:
     """Synchronise the stream; return and clear the device status word."""
     return int(lib().ringattn_get_error(_stream(stream)))

@@ -352,6 +352,24 @@ int blockwise_ffn_bwd(const void* x, const void* w1, const void* w2, const void*
   return launch_ffn_bwd_tc(x, w1, w2, w3, dy, dx, dw1, dw2, dw3, T, d_model, d_ff, chunk, workspace, st);
 }
 
+int ringattn_accumulate(float* acc, const void* x, int64_t n, int dtype, void* stream) {
+  if (n < 0) return RA_ERR_ARG;
+  if (dtype != RA_BF16 && dtype != RA_F32) return RA_ERR_DTYPE;
+  if (n == 0) return RA_OK;
+  if (!acc || !x) return RA_ERR_ARG;
+  if (!aligned16(acc) || !aligned16(x)) return RA_ERR_ALIGN;
+  return launch_accumulate(acc, x, n, dtype, static_cast<cudaStream_t>(stream));
+}
+
+int ringattn_cast(const float* x, void* out, int64_t n, int dtype, void* stream) {
+  if (n < 0) return RA_ERR_ARG;
+  if (dtype != RA_BF16 && dtype != RA_F32) return RA_ERR_DTYPE;
+  if (n == 0) return RA_OK;
+  if (!x || !out) return RA_ERR_ARG;
+  if (!aligned16(x) || !aligned16(out)) return RA_ERR_ALIGN;
+  return launch_cast(x, out, n, dtype, static_cast<cudaStream_t>(stream));
+}
+
 int ringattn_get_error(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return RA_ERR_CUDA;

@@ -125,12 +125,6 @@ __device__ __forceinline__ uint64_t tile_desc(uint32_t tile, int kk) {
   return MN ? sdesc_sw128(tile + kk * 2048, 8192, 1024) : sdesc_sw128(tile + kk * 32, 16, 1024);
 }
 
-__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
-  uint4 q;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(q.x), "=r"(q.y), "=r"(q.z), "=r"(q.w) : "r"(addr));
-  return q;
-}
-
 // eight floats -> four packed bf16 pairs -> one swizzled 16-byte unit
 __device__ __forceinline__ void st_unit_bf16(uint32_t row_base_box, uint32_t unit, uint32_t sw, const float* v) {
   st_shared_v4(row_base_box + ((unit ^ sw) << 4), pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),

@@ -110,6 +110,10 @@ int launch_rmsnorm_bwd(const void* x, const void* g, const float* rstd, const vo
                        float* dg, float* partial, int64_t T, int64_t d_model, cudaStream_t stream);
 size_t rmsnorm_dg_partial_floats(int64_t T, int64_t d_model);
 
+// acc[i] += x[i] (x of dtype RA_BF16 or RA_F32); out[i] = x[i] rounded to dtype (csrc/elementwise.cu).
+int launch_accumulate(float* acc, const void* x, int64_t n, int dtype, cudaStream_t stream);
+int launch_cast(const float* x, void* out, int64_t n, int dtype, cudaStream_t stream);
+
 int launch_selftest_timeout(int timeout_us, cudaStream_t stream);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point.

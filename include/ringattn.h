@@ -319,6 +319,17 @@ RA_API int blockwise_ffn_bwd(const void* x, const void* w1, const void* w2, cons
                              int64_t T, int64_t d_model, int64_t d_ff, int64_t chunk, int dtype,
                              void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * ringattn_accumulate -- acc[i] += x[i] for i < n; acc fp32, x of `dtype`.
+ * ringattn_cast       -- out[i] = x[i] rounded to `dtype` (RNE); x fp32.
+ * The multi-device ring (chapterpal "Ring Attention", definition: key/value
+ * blocks circulate between devices) uses them to sum per-pair gradients in
+ * fp32 -- the key/value gradients travel with their blocks -- and to round
+ * the fp32 accumulators at the end.  Pointers 16-byte aligned; n may be 0.
+ */
+RA_API int ringattn_accumulate(float* acc, const void* x, int64_t n, int dtype, void* stream);
+RA_API int ringattn_cast(const float* x, void* out, int64_t n, int dtype, void* stream);
+
 /* ---------------------------------------------------------------------------
  * One blockwise transformer layer (paper abstract: self-attention and the
  * feed-forward both computed blockwise, for training).  Pre-norm decoder

@@ -13,7 +13,7 @@ from exact_blockwise_long_b200.synthetic import to_f64
 # Tolerances (max absolute error against the fp64 oracle).
 TOL_F32 = 1e-4          # fp32 path, O and LSE
 TOL_BF16_O = 2e-2       # bf16 inputs, fp32 accumulation: O
-TOL_BF16_LSE = 1e-2     # bf16 path LSE (the pages state none)
+TOL_BF16_LSE = 1e-2     # bf16 path LSE: the pages state none; half the O bound
 TOL_BF16_GRAD = 5e-2    # dQ, dK, dV
 
 

@@ -1,9 +1,12 @@
 """GPU parity of the blockwise SwiGLU feed-forward (tcgen05 GEMMs) against
 the fp64 oracle on the same seeded bf16 input bits.
 
-Tolerance (derived in the design doc): |y_gpu - y_ref| <= 2^-8 |y_ref| + 0.03.
-The relative part covers the final bf16 rounding of y (2^-9) with margin;
-the absolute part covers h rounded to bf16 before the down projection."""
+Tolerance: |y_gpu - y_ref| <= 2^-8 |y_ref| + 0.03.  The relative part
+covers the final bf16 rounding of y (2^-9) with margin.  The absolute part
+covers h rounded to bf16 (relative 2^-9) before the down projection: y sums
+d_ff = 11008 products with w ~ N(0, 0.02^2) and |h| about 1.2, so the
+rounding gives about 2.7e-3 rms in y, about 0.015 at 5.5 sigma over 8M
+outputs."""
 
 import numpy as np
 import pytest
