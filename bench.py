@@ -65,7 +65,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (smaller profiling cases)")
-    ap.add_argument("--tokens", type=int, default=0, help="override the sequence length of layer7b_full")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the sequence length of layer7b_full or the cache length of decode_n128k")
     return ap.parse_args()
 
 
@@ -291,6 +292,8 @@ def run_decode(args, ra, dev, rank, world, dist):
     from dataclasses import replace
     from exact_blockwise_long_b200.synthetic import DECODE_WORKLOADS, decode_inputs
     w = DECODE_WORKLOADS[args.workload]
+    if args.tokens:  # a shorter cache (smaller profiling cases)
+        w = replace(w, N=args.tokens)
     q, k, v = decode_inputs(replace(w, seed=w.seed + 1000 * rank), device=dev)
     out = torch.empty_like(q)
     lse = torch.empty((w.B, w.H), device=dev, dtype=torch.float32)
