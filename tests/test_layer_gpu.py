@@ -70,6 +70,7 @@ CASES = [
     (1, 1024, 2, 128, 384, 4, 128, 128, 256, True),
     (2, 512, 4, 64, 512, 2, 128, 256, 512, True),
     (1, 768, 2, 128, 256, 3, 256, 128, 256, False),
+    (1, 4096, 2, 128, 256, 2, 256, 512, 1024, True),  # four FFN chunks, long weight-gradient K
 ]
 
 
