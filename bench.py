@@ -42,14 +42,14 @@ METRIC = "ring-attn fwd+bwd TFLOP/s & tokens/s on 1 B200; % of BF16 tensor peak"
 # (heads are independent units; see profiles/*_n32k_d128_h8.md).
 NCU_TRAFFIC = {
     ("bwd_kv_kernel", "n32k_d128"): {
-        "bytes": 4 * (272.112128e6 + 107.426816e6),
-        "sha256": "1e5d1c805c75bc9da5373177b94fe9ffc8ed319fd715584d09866ecbff829fda"},
+        "bytes": 4 * (272.113664e6 + 104.500992e6),
+        "sha256": "79e59b3f198f9446fd9f59500a14cd01c91fa2c9a9609c3ae931a483fce5ab9c"},
     ("bwd_q_kernel", "n32k_d128"): {
-        "bytes": 4 * (271.273472e6 + 51.107840e6),
-        "sha256": "1e5d1c805c75bc9da5373177b94fe9ffc8ed319fd715584d09866ecbff829fda"},
+        "bytes": 4 * (271.004928e6 + 48.961280e6),
+        "sha256": "79e59b3f198f9446fd9f59500a14cd01c91fa2c9a9609c3ae931a483fce5ab9c"},
     ("fwd_tc2_kernel", "n32k_d128"): {
-        "bytes": 4 * (202.958592e6 + 49.582848e6),
-        "sha256": "e9db5aae1017ae8e993d973016b04ffacdea9fd4f4df0e639cd340068e47deb0"},
+        "bytes": 4 * (202.573056e6 + 48.696576e6),
+        "sha256": "5c686052862a91d3ec7544ef7ec3b53956e0efd7f35b73a76a07e6677b666c14"},
 }
 
 
