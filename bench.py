@@ -60,7 +60,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="n32k_d128",
                     choices=["n32k_d128", "n8k_d64_causal", "n8k_d64_full", "layer7b", "layer7b_full",
-                             "n1m_d128", "n32k_d128_gqa8", "decode_n128k"])
+                             "n1m_d128", "n32k_d128_gqa8", "decode_n128k", "n32k_d128_step", "merge_n32k"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -284,6 +284,81 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # the native arm
 # ---------------------------------------------------------------------------
+
+def run_step_mode(args, ra, dev, rank, world, dist):
+    """Auxiliary workloads of the 32k shapes.
+
+    n32k_d128_step: the causal forward as S ring steps (ringattn_fwd_step,
+    each merging its partial exactly into fp32 accumulators in HBM), the
+    per-step building block of a multi-device ring; compare its TFLOP/s with
+    the fused whole-ring forward.  merge_n32k: the standalone exact merge
+    (ringattn_merge) of two fp32 partials of every row, HBM-bound."""
+    import torch
+    from dataclasses import replace
+    from exact_blockwise_long_b200.synthetic import WORKLOADS, attention_inputs
+    w = replace(WORKLOADS["n32k_d128"], bwd=False)
+    q, k, v, _ = attention_inputs(replace(w, seed=w.seed + 1000 * rank), device=dev)
+    B, H, N, D = q.shape
+    stream = torch.cuda.current_stream()
+    o_acc = torch.empty((B, H, N, D), device=dev, dtype=torch.float32)
+    lse_acc = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+    if args.workload == "n32k_d128_step":
+        def step():
+            o_acc.zero_()
+            lse_acc.fill_(float("-inf"))
+            for t in range(w.S):
+                ra.ringattn_fwd_step(q, k, v, o_acc, lse_acc, w.S, w.q_chunk, w.k_chunk, w.causal, t)
+        launches = w.S
+    else:
+        o_b = torch.randn((B, H, N, D), device=dev)
+        l_b = torch.randn((B, H, N), device=dev)
+        o_acc.normal_()
+        lse_acc.normal_()
+
+        def step():
+            ra.ringattn_merge(o_acc, lse_acc, o_b, l_b)
+        launches = 1
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if ra.ringattn_get_error() != 0:
+        raise RuntimeError("device status word set during the timed region")
+    ms = max_over_ranks(a.elapsed_time(b) / args.steps, dist if world > 1 else None, dev)
+    pk = peaks()
+    if args.workload == "n32k_d128_step":
+        fl = attn_fwd_flops(w)
+        tf = whole_job_tflops(fl, world, ms)
+        return {"metric": METRIC, "value": tf, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": f"n32k_d128_step: causal forward as {w.S} ring steps merged into fp32 "
+                                       f"HBM accumulators, B={B}, H={H}, N={N}, d={D}"},
+                "roofline": {"bound": "tensor", "kernel": "fwd_tc2_kernel (step mode)", "achieved": tf,
+                             "peak": pk["bf16_sustained"], "unit": "TFLOP/s", "frac": tf / pk["bf16_sustained"],
+                             "traffic": None, "peak_kind": f"bf16 dense, sustained ({pk['source']})"},
+                "gpu_launches": launches * args.steps, "clocks": clk}
+    rows = B * H * N
+    nbytes = rows * (3 * D * 4 + 3 * 4)  # read o_a, o_b, lse_a, lse_b; write o_a, lse_a
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"metric": "ringattn_merge HBM throughput (auxiliary)", "value": gbs * world, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"merge_n32k: exact merge of two fp32 partials of {rows} rows, d={D}"},
+            "roofline": {"bound": "hbm", "kernel": "merge_kernel", "achieved": gbs, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                         "peak_kind": f"HBM copy ({pk['source']})"},
+            "gpu_launches": launches * args.steps, "clocks": clk}
+
 
 def run_decode(args, ra, dev, rank, world, dist):
     """One decode step (new token per head against the sharded cache) per
@@ -585,8 +660,9 @@ def main():
     from dataclasses import replace
     from exact_blockwise_long_b200.synthetic import attention_inputs, ffn_inputs
 
-    if args.workload.startswith("decode") or args.workload == "layer7b_full":
-        runner = run_decode if args.workload.startswith("decode") else run_layer
+    if args.workload.startswith("decode") or args.workload in ("layer7b_full", "n32k_d128_step", "merge_n32k"):
+        runner = (run_decode if args.workload.startswith("decode") else
+                  run_layer if args.workload == "layer7b_full" else run_step_mode)
         line = runner(args, ra, dev, rank, world, dist)
         if world > 1:
             dist.barrier()

@@ -17,6 +17,31 @@ namespace {
 
 constexpr int kWarps = 8;
 
+// Weights of the two partials of one row; (-inf, anything) is the neutral
+// element and never enters a subtraction.
+__device__ __forceinline__ void merge_weights(float la, float lb, float& wa, float& wb, float& lse) {
+  const bool a_empty = (la == -INFINITY), b_empty = (lb == -INFINITY);
+  if (!a_empty && !b_empty) {
+    const float m = fmaxf(la, lb);
+    const float ea = expf(la - m), eb = expf(lb - m);
+    const float tot = ea + eb;
+    lse = m + logf(tot);
+    wa = ea / tot;
+    wb = eb / tot;
+  } else if (!b_empty) {
+    wa = 0.f;
+    wb = 1.f;
+    lse = lb;
+  } else {  // right side empty: the left one stands; both empty: zero row, lse -inf
+    wa = a_empty ? 0.f : 1.f;
+    wb = 0.f;
+    lse = la;
+  }
+}
+
+// One warp per row pair per iteration: every load of both rows (the two
+// LSEs and the D-float rows of both partials) is issued before any of them
+// is used, so a row costs one memory round trip, not two.
 __global__ void __launch_bounds__(kWarps * 32) merge_kernel(float* __restrict__ o_a, float* __restrict__ lse_a,
                                                             const float* __restrict__ o_b,
                                                             const float* __restrict__ lse_b, int64_t rows,
@@ -24,39 +49,46 @@ __global__ void __launch_bounds__(kWarps * 32) merge_kernel(float* __restrict__ 
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * kWarps;
-  for (int64_t row = warp0; row < rows; row += nwarps) {
-    const float la = lse_a[row];
-    const float lb = __ldg(&lse_b[row]);
-    float4* pa = reinterpret_cast<float4*>(o_a + row * (int64_t)D4 * 4);
-    const float4* pb = reinterpret_cast<const float4*>(o_b + row * (int64_t)D4 * 4);
-    const bool a_empty = (la == -INFINITY), b_empty = (lb == -INFINITY);
-    if (b_empty && !a_empty) continue;  // neutral element on the right
-    float wa = 0.f, wb = 0.f, lse = -INFINITY;
-    if (!a_empty && !b_empty) {
-      const float m = fmaxf(la, lb);
-      const float ea = expf(la - m), eb = expf(lb - m);
-      const float tot = ea + eb;
-      lse = m + logf(tot);
-      wa = ea / tot;
-      wb = eb / tot;
-    } else if (!b_empty) {
-      wb = 1.f;
-      lse = lb;
-    }
+  for (int64_t r0 = warp0; r0 < rows; r0 += 2 * nwarps) {
+    const int64_t r1 = r0 + nwarps;
+    const bool has1 = r1 < rows;
+    const float la0 = lse_a[r0], lb0 = __ldg(&lse_b[r0]);
+    const float la1 = has1 ? lse_a[r1] : -INFINITY, lb1 = has1 ? __ldg(&lse_b[r1]) : -INFINITY;
+    float4* pa0 = reinterpret_cast<float4*>(o_a + r0 * (int64_t)D4 * 4);
+    const float4* pb0 = reinterpret_cast<const float4*>(o_b + r0 * (int64_t)D4 * 4);
+    float4* pa1 = reinterpret_cast<float4*>(o_a + r1 * (int64_t)D4 * 4);
+    const float4* pb1 = reinterpret_cast<const float4*>(o_b + r1 * (int64_t)D4 * 4);
     for (int c = lane; c < D4; c += 32) {
-      float4 r;
-      if (a_empty && b_empty) {
-        r = make_float4(0.f, 0.f, 0.f, 0.f);
-      } else if (a_empty) {
-        r = __ldg(&pb[c]);
-      } else {
-        const float4 x = pa[c];
-        const float4 y = __ldg(&pb[c]);
-        r = make_float4(wa * x.x + wb * y.x, wa * x.y + wb * y.y, wa * x.z + wb * y.z, wa * x.w + wb * y.w);
+      const float4 x0 = pa0[c], y0 = __ldg(&pb0[c]);
+      float4 x1 = make_float4(0.f, 0.f, 0.f, 0.f), y1 = x1;
+      if (has1) {
+        x1 = pa1[c];
+        y1 = __ldg(&pb1[c]);
       }
-      pa[c] = r;
+      float wa, wb, l;
+      merge_weights(la0, lb0, wa, wb, l);
+      // an empty side contributes nothing even if its payload is not finite
+      pa0[c] = make_float4((wa != 0.f ? wa * x0.x : 0.f) + (wb != 0.f ? wb * y0.x : 0.f),
+                           (wa != 0.f ? wa * x0.y : 0.f) + (wb != 0.f ? wb * y0.y : 0.f),
+                           (wa != 0.f ? wa * x0.z : 0.f) + (wb != 0.f ? wb * y0.z : 0.f),
+                           (wa != 0.f ? wa * x0.w : 0.f) + (wb != 0.f ? wb * y0.w : 0.f));
+      if (has1) {
+        merge_weights(la1, lb1, wa, wb, l);
+        pa1[c] = make_float4((wa != 0.f ? wa * x1.x : 0.f) + (wb != 0.f ? wb * y1.x : 0.f),
+                             (wa != 0.f ? wa * x1.y : 0.f) + (wb != 0.f ? wb * y1.y : 0.f),
+                             (wa != 0.f ? wa * x1.z : 0.f) + (wb != 0.f ? wb * y1.z : 0.f),
+                             (wa != 0.f ? wa * x1.w : 0.f) + (wb != 0.f ? wb * y1.w : 0.f));
+      }
     }
-    if (lane == 0) lse_a[row] = lse;
+    if (lane == 0) {
+      float wa, wb, l;
+      merge_weights(la0, lb0, wa, wb, l);
+      lse_a[r0] = l;
+      if (has1) {
+        merge_weights(la1, lb1, wa, wb, l);
+        lse_a[r1] = l;
+      }
+    }
   }
 }
 
