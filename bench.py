@@ -257,8 +257,14 @@ def run_reference(args):
         sampler = lambda: layer_oracle_sample(lw)  # noqa: E731
         config = {"workload": f"{lw.name}: one blockwise transformer layer fwd+bwd, N={lw.N}, H={lw.H}, "
                               f"d={lw.D}, d_ff={lw.d_ff}, S={lw.S}"}
+    elif args.workload == "merge_n32k":
+        sampler = merge_oracle_sample
+        config = {"workload": "merge_n32k: exact merge of two fp32 partials per row, d=128"}
     else:
-        aw, fw = workload(args.workload)
+        name = "n32k_d128" if args.workload == "n32k_d128_step" else args.workload
+        aw, fw = workload(name)
+        if args.workload == "n32k_d128_step":
+            aw = replace(aw, bwd=False)  # the step-mode workload is the forward
         if args.heads:
             aw = replace(aw, H=args.heads)
         sampler = lambda: oracle_sample(aw, fw)  # noqa: E731
@@ -470,6 +476,26 @@ def decode_oracle_sample(w, min_seconds=2.0):
         threads = os.cpu_count()
     desc = f"fp64 oracle (numpy) decode of {groups} (batch, key/value head) group(s) of {G} query heads, N={w.N}"
     return dt, 4.0 * G * w.N * w.D * groups, desc, threads
+
+
+def merge_oracle_sample(rows=1 << 18, D=128):
+    """The fp64 oracle's exact merge on `rows` rows of random partials (about
+    a quarter of the merge workload's rows).  Returns (seconds, the merge's
+    FLOPs counted as 3 per output element, desc, threads)."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(11)
+    o_a, o_b = rng.standard_normal((rows, D)), rng.standard_normal((rows, D))
+    l_a, l_b = rng.standard_normal(rows) * 5, rng.standard_normal(rows) * 5
+    t0 = time.perf_counter()
+    oracle.lse_merge(o_a, l_a, o_b, l_b)
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    return dt, 3.0 * rows * D, f"fp64 oracle (numpy) lse_merge of {rows} rows of d={D}", threads
 
 
 def run_layer(args, ra, dev, rank, world, dist):
