@@ -42,11 +42,11 @@ METRIC = "ring-attn fwd+bwd TFLOP/s & tokens/s on 1 B200; % of BF16 tensor peak"
 # (heads are independent units; see profiles/*_n32k_d128_h8.md).
 NCU_TRAFFIC = {
     ("bwd_kv_kernel", "n32k_d128"): {
-        "bytes": 4 * (272.113664e6 + 104.500992e6),
-        "sha256": "79e59b3f198f9446fd9f59500a14cd01c91fa2c9a9609c3ae931a483fce5ab9c"},
+        "bytes": 4 * (272.233984e6 + 103.432192e6),
+        "sha256": "c874611cfb2c61df7872652125c6ea89c7b4fc8e5a4e900c3b5b996c615147b0"},
     ("bwd_q_kernel", "n32k_d128"): {
-        "bytes": 4 * (271.004928e6 + 48.961280e6),
-        "sha256": "79e59b3f198f9446fd9f59500a14cd01c91fa2c9a9609c3ae931a483fce5ab9c"},
+        "bytes": 4 * (271.248384e6 + 47.282432e6),
+        "sha256": "c874611cfb2c61df7872652125c6ea89c7b4fc8e5a4e900c3b5b996c615147b0"},
     ("fwd_tc2_kernel", "n32k_d128"): {
         "bytes": 4 * (202.573056e6 + 48.696576e6),
         "sha256": "5c686052862a91d3ec7544ef7ec3b53956e0efd7f35b73a76a07e6677b666c14"},

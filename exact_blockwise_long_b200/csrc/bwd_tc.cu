@@ -39,6 +39,12 @@ constexpr int kT = 128;        // rows per tile (TMEM lanes)
 constexpr int kSt = 2;         // streamed-tile stages
 constexpr int kThreads = 384;   // 4 role warps + two element-wise warpgroups
 constexpr int kHalf = 64;      // score columns per element-wise warpgroup
+// At d = 64 the four matmuls of a dK/dV step take half as long as at
+// d = 128 while the exponentials do not, so the MUFU would bound that pass:
+// there every second exponential pair is computed by ex2_poly2 on the
+// FMA/integer pipes (0.76 -> 0.72 ms on the causal 8k workload).  Everywhere
+// else all stay on the MUFU: moving some was measured no faster at d = 128
+// and slower in the dQ pass.
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t FULL = 0xffffffffu;
@@ -345,8 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < kHalf; c += 2) {
         const float2 t = fma2(make_float2(P[c], P[c + 1]), sl22, make_float2(-lse2[c], -lse2[c + 1]));
-        P[c] = ex2_approx(t.x);
-        P[c + 1] = ex2_approx(t.y);
+        const float2 e = (D == 64 && (c / 2) % 2 == 1) ? ex2_poly2(t) : make_float2(ex2_approx(t.x), ex2_approx(t.y));
+        P[c] = e.x;
+        P[c + 1] = e.y;
       }
       if (diag) {
 #pragma unroll
