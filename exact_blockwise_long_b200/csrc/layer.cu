@@ -68,9 +68,12 @@ Saved carve_saved(void* p, int64_t B, int64_t N, int64_t H, int64_t D) {
 bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // shape rules shared by forward and backward
+// kNoTokens: a valid request with an empty batch (B == 0)
+constexpr int kNoTokens = 1;
+
 int check_layer(int64_t B, int64_t N, int64_t H, int64_t D, int64_t d_ff, int S, int q_chunk, int k_chunk,
                 int ffn_chunk, int causal) {
-  if (B <= 0 || N <= 0 || H <= 0 || D <= 0 || d_ff <= 0 || S <= 0 || q_chunk <= 0 || k_chunk <= 0 ||
+  if (B < 0 || N <= 0 || H <= 0 || D <= 0 || d_ff <= 0 || S <= 0 || q_chunk <= 0 || k_chunk <= 0 ||
       ffn_chunk <= 0)
     return RA_ERR_ARG;
   if (causal != 0 && causal != 1) return RA_ERR_ARG;
@@ -83,7 +86,7 @@ int check_layer(int64_t B, int64_t N, int64_t H, int64_t D, int64_t d_ff, int S,
   const int64_t T = B * N;
   if (T % ffn_chunk || ffn_chunk % 128 || d_ff % 128) return RA_ERR_SHAPE;
   if (B * H * N > (int64_t)INT32_MAX / 2 || d_ff > INT32_MAX / 4) return RA_ERR_UNSUPPORTED;
-  return RA_OK;
+  return B == 0 ? kNoTokens : RA_OK;
 }
 
 GemmOperand plain(const void* p, int64_t rows, int64_t cols, int mn) {
@@ -149,6 +152,7 @@ int blockwise_layer_fwd(const void* x, const void* g_attn, const void* wq, const
                         int S, int q_chunk, int k_chunk, int causal, int ffn_chunk, float eps, void* workspace,
                         size_t workspace_bytes, void* const* marks, void* stream) {
   int rc = check_layer(B, N, H, D, d_ff, S, q_chunk, k_chunk, ffn_chunk, causal);
+  if (rc == kNoTokens) return RA_OK;  // no tokens: nothing to compute
   if (rc != RA_OK) return rc;
   if (!(eps > 0.f)) return RA_ERR_ARG;
   const void* ptrs[] = {x, g_attn, wq, wk, wv, wo, g_ffn, w1, w2, w3, y, saved, workspace};
@@ -194,6 +198,18 @@ int blockwise_layer_bwd(const void* x, const void* g_attn, const void* wq, const
                         int causal, int ffn_chunk, void* workspace, size_t workspace_bytes, void* const* marks,
                         void* stream) {
   int rc = check_layer(B, N, H, D, d_ff, S, q_chunk, k_chunk, ffn_chunk, causal);
+  if (rc == kNoTokens) {  // no tokens: every parameter gradient is zero
+    const size_t dm = (size_t)(H * D), ff = (size_t)d_ff;
+    float* grads[] = {dg_attn, dwq, dwk, dwv, dwo, dg_ffn, dw1, dw2, dw3};
+    const size_t n[] = {dm, dm * dm, dm * dm, dm * dm, dm * dm, dm, ff * dm, dm * ff, ff * dm};
+    for (int i = 0; i < 9; ++i) {
+      if (!grads[i]) return RA_ERR_ARG;
+      if (!a16(grads[i])) return RA_ERR_ALIGN;
+    }
+    for (int i = 0; i < 9; ++i)
+      if (cudaMemsetAsync(grads[i], 0, n[i] * 4, static_cast<cudaStream_t>(stream)) != cudaSuccess) return RA_ERR_CUDA;
+    return RA_OK;
+  }
   if (rc != RA_OK) return rc;
   const void* ptrs[] = {x,   g_attn, wq,  wk,  wv,     wo,  g_ffn, w1,  w2,  w3,       saved,
                         dy,  dx,     dg_attn, dwq, dwk, dwv, dwo, dg_ffn, dw1, dw2, dw3, workspace};

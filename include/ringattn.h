@@ -348,6 +348,8 @@ RA_API int ringattn_cast(const float* x, void* out, int64_t n, int dtype, void* 
  *     k, v, o, x2, xn2, lse, both rstd) and read by the backward
  *   gradients: dx bf16; dg_attn, dg_ffn [H*D] fp32; dwq, dwk, dwv, dwo,
  *     dw1, dw2, dw3 fp32 in the weights' shapes (written, not accumulated)
+ * B == 0 is valid: the forward does nothing and the backward zeroes the
+ * nine parameter gradients (token pointers may then be null).
  * Rules: D in {64, 128}; H*D in {256, 512, 1024, 2048, 4096}; N % 128 == 0;
  * the attention's shard and chunk rules (N % S, shard % chunk, chunks
  * multiples of 128); (B*N) % ffn_chunk == 0, ffn_chunk and d_ff multiples

@@ -124,3 +124,67 @@ def test_product_path_has_no_oracle_or_fallback():
         if fn.endswith(".py"):
             src = open(os.path.join(pkg, fn)).read()
             assert "import oracle" not in src and "from oracle" not in src, fn
+
+
+def test_ffn_bwd_contract(L):
+    f = L.blockwise_ffn_bwd
+    ws = L.blockwise_ffn_bwd_workspace_size(2048, 11008, 0)
+    assert ws == 2048 * 11008 * (4 + 3 * 2)          # dh fp32 + dg, du, h bf16
+    assert L.blockwise_ffn_bwd_workspace_size(2048, 11008, 1) == 0
+    ptrs = [FAKE] * 9
+    assert f(*ptrs, 4000, 4096, 11008, 2048, 0, FAKE, ws, None) == -2          # T % chunk
+    assert f(*ptrs, 4096, 4096, 11000, 2048, 0, FAKE, ws, None) == -2          # d_ff % 128
+    assert f(*ptrs, 4096, 4096, 11008, 2048, 1, FAKE, ws, None) == -5          # fp32 not built
+    assert f(*ptrs, 4096, 4096, 11008, 2048, 9, FAKE, ws, None) == -3
+    assert f(*ptrs, 4096, 4096, 11008, 2048, 0, FAKE, ws - 16, None) == -8
+    assert f(*([MIS] + ptrs[1:]), 4096, 4096, 11008, 2048, 0, FAKE, ws, None) == -4
+    assert f(*([FAKE] * 6 + [None] + [FAKE] * 2), 4096, 4096, 11008, 2048, 0, FAKE, ws, None) == -1
+
+
+def test_layer_contract(L):
+    B, N, H, D, dff = 1, 4096, 32, 128, 11008
+    saved = L.blockwise_layer_saved_size(B, N, H, D)
+    dm = H * D
+    assert saved >= 7 * N * dm * 2 + 3 * N * 4        # seven bf16 activations, lse and two rstd rows
+    fws = L.blockwise_layer_fwd_workspace_size(2048, dff)
+    bws = L.blockwise_layer_bwd_workspace_size(B, N, H, D, dff, 2048)
+    assert fws == 2048 * dff * 2 and bws > 7 * N * dm * 2
+    fwd = L.blockwise_layer_fwd
+    p12 = [FAKE] * 12
+
+    def fw(*, ptrs=p12, B=B, N=N, H=H, D=D, dff=dff, S=2, qc=2048, kc=2048, causal=1, fc=2048, eps=1e-5,
+           sv=saved, ws=FAKE, wsb=fws):
+        return fwd(*ptrs, sv, B, N, H, D, dff, S, qc, kc, causal, fc, eps, ws, wsb, None, None)
+
+    assert fw(S=3) == -2                 # N % S
+    assert fw(D=96) == -5                # head dim
+    assert fw(H=24) == -5                # d_model 3072 not built (RMS norm rows)
+    assert fw(fc=1000) == -2             # ffn chunk
+    assert fw(eps=0.0) == -1
+    assert fw(sv=saved - 1) == -8
+    assert fw(wsb=fws - 1) == -8
+    assert fw(ptrs=[None] + p12[1:]) == -1
+    assert fw(ptrs=p12[:5] + [MIS] + p12[6:]) == -4
+    assert fw(B=0, ptrs=[None] * 12, ws=None, wsb=0) == 0   # no tokens: nothing to do
+    bwd = L.blockwise_layer_bwd
+    grads = [FAKE] * 9
+
+    def bw(*, B=B, S=2, g=grads, wsb=bws):
+        return bwd(*([FAKE] * 11), saved, FAKE, FAKE, *g, B, N, H, D, dff, S, 2048, 2048, 1, 2048, FAKE, wsb,
+                   None, None)
+
+    assert bw(S=3) == -2
+    assert bw(wsb=bws - 1) == -8
+    assert bw(g=[None] + grads[1:]) == -1
+    assert bw(B=0, g=[MIS] + grads[1:]) == -4   # no tokens: the gradients must still be valid
+
+
+def test_accumulate_and_cast_contract(L):
+    assert L.ringattn_accumulate(None, FAKE, 16, 0, None) == -1
+    assert L.ringattn_accumulate(FAKE, FAKE, -1, 0, None) == -1
+    assert L.ringattn_accumulate(FAKE, FAKE, 16, 5, None) == -3
+    assert L.ringattn_accumulate(MIS, FAKE, 16, 0, None) == -4
+    assert L.ringattn_accumulate(None, None, 0, 0, None) == 0   # nothing to do
+    assert L.ringattn_cast(FAKE, None, 16, 0, None) == -1
+    assert L.ringattn_cast(FAKE, MIS, 16, 0, None) == -4
+    assert L.ringattn_cast(None, None, 0, 1, None) == 0
