@@ -115,3 +115,20 @@ def test_layer_bad_shapes():
         ra.blockwise_layer_fwd(x, params, y, saved, 1, 1024, 2, 128, 3, 128, 128, True, 256, fws)
     with pytest.raises(RingAttnError):   # the saved buffer is too small
         ra.blockwise_layer_fwd(x, params, y, saved[:1024], 1, 1024, 2, 128, 4, 128, 128, True, 256, fws)
+
+
+def test_layer_empty_batch():
+    """No tokens: the forward does nothing, the backward zeroes the nine
+    parameter gradients."""
+    import exact_blockwise_long_b200 as ra
+    w = LayerWorkload("t", 1, 256, 2, 128, 256, 2, 128, 128, 256, 8)
+    x, params, dy = layer_inputs(w)
+    grads = tuple(torch.full(p.shape, 3.0, device="cuda", dtype=torch.float32) for p in params)
+    e = x[:0]
+    empty = torch.empty(0, device="cuda", dtype=torch.uint8)
+    assert ra.lib().blockwise_layer_fwd(*([None] * 12), 0, 0, 256, 2, 128, 256, 2, 128, 128, 1, 256, 1e-5, None,
+                                        0, None, None) == 0
+    ra.blockwise_layer_bwd(e, params, empty, dy[:0], torch.empty_like(e), grads, 0, 256, 2, 128, 2, 128, 128,
+                           True, 256, empty)
+    assert ra.ringattn_get_error() == 0
+    assert all(torch.count_nonzero(g) == 0 for g in grads)
