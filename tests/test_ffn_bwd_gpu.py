@@ -141,3 +141,35 @@ def test_ffn_bwd_7b_shape_sampled():
     check(to_f64(dw1[ui]), r1, t1, False)
     check(to_f64(dw2[:, ui]), r2, t2, False)
     check(to_f64(dw3[ui]), r3, t3, False)
+
+
+@pytest.mark.slow
+def test_ffn_bwd_7b_full_size_sampled():
+    """The layer workload's FFN backward at full size (131072 tokens, 64
+    chunks): 16 seeded dx rows, and the weight gradients of 8 seeded hidden
+    units summed over all tokens (the oracle runs on 8192-token slices of
+    those units and adds the slices up in fp64)."""
+    w = FFN_WORKLOADS["layer7b_ffn"]
+    x, w1, w2, w3, dy = ffn_inputs(w, with_dy=True)
+    dx, dw1, dw2, dw3 = run_ffn_bwd(x, w1, w2, w3, dy, w.chunk)
+    rng = np.random.default_rng(w.seed + 5000)
+    rows = np.sort(rng.choice(w.T, 16, replace=False))
+    rows[0], rows[-1] = 0, w.T - 1
+    units = np.sort(rng.choice(w.d_ff, 8, replace=False))
+    W1, W2, W3 = to_f64(w1), to_f64(w2), to_f64(w3)
+    ri = torch.as_tensor(rows, device="cuda")
+    xs, dys = to_f64(x[ri]), to_f64(dy[ri])
+    check(to_f64(dx[ri]), oracle.swiglu_ffn_backward(xs, W1, W2, W3, dys)[0],
+          oracle.swiglu_ffn_backward_terms(xs, W1, W2, W3, dys)[0], final_round=True)
+    ref = [np.zeros((len(units), w.d_model)), np.zeros((w.d_model, len(units))), np.zeros((len(units), w.d_model))]
+    trm = [np.zeros_like(r) for r in ref]
+    for c0 in range(0, w.T, 8192):
+        sub = (to_f64(x[c0:c0 + 8192]), W1[units], W2[:, units], W3[units], to_f64(dy[c0:c0 + 8192]))
+        _, r1, r2, r3 = oracle.swiglu_ffn_backward(*sub)
+        _, t1, t2, t3 = oracle.swiglu_ffn_backward_terms(*sub)
+        for acc, part in zip(ref + trm, (r1, r2, r3, t1, t2, t3)):
+            acc += part
+    ui = torch.as_tensor(units, device="cuda")
+    check(to_f64(dw1[ui]), ref[0], trm[0], False)
+    check(to_f64(dw2[:, ui]), ref[1], trm[1], False)
+    check(to_f64(dw3[ui]), ref[2], trm[2], False)
