@@ -16,7 +16,7 @@ namespace ra {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kDgRows = 256;  // rows per dg partial
+constexpr int kDgRows = 64;  // rows per dg partial
 
 __device__ __forceinline__ void unpack8(const uint4& q, float (&f)[8]) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
@@ -107,34 +107,73 @@ __global__ void __launch_bounds__(kWarps * 32)
   }
 }
 
-// partial[blk][c] = sum over the rows of block blk of dxn[t][c] * x[t][c] * rstd[t]
-// (each thread owns two adjacent columns)
-__global__ void __launch_bounds__(256) rmsnorm_dg_partial_kernel(const uint32_t* __restrict__ x,
-                                                                 const uint32_t* __restrict__ dxn,
-                                                                 const float* __restrict__ rstd,
-                                                                 float* __restrict__ partial, int T, int dm) {
-  const int cp = blockIdx.x * 256 + threadIdx.x;  // column pair
-  if (2 * cp >= dm) return;
+// partial[blk][c] = sum over the rows of block blk of dxn[t][c] * x[t][c] * rstd[t].
+// Each thread owns eight adjacent columns (16-byte loads) and walks the
+// block's rows four at a time, so eight independent loads are in flight.
+constexpr int kDgThreads = 128;  // x 8 columns = 1024 columns per CTA
+__global__ void __launch_bounds__(kDgThreads) rmsnorm_dg_partial_kernel(const uint4* __restrict__ x,
+                                                                        const uint4* __restrict__ dxn,
+                                                                        const float* __restrict__ rstd,
+                                                                        float* __restrict__ partial, int T, int dm) {
+  const int v = blockIdx.x * kDgThreads + threadIdx.x;  // 8-column group
+  const int nv = dm / 8;
+  if (v >= nv) return;
   const int t0 = blockIdx.y * kDgRows;
   const int t1 = min(T, t0 + kDgRows);
-  float a0 = 0.f, a1 = 0.f;
-  for (int t = t0; t < t1; ++t) {
-    const uint32_t xv = x[(size_t)t * (dm / 2) + cp], dv = dxn[(size_t)t * (dm / 2) + cp];
-    const float r = rstd[t];
-    a0 = fmaf(__uint_as_float(dv << 16), __uint_as_float(xv << 16) * r, a0);
-    a1 = fmaf(__uint_as_float(dv & 0xffff0000u), __uint_as_float(xv & 0xffff0000u) * r, a1);
+  float a[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) a[e] = 0.f;
+  int t = t0;
+  for (; t + 4 <= t1; t += 4) {
+    uint4 xv[4], dv[4];
+    float r[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      xv[u] = x[(size_t)(t + u) * nv + v];
+      dv[u] = dxn[(size_t)(t + u) * nv + v];
+      r[u] = rstd[t + u];
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float xf[8], df[8];
+      unpack8(xv[u], xf);
+      unpack8(dv[u], df);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) a[e] = fmaf(df[e], xf[e] * r[u], a[e]);
+    }
   }
-  partial[(size_t)blockIdx.y * dm + 2 * cp] = a0;
-  partial[(size_t)blockIdx.y * dm + 2 * cp + 1] = a1;
+  for (; t < t1; ++t) {
+    float xf[8], df[8];
+    unpack8(x[(size_t)t * nv + v], xf);
+    unpack8(dxn[(size_t)t * nv + v], df);
+    const float r = rstd[t];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) a[e] = fmaf(df[e], xf[e] * r, a[e]);
+  }
+  float4* dst = reinterpret_cast<float4*>(partial + (size_t)blockIdx.y * dm + (size_t)v * 8);
+  dst[0] = make_float4(a[0], a[1], a[2], a[3]);
+  dst[1] = make_float4(a[4], a[5], a[6], a[7]);
 }
 
+// dg[c] = sum over the blocks of partial[blk][c], in a fixed order: warp w
+// of a CTA sums blocks w, w + 8, ... for 32 adjacent columns, then the eight
+// warp sums are added in warp order.
 __global__ void __launch_bounds__(256) rmsnorm_dg_reduce_kernel(const float* __restrict__ partial, int nblk, int dm,
                                                                 float* __restrict__ dg) {
-  const int c = blockIdx.x * 256 + threadIdx.x;
-  if (c >= dm) return;
+  __shared__ float sh[8][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c = blockIdx.x * 32 + lane;
   float s = 0.f;
-  for (int b = 0; b < nblk; ++b) s += partial[(size_t)b * dm + c];
-  dg[c] = s;
+  if (c < dm)
+    for (int b = warp; b < nblk; b += 8) s += partial[(size_t)b * dm + c];
+  sh[warp][lane] = s;
+  __syncthreads();
+  if (warp == 0 && c < dm) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += sh[w][lane];
+    dg[c] = t;
+  }
 }
 
 template <int V>
@@ -189,10 +228,10 @@ int launch_rmsnorm_bwd(const void* x, const void* g, const float* rstd, const vo
   }
   if (rc != RA_OK) return rc;
   const int nblk = (int)((T + kDgRows - 1) / kDgRows);
-  const dim3 pgrid((unsigned)((d_model / 2 + 255) / 256), (unsigned)nblk);
-  rmsnorm_dg_partial_kernel<<<pgrid, 256, 0, stream>>>((const uint32_t*)x, (const uint32_t*)dxn, rstd, partial,
-                                                       (int)T, (int)d_model);
-  rmsnorm_dg_reduce_kernel<<<(unsigned)((d_model + 255) / 256), 256, 0, stream>>>(partial, nblk, (int)d_model, dg);
+  const dim3 pgrid((unsigned)((d_model / 8 + kDgThreads - 1) / kDgThreads), (unsigned)nblk);
+  rmsnorm_dg_partial_kernel<<<pgrid, kDgThreads, 0, stream>>>((const uint4*)x, (const uint4*)dxn, rstd, partial,
+                                                              (int)T, (int)d_model);
+  rmsnorm_dg_reduce_kernel<<<(unsigned)((d_model + 31) / 32), 256, 0, stream>>>(partial, nblk, (int)d_model, dg);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
