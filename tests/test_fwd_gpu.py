@@ -97,9 +97,11 @@ def test_bf16_sharp_softmax_rescale_path():
 
 
 def test_bf16_deterministic():
+    """Race check by repetition: a missing wait would show up as run-to-run
+    differences, so twenty runs must give identical bits."""
     q, k, v, _ = small_attention_inputs(1, 4, 2048, 128, 7)
     o1, l1 = run_fwd(q, k, v, 4, 256, 256, True)
-    for _ in range(5):
+    for _ in range(20):
         o2, l2 = run_fwd(q, k, v, 4, 256, 256, True)
         assert torch.equal(o1, o2) and torch.equal(l1, l2)
 

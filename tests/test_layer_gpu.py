@@ -132,3 +132,15 @@ def test_layer_empty_batch():
                            True, 256, empty)
     assert ra.ringattn_get_error() == 0
     assert all(torch.count_nonzero(g) == 0 for g in grads)
+
+
+def test_layer_bit_reproducible():
+    """Every reduction is in a fixed order (TMA adds in stream order, split-K
+    adds onto zero, ordered dg sums): repeated runs give identical bits."""
+    w = LayerWorkload("t", 1, 1024, 2, 128, 384, 4, 128, 128, 256, 71, w_std=256 ** -0.5)
+    x, params, dy = layer_inputs(w)
+    a = run_layer(w, x, params, dy)
+    for _ in range(3):
+        b = run_layer(w, x, params, dy)
+        assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+        assert all(torch.equal(p, q) for p, q in zip(a[2], b[2]))
