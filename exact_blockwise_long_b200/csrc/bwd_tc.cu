@@ -164,7 +164,7 @@ struct KVLayout {
   static constexpr int kDO = kQ + kSt * kTile;
   static constexpr int kVec = kDO + kSt * kTile;  // per stage: lse*log2e [128], D [128]
   static constexpr int kBar = kVec + kSt * 1024;
-  static constexpr int kNumBars = 1 + 2 * kSt + 5;
+  static constexpr int kNumBars = 1 + 2 * kSt + 6;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4;
@@ -180,7 +180,10 @@ static_assert(KVLayout<128>::kAlloc <= 232448, "dK/dV tile set exceeds shared me
 // has itself read, so the A operand of dV (dK) sits in columns [0,32) and
 // [64,96).
 // MMA order per step n: dP_n, dV_n, S_{n+1}, dK_n (S_0 first); S_{n+1} is
-// issued as soon as dV_n has read P_n out of the S columns.
+// issued as soon as dV_n has read P_n out of the S columns.  P^T is
+// published in two halves (queries {0-31, 64-95}, then {32-63, 96-127}), so
+// the first half of dV runs while the second half of the exponentials is
+// computed.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -214,7 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_qe = bar_qf + kSt;
   uint64_t* bar_sf = bar_qe + kSt;   // S^T computed
   uint64_t* bar_dpf = bar_sf + 1;    // dP^T computed
-  uint64_t* bar_pr = bar_dpf + 1;    // P^T written to TMEM
+  uint64_t* bar_ph = bar_dpf + 1;    // first half of P^T (queries [0,32) and [64,96)) written to TMEM
+  uint64_t* bar_pr = bar_ph + 1;     // all of P^T written to TMEM
   uint64_t* bar_dsr = bar_pr + 1;    // dS^T written to TMEM
   uint64_t* bar_done = bar_dsr + 1;  // dK, dV final
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + LY::kTmemSlot);
@@ -228,6 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar_sf, 1);
     mbar_init(bar_dpf, 1);
+    mbar_init(bar_ph, 2 * 128);
     mbar_init(bar_pr, 2 * 128);
     mbar_init(bar_dsr, 2 * 128);
     mbar_init(bar_done, 1);
@@ -307,13 +312,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                       kk > 0 ? 1u : 0u);
         }
         mma_commit(bar_dpf);
-        // dV += P^T dO
-        if (!(ok = mbar_wait(bar_pr, n & 1, p.st, abort_flag))) break;
-        tc_fence_after();
+        // dV += P^T dO in two halves: queries {0-31, 64-95} as soon as the
+        // element-wise warps have published them, then {32-63, 96-127}
 #pragma unroll
-        for (int kk = 0; kk < kT / 16; ++kk)
-          mma_bf16_ts(tDV, tS + a_col(kk), sdesc_sw128(dob + kk * 2048, LY::kSlab, 1024), idTS,
-                      (n > 0 || kk > 0) ? 1u : 0u);
+        for (int half = 0; half < 2; ++half) {
+          if (!(ok = mbar_wait(half ? bar_pr : bar_ph, n & 1, p.st, abort_flag))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int kk = (j >> 1) * 4 + half * 2 + (j & 1);
+            mma_bf16_ts(tDV, tS + a_col(kk), sdesc_sw128(dob + kk * 2048, LY::kSlab, 1024), idTS,
+                        (n > 0 || half > 0 || j > 0) ? 1u : 0u);
+          }
+        }
+        if (!ok) break;
         // S^T of the next query tile into the columns dV has just read
         if (n + 1 < n_total) {
           const int st1 = (n + 1) % kSt;
@@ -348,27 +360,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* dvec = lse2 + 128;
       float P[kHalf];
       load_row64(cS, P);
+      // P^T (bf16) over the first 32 columns this group read, formed and
+      // published in two halves of 32 queries so that dV starts on the first
 #pragma unroll
-      for (int c = 0; c < kHalf; c += 2) {
-        const float2 t = fma2(make_float2(P[c], P[c + 1]), sl22, make_float2(-lse2[c], -lse2[c + 1]));
-        const float2 e = (D == 64 && (c / 2) % 2 == 1) ? ex2_poly2(t) : make_float2(ex2_approx(t.x), ex2_approx(t.y));
-        P[c] = e.x;
-        P[c + 1] = e.y;
-      }
-      if (diag) {
+      for (int half = 0; half < 2; ++half) {
 #pragma unroll
-        for (int c = 0; c < kHalf; ++c)
-          if (r > h * kHalf + c) P[c] = 0.f;  // key r is in the future of the query
-      }
-      {
-        uint32_t pk[32];
+        for (int c = 32 * half; c < 32 * half + 32; c += 2) {
+          const float2 t = fma2(make_float2(P[c], P[c + 1]), sl22, make_float2(-lse2[c], -lse2[c + 1]));
+          const float2 e = (D == 64 && (c / 2) % 2 == 1) ? ex2_poly2(t) : make_float2(ex2_approx(t.x), ex2_approx(t.y));
+          P[c] = e.x;
+          P[c + 1] = e.y;
+        }
+        if (diag) {
 #pragma unroll
-        for (int x = 0; x < 32; ++x) pk[x] = pack_bf16x2(P[2 * x], P[2 * x + 1]);
-        tmem_st32(cS, pk);
+          for (int c = 32 * half; c < 32 * half + 32; ++c)
+            if (r > h * kHalf + c) P[c] = 0.f;  // key r is in the future of the query
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) pk[x] = pack_bf16x2(P[32 * half + 2 * x], P[32 * half + 2 * x + 1]);
+        tmem_st16(cS + 16 * half, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(half ? bar_pr : bar_ph);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar_pr);
 
       if (!__all_sync(FULL, mbar_wait(bar_dpf, n & 1, p.st, abort_flag))) return false;
       tc_fence_after();
