@@ -49,6 +49,31 @@ int make_tmap_bf16_2d(void* tmap, const void* base, uint64_t inner, uint64_t row
                       box_rows);
 }
 
+int make_tmap_bf16_tile(void* tmap, const void* base, uint64_t D, uint64_t rows, uint32_t box_rows) {
+  if (D % 64 != 0 || D == 0) return RA_ERR_ARG;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return RA_ERR_CUDA;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  // dimensions: element within a 64-wide slab, row, slab (stride 128 B)
+  cuuint64_t dims[3] = {64, rows, D / 64};
+  cuuint64_t strides[2] = {D * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, (cuuint32_t)(D / 64)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(reinterpret_cast<CUtensorMap*>(tmap), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                        const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? RA_OK : RA_ERR_CUDA;
+}
+
 int make_tmap_f32_2d(void* tmap, const void* base, uint64_t inner, uint64_t rows, uint64_t row_pitch_bytes,
                      uint32_t box_inner, uint32_t box_rows) {
   return make_tmap_2d(tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, inner, rows, row_pitch_bytes, box_inner,

@@ -256,22 +256,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmDO);
       mbar_arrive_expect_tx(bar_kv, 2 * LY::kTile);
-#pragma unroll
-      for (int s = 0; s < D / 64; ++s) {
-        tma_load_2d(sK + s * LY::kSlab, &tmK, bar_kv, s * 64, krow0);
-        tma_load_2d(sV + s * LY::kSlab, &tmV, bar_kv, s * 64, krow0);
-      }
+      tma_load_tile(sK, &tmK, bar_kv, krow0);
+      tma_load_tile(sV, &tmV, bar_kv, krow0);
       int n = 0;
       walk.run([&](int qbh, int qt, bool) {
         const int st = n % kSt;
         const int qrow = qbh * p.N + qt * kT;
         if (!mbar_wait(&bar_qe[st], ((n / kSt) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_qf[st], 2 * LY::kTile + 1024);
-#pragma unroll
-        for (int s = 0; s < D / 64; ++s) {
-          tma_load_2d(sQ + st * LY::kTile + s * LY::kSlab, &tmQ, &bar_qf[st], s * 64, qrow);
-          tma_load_2d(sDO + st * LY::kTile + s * LY::kSlab, &tmDO, &bar_qf[st], s * 64, qrow);
-        }
+        tma_load_tile(sQ + st * LY::kTile, &tmQ, &bar_qf[st], qrow);
+        tma_load_tile(sDO + st * LY::kTile, &tmDO, &bar_qf[st], qrow);
         bulk_load(sVec + st * 256, p.lse2 + qrow, 512, &bar_qf[st]);
         bulk_load(sVec + st * 256 + 128, p.dvec + qrow, 512, &bar_qf[st]);
         ++n;
@@ -528,25 +522,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmDO);
       mbar_arrive_expect_tx(bar_qd, 2 * LY::kTile);
-#pragma unroll
-      for (int s = 0; s < D / 64; ++s) {
-        tma_load_2d(sQ + s * LY::kSlab, &tmQ, bar_qd, s * 64, qrow0);
-        tma_load_2d(sDO + s * LY::kSlab, &tmDO, bar_qd, s * 64, qrow0);
-      }
+      tma_load_tile(sQ, &tmQ, bar_qd, qrow0);
+      tma_load_tile(sDO, &tmDO, bar_qd, qrow0);
       int n = 0;
       walk.run([&](int kt, bool) {
         const int ks = n % kKStQ, vs = n % kSt;
         const int krow = kv_head_of(bh, p.H, p.G) * p.N + kt * kT;
         if (!mbar_wait(&bar_ke[ks], ((n / kKStQ) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_kf[ks], LY::kTile);
-#pragma unroll
-        for (int s = 0; s < D / 64; ++s)
-          tma_load_2d(sK + ks * LY::kTile + s * LY::kSlab, &tmK, &bar_kf[ks], s * 64, krow);
+        tma_load_tile(sK + ks * LY::kTile, &tmK, &bar_kf[ks], krow);
         if (!mbar_wait(&bar_ve[vs], ((n / kSt) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_vf[vs], LY::kTile);
-#pragma unroll
-        for (int s = 0; s < D / 64; ++s)
-          tma_load_2d(sV + vs * LY::kTile + s * LY::kSlab, &tmV, &bar_vf[vs], s * 64, krow);
+        tma_load_tile(sV + vs * LY::kTile, &tmV, &bar_vf[vs], krow);
         ++n;
         return true;
       });
@@ -730,10 +717,10 @@ int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* d
 
   alignas(64) CUtensorMap tq, tk, tv, tdo;
   const int64_t kv_rows = a.B * a.Hkv * a.N;
-  if (make_tmap_bf16_2d(&tq, a.q, D, rows, D * 2, 64, kT) != RA_OK) return RA_ERR_CUDA;
-  if (make_tmap_bf16_2d(&tk, a.k, D, kv_rows, D * 2, 64, kT) != RA_OK) return RA_ERR_CUDA;
-  if (make_tmap_bf16_2d(&tv, a.v, D, kv_rows, D * 2, 64, kT) != RA_OK) return RA_ERR_CUDA;
-  if (make_tmap_bf16_2d(&tdo, dout, D, rows, D * 2, 64, kT) != RA_OK) return RA_ERR_CUDA;
+  if (make_tmap_bf16_tile(&tq, a.q, D, rows, kT) != RA_OK) return RA_ERR_CUDA;
+  if (make_tmap_bf16_tile(&tk, a.k, D, kv_rows, kT) != RA_OK) return RA_ERR_CUDA;
+  if (make_tmap_bf16_tile(&tv, a.v, D, kv_rows, kT) != RA_OK) return RA_ERR_CUDA;
+  if (make_tmap_bf16_tile(&tdo, dout, D, rows, kT) != RA_OK) return RA_ERR_CUDA;
   BParams p{};
   p.lse2 = lse2;
   p.dvec = dvec;

@@ -115,6 +115,20 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, ui
       : "memory");
 }
 
+// One row-tile of a [rows x D] bf16 tensor (D a multiple of 64) through a
+// map made by make_tmap_bf16_tile: all D / 64 slabs of box_rows x 128 B in one
+// load, landing slab after slab with the 128-byte swizzle, i.e. exactly what
+// D / 64 2-D loads of the slabs would write.  One box per tile matters: a
+// CTA's tensor-memory loads progress box by box, so a single 32 KB box
+// arrives in about the time of one 16 KB box.
+__device__ __forceinline__ void tma_load_tile(void* smem_dst, const void* tmap, uint64_t* bar, int row) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %3}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(0), "r"(row)
+      : "memory");
+}
+
 // Untiled bulk copy global -> shared (16-byte aligned addresses, size a
 // multiple of 16), completing transaction bytes on `bar`.
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {

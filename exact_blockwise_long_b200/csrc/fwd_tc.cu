@@ -150,14 +150,18 @@ __device__ __forceinline__ float row_max(const float (&s)[kBN]) {
 // P = 2^(s * scale * log2(e) - m) as bf16 pairs over the first 64 columns of
 // the tile's TMEM (P of keys 2c, 2c+1 in column c); returns the row sum of
 // the fp32 probabilities.  Masked scores are -inf and give exactly 0.
-// One pair in kEx2PolyEvery is computed by ex2_poly2 on the FMA/integer
-// pipes, the rest by the MUFU: each 128 x 128 tile needs as many MUFU cycles
-// for its exponentials as tensor cycles for its two matmuls, so moving part
-// of them off the MUFU shortens the softmax's critical path.
+// One pair in PolyEvery is computed by ex2_poly2 on the FMA/integer pipes,
+// the rest by the MUFU: each 128 x 128 tile needs as many MUFU cycles for its
+// exponentials as tensor cycles for its two matmuls, so moving part of them
+// off the MUFU shortens the softmax's critical path.  Measured best: one pair
+// in four at d = 128, one in three at d = 64 (whose matmuls take half as
+// long); one in two is slower at both.
 // With bar_half, the first half of P (keys 0-63) is published on it as soon
 // as it is in TMEM, so the P V matmul over those keys can start while the
 // second half is computed.
-constexpr int kEx2PolyEvery = 4;
+template <int D>
+constexpr int kEx2PolyEvery = D == 64 ? 3 : 4;
+template <int PolyEvery>
 __device__ __forceinline__ float exp_store(const float (&s)[kBN], uint32_t tS, float sl2, float m,
                                            uint64_t* bar_half = nullptr) {
   const float2 k2 = make_float2(sl2, sl2), nm2 = make_float2(-m, -m);
@@ -170,7 +174,7 @@ __device__ __forceinline__ float exp_store(const float (&s)[kBN], uint32_t tS, f
 #pragma unroll
     for (int x = 0; x < 32; ++x) {
       const float2 t = fma2(make_float2(s[h * 64 + 2 * x], s[h * 64 + 2 * x + 1]), k2, nm2);
-      const float2 pr = (x % kEx2PolyEvery == kEx2PolyEvery - 1) ? ex2_poly2(t)
+      const float2 pr = (x % PolyEvery == PolyEvery - 1) ? ex2_poly2(t)
                                                                 : make_float2(ex2_approx(t.x), ex2_approx(t.y));
       acc[x & 3] = add2(acc[x & 3], pr);
       pk[x] = pack_bf16x2(pr.x, pr.y);
@@ -334,22 +338,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       mbar_arrive_expect_tx(bar_q, LY::kTileBytes);
-#pragma unroll
-      for (int s = 0; s < D / 64; ++s) tma_load_2d(sQ + s * LY::kSlabBytes, &tmQ, bar_q, s * 64, qrow0);
+      tma_load_tile(sQ, &tmQ, bar_q, qrow0);
       int n = 0;
       walk.run([&](int kt, bool) {
         const int krow = kv_head_of(bh, p.H, p.G) * p.N + kt * kBN;
         const int ks = n % kKSt, vs = n % kVSt;
         if (!mbar_wait(&bar_ke[ks], ((n / kKSt) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_kf[ks], LY::kTileBytes);
-#pragma unroll
-        for (int s = 0; s < D / 64; ++s)
-          tma_load_2d(sK + ks * LY::kTileBytes + s * LY::kSlabBytes, &tmK, &bar_kf[ks], s * 64, krow);
+        tma_load_tile(sK + ks * LY::kTileBytes, &tmK, &bar_kf[ks], krow);
         if (!mbar_wait(&bar_ve[vs], ((n / kVSt) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_vf[vs], LY::kTileBytes);
-#pragma unroll
-        for (int s = 0; s < D / 64; ++s)
-          tma_load_2d(sV + vs * LY::kTileBytes + s * LY::kSlabBytes, &tmV, &bar_vf[vs], s * 64, krow);
+        tma_load_tile(sV + vs * LY::kTileBytes, &tmV, &bar_vf[vs], krow);
         ++n;
         return true;
       });
@@ -431,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         rescale_o<D>(tO + lane_off, alpha);
         m_run = m_new;
       }
-      const float rowsum = exp_store(s, tS, sl2, m_run);
+      const float rowsum = exp_store<kEx2PolyEvery<D>>(s, tS, sl2, m_run);
       tmem_st_wait();
       l_run += rowsum;
       tc_fence_before();
@@ -606,23 +605,17 @@ __global__ void __launch_bounds__(kThreads2, 1)
       mbar_arrive_expect_tx(bar_q, 2 * LY::kTileBytes);
 #pragma unroll
       for (int t = 0; t < 2; ++t)
-#pragma unroll
-        for (int s = 0; s < D / 64; ++s)
-          tma_load_2d(sQ + t * LY::kTileBytes + s * LY::kSlabBytes, &tmQ, bar_q, s * 64, qrow0 + t * kBM);
+        tma_load_tile(sQ + t * LY::kTileBytes, &tmQ, bar_q, qrow0 + t * kBM);
       int n = 0;
       walk.run([&](int kt, bool, bool, bool) {
         const int krow = kv_head_of(bh, p.H, p.G) * p.N + kt * kBN;
         const int ks = n % kKSt, vs = n % kVSt;
         if (!mbar_wait(&bar_ke[ks], ((n / kKSt) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_kf[ks], LY::kTileBytes);
-#pragma unroll
-        for (int s = 0; s < D / 64; ++s)
-          tma_load_2d(sK + ks * LY::kTileBytes + s * LY::kSlabBytes, &tmK, &bar_kf[ks], s * 64, krow);
+        tma_load_tile(sK + ks * LY::kTileBytes, &tmK, &bar_kf[ks], krow);
         if (!mbar_wait(&bar_ve[vs], ((n / kVSt) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_vf[vs], LY::kTileBytes);
-#pragma unroll
-        for (int s = 0; s < D / 64; ++s)
-          tma_load_2d(sV + vs * LY::kTileBytes + s * LY::kSlabBytes, &tmV, &bar_vf[vs], s * 64, krow);
+        tma_load_tile(sV + vs * LY::kTileBytes, &tmV, &bar_vf[vs], krow);
         ++n;
         return true;
       });
@@ -715,7 +708,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
         rescale_o<D>(tO, alpha);
         m_run = m_new;
       }
-      const float rowsum = exp_store(s, tS, sl2, m_run, &bar_ph[tile]);
+      const float rowsum = exp_store<kEx2PolyEvery<D>>(s, tS, sl2, m_run, &bar_ph[tile]);
       tmem_st_wait();
       l_run += rowsum;
       tc_fence_before();
@@ -743,9 +736,9 @@ int launch_d(const AttnArgs& a, void* out, float* lse, float* o_acc, float* lse_
   alignas(64) CUtensorMap tq, tk, tv;
   const uint64_t rows = (uint64_t)(a.B * a.H * a.N);
   const uint64_t kv_rows = (uint64_t)(a.B * a.Hkv * a.N);
-  if (make_tmap_bf16_2d(&tq, a.q, D, rows, D * 2, 64, kBM) != RA_OK) return RA_ERR_CUDA;
-  if (make_tmap_bf16_2d(&tk, a.k, D, kv_rows, D * 2, 64, kBN) != RA_OK) return RA_ERR_CUDA;
-  if (make_tmap_bf16_2d(&tv, a.v, D, kv_rows, D * 2, 64, kBN) != RA_OK) return RA_ERR_CUDA;
+  if (make_tmap_bf16_tile(&tq, a.q, D, rows, kBM) != RA_OK) return RA_ERR_CUDA;
+  if (make_tmap_bf16_tile(&tk, a.k, D, kv_rows, kBN) != RA_OK) return RA_ERR_CUDA;
+  if (make_tmap_bf16_tile(&tv, a.v, D, kv_rows, kBN) != RA_OK) return RA_ERR_CUDA;
   Params p{};
   p.out = (__nv_bfloat16*)out;
   p.lse = lse;

@@ -123,6 +123,10 @@ int make_tmap_bf16_2d(void* tmap /* CUtensorMap* */, const void* base, uint64_t 
                       uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_rows);
 
 // The same for a 2-D fp32 map (box inner extent at most 32 elements).
+// 3-D map over a [rows x D] bf16 tensor whose box is one row-tile of box_rows
+// rows with all D / 64 slabs (for tma_load_tile).
+int make_tmap_bf16_tile(void* tmap /* CUtensorMap* */, const void* base, uint64_t D, uint64_t rows,
+                        uint32_t box_rows);
 int make_tmap_f32_2d(void* tmap /* CUtensorMap* */, const void* base, uint64_t inner, uint64_t rows,
                      uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_rows);
 
