@@ -50,6 +50,8 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t FULL = 0xffffffffu;
 
 struct BParams {
+  const __nv_bfloat16* q;     // [BH*N, D]
+  const __nv_bfloat16* dout;  // [BH*N, D]
   const float* lse2;   // lse * log2(e)    [BH*N]
   const float* dvec;   // D_i = dO_i . O_i  [BH*N]
   __nv_bfloat16* dq;
@@ -423,18 +425,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ===========================================================================
 // dQ: query tile stationary
 // ===========================================================================
-constexpr int kKStQ = 3;  // K stages of the dQ pass (K is held from S until dQ)
-
 template <int D>
 struct QLayout {
   static constexpr int kTile = kT * D * 2;
   static constexpr int kSlab = kT * 128;
-  static constexpr int kQ = 0;
-  static constexpr int kDO = kQ + kTile;
-  static constexpr int kK = kDO + kTile;
-  static constexpr int kV = kK + kKStQ * kTile;
-  static constexpr int kBar = kV + kSt * kTile;
-  static constexpr int kNumBars = 1 + 2 * kKStQ + 2 * kSt + 2 + 3;
+  static constexpr int kKSt = D == 64 ? 6 : 4;  // K held from S until dQ
+  static constexpr int kVSt = D == 64 ? 6 : 3;  // V held for dP
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + kKSt * kTile;
+  static constexpr int kBar = kV + kVSt * kTile;
+  static constexpr int kNumBars = 1 + 2 * kKSt + 2 * kVSt + 5;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4;
@@ -442,14 +442,19 @@ struct QLayout {
 };
 static_assert(QLayout<128>::kAlloc <= 232448, "dQ tile set exceeds shared memory");
 
-// Warp roles: warp 0 TMA producer (Q, dO once; K, V per step), warp 1 MMA
-// issuer, warp 2 TMEM allocator, warps 4-7 and 8-11 one thread per query
-// row each, the first warpgroup on key columns [0,64), the second on
-// [64,128): P, dS and half of the dQ epilogue.  Each warpgroup writes its
-// bf16 dS over the first 32 of the S columns it has itself read, so the A
-// operand of dQ sits in columns [0,32) and [64,96) of that step's S buffer.
-// MMA order per step n: dP_n, S_{n+1}, dQ_n (S_0 first); S is double
-// buffered so the next scores are ready when a row's dS is done.
+// Warp roles: warp 0 TMA producer (K, V per step), warp 1 MMA issuer,
+// warp 2 TMEM allocator, warps 4-7 and 8-11 one thread per query row each,
+// the first warpgroup on key columns [0,64), the second on [64,128): P, dS
+// and half of the dQ epilogue.  The stationary Q and dO tiles live in tensor
+// memory (written once by the element-wise warps), so all three matmuls take
+// their A operand from TMEM and shared memory holds only the K, V ring:
+// operand reads per step drop from 160 KB to 96 KB at d = 128 and the ring
+// is 4 + 3 tiles deep.  TMEM: S [0,128), dP [128,256), dQ [256,256+D),
+// Q [384,384+D/2), dO [448,448+D/2).  Each warpgroup writes its bf16 dS
+// over the first 32 of the dP columns it has itself read (A operand of dQ in
+// columns [0,32) and [64,96) of dP).
+// MMA order per step n: dP_n, S_{n+1} (as soon as both warpgroups have
+// loaded S_n), dQ_n; S_0 first.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -470,35 +475,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   const RingWalkQ walk{(qt * kT) / p.L, p.S, tps, qt, p.causal};
   const int n_total = walk.count();
 
-  uint8_t* sQ = smem + LY::kQ;
-  uint8_t* sDO = smem + LY::kDO;
   uint8_t* sK = smem + LY::kK;
   uint8_t* sV = smem + LY::kV;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + LY::kBar);
-  uint64_t* bar_qd = bars;
+  uint64_t* bar_qd = bars;                 // Q and dO written to TMEM
   uint64_t* bar_kf = bar_qd + 1;
-  uint64_t* bar_ke = bar_kf + kKStQ;
-  uint64_t* bar_vf = bar_ke + kKStQ;
-  uint64_t* bar_ve = bar_vf + kSt;
-  uint64_t* bar_sf = bar_ve + kSt;   // [2] S buffer b computed
-  uint64_t* bar_dpf = bar_sf + 2;    // dP computed
-  uint64_t* bar_dsr = bar_dpf + 1;   // dS written to TMEM
-  uint64_t* bar_done = bar_dsr + 1;  // dQ final
+  uint64_t* bar_ke = bar_kf + LY::kKSt;
+  uint64_t* bar_vf = bar_ke + LY::kKSt;
+  uint64_t* bar_ve = bar_vf + LY::kVSt;
+  uint64_t* bar_sf = bar_ve + LY::kVSt;    // S computed
+  uint64_t* bar_sfree = bar_sf + 1;        // S loaded by both warpgroups
+  uint64_t* bar_dpf = bar_sfree + 1;       // dP computed
+  uint64_t* bar_dsr = bar_dpf + 1;         // dS written to TMEM
+  uint64_t* bar_done = bar_dsr + 1;        // dQ final
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + LY::kTmemSlot);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LY::kAbort);
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_qd, 1);
-    for (int s = 0; s < kKStQ; ++s) {
+    mbar_init(bar_qd, 2 * 128);
+    for (int s = 0; s < LY::kKSt; ++s) {
       mbar_init(&bar_kf[s], 1);
       mbar_init(&bar_ke[s], 1);
     }
-    for (int s = 0; s < kSt; ++s) {
+    for (int s = 0; s < LY::kVSt; ++s) {
       mbar_init(&bar_vf[s], 1);
       mbar_init(&bar_ve[s], 1);
     }
-    mbar_init(&bar_sf[0], 1);
-    mbar_init(&bar_sf[1], 1);
+    mbar_init(bar_sf, 1);
+    mbar_init(bar_sfree, 2 * 128);
     mbar_init(bar_dpf, 1);
     mbar_init(bar_dsr, 2 * 128);
     mbar_init(bar_done, 1);
@@ -513,25 +517,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tDP = tmem + 256, tDQ = tmem + 384;
+  const uint32_t tS = tmem, tDP = tmem + 128, tDQ = tmem + 256, tQ = tmem + 384, tDO = tmem + 448;
 
   if (warp == 0) {
     if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      tma_prefetch_desc(&tmDO);
-      mbar_arrive_expect_tx(bar_qd, 2 * LY::kTile);
-      tma_load_tile(sQ, &tmQ, bar_qd, qrow0);
-      tma_load_tile(sDO, &tmDO, bar_qd, qrow0);
       int n = 0;
       walk.run([&](int kt, bool) {
-        const int ks = n % kKStQ, vs = n % kSt;
+        const int ks = n % LY::kKSt, vs = n % LY::kVSt;
         const int krow = kv_head_of(bh, p.H, p.G) * p.N + kt * kT;
-        if (!mbar_wait(&bar_ke[ks], ((n / kKStQ) & 1) ^ 1, p.st, abort_flag)) return false;
+        if (!mbar_wait(&bar_ke[ks], ((n / LY::kKSt) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_kf[ks], LY::kTile);
         tma_load_tile(sK + ks * LY::kTile, &tmK, &bar_kf[ks], krow);
-        if (!mbar_wait(&bar_ve[vs], ((n / kSt) & 1) ^ 1, p.st, abort_flag)) return false;
+        if (!mbar_wait(&bar_ve[vs], ((n / LY::kVSt) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_vf[vs], LY::kTile);
         tma_load_tile(sV + vs * LY::kTile, &tmV, &bar_vf[vs], krow);
         ++n;
@@ -540,50 +539,52 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idSS = idesc_bf16_f32(kT, kT, false, false);  // K-major x K-major
-      constexpr uint32_t idDQ = idesc_bf16_f32(kT, D, false, true);    // TMEM dS x MN-major K
-      const uint32_t q_base = smem_u32(sQ), do_base = smem_u32(sDO);
+      constexpr uint32_t idS = idesc_bf16_f32(kT, kT, false, false);  // TMEM A x K-major B
+      constexpr uint32_t idDQ = idesc_bf16_f32(kT, D, false, true);   // TMEM dS x MN-major K
       const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV);
       auto a_col = [](int kk) -> uint32_t { return kk < 4 ? kk * 8 : 64 + (kk - 4) * 8; };
+      // S_n = Q K_n^T, Q from TMEM (columns 8 kk hold d elements [16 kk, 16 kk + 16))
       auto issue_s = [&](int n) -> bool {
-        const int ks = n % kKStQ;
-        if (!mbar_wait(&bar_kf[ks], (n / kKStQ) & 1, p.st, abort_flag)) return false;
+        const int ks = n % LY::kKSt;
+        if (!mbar_wait(&bar_kf[ks], (n / LY::kKSt) & 1, p.st, abort_flag)) return false;
         tc_fence_after();
         const uint32_t kb = k_base + ks * LY::kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * LY::kSlab + (kk & 3) * 32;
-          mma_bf16_ss(tmem + (n & 1) * 128, sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
-                      idSS, kk > 0 ? 1u : 0u);
+          mma_bf16_ts(tS, tQ + kk * 8, sdesc_sw128(kb + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bar_sf[n & 1]);
+        mma_commit(bar_sf);
         return true;
       };
-      bool ok = mbar_wait(bar_qd, 0, p.st, abort_flag) && issue_s(0);
+      bool ok = mbar_wait(bar_qd, 0, p.st, abort_flag);
+      if (ok) tc_fence_after();
+      ok = ok && issue_s(0);
       for (int n = 0; ok && n < n_total; ++n) {
-        const int ks = n % kKStQ, vs = n % kSt;
-        // dP = dO V^T (its columns were last read for dS of the previous step)
-        if (!(ok = mbar_wait(&bar_vf[vs], (n / kSt) & 1, p.st, abort_flag))) break;
+        const int ks = n % LY::kKSt, vs = n % LY::kVSt;
+        // dP = dO V^T, dO from TMEM; its columns were last read by dQ of the previous step
+        if (!(ok = mbar_wait(&bar_vf[vs], (n / LY::kVSt) & 1, p.st, abort_flag))) break;
         tc_fence_after();
         const uint32_t vb = v_base + vs * LY::kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * LY::kSlab + (kk & 3) * 32;
-          mma_bf16_ss(tDP, sdesc_sw128(do_base + off, 16, 1024), sdesc_sw128(vb + off, 16, 1024), idSS,
-                      kk > 0 ? 1u : 0u);
+          mma_bf16_ts(tDP, tDO + kk * 8, sdesc_sw128(vb + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
         }
         mma_commit(bar_dpf);
         mma_commit(&bar_ve[vs]);
-        // scores of the next key tile into the other S buffer
-        if (n + 1 < n_total && !(ok = issue_s(n + 1))) break;
-        // dQ += dS K, dS read from this step's S buffer
+        // scores of the next key tile once both warpgroups have read this one's
+        if (n + 1 < n_total) {
+          if (!(ok = mbar_wait(bar_sfree, n & 1, p.st, abort_flag))) break;
+          if (!(ok = issue_s(n + 1))) break;
+        }
+        // dQ += dS K, dS read from the dP columns
         if (!(ok = mbar_wait(bar_dsr, n & 1, p.st, abort_flag))) break;
         tc_fence_after();
         const uint32_t kb = k_base + ks * LY::kTile;
-        const uint32_t tds = tmem + (n & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < kT / 16; ++kk)
-          mma_bf16_ts(tDQ, tds + a_col(kk), sdesc_sw128(kb + kk * 2048, LY::kSlab, 1024), idDQ,
+          mma_bf16_ts(tDQ, tDP + a_col(kk), sdesc_sw128(kb + kk * 2048, LY::kSlab, 1024), idDQ,
                       (n > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bar_ke[ks]);
       }
@@ -596,13 +597,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float nl2 = -p.lse2[qrow0 + r];
     const float Dr = p.dvec[qrow0 + r];
     const float2 sl22 = make_float2(p.scale_log2, p.scale_log2), nl22 = make_float2(nl2, nl2);
+    // this row's Q and dO, d elements [D/2 h, D/2 h + D/2), into TMEM as bf16
+    // pairs (column 8 kk + j holds elements 16 kk + 2 j, 16 kk + 2 j + 1)
+    {
+      const uint4* gq = reinterpret_cast<const uint4*>(p.q + ((size_t)qrow0 + r) * D + h * (D / 2));
+      const uint4* gd = reinterpret_cast<const uint4*>(p.dout + ((size_t)qrow0 + r) * D + h * (D / 2));
+      uint32_t wq[D / 4], wd[D / 4];
+#pragma unroll
+      for (int x = 0; x < D / 16; ++x) {
+        const uint4 a = __ldg(gq + x), b = __ldg(gd + x);
+        wq[4 * x] = a.x; wq[4 * x + 1] = a.y; wq[4 * x + 2] = a.z; wq[4 * x + 3] = a.w;
+        wd[4 * x] = b.x; wd[4 * x + 1] = b.y; wd[4 * x + 2] = b.z; wd[4 * x + 3] = b.w;
+      }
+      if constexpr (D == 128) {
+        tmem_st32(tQ + lane_off + h * 32, wq);
+        tmem_st32(tDO + lane_off + h * 32, wd);
+      } else {
+        tmem_st16(tQ + lane_off + h * 16, wq);
+        tmem_st16(tDO + lane_off + h * 16, wd);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_qd);
+    }
+    const uint32_t cS = tS + lane_off + h * kHalf, cDP = tDP + lane_off + h * kHalf;
     int n = 0;
     const bool ok = walk.run([&](int, bool diag) {
-      if (!__all_sync(FULL, mbar_wait(&bar_sf[n & 1], (n >> 1) & 1, p.st, abort_flag))) return false;
+      if (!__all_sync(FULL, mbar_wait(bar_sf, n & 1, p.st, abort_flag))) return false;
       tc_fence_after();
-      const uint32_t cS = tmem + (n & 1) * 128 + lane_off + h * kHalf;
       float P[kHalf];
       load_row64(cS, P);
+      tc_fence_before();
+      mbar_arrive(bar_sfree);  // the S columns may take the next tile's scores
 #pragma unroll
       for (int c = 0; c < kHalf; c += 2) {
         const float2 t = fma2(make_float2(P[c], P[c + 1]), sl22, nl22);
@@ -618,8 +644,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       {
         uint32_t a[32], b[32];
-        tmem_ld32(tDP + lane_off + h * kHalf, a);
-        tmem_ld32(tDP + lane_off + h * kHalf + 32, b);
+        tmem_ld32(cDP, a);
+        tmem_ld32(cDP + 32, b);
         tmem_ld_wait();
         uint32_t pk[32];
 #pragma unroll
@@ -629,7 +655,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[16 + x] = pack_bf16x2(P[32 + 2 * x] * (__uint_as_float(b[2 * x]) - Dr),
                                    P[33 + 2 * x] * (__uint_as_float(b[2 * x + 1]) - Dr));
         }
-        tmem_st32(cS, pk);  // bf16 dS over this group's first 32 S columns (already read)
+        tmem_st32(cDP, pk);  // bf16 dS over this group's first 32 dP columns (already read)
       }
       tmem_st_wait();
       tc_fence_before();
@@ -722,6 +748,8 @@ int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* d
   if (make_tmap_bf16_tile(&tv, a.v, D, kv_rows, kT) != RA_OK) return RA_ERR_CUDA;
   if (make_tmap_bf16_tile(&tdo, dout, D, rows, kT) != RA_OK) return RA_ERR_CUDA;
   BParams p{};
+  p.q = (const __nv_bfloat16*)a.q;
+  p.dout = (const __nv_bfloat16*)dout;
   p.lse2 = lse2;
   p.dvec = dvec;
   p.dq = (__nv_bfloat16*)dq;
