@@ -42,14 +42,14 @@ METRIC = "ring-attn fwd+bwd TFLOP/s & tokens/s on 1 B200; % of BF16 tensor peak"
 # (heads are independent units; see profiles/*_n32k_d128_h8.md).
 NCU_TRAFFIC = {
     ("bwd_kv_kernel", "n32k_d128"): {
-        "bytes": 4 * (272.233984e6 + 103.432192e6),
-        "sha256": "c874611cfb2c61df7872652125c6ea89c7b4fc8e5a4e900c3b5b996c615147b0"},
+        "bytes": 4 * (271.702016e6 + 100.289024e6),
+        "sha256": "687afa776acab599fc6dcb31a37a8874692859b9ba313bc553a98a778ff20e33"},
     ("bwd_q_kernel", "n32k_d128"): {
-        "bytes": 4 * (271.248384e6 + 47.282432e6),
-        "sha256": "c874611cfb2c61df7872652125c6ea89c7b4fc8e5a4e900c3b5b996c615147b0"},
+        "bytes": 4 * (270.872320e6 + 47.599616e6),
+        "sha256": "687afa776acab599fc6dcb31a37a8874692859b9ba313bc553a98a778ff20e33"},
     ("fwd_tc2_kernel", "n32k_d128"): {
-        "bytes": 4 * (202.573056e6 + 48.696576e6),
-        "sha256": "5c686052862a91d3ec7544ef7ec3b53956e0efd7f35b73a76a07e6677b666c14"},
+        "bytes": 4 * (202.305536e6 + 48.263936e6),
+        "sha256": "b9611e372d9d56c91c6de605248d55ae1557c659a94ef3f86ba6439a0cbf8bbd"},
 }
 
 
