@@ -43,10 +43,10 @@ METRIC = "ring-attn fwd+bwd TFLOP/s & tokens/s on 1 B200; % of BF16 tensor peak"
 NCU_TRAFFIC = {
     ("bwd_kv_kernel", "n32k_d128"): {
         "bytes": 4 * (271.702016e6 + 100.289024e6),
-        "sha256": "687afa776acab599fc6dcb31a37a8874692859b9ba313bc553a98a778ff20e33"},
+        "sha256": "18edf75c7b519d87cc6c86c3cc0ab11538ca312545a3fac0b35d6550cdca6bf2"},
     ("bwd_q_kernel", "n32k_d128"): {
         "bytes": 4 * (270.872320e6 + 47.599616e6),
-        "sha256": "687afa776acab599fc6dcb31a37a8874692859b9ba313bc553a98a778ff20e33"},
+        "sha256": "18edf75c7b519d87cc6c86c3cc0ab11538ca312545a3fac0b35d6550cdca6bf2"},
     ("fwd_tc2_kernel", "n32k_d128"): {
         "bytes": 4 * (202.305536e6 + 48.263936e6),
         "sha256": "b9611e372d9d56c91c6de605248d55ae1557c659a94ef3f86ba6439a0cbf8bbd"},

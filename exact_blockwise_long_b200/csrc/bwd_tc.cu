@@ -23,10 +23,11 @@
 //                 dP^T = V dO^T   (TMEM [128,256))
 //                 dV  += P^T dO   (P^T bf16 over S^T, A operand from TMEM)
 //                 dK  += dS^T Q   (dS^T bf16 over dP^T, A operand from TMEM)
-//   dQ          per (query tile, key tile) 3 tcgen05 MMAs:
-//                 S    = Q K^T    (TMEM [0,128) / [128,256), double buffered)
-//                 dP   = dO V^T   (TMEM [256,384))
-//                 dQ  += dS K     (dS bf16 over S, A operand from TMEM)
+//   dQ          per (query tile, key tile) 3 tcgen05 MMAs, Q and dO held in
+//               TMEM as their A operands:
+//                 S    = Q K^T    (TMEM [0,128))
+//                 dP   = dO V^T   (TMEM [128,256))
+//                 dQ  += dS K     (dS bf16 over dP, A operand from TMEM)
 #include <math.h>
 
 #include "common.cuh"
