@@ -36,7 +36,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 template <int D, int G>
 struct DLayout {
   static constexpr int kTile = kKeys * D * 2;
-  static constexpr int kSlab = kKeys * 128;
   static constexpr int kK = 0;
   static constexpr int kV = kK + kStages * kTile;
   static constexpr int kQ = kV + kStages * kTile;            // fp32 [G][D]
@@ -117,11 +116,8 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(const __grid_c
     const int s = t % kStages;
     const int row = kvbh * p.N + k0 + t * kKeys;
     mbar_arrive_expect_tx(&bar_full[s], 2 * LY::kTile);
-#pragma unroll
-    for (int sl = 0; sl < D / 64; ++sl) {
-      tma_load_2d(sK + s * LY::kTile + sl * LY::kSlab, &tmK, &bar_full[s], sl * 64, row);
-      tma_load_2d(sV + s * LY::kTile + sl * LY::kSlab, &tmV, &bar_full[s], sl * 64, row);
-    }
+    tma_load_tile(sK + s * LY::kTile, &tmK, &bar_full[s], row);
+    tma_load_tile(sV + s * LY::kTile, &tmV, &bar_full[s], row);
   };
   if (tid == 0) {
     tma_prefetch_desc(&tmK);
@@ -287,8 +283,8 @@ int launch_d(const void* q, const void* k, const void* v, void* out, float* lse,
   const int L = (int)((N + S - 1) / S);
   alignas(64) CUtensorMap tk, tv;
   const uint64_t kv_rows = (uint64_t)(B * Hkv * N);
-  if (make_tmap_bf16_2d(&tk, k, D, kv_rows, D * 2, 64, kKeys) != RA_OK) return RA_ERR_CUDA;
-  if (make_tmap_bf16_2d(&tv, v, D, kv_rows, D * 2, 64, kKeys) != RA_OK) return RA_ERR_CUDA;
+  if (make_tmap_bf16_tile(&tk, k, D, kv_rows, kKeys) != RA_OK) return RA_ERR_CUDA;
+  if (make_tmap_bf16_tile(&tv, v, D, kv_rows, kKeys) != RA_OK) return RA_ERR_CUDA;
   DParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.part_lse = static_cast<float*>(workspace);
