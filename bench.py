@@ -42,13 +42,13 @@ METRIC = "ring-attn fwd+bwd TFLOP/s & tokens/s on 1 B200; % of BF16 tensor peak"
 # (heads are independent units; see profiles/*_n32k_d128_h8.md).
 NCU_TRAFFIC = {
     ("bwd_kv_kernel", "n32k_d128"): {
-        "bytes": 4 * (271.702016e6 + 100.289024e6),
-        "sha256": "18edf75c7b519d87cc6c86c3cc0ab11538ca312545a3fac0b35d6550cdca6bf2"},
+        "bytes": 4 * (272.243200e6 + 101.754624e6),
+        "sha256": "cbc4330a94949a94c161a59bf5be8c407f2ec2c6336d4b56842b3501eb8472a5"},
     ("bwd_q_kernel", "n32k_d128"): {
-        "bytes": 4 * (270.872320e6 + 47.599616e6),
-        "sha256": "18edf75c7b519d87cc6c86c3cc0ab11538ca312545a3fac0b35d6550cdca6bf2"},
+        "bytes": 4 * (271.136512e6 + 49.010432e6),
+        "sha256": "cbc4330a94949a94c161a59bf5be8c407f2ec2c6336d4b56842b3501eb8472a5"},
     ("fwd_tc2_kernel", "n32k_d128"): {
-        "bytes": 4 * (202.305536e6 + 48.263936e6),
+        "bytes": 4 * (201.815040e6 + 47.820032e6),
         "sha256": "b9611e372d9d56c91c6de605248d55ae1557c659a94ef3f86ba6439a0cbf8bbd"},
 }
 
@@ -141,16 +141,58 @@ def peaks():
 
 
 class ClockSampler:
+    """SM clock, power and clock-event reasons of one GPU while the timed
+    region runs: NVML polled every 10 ms from a thread (nvidia-smi's 100 ms
+    loop is the fallback), so even a short timed region gets samples."""
+
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40}
 
     def __init__(self, index):
         self.index = index
         self.proc = None
+        self.thread = None
+        self.samples = []  # (sm_mhz, power_w, reason_bits)
+        self.max_mhz = None
         self.path = os.path.join("/tmp", f"ra_clocks_{os.getpid()}.csv")
 
     def start(self):
+        try:
+            import threading
+            import pynvml
+            pynvml.nvmlInit()
+            h = None
+            try:  # the CUDA device by PCI address (CUDA and NVML numbering can differ)
+                pr = torch.cuda.get_device_properties(self.index)
+                bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+                h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                h = None
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.stop_evt = threading.Event()
+
+            def poll():
+                while not self.stop_evt.is_set():
+                    try:
+                        self.samples.append((float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)),
+                                             pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0, int(reasons_fn(h))))
+                    except Exception:
+                        pass
+                    self.stop_evt.wait(0.01)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.thread = None
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
@@ -159,7 +201,20 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
+    def _summary(self, sm, power, reasons, mx, source):
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0, "source": source}
+        loaded = [s for s, p in zip(sm, power) if p > 300] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "samples_under_load": len(loaded), "source": source}
+
     def stop(self):
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=5)
+            reasons = {nm for nm, bit in self.REASON_BITS.items() if any(r & bit for _, _, r in self.samples)}
+            return self._summary([x[0] for x in self.samples], [x[1] for x in self.samples], reasons,
+                                 self.max_mhz, "nvml, 10 ms")
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -184,11 +239,7 @@ class ClockSampler:
                 if val.lower().startswith("active"):
                     reasons.add(nm)
         os.unlink(self.path)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
-        loaded = [s for s, p in zip(sm, power) if p > 300] or sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm), "samples_under_load": len(loaded)}
+        return self._summary(sm, power, reasons, mx, "nvidia-smi, 100 ms")
 
 
 # ---------------------------------------------------------------------------

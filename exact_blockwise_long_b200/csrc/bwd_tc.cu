@@ -458,8 +458,7 @@ static_assert(QLayout<128>::kAlloc <= 232448, "dQ tile set exceeds shared memory
 // loaded S_n), dQ_n; S_0 first.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+    bwd_q_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const BParams p) {
   using LY = QLayout<D>;
   extern __shared__ uint8_t smem_q[];
@@ -782,7 +781,7 @@ int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* d
     p.group = head_group(p.num_tiles, p.BH, (double)a.N * D * 4 * 2, 100.0e6);
     auto kern = bwd_q_kernel<D>;
     if (set_smem_attr((const void*)kern, QLayout<D>::kAlloc) != RA_OK) return RA_ERR_CUDA;
-    kern<<<(unsigned)(p.BH * p.num_tiles), kThreads, QLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
+    kern<<<(unsigned)(p.BH * p.num_tiles), kThreads, QLayout<D>::kAlloc, stream>>>(tk, tv, p);
     if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
   }
   return RA_OK;
