@@ -904,53 +904,78 @@ def main():
 
     # End to end through the public API: every step copies its inputs from
     # pinned host memory and reads its results back.  Two device buffer sets
-    # let step j+1's host-to-device copy and step j-1's device-to-host copy
-    # run on their own streams while step j computes.
+    # let step j+1's host-to-device copies and step j-1's device-to-host
+    # copies run on their own streams while step j computes.  Each tensor
+    # moves as soon as it can: q, k, v first and dO (and the FFN's x, dy)
+    # behind them while the forward runs; O and LSE go back while the
+    # backward runs, dK and dV while the dQ pass runs, dQ last.
     if not args.no_e2e:
-        in0 = [q, k, v] + ([do] if aw.bwd else []) + ([x, dy] if fw is not None else [])
-        out0 = [o, lse] + ([dq, dk, dv] if aw.bwd else []) + ([y, dx, dw1, dw2, dw3] if fw is not None else [])
-        hin = [t.cpu().pin_memory() for t in in0]
-        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in out0]
-        ins = [in0, [torch.empty_like(t) for t in in0]]
-        outs = [out0, [torch.empty_like(t) for t in out0]]
-        h2d = sum(t.numel() * t.element_size() for t in hin)
-        d2h = sum(t.numel() * t.element_size() for t in hout)
+        in_f0 = [q, k, v]
+        in_b0 = ([do] if aw.bwd else []) + ([x, dy] if fw is not None else [])
+        out_f0 = [o, lse]
+        out_kv0 = [dk, dv] if aw.bwd else []
+        out_b0 = ([dq] if aw.bwd else []) + ([y, dx, dw1, dw2, dw3] if fw is not None else [])
+        groups0 = [in_f0, in_b0, out_f0, out_kv0, out_b0]
+        hgrp = [[t.cpu().pin_memory() for t in g_] for g_ in groups0[:2]] + \
+               [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in g_] for g_ in groups0[2:]]
+        dev_sets = [groups0, [[torch.empty_like(t) for t in g_] for g_ in groups0]]
+        h2d = sum(t.numel() * t.element_size() for g_ in hgrp[:2] for t in g_)
+        d2h = sum(t.numel() * t.element_size() for g_ in hgrp[2:] for t in g_)
         e2e_steps = max(3, args.steps)  # as many as the device-timed loop: pipeline fill and drain amortise alike
         s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-        in_ready = [event(), event()]
-        done = [event(), event()]
-        copied = [event(), event()]
+        f_in, b_in, f_done, kv_done, done, copied = ([event(), event()] for _ in range(6))
+        split_bwd = aw.bwd and not gqa
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         a, b = event(), event()
         a.record(stream)
         s_in.wait_event(a)
+
+        def to_host(dev_group, host_group):
+            with torch.cuda.stream(s_out):
+                for h, d_ in zip(host_group, dev_group):
+                    h.copy_(d_, non_blocking=True)
+
         for j in range(e2e_steps):
             bi = j % 2
+            in_f, in_b, out_f, out_kv, out_b = dev_sets[bi]
             if j >= 2:
                 s_in.wait_event(done[bi])  # step j-2 no longer reads these inputs
             with torch.cuda.stream(s_in):
-                for h, d_ in zip(hin, ins[bi]):
+                for h, d_ in zip(hgrp[0], in_f):
                     d_.copy_(h, non_blocking=True)
-            in_ready[bi].record(s_in)
-            stream.wait_event(in_ready[bi])
+                f_in[bi].record(s_in)
+                for h, d_ in zip(hgrp[1], in_b):
+                    d_.copy_(h, non_blocking=True)
+                b_in[bi].record(s_in)
+            stream.wait_event(f_in[bi])
             if j >= 2:
                 stream.wait_event(copied[bi])  # step j-2's results have been read back
-            qq, kk, vv = ins[bi][0], ins[bi][1], ins[bi][2]
-            oo, ll = outs[bi][0], outs[bi][1]
+            qq, kk, vv = in_f
+            oo, ll = out_f
             fwd_call(qq, kk, vv, oo, ll)
-            if aw.bwd:
-                bwd_call(qq, kk, vv, oo, ll, ins[bi][3], outs[bi][2], outs[bi][3], outs[bi][4])
+            f_done[bi].record(stream)
+            s_out.wait_event(f_done[bi])
+            to_host(out_f, hgrp[2])
+            stream.wait_event(b_in[bi])
+            if split_bwd:
+                ra.ringattn_bwd_phase(qq, kk, vv, oo, ll, in_b[0], out_b[0], out_kv[0], out_kv[1], *cfg, ws, 3)
+                kv_done[bi].record(stream)
+                s_out.wait_event(kv_done[bi])
+                to_host(out_kv, hgrp[3])
+                ra.ringattn_bwd_phase(qq, kk, vv, oo, ll, in_b[0], out_b[0], out_kv[0], out_kv[1], *cfg, ws, 4)
+            elif aw.bwd:
+                bwd_call(qq, kk, vv, oo, ll, in_b[0], out_b[0], out_kv[0], out_kv[1])
             if fw is not None:
-                xx, gy = ins[bi][-2], ins[bi][-1]
-                ra.blockwise_ffn(xx, w1, w2, w3, outs[bi][-5], fw.chunk, ffn_ws)
-                ra.blockwise_ffn_bwd(xx, w1, w2, w3, gy, *outs[bi][-4:], fw.chunk, ffn_bws)
+                xx, gy = in_b[-2], in_b[-1]
+                ra.blockwise_ffn(xx, w1, w2, w3, out_b[-5], fw.chunk, ffn_ws)
+                ra.blockwise_ffn_bwd(xx, w1, w2, w3, gy, *out_b[-4:], fw.chunk, ffn_bws)
             done[bi].record(stream)
             s_out.wait_event(done[bi])
-            with torch.cuda.stream(s_out):
-                for h, d_ in zip(hout, outs[bi]):
-                    h.copy_(d_, non_blocking=True)
+            if not split_bwd:
+                to_host(out_kv, hgrp[3])
+            to_host(out_b, hgrp[4])
             copied[bi].record(s_out)
         stream.wait_event(copied[(e2e_steps - 1) % 2])
         if e2e_steps > 1:
