@@ -142,7 +142,7 @@ def ringattn_bwd(q, k, v, out, lse, dout, dq, dk, dv, S, q_chunk, k_chunk, causa
 
 def ringattn_bwd_phase(q, k, v, out, lse, dout, dq, dk, dv, S, q_chunk, k_chunk, causal, workspace, phase_mask,
                        scale=0.0, stream=None):
-    """Run the selected phases of ringattn_bwd (bit 0 preprocess, 1 main, 2 dQ convert)."""
+    """Run the selected launches of ringattn_bwd: bit 0 preprocess, bit 1 the dK/dV pass, bit 2 the dQ pass."""
     B, H, N, D = _bhnd(q)
     nbytes = workspace.numel() * workspace.element_size()
     call("ringattn_bwd_phase", _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), _dev(lse, "lse"),
