@@ -117,10 +117,11 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, ui
 
 // One row-tile of a [rows x D] bf16 tensor (D a multiple of 64) through a
 // map made by make_tmap_bf16_tile: all D / 64 slabs of box_rows x 128 B in one
-// load, landing slab after slab with the 128-byte swizzle, i.e. exactly what
-// D / 64 2-D loads of the slabs would write.  One box per tile matters: a
-// CTA's tensor-memory loads progress box by box, so a single 32 KB box
-// arrives in about the time of one 16 KB box.
+// TMA load, landing slab after slab with the 128-byte swizzle, i.e. exactly
+// what D / 64 2-D loads of the slabs would write, with one instruction and one
+// box per tile.  (A single CTA streaming boxes alone moved 16 KB boxes at
+// about 26 B/clk and 32 KB boxes at 44-51 B/clk; inside the attention kernels
+// the change of box count did not change their timing.)
 __device__ __forceinline__ void tma_load_tile(void* smem_dst, const void* tmap, uint64_t* bar, int row) {
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
