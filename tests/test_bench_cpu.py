@@ -1,0 +1,72 @@
+"""bench.py host logic on CPU: the clock sampler against a fake NVML."""
+
+import sys
+import time
+import types
+
+import bench
+
+
+def _fake_nvml(clocks, powers_mw, reasons):
+    """A stand-in for the pynvml module that replays fixed readings."""
+    state = {"i": 0}
+    m = types.ModuleType("pynvml")
+    m.NVML_CLOCK_SM = 1
+
+    def nxt(seq):
+        return seq[min(state["i"], len(seq) - 1)]
+
+    def reason(h):  # the sampler reads clock, power, reasons: advance after the last
+        v = nxt(reasons)
+        state["i"] += 1
+        return v
+
+    m.nvmlInit = lambda: None
+    m.nvmlDeviceGetHandleByPciBusId = lambda bus: (_ for _ in ()).throw(RuntimeError("no PCI match"))
+    m.nvmlDeviceGetHandleByIndex = lambda i: ("handle", i)
+    m.nvmlDeviceGetMaxClockInfo = lambda h, kind: 1965
+    m.nvmlDeviceGetClockInfo = lambda h, kind: nxt(clocks)
+    m.nvmlDeviceGetPowerUsage = lambda h: nxt(powers_mw)
+    m.nvmlDeviceGetCurrentClocksEventReasons = reason
+    return m
+
+
+def test_clock_sampler_reads_nvml(monkeypatch):
+    fake = _fake_nvml([1965, 1600, 1580, 1580, 1580], [120_000, 990_000, 995_000, 993_000, 994_000],
+                      [0x0, 0x4, 0x4, 0x4, 0x4])
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    c = bench.ClockSampler(0)
+    c.start()
+    time.sleep(0.15)
+    out = c.stop()
+    assert out["source"] == "nvml, 10 ms"
+    assert out["samples"] >= 5
+    assert out["sm_max_mhz"] == 1965.0
+    # samples under load (> 300 W) only: the idle 1965 MHz reading is left out
+    assert out["sm_mhz"] == 1580.0
+    assert out["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_sampler_flags_thermal_and_hw_slowdown(monkeypatch):
+    fake = _fake_nvml([1200], [800_000], [0x8 | 0x40 | 0x20])
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    c = bench.ClockSampler(0)
+    c.start()
+    time.sleep(0.05)
+    out = c.stop()
+    assert out["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"]
+
+
+def test_clock_sampler_without_nvml_or_smi(monkeypatch):
+    broken = types.ModuleType("pynvml")
+
+    def fail():
+        raise RuntimeError("no driver")
+
+    broken.nvmlInit = fail
+    monkeypatch.setitem(sys.modules, "pynvml", broken)
+    monkeypatch.setattr(bench.subprocess, "Popen", lambda *a, **k: (_ for _ in ()).throw(FileNotFoundError()))
+    c = bench.ClockSampler(0)
+    c.start()
+    out = c.stop()
+    assert out["sm_mhz"] is None
