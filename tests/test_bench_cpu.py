@@ -70,3 +70,15 @@ def test_clock_sampler_without_nvml_or_smi(monkeypatch):
     c.start()
     out = c.stop()
     assert out["sm_mhz"] is None
+
+
+def test_clocks_rejected_rules():
+    ok = {"sm_mhz": 1580.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert not bench.clocks_rejected(ok)
+    assert not bench.clocks_rejected({"sm_mhz": 1960.0, "sm_max_mhz": 1965.0, "reasons": []})
+    for r in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"):
+        assert bench.clocks_rejected({"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": [r]})
+    # stuck low with no reason: a leftover clock lock
+    assert bench.clocks_rejected({"sm_mhz": 1000.0, "sm_max_mhz": 1965.0, "reasons": []})
+    # no samples at all is not a rejection
+    assert not bench.clocks_rejected({"sm_mhz": None, "sm_max_mhz": None, "reasons": []})
