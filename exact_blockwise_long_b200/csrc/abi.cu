@@ -171,7 +171,7 @@ int check_attn(const void* q, const void* k, const void* v, int64_t B, int64_t H
   if (L % q_chunk || L % k_chunk) return RA_ERR_SHAPE;
   const int tile = (dtype == RA_BF16) ? 128 : 64;
   if (q_chunk % tile || k_chunk % tile) return RA_ERR_SHAPE;
-  if (B * H * N > (int64_t)INT32_MAX) return RA_ERR_UNSUPPORTED;  // row index of the 2-D TMA view
+  if (B * H * N > (int64_t)INT32_MAX) return RA_ERR_UNSUPPORTED;  // row coordinate of the TMA tile maps (int32)
   if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return RA_ERR_ALIGN;
   return RA_OK;
 }
