@@ -14,7 +14,7 @@ compute dtype with round-to-nearest-even.
 
 from __future__ import annotations
 
-from dataclasses import dataclass, field
+from dataclasses import dataclass
 
 import numpy as np
 import torch

@@ -2,7 +2,6 @@
 every entry point include/ringattn.h declares, and rejects bad arguments
 before touching the device."""
 
-import ctypes
 import os
 import re
 

@@ -2,7 +2,6 @@
 the fused ring-step + merge mode and the standalone merge kernel, against
 the fp64 oracle on the same seeded input bits."""
 
-import itertools
 
 import numpy as np
 import pytest

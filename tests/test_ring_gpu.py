@@ -3,7 +3,6 @@ of the accumulate / cast kernels.  One GPU only: the ring's ranks are
 emulated one after another in this process (no rank waits on another), or
 run as a process group of one."""
 
-import numpy as np
 import pytest
 import torch
 

@@ -7,7 +7,6 @@ static scratch array, and refuse problems larger than that array.
 This file is collected last on purpose: it runs after every other test, and
 it also passes on its own in a fresh process."""
 
-import ctypes
 
 import pytest
 import torch
