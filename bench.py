@@ -39,7 +39,7 @@ METRIC = "ring-attn fwd+bwd TFLOP/s & tokens/s on 1 B200; % of BF16 tensor peak"
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
 # source it was taken on (sha256 of the source file).
 # Captured on 8 heads of the n32k_d128 workload and scaled x4 to its 32 heads
-# (heads are independent units; see profiles/*_n32k_d128_h8.md).
+# (heads are independent units).
 NCU_TRAFFIC = {
     ("bwd_kv_kernel", "n32k_d128"): {
         "bytes": 4 * (272.243200e6 + 101.754624e6),
@@ -128,6 +128,16 @@ def describe(aw, fw):
 # ---------------------------------------------------------------------------
 # peaks, clocks
 # ---------------------------------------------------------------------------
+
+def tensor_peak(pk, region_ms):
+    """The bf16 peak a timed region is held against: the burst figure for a
+    region shorter than the seconds a power-capped steady state takes to set
+    in, the sustained one for a longer region.  Returns (peak, description,
+    the other figure)."""
+    if region_ms >= 3000.0:
+        return pk["bf16_sustained"], f"bf16 dense, sustained ({pk['source']}; timed region >= 3 s)", pk["bf16_burst"]
+    return pk["bf16_burst"], f"bf16 dense, burst ({pk['source']}; timed region < 3 s)", pk["bf16_sustained"]
+
 
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -420,8 +430,9 @@ def run_step_mode(args, ra, dev, rank, world, dist):
                 "config": {"workload": f"n32k_d128_step: causal forward as {w.S} ring steps merged into fp32 "
                                        f"HBM accumulators, B={B}, H={H}, N={N}, d={D}"},
                 "roofline": {"bound": "tensor", "kernel": "fwd_tc2_kernel (step mode)", "achieved": tf,
-                             "peak": pk["bf16_sustained"], "unit": "TFLOP/s", "frac": tf / pk["bf16_sustained"],
-                             "traffic": None, "peak_kind": f"bf16 dense, sustained ({pk['source']})"},
+                             "peak": tensor_peak(pk, ms * args.steps)[0], "unit": "TFLOP/s",
+                             "frac": tf / tensor_peak(pk, ms * args.steps)[0], "traffic": None,
+                             "peak_kind": tensor_peak(pk, ms * args.steps)[1]},
                 "gpu_launches": launches * args.steps, "clocks": clk}
     rows = B * H * N
     nbytes = rows * (3 * D * 4 + 3 * 4)  # read o_a, o_b, lse_a, lse_b; write o_a, lse_a
@@ -637,10 +648,16 @@ def run_layer(args, ra, dev, rank, world, dist):
     def avg(fn):
         return sum(fn(s0, fm, bm) for s0, fm, bm in spans) / len(spans)
 
+    fwd_name = ra.ringattn_kernel_plan(0, w.N, w.D, torch.bfloat16, w.S)
+    bwd_plan = ra.ringattn_kernel_plan(1, w.N, w.D, torch.bfloat16, w.S)
+    # the layer records a mark after the attention backward's preprocess, its
+    # main pass and its last launch (the dQ conversion, or the split dQ pass)
+    main, last = (("bwd_fused_kernel", 2.5), ("bwd_dq_convert_kernel", 0.0)) if "bwd_fused_kernel" in bwd_plan \
+        else (("bwd_kv_kernel", 2.0), ("bwd_q_kernel", 0.5))
     kernels = {
-        "fwd_tc2_kernel": (avg(lambda s0, fm, bm: fm[1].elapsed_time(fm[2])), af, "fwd_tc.cu"),
-        "bwd_kv_kernel": (avg(lambda s0, fm, bm: bm[4].elapsed_time(bm[5])), 2.0 * af, "bwd_tc.cu"),
-        "bwd_q_kernel": (avg(lambda s0, fm, bm: bm[5].elapsed_time(bm[6])), 0.5 * af, "bwd_tc.cu"),
+        fwd_name: (avg(lambda s0, fm, bm: fm[1].elapsed_time(fm[2])), af, "fwd_tc.cu"),
+        main[0]: (avg(lambda s0, fm, bm: bm[4].elapsed_time(bm[5])), main[1] * af, "bwd_tc.cu"),
+        last[0]: (avg(lambda s0, fm, bm: bm[5].elapsed_time(bm[6])), last[1] * af, "bwd_tc.cu"),
         "gemm_kernel[projections]": (avg(lambda s0, fm, bm: fm[0].elapsed_time(fm[1]) + fm[2].elapsed_time(fm[3]) +
                                          bm[1].elapsed_time(bm[3]) + bm[6].elapsed_time(bm[8])), proj,
                                      "gemm_tc.cu"),
@@ -654,10 +671,11 @@ def run_layer(args, ra, dev, rank, world, dist):
     src = os.path.join(ROOT, "exact_blockwise_long_b200", "csrc", ksrc)
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
     tr = NCU_TRAFFIC.get((kname, args.workload))
-    roof = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": pk["bf16_sustained"],
-            "unit": "TFLOP/s", "frac": achieved / pk["bf16_sustained"],
+    peak, peak_kind, other = tensor_peak(pk, ms * args.steps)
+    roof = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak,
             "traffic": tr["bytes"] if tr and tr["sha256"] == sha else None,
-            "peak_kind": f"bf16 dense, sustained ({pk['source']})", "frac_of_burst": achieved / pk["bf16_burst"],
+            "peak_kind": peak_kind, "frac_of_other_peak": achieved / other,
             "kernel_ms": kms,
             "kernels": {k_: {"ms": v_[0], "algorithmic_tflops": v_[1] / (v_[0] * 1e-3) / 1e12}
                         for k_, v_ in kernels.items()}}
@@ -670,7 +688,7 @@ def run_layer(args, ra, dev, rank, world, dist):
                                    f"ffn_chunk={w.ffn_chunk}, {'causal' if w.causal else 'non-causal'}",
                        "B": w.B, "seq_len": w.N, "H": w.H, "head_dim": w.D, "d_ff": w.d_ff, "shards": w.S,
                        "l2": "inputs larger than L2 (no flush between steps)"},
-            "tokens_per_s": w.T * world / (ms * 1e-3), "pct_of_bf16_peak": 100.0 * value / world / pk["bf16_sustained"],
+            "tokens_per_s": w.T * world / (ms * 1e-3), "pct_of_bf16_peak": 100.0 * value / world / peak,
             "roofline": roof, "gpu_launches": launches_per_step * args.steps, "clocks": clk}
 
     if not args.no_e2e:
@@ -790,6 +808,13 @@ def main():
     stream = torch.cuda.current_stream()
     cfg = (aw.S, aw.q_chunk, aw.k_chunk, aw.causal)
     gqa = aw.kv_heads != aw.H
+    # the kernels the library launches for this shape on this device
+    fwd_name = ra.ringattn_kernel_plan(0, aw.N, aw.D, torch.bfloat16, aw.S)
+    bwd_plan = ra.ringattn_kernel_plan(1, aw.N, aw.D, torch.bfloat16, aw.S) if aw.bwd else ""
+    fused = "bwd_fused_kernel" in bwd_plan
+    # backward phases timed one by one: preprocess, main pass, last pass
+    bwd_phases = (1, 8, 16) if fused else (1, 2, 4)
+    bwd_names = ("bwd_fused_kernel", "bwd_dq_convert_kernel") if fused else ("bwd_kv_kernel", "bwd_q_kernel")
 
     def fwd_call(qq, kk, vv, oo, ll):
         if gqa:
@@ -823,15 +848,10 @@ def main():
                 e[4].record(stream)
             launches += 3
         elif aw.bwd:
-            ra.ringattn_bwd_phase(q, k, v, o, lse, do, dq, dk, dv, *cfg, ws, 1)
-            if timed:
-                e[2].record(stream)
-            ra.ringattn_bwd_phase(q, k, v, o, lse, do, dq, dk, dv, *cfg, ws, 2)
-            if timed:
-                e[3].record(stream)
-            ra.ringattn_bwd_phase(q, k, v, o, lse, do, dq, dk, dv, *cfg, ws, 4)
-            if timed:
-                e[4].record(stream)
+            for i, m in enumerate(bwd_phases):
+                ra.ringattn_bwd_phase(q, k, v, o, lse, do, dq, dk, dv, *cfg, ws, m)
+                if timed:
+                    e[2 + i].record(stream)
             launches += 3
         if fw is not None:
             if timed:
@@ -847,8 +867,8 @@ def main():
             if aw.bwd and gqa:
                 ev.setdefault("bwd", []).append((e[1], e[4]))
             elif aw.bwd:
-                ev.setdefault("bwd_kv", []).append((e[2], e[3]))
-                ev.setdefault("bwd_q", []).append((e[3], e[4]))
+                ev.setdefault("bwd_main", []).append((e[2], e[3]))
+                ev.setdefault("bwd_last", []).append((e[3], e[4]))
         return launches
 
     for _ in range(args.warmup):
@@ -896,18 +916,25 @@ def main():
     def mean_ms(pairs):
         return sum(a.elapsed_time(b) for a, b in pairs) / len(pairs)
 
-    # Algorithmic FLOPs per launch: the forward's two matmuls; the dK/dV
-    # kernel's four (S, dP, dV, dK), the dQ kernel's one (dQ; its S and dP
-    # are recomputation, not credited): 2 + 4 + 1 = 7 = 3.5 x the forward's 2.
+    # Algorithmic FLOPs per launch: the forward's two matmuls (S, PV); the
+    # fused backward pass's five (S, dP, dV, dK, dQ); or, split, the dK/dV
+    # kernel's four and the dQ kernel's one (its S and dP are recomputation,
+    # not credited): 2 + 5 = 7 = 3.5 x the forward's 2 either way.
     fwd_fl = attn_fwd_flops(aw)
-    fwd_name = "fwd_tc2_kernel" if (aw.N // aw.S) % 256 == 0 else "fwd_tc_kernel"
     kernels = {fwd_name: (mean_ms(ev["fwd"]), fwd_fl, "fwd_tc.cu")}
+    hbm = {}
     if aw.bwd and gqa:
-        # one call: preprocess + dK/dV + dQ launches, timed together
-        kernels["bwd_kv_kernel+bwd_q_kernel"] = (mean_ms(ev["bwd"]), 2.5 * fwd_fl, "bwd_tc.cu")
+        # one call: all the backward's launches, timed together
+        kernels[bwd_plan.replace("bwd_preprocess_kernel+", "")] = (mean_ms(ev["bwd"]), 2.5 * fwd_fl, "bwd_tc.cu")
+    elif aw.bwd and fused:
+        kernels["bwd_fused_kernel"] = (mean_ms(ev["bwd_main"]), 2.5 * fwd_fl, "bwd_tc.cu")
+        # the conversion reads the fp32 accumulator and writes bf16 dq
+        conv_ms = mean_ms(ev["bwd_last"])
+        conv_bytes = aw.B * aw.H * aw.N * aw.D * 6.0
+        hbm["bwd_dq_convert_kernel"] = {"ms": conv_ms, "gbs": conv_bytes / (conv_ms * 1e-3) / 1e9}
     elif aw.bwd:
-        kernels["bwd_kv_kernel"] = (mean_ms(ev["bwd_kv"]), 2.0 * fwd_fl, "bwd_tc.cu")
-        kernels["bwd_q_kernel"] = (mean_ms(ev["bwd_q"]), 0.5 * fwd_fl, "bwd_tc.cu")
+        kernels["bwd_kv_kernel"] = (mean_ms(ev["bwd_main"]), 2.0 * fwd_fl, "bwd_tc.cu")
+        kernels["bwd_q_kernel"] = (mean_ms(ev["bwd_last"]), 0.5 * fwd_fl, "bwd_tc.cu")
     kname = max(kernels, key=lambda k_: kernels[k_][0])
     if fw is not None:
         # the feed-forward's forward and backward GEMMs, timed together
@@ -918,18 +945,21 @@ def main():
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
     tr = NCU_TRAFFIC.get((kname, args.workload))
     traffic = tr["bytes"] if tr and tr["sha256"] == sha else None
-    roof = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": pk["bf16_sustained"],
-            "unit": "TFLOP/s", "frac": achieved / pk["bf16_sustained"], "traffic": traffic,
-            "peak_kind": f"bf16 dense, sustained ({pk['source']})",
-            "frac_of_burst": achieved / pk["bf16_burst"], "kernel_ms": kms,
+    peak, peak_kind, other = tensor_peak(pk, ms_step * args.steps)
+    roof = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
+            "frac_of_other_peak": achieved / other, "kernel_ms": kms,
             "kernels": {k_: {"ms": v_[0], "algorithmic_tflops": v_[1] / (v_[0] * 1e-3) / 1e12}
                         for k_, v_ in kernels.items()}}
+    if hbm:
+        roof["hbm_kernels"] = hbm
 
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": describe(aw, fw),
-            "tokens_per_s": tokens_s, "pct_of_bf16_peak": 100.0 * value / world / pk["bf16_sustained"],
-            "roofline": roof, "gpu_launches": launches, "clocks": clk}
+            "tokens_per_s": tokens_s, "pct_of_bf16_peak": 100.0 * value / world / peak,
+            "roofline": roof, "gpu_launches": launches, "clocks": clk,
+            "kernel_plan": {"fwd": fwd_name, "bwd": bwd_plan or None}}
 
     # End to end through the public API: every step copies its inputs from
     # pinned host memory and reads its results back.  Two device buffer sets
@@ -989,11 +1019,14 @@ def main():
             to_host(out_f, hgrp[2])
             stream.wait_event(b_in[bi])
             if split_bwd:
-                ra.ringattn_bwd_phase(qq, kk, vv, oo, ll, in_b[0], out_b[0], out_kv[0], out_kv[1], *cfg, ws, 3)
+                # dk, dv are final after the main pass: they go back while the last pass runs
+                ra.ringattn_bwd_phase(qq, kk, vv, oo, ll, in_b[0], out_b[0], out_kv[0], out_kv[1], *cfg, ws,
+                                      bwd_phases[0] | bwd_phases[1])
                 kv_done[bi].record(stream)
                 s_out.wait_event(kv_done[bi])
                 to_host(out_kv, hgrp[3])
-                ra.ringattn_bwd_phase(qq, kk, vv, oo, ll, in_b[0], out_b[0], out_kv[0], out_kv[1], *cfg, ws, 4)
+                ra.ringattn_bwd_phase(qq, kk, vv, oo, ll, in_b[0], out_b[0], out_kv[0], out_kv[1], *cfg, ws,
+                                      bwd_phases[2])
             elif aw.bwd:
                 bwd_call(qq, kk, vv, oo, ll, in_b[0], out_b[0], out_kv[0], out_kv[1])
             if fw is not None:

@@ -31,6 +31,7 @@ _SZ = ctypes.c_size_t
 SIGNATURES = {
     "ringattn_version": (_I, []),
     "ringattn_status_string": (ctypes.c_char_p, [_I]),
+    "ringattn_kernel_plan": (ctypes.c_char_p, [_I, _I64, _I64, _I, _I]),
     "ringattn_fwd": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _F, _P]),
     "ringattn_fwd_gqa": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _F, _P]),
     "ringattn_bwd_gqa": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I,

@@ -119,6 +119,14 @@ def ringattn_merge(o_a, lse_a, o_b, lse_b, stream=None):
     return o_a, lse_a
 
 
+def ringattn_kernel_plan(op, N, D, dtype, S):
+    """Names of the kernels ringattn_fwd (op 0) or ringattn_bwd (op 1) launch
+    for this shape on the current device, joined by '+'; None if invalid."""
+    r = lib().ringattn_kernel_plan(int(op), int(N), int(D), _DT[dtype] if not isinstance(dtype, int) else dtype,
+                                   int(S))
+    return r.decode() if r is not None else None
+
+
 def ringattn_bwd_workspace_size(B, H, N, D) -> int:
     return int(lib().ringattn_bwd_workspace_size(int(B), int(H), int(N), int(D)))
 
@@ -142,7 +150,9 @@ def ringattn_bwd(q, k, v, out, lse, dout, dq, dk, dv, S, q_chunk, k_chunk, causa
 
 def ringattn_bwd_phase(q, k, v, out, lse, dout, dq, dk, dv, S, q_chunk, k_chunk, causal, workspace, phase_mask,
                        scale=0.0, stream=None):
-    """Run the selected launches of ringattn_bwd: bit 0 preprocess, bit 1 the dK/dV pass, bit 2 the dQ pass."""
+    """Run the selected backward launches: bit 0 preprocess, bits 1-2 the split
+    (deterministic) dK/dV and dQ passes, bit 3 the fused pass, bit 4 the dQ
+    conversion (include/ringattn.h, ringattn_bwd_phase)."""
     B, H, N, D = _bhnd(q)
     nbytes = workspace.numel() * workspace.element_size()
     call("ringattn_bwd_phase", _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), _dev(lse, "lse"),
@@ -153,9 +163,9 @@ def ringattn_bwd_phase(q, k, v, out, lse, dout, dq, dk, dv, S, q_chunk, k_chunk,
 
 
 def ringattn_bwd_noalloc(q, k, v, out, lse, dout, dq, dk, dv, S, q_chunk, k_chunk, causal, scale=0.0, stream=None):
-    """ringattn_bwd without a workspace: the library's fixed static scratch is
-    used instead, for callers that cannot allocate device memory.  Calls must
-    not overlap on the GPU (they share that scratch)."""
+    """The deterministic backward without a workspace: the library's fixed
+    static scratch is used instead, for callers that cannot allocate device
+    memory.  Calls must not overlap on the GPU (they share that scratch)."""
     B, H, N, D = _bhnd(q)
     for t in (k, v, out, dout, dq, dk, dv):
         if t.shape != q.shape or t.dtype != q.dtype:

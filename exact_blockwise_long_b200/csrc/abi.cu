@@ -199,6 +199,15 @@ const char* ringattn_status_string(int status) {
   }
 }
 
+const char* ringattn_kernel_plan(int op, int64_t N, int64_t D, int dtype, int S) {
+  if (N <= 0 || S <= 0 || N % S) return nullptr;
+  if (D != 64 && D != 128) return nullptr;
+  if (dtype != RA_BF16 && dtype != RA_F32) return nullptr;
+  if (op == 0) return dtype == RA_F32 ? "fwd_simt_kernel" : fwd_tc_kernel_name(N / S, D);
+  if (op == 1) return dtype == RA_BF16 ? bwd_tc_kernel_names(D) : nullptr;
+  return nullptr;
+}
+
 int ringattn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t H,
                  int64_t N, int64_t D, int dtype, int S, int q_chunk, int k_chunk, int causal, float scale,
                  void* stream) {
@@ -247,32 +256,59 @@ int ringattn_merge(float* o_a, float* lse_a, const float* o_b, const float* lse_
 }
 
 size_t ringattn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D) {
-  if (B <= 0 || H <= 0 || N <= 0 || D <= 0) return 0;  // empty problems need no workspace
-  const size_t dvec = (size_t)B * H * N * sizeof(float);
-  return 2 * ((dvec + 255) & ~(size_t)255);
+  return bwd_workspace_bytes(B, H, N, D, bwd_fused_supported(D));  // 0 for empty problems
 }
 
-namespace {
-int bwd_impl(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
-             void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t D, int dtype, int S,
-             int q_chunk, int k_chunk, int causal, float scale, void* workspace, size_t workspace_bytes,
-             int phase_mask, void* stream) {
-  if (phase_mask <= 0 || phase_mask > 7) return RA_ERR_ARG;
+}  // extern "C"
+
+namespace ra {
+
+int check_bwd_args(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+                   const void* dq, const void* dk, const void* dv, int64_t B, int64_t H, int64_t Hkv, int64_t N,
+                   int64_t D, int dtype, int S, int q_chunk, int k_chunk, int causal, int phase_mask) {
+  if (phase_mask <= 0 || phase_mask > kPhaseAll) return RA_ERR_ARG;
   if (Hkv < 0 || (Hkv == 0 && H != 0) || (Hkv > 0 && H % Hkv != 0)) return RA_ERR_ARG;
   int rc = check_attn(q, k, v, B, H, N, D, dtype, S, q_chunk, k_chunk, causal);
-  if (rc == kEmpty) return dtype == RA_BF16 ? RA_OK : RA_ERR_UNSUPPORTED;
+  if (rc == kEmpty) return dtype == RA_BF16 ? kBwdEmpty : RA_ERR_UNSUPPORTED;
   if (rc != RA_OK) return rc;
   if (!out || !lse || !dout || !dq || !dk || !dv) return RA_ERR_ARG;
   if (!aligned16(out) || !aligned16(lse) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) ||
       !aligned16(dv))
     return RA_ERR_ALIGN;
   if (dtype != RA_BF16) return RA_ERR_UNSUPPORTED;
-  if (!workspace || workspace_bytes < ringattn_bwd_workspace_size(B, H, N, D)) return RA_ERR_WORKSPACE;
+  if ((phase_mask & (kPhaseFused | kPhaseConvert)) && !bwd_fused_supported(D)) return RA_ERR_UNSUPPORTED;
+  return RA_OK;
+}
+
+int run_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+            void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t D, int S,
+            int q_chunk, int k_chunk, int causal, float scale, void* workspace, size_t workspace_bytes,
+            int phase_mask, void* stream) {
+  AttnArgs a{q, k, v, B, H, N, D, RA_BF16, S, q_chunk, k_chunk, causal, resolve_scale(scale, D), Hkv};
+  return launch_bwd_tc(a, out, lse, dout, dq, dk, dv, workspace, workspace_bytes, phase_mask,
+                       static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace ra
+
+namespace {
+int bwd_impl(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+             void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t D, int dtype, int S,
+             int q_chunk, int k_chunk, int causal, float scale, void* workspace, size_t workspace_bytes,
+             int phase_mask, void* stream) {
+  const int rc = check_bwd_args(q, k, v, out, lse, dout, dq, dk, dv, B, H, Hkv, N, D, dtype, S, q_chunk, k_chunk,
+                                causal, phase_mask);
+  if (rc == kBwdEmpty) return RA_OK;
+  if (rc != RA_OK) return rc;
+  const bool fused = (phase_mask & (kPhaseFused | kPhaseConvert)) != 0;
+  if (!workspace || workspace_bytes < bwd_workspace_bytes(B, H, N, D, fused)) return RA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return RA_ERR_ALIGN;
-  AttnArgs a{q, k, v, B, H, N, D, dtype, S, q_chunk, k_chunk, causal, resolve_scale(scale, D), Hkv};
-  return launch_bwd_tc(a, out, lse, dout, dq, dk, dv, workspace, phase_mask, static_cast<cudaStream_t>(stream));
+  return run_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, H, Hkv, N, D, S, q_chunk, k_chunk, causal, scale,
+                 workspace, workspace_bytes, phase_mask, stream);
 }
 }  // namespace
+
+extern "C" {
 
 int ringattn_bwd_phase(const void* q, const void* k, const void* v, const void* out, const float* lse,
                        const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N, int64_t D,
@@ -287,15 +323,15 @@ int ringattn_bwd_gqa(const void* q, const void* k, const void* v, const void* ou
                      int64_t D, int dtype, int S, int q_chunk, int k_chunk, int causal, float scale,
                      void* workspace, size_t workspace_bytes, void* stream) {
   return bwd_impl(q, k, v, out, lse, dout, dq, dk, dv, B, H, Hkv, N, D, dtype, S, q_chunk, k_chunk, causal, scale,
-                  workspace, workspace_bytes, 7, stream);
+                  workspace, workspace_bytes, bwd_default_phases(D), stream);
 }
 
 int ringattn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
                  const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N, int64_t D,
                  int dtype, int S, int q_chunk, int k_chunk, int causal, float scale, void* workspace,
                  size_t workspace_bytes, void* stream) {
-  return ringattn_bwd_phase(q, k, v, out, lse, dout, dq, dk, dv, B, H, N, D, dtype, S, q_chunk, k_chunk, causal,
-                            scale, workspace, workspace_bytes, 7, stream);
+  return bwd_impl(q, k, v, out, lse, dout, dq, dk, dv, B, H, H, N, D, dtype, S, q_chunk, k_chunk, causal, scale,
+                  workspace, workspace_bytes, bwd_default_phases(D), stream);
 }
 
 size_t ringattn_decode_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D, int S, int k_chunk) {

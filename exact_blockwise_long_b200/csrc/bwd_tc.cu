@@ -49,6 +49,7 @@ constexpr int kHalf = 64;      // score columns per element-wise warpgroup
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t FULL = 0xffffffffu;
+constexpr int kMaxDynSmem = 232448;  // 227 KB: the most dynamic shared memory one CTA may use
 
 struct BParams {
   const __nv_bfloat16* q;     // [BH*N, D]
@@ -58,6 +59,8 @@ struct BParams {
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
+  float* dqacc;        // fused pass: fp32 dQ accumulator [BH*N, D] (unscaled)
+  int smem_alloc;      // fused pass: dynamic shared memory bytes of the launch
   int BH, N, S, L, causal, num_tiles;
   int H, G;            // query heads; query heads per key/value head
   int BHkv;            // batch x key/value heads
@@ -173,7 +176,7 @@ struct KVLayout {
   static constexpr int kBytes = kAbort + 4;
   static constexpr int kAlloc = kBytes + 1024;
 };
-static_assert(KVLayout<128>::kAlloc <= 232448, "dK/dV tile set exceeds shared memory");
+static_assert(KVLayout<128>::kAlloc <= kMaxDynSmem, "dK/dV tile set exceeds shared memory");
 
 // Warp roles: warp 0 TMA producer (K, V once; Q, dO, lse, D per step),
 // warp 1 MMA issuer, warp 2 TMEM allocator, warps 4-7 and 8-11 one thread
@@ -424,6 +427,342 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ===========================================================================
+// dK, dV and dQ in one pass: key/value tile stationary, dQ reduced in fp32
+// ===========================================================================
+// The dK/dV loop above plus a fifth matmul per tile pair,
+//   dQ^T_n = K^T dS^T_n   (M = d, N = 128 queries, K = 128 keys),
+// whose 128 x 128 fp32 result is added into an fp32 dQ accumulator in HBM
+// (L2-resident for the head group in flight) by the element-wise warps.  It
+// replaces the query-stationary pass, which recomputes S and dP (two of its
+// three matmuls) to avoid those additions.  The sum over key tiles then runs
+// in whatever order the CTAs reach L2, so dQ is reproducible only up to fp32
+// summation order; dK and dV are still written once per key tile.
+//
+// Both operands of dQ^T come from shared memory: K (stationary, read as an
+// MN-major A operand) and dS^T (MN-major B), which the element-wise warps
+// write beside their TMEM copy.  Tensor memory holds S^T [0,128),
+// dP^T [128,256), dK [256,384), dV [384,512): dQ^T has no columns of its own
+// and lands in the dP^T columns after dK has read dS^T from them; the next
+// dP^T is issued once the element-wise warps have loaded dQ^T out.
+// MMA order per step n: dV_n (two halves), dP_n, S_{n+1}, dK_n, dQ^T_n.
+// Element-wise order per step n: P^T_n, then dQ^T_{n-1} drained (loaded,
+// released, its 64 columns per thread reduced into HBM), then dS^T_n.
+template <int D>
+struct FusedLayout {
+  static constexpr int kTile = kT * D * 2;
+  static constexpr int kSlab = kT * 128;
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + kTile;
+  static constexpr int kQ = kV + kTile;
+  static constexpr int kDO = kQ + kSt * kTile;
+  static constexpr int kDS = kDO + kSt * kTile;  // dS^T bf16 [128 keys x 128 queries], two 64-query slabs
+  static constexpr int kVec = kDS + kT * kT * 2;  // per stage: lse*log2e [128], D [128]
+  static constexpr int kBar = kVec + kSt * 1024;
+  static constexpr int kNumBars = 1 + 2 * kSt + 8;
+  static constexpr int kTmemSlot = kBar + kNumBars * 8;
+  static constexpr int kAbort = kTmemSlot + 4;
+  static constexpr int kBytes = kAbort + 4;
+  // The tiles need a 1024-byte aligned base.  At d = 128 the layout leaves
+  // less than 1024 bytes of the 227 KB a CTA may hold for aligning it, so
+  // the launch asks for the maximum and the kernel checks its base.
+  static constexpr int kAlloc = kBytes + 1024 <= kMaxDynSmem ? kBytes + 1024 : kMaxDynSmem;
+};
+static_assert(FusedLayout<128>::kBytes <= kMaxDynSmem, "fused backward tile set exceeds shared memory");
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                     const BParams p) {
+  static_assert(D == 128, "dQ^T takes all 128 TMEM lanes: M = d = 128");
+  using LY = FusedLayout<D>;
+  extern __shared__ uint8_t smem_fu[];
+  const uint32_t pad = (1024 - (smem_u32(smem_fu) & 1023)) & 1023;
+  if (pad + LY::kBytes > (uint32_t)p.smem_alloc) {
+    // the shared-memory window cannot hold the aligned tile set: report, do nothing
+    if (threadIdx.x == 0) atomicExch(p.st.word, (int)RA_ERR_UNSUPPORTED);
+    return;
+  }
+  uint8_t* smem = smem_fu + pad;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  int kvbh, kt;
+  grouped_order((int)blockIdx.x, p.num_tiles, p.BHkv, p.group, kvbh, kt);
+  const int krow0 = kvbh * p.N + kt * kT;
+  const int tps = p.L / kT;
+  const int Hkv = p.H / p.G;
+  const int qbh0 = (kvbh / Hkv) * p.H + (kvbh % Hkv) * p.G;
+  const RingWalkKV walk{(kt * kT) / p.L, p.S, tps, kt, p.causal, qbh0, p.G};
+  const int n_total = walk.count();
+
+  uint8_t* sK = smem + LY::kK;
+  uint8_t* sV = smem + LY::kV;
+  uint8_t* sQ = smem + LY::kQ;
+  uint8_t* sDO = smem + LY::kDO;
+  uint8_t* sDS = smem + LY::kDS;
+  float* sVec = reinterpret_cast<float*>(smem + LY::kVec);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + LY::kBar);
+  uint64_t* bar_kv = bars;
+  uint64_t* bar_qf = bar_kv + 1;
+  uint64_t* bar_qe = bar_qf + kSt;
+  uint64_t* bar_sf = bar_qe + kSt;   // S^T computed
+  uint64_t* bar_dpf = bar_sf + 1;    // dP^T computed
+  uint64_t* bar_ph = bar_dpf + 1;    // first half of P^T written to TMEM
+  uint64_t* bar_pr = bar_ph + 1;     // all of P^T written to TMEM
+  uint64_t* bar_dsr = bar_pr + 1;    // dS^T written to TMEM and shared memory
+  uint64_t* bar_dqf = bar_dsr + 1;   // dQ^T computed (in the dP^T columns)
+  uint64_t* bar_dqe = bar_dqf + 1;   // dQ^T loaded out: the dP^T columns are free
+  uint64_t* bar_done = bar_dqe + 1;  // dK, dV final
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + LY::kTmemSlot);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LY::kAbort);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_kv, 1);
+    for (int s = 0; s < kSt; ++s) {
+      mbar_init(&bar_qf[s], 1);
+      mbar_init(&bar_qe[s], 1);
+    }
+    mbar_init(bar_sf, 1);
+    mbar_init(bar_dpf, 1);
+    mbar_init(bar_ph, 2 * 128);
+    mbar_init(bar_pr, 2 * 128);
+    mbar_init(bar_dsr, 2 * 128);
+    mbar_init(bar_dqf, 1);
+    mbar_init(bar_dqe, 2 * 128);
+    mbar_init(bar_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tDP = tmem + 128, tDK = tmem + 256, tDV = tmem + 384;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+      mbar_arrive_expect_tx(bar_kv, 2 * LY::kTile);
+      tma_load_tile(sK, &tmK, bar_kv, krow0);
+      tma_load_tile(sV, &tmV, bar_kv, krow0);
+      int n = 0;
+      walk.run([&](int qbh, int qt, bool) {
+        const int st = n % kSt;
+        const int qrow = qbh * p.N + qt * kT;
+        if (!mbar_wait(&bar_qe[st], ((n / kSt) & 1) ^ 1, p.st, abort_flag)) return false;
+        mbar_arrive_expect_tx(&bar_qf[st], 2 * LY::kTile + 1024);
+        tma_load_tile(sQ + st * LY::kTile, &tmQ, &bar_qf[st], qrow);
+        tma_load_tile(sDO + st * LY::kTile, &tmDO, &bar_qf[st], qrow);
+        bulk_load(sVec + st * 256, p.lse2 + qrow, 512, &bar_qf[st]);
+        bulk_load(sVec + st * 256 + 128, p.dvec + qrow, 512, &bar_qf[st]);
+        ++n;
+        return true;
+      });
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idSS = idesc_bf16_f32(kT, kT, false, false);  // K-major x K-major
+      constexpr uint32_t idTS = idesc_bf16_f32(kT, D, false, true);    // TMEM A x MN-major B
+      constexpr uint32_t idDQ = idesc_bf16_f32(D, kT, true, true);     // MN-major K^T x MN-major dS^T
+      const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV);
+      const uint32_t q_base = smem_u32(sQ), do_base = smem_u32(sDO), ds_base = smem_u32(sDS);
+      auto a_col = [](int kk) -> uint32_t { return kk < 4 ? kk * 8 : 64 + (kk - 4) * 8; };
+      auto issue_s = [&](int st) {
+        const uint32_t qb = q_base + st * LY::kTile;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * LY::kSlab + (kk & 3) * 32;
+          mma_bf16_ss(tS, sdesc_sw128(k_base + off, 16, 1024), sdesc_sw128(qb + off, 16, 1024), idSS,
+                      kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_sf);
+      };
+      bool ok = mbar_wait(bar_kv, 0, p.st, abort_flag) && mbar_wait(&bar_qf[0], 0, p.st, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+      }
+      for (int n = 0; ok && n < n_total; ++n) {
+        const int st = n % kSt;
+        const uint32_t qb = q_base + st * LY::kTile, dob = do_base + st * LY::kTile;
+        // dV += P^T dO in two halves as the element-wise warps publish them
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          if (!(ok = mbar_wait(half ? bar_pr : bar_ph, n & 1, p.st, abort_flag))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int kk = (j >> 1) * 4 + half * 2 + (j & 1);
+            mma_bf16_ts(tDV, tS + a_col(kk), sdesc_sw128(dob + kk * 2048, LY::kSlab, 1024), idTS,
+                        (n > 0 || half > 0 || j > 0) ? 1u : 0u);
+          }
+        }
+        if (!ok) break;
+        // dP^T = V dO^T into the dP^T columns, once dQ^T_{n-1} has left them
+        if (n > 0 && !(ok = mbar_wait(bar_dqe, (n - 1) & 1, p.st, abort_flag))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * LY::kSlab + (kk & 3) * 32;
+          mma_bf16_ss(tDP, sdesc_sw128(v_base + off, 16, 1024), sdesc_sw128(dob + off, 16, 1024), idSS,
+                      kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_dpf);
+        // S^T of the next query tile into the columns dV has read
+        if (n + 1 < n_total) {
+          const int st1 = (n + 1) % kSt;
+          if (!(ok = mbar_wait(&bar_qf[st1], ((n + 1) / kSt) & 1, p.st, abort_flag))) break;
+          tc_fence_after();
+          issue_s(st1);
+        }
+        if (!(ok = mbar_wait(bar_dsr, n & 1, p.st, abort_flag))) break;
+        tc_fence_after();
+        // dK += dS^T Q (dS^T from the dP^T columns)
+#pragma unroll
+        for (int kk = 0; kk < kT / 16; ++kk)
+          mma_bf16_ts(tDK, tDP + a_col(kk), sdesc_sw128(qb + kk * 2048, LY::kSlab, 1024), idTS,
+                      (n > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bar_qe[st]);  // Q_n and dO_n are no longer read
+        // dQ^T = K^T dS^T over the dP^T columns (dK has been issued before it)
+#pragma unroll
+        for (int kk = 0; kk < kT / 16; ++kk)
+          mma_bf16_ss(tDP, sdesc_sw128(k_base + kk * 2048, LY::kSlab, 1024),
+                      sdesc_sw128(ds_base + kk * 2048, LY::kSlab, 1024), idDQ, kk > 0 ? 1u : 0u);
+        mma_commit(bar_dqf);
+      }
+      mma_commit(bar_done);
+    }
+  } else if (warp >= 4) {
+    const int h = (warp >> 2) - 1;          // query columns [64 h, 64 h + 64)
+    const int r = (warp & 3) * 32 + lane;   // key row of S^T, dP^T = TMEM lane; d index of dQ^T
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t cS = tS + lane_off + h * kHalf, cDP = tDP + lane_off + h * kHalf;
+    const float2 sl22 = make_float2(p.scale_log2, p.scale_log2);
+    // this thread's row of the dS^T tile in shared memory: slab h, 128-byte
+    // swizzled row r (16-byte chunk j stored at chunk j ^ (r % 8))
+    const uint32_t ds_row = smem_u32(sDS) + h * LY::kSlab + r * 128;
+    // dQ^T of step m (query rows qrow .. qrow + 127): load this thread's 64
+    // columns, free the dP^T columns, then add them into the accumulator.
+    auto drain_dq = [&](int m, int qrow, bool release) -> bool {
+      if (!__all_sync(FULL, mbar_wait(bar_dqf, m & 1, p.st, abort_flag))) return false;
+      tc_fence_after();
+      uint32_t a[32], b[32];
+      tmem_ld32(cDP, a);
+      tmem_ld32(cDP + 32, b);
+      tmem_ld_wait();
+      if (release) {
+        tc_fence_before();
+        mbar_arrive(bar_dqe);
+      }
+      float* dst = p.dqacc + ((size_t)qrow + h * kHalf) * D + r;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) red_add_f32(dst + (size_t)c * D, __uint_as_float(a[c]));
+#pragma unroll
+      for (int c = 0; c < 32; ++c) red_add_f32(dst + (size_t)(32 + c) * D, __uint_as_float(b[c]));
+      return true;
+    };
+    int n = 0, prev_qrow = 0;
+    const bool ok = walk.run([&](int qbh, int qt, bool diag) {
+      const int st = n % kSt;
+      if (!__all_sync(FULL, mbar_wait(&bar_qf[st], (n / kSt) & 1, p.st, abort_flag))) return false;
+      if (!__all_sync(FULL, mbar_wait(bar_sf, n & 1, p.st, abort_flag))) return false;
+      tc_fence_after();
+      const float* lse2 = sVec + st * 256 + h * kHalf;
+      const float* dvec = lse2 + 128;
+      float P[kHalf];
+      load_row64(cS, P);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int c = 32 * half; c < 32 * half + 32; c += 2) {
+          const float2 t = fma2(make_float2(P[c], P[c + 1]), sl22, make_float2(-lse2[c], -lse2[c + 1]));
+          P[c] = ex2_approx(t.x);
+          P[c + 1] = ex2_approx(t.y);
+        }
+        if (diag) {
+#pragma unroll
+          for (int c = 32 * half; c < 32 * half + 32; ++c)
+            if (r > h * kHalf + c) P[c] = 0.f;  // key r is in the future of the query
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) pk[x] = pack_bf16x2(P[32 * half + 2 * x], P[32 * half + 2 * x + 1]);
+        tmem_st16(cS + 16 * half, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(half ? bar_pr : bar_ph);
+      }
+      // the previous step's dQ^T: its columns are needed for this step's dP^T
+      if (n > 0 && !drain_dq(n - 1, prev_qrow, true)) return false;
+
+      if (!__all_sync(FULL, mbar_wait(bar_dpf, n & 1, p.st, abort_flag))) return false;
+      tc_fence_after();
+      {
+        uint32_t a[32], b[32];
+        tmem_ld32(cDP, a);
+        tmem_ld32(cDP + 32, b);
+        tmem_ld_wait();
+        uint32_t pk[32];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const int q = 2 * x;
+          pk[x] = pack_bf16x2(P[q] * (__uint_as_float(a[2 * x]) - dvec[q]),
+                              P[q + 1] * (__uint_as_float(a[2 * x + 1]) - dvec[q + 1]));
+          pk[16 + x] = pack_bf16x2(P[32 + q] * (__uint_as_float(b[2 * x]) - dvec[32 + q]),
+                                   P[33 + q] * (__uint_as_float(b[2 * x + 1]) - dvec[33 + q]));
+        }
+        tmem_st32(cDP, pk);  // bf16 dS^T over the first 32 of this group's dP^T columns
+        // the same 64 bf16 values as row r of slab h of the shared-memory dS^T
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          st_shared_v4(ds_row + ((j ^ (r & 7)) << 4), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar_dsr);
+      prev_qrow = qbh * p.N + qt * kT;
+      ++n;
+      return true;
+    });
+    bool fin = ok;
+    if (fin && n > 0) fin = drain_dq(n - 1, prev_qrow, false);
+    if (fin && __all_sync(FULL, mbar_wait(bar_done, 0, p.st, abort_flag))) {
+      tc_fence_after();
+      const size_t row = (size_t)krow0 + r;
+      store_acc_row<D / 2>(tDK + lane_off + h * (D / 2), p.scale, p.dk + row * D + h * (D / 2));
+      store_acc_row<D / 2>(tDV + lane_off + h * (D / 2), 1.f, p.dv + row * D + h * (D / 2));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// dq = bf16(scale * dQ accumulator), four elements per thread per step;
+// HBM-bound (reads 4 B, writes 2 B per element).
+__global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const float4* __restrict__ acc,
+                                                             uint2* __restrict__ dq, float scale, int64_t n4) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
+    const float4 a = acc[i];
+    dq[i] = make_uint2(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale));
+  }
+}
+
+// ===========================================================================
 // dQ: query tile stationary
 // ===========================================================================
 template <int D>
@@ -441,7 +780,7 @@ struct QLayout {
   static constexpr int kBytes = kAbort + 4;
   static constexpr int kAlloc = kBytes + 1024;
 };
-static_assert(QLayout<128>::kAlloc <= 232448, "dQ tile set exceeds shared memory");
+static_assert(QLayout<128>::kAlloc <= kMaxDynSmem, "dQ tile set exceeds shared memory");
 
 // Warp roles: warp 0 TMA producer (K, V per step), warp 1 MMA issuer,
 // warp 2 TMEM allocator, warps 4-7 and 8-11 one thread per query row each,
@@ -677,12 +1016,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// D_i = dO_i . O_i and lse_i * log2(e); one warp per row; HBM-bound.
+// D_i = dO_i . O_i and lse_i * log2(e); with dqacc, also zeroes row i of
+// the fp32 dQ accumulator.  One warp per row; HBM-bound.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ out,
                                                              const __nv_bfloat16* __restrict__ dout,
                                                              const float* __restrict__ lse, float* __restrict__ dvec,
-                                                             float* __restrict__ lse2, int64_t rows) {
+                                                             float* __restrict__ lse2, float* __restrict__ dqacc,
+                                                             int64_t rows) {
   constexpr int E = D / 32;  // elements per lane (2 or 4)
   const int lane = threadIdx.x & 31;
   const int64_t w0 = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -713,6 +1054,11 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16
       dvec[row] = acc;
       lse2[row] = lse[row] * kLog2e;
     }
+    if (dqacc) {
+      float4* z = reinterpret_cast<float4*>(dqacc + row * D);
+#pragma unroll
+      for (int c = lane; c < D / 4; c += 32) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
 }
 
@@ -723,23 +1069,50 @@ int sm_count() {
 }
 
 template <int D>
+int launch_passes(const AttnArgs& a, const void* dout, void* dq, void* dk, void* dv, const float* dvec,
+                  const float* lse2, float* dqacc, int phase_mask, cudaStream_t stream);
+
+template <int D>
 int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* dout, void* dq, void* dk, void* dv,
-             void* workspace, int phase_mask, cudaStream_t stream) {
+             void* workspace, size_t workspace_bytes, int phase_mask, cudaStream_t stream) {
   const int64_t rows = a.B * a.H * a.N;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const size_t vec_bytes = ((size_t)rows * 4 + 255) & ~(size_t)255;
   float* dvec = reinterpret_cast<float*>(ws);
   float* lse2 = reinterpret_cast<float*>(ws + vec_bytes);
+  // the fused pass's fp32 dQ accumulator follows the two row vectors
+  float* dqacc = (bwd_fused_supported(D) && workspace_bytes >= bwd_workspace_bytes(a.B, a.H, a.N, D, true))
+                     ? reinterpret_cast<float*>(ws + 2 * vec_bytes)
+                     : nullptr;
+  if ((phase_mask & (kPhaseFused | kPhaseConvert)) && !dqacc) return RA_ERR_WORKSPACE;
 
-  if (phase_mask & 1) {
+  if (phase_mask & kPhasePre) {
     const int64_t want = (rows + 7) / 8;
     const int64_t cap = (int64_t)sm_count() * 16;
     const unsigned grid = (unsigned)(want < cap ? want : cap);
     bwd_preprocess_kernel<D><<<grid, 256, 0, stream>>>((const __nv_bfloat16*)out, (const __nv_bfloat16*)dout, lse,
-                                                       dvec, lse2, rows);
+                                                       dvec, lse2, dqacc, rows);
     if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
   }
-  if ((phase_mask & 6) == 0) return RA_OK;
+  if (phase_mask & (kPhaseKV | kPhaseQ | kPhaseFused)) {
+    const int rc = launch_passes<D>(a, dout, dq, dk, dv, dvec, lse2, dqacc, phase_mask, stream);
+    if (rc != RA_OK) return rc;
+  }
+  if (phase_mask & kPhaseConvert) {
+    const int64_t n4 = rows * D / 4;
+    const int64_t want = (n4 + 255) / 256, cap = (int64_t)sm_count() * 8;
+    bwd_dq_convert_kernel<<<(unsigned)(want < cap ? want : cap), 256, 0, stream>>>(
+        reinterpret_cast<const float4*>(dqacc), reinterpret_cast<uint2*>(dq), a.scale, n4);
+    if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
+  }
+  return RA_OK;
+}
+
+// The tensor-core passes selected by phase_mask (kPhaseKV, kPhaseQ, kPhaseFused).
+template <int D>
+int launch_passes(const AttnArgs& a, const void* dout, void* dq, void* dk, void* dv, const float* dvec,
+                  const float* lse2, float* dqacc, int phase_mask, cudaStream_t stream) {
+  const int64_t rows = a.B * a.H * a.N;
 
   alignas(64) CUtensorMap tq, tk, tv, tdo;
   const int64_t kv_rows = a.B * a.Hkv * a.N;
@@ -768,7 +1141,8 @@ int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* d
   p.scale_log2 = a.scale * kLog2e;
   int rc = current_status(&p.st);
   if (rc != RA_OK) return rc;
-  if (phase_mask & 2) {
+  p.dqacc = dqacc;
+  if (phase_mask & kPhaseKV) {
     // per key/value head: K, V and its query heads' Q, dO stream through L2
     p.group = head_group(p.num_tiles, p.BHkv, (double)a.N * D * 2 * (2 + 2 * p.G), 100.0e6);
     auto kern = bwd_kv_kernel<D>;
@@ -776,7 +1150,7 @@ int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* d
     kern<<<(unsigned)(p.BHkv * p.num_tiles), kThreads, KVLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
     if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
   }
-  if (phase_mask & 4) {
+  if (phase_mask & kPhaseQ) {
     // per query head: Q, dO, K, V (bf16) stream through L2
     p.group = head_group(p.num_tiles, p.BH, (double)a.N * D * 4 * 2, 100.0e6);
     auto kern = bwd_q_kernel<D>;
@@ -784,15 +1158,50 @@ int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* d
     kern<<<(unsigned)(p.BH * p.num_tiles), kThreads, QLayout<D>::kAlloc, stream>>>(tk, tv, p);
     if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
   }
+  if (phase_mask & kPhaseFused) {
+    if constexpr (D == 128) {
+      // per key/value head: K, V, its query heads' Q, dO (bf16) and their
+      // fp32 dQ accumulator rows stay in L2 while the head group is in flight
+      p.group = head_group(p.num_tiles, p.BHkv, (double)a.N * D * (2.0 * (2 + 2 * p.G) + 4.0 * p.G), 100.0e6);
+      p.smem_alloc = FusedLayout<D>::kAlloc;
+      auto kern = bwd_fused_kernel<D>;
+      if (set_smem_attr((const void*)kern, FusedLayout<D>::kAlloc) != RA_OK) return RA_ERR_CUDA;
+      kern<<<(unsigned)(p.BHkv * p.num_tiles), kThreads, FusedLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
+      if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
+    } else {
+      return RA_ERR_UNSUPPORTED;
+    }
+  }
   return RA_OK;
 }
 
 }  // namespace
 
+bool bwd_fused_supported(int64_t D) { return D == 128; }
+
+size_t bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t D, bool fused) {
+  if (B <= 0 || H <= 0 || N <= 0 || D <= 0) return 0;
+  const size_t rows = (size_t)B * H * N;
+  const size_t vec = (rows * 4 + 255) & ~(size_t)255;
+  return 2 * vec + (fused ? rows * (size_t)D * 4 : 0);
+}
+
+int bwd_default_phases(int64_t D) {
+  return bwd_fused_supported(D) ? (kPhasePre | kPhaseFused | kPhaseConvert) : (kPhasePre | kPhaseKV | kPhaseQ);
+}
+
+const char* bwd_tc_kernel_names(int64_t D) {
+  if (D != 64 && D != 128) return nullptr;
+  return bwd_fused_supported(D) ? "bwd_preprocess_kernel+bwd_fused_kernel+bwd_dq_convert_kernel"
+                                : "bwd_preprocess_kernel+bwd_kv_kernel+bwd_q_kernel";
+}
+
 int launch_bwd_tc(const AttnArgs& a, const void* out, const float* lse, const void* dout, void* dq, void* dk,
-                  void* dv, void* workspace, int phase_mask, cudaStream_t stream) {
-  if (a.D == 64) return launch_d<64>(a, out, lse, dout, dq, dk, dv, workspace, phase_mask, stream);
-  if (a.D == 128) return launch_d<128>(a, out, lse, dout, dq, dk, dv, workspace, phase_mask, stream);
+                  void* dv, void* workspace, size_t workspace_bytes, int phase_mask, cudaStream_t stream) {
+  if (a.D == 64)
+    return launch_d<64>(a, out, lse, dout, dq, dk, dv, workspace, workspace_bytes, phase_mask, stream);
+  if (a.D == 128)
+    return launch_d<128>(a, out, lse, dout, dq, dk, dv, workspace, workspace_bytes, phase_mask, stream);
   return RA_ERR_UNSUPPORTED;
 }
 

@@ -184,6 +184,11 @@ __device__ __forceinline__ void red_add_v4(float* gptr, float a, float b, float 
                : "memory");
 }
 
+// Scalar fp32 reduction into global memory (performed at L2; no return value).
+__device__ __forceinline__ void red_add_f32(float* gptr, float a) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(gptr), "f"(a) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // tcgen05: tensor memory and the 5th-generation tensor core
 // ---------------------------------------------------------------------------

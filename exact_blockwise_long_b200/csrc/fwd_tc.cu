@@ -32,6 +32,8 @@
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O [256, 256+D).
 #include <math.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -475,7 +477,7 @@ constexpr int kThreads2 = 384;
 // the softmax warpgroups rise to kSoftmaxRegs, the producer/MMA warpgroup
 // drops to kOtherRegs: 256 x 208 + 128 x 88 = 64512.  Per sub-partition:
 // 2 x 32 x 208 + 32 x 88 = 16128 of 16384.  The host launches this kernel
-// only when the compiled register count equals kLaunchRegs.
+// only when the compiled register count equals kLaunchRegs (tc2_usable).
 constexpr int kLaunchRegs = 168;
 constexpr uint32_t kSoftmaxRegs = 208;
 constexpr uint32_t kOtherRegs = 88;
@@ -730,6 +732,28 @@ __global__ void __launch_bounds__(kThreads2, 1)
   }
 }
 
+// Whether fwd_tc2_kernel<D> may run on the current device: its register
+// split (setmaxnreg) is sized for exactly kLaunchRegs registers per thread at
+// launch, so a build that compiled it to another count must not launch it
+// (a split larger than the launch's registers would wait forever).  Decided
+// once per device and cached; ringattn_kernel_plan reports the outcome.
+template <int D>
+bool tc2_usable() {
+  constexpr int kMaxDev = 64;
+  static std::mutex mu;
+  static signed char known[kMaxDev] = {};  // 0 unknown, 1 usable, -1 not
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return false;
+  std::lock_guard<std::mutex> lk(mu);
+  if (known[dev] == 0) {
+    cudaFuncAttributes fa;
+    const bool ok = cudaFuncGetAttributes(&fa, (const void*)fwd_tc2_kernel<D>) == cudaSuccess &&
+                    fa.numRegs == kLaunchRegs;
+    known[dev] = ok ? 1 : -1;
+  }
+  return known[dev] > 0;
+}
+
 template <int D>
 int launch_d(const AttnArgs& a, void* out, float* lse, float* o_acc, float* lse_acc, int step,
              cudaStream_t stream) {
@@ -756,12 +780,7 @@ int launch_d(const AttnArgs& a, void* out, float* lse, float* o_acc, float* lse_
   p.scale_log2 = a.scale * 1.4426950408889634f;
   int rc = current_status(&p.st);
   if (rc != RA_OK) return rc;
-  bool two_tiles = (p.L % (2 * kBM) == 0);
-  if (two_tiles) {
-    cudaFuncAttributes fa;
-    two_tiles = cudaFuncGetAttributes(&fa, (const void*)fwd_tc2_kernel<D>) == cudaSuccess &&
-                fa.numRegs == kLaunchRegs;
-  }
+  const bool two_tiles = (p.L % (2 * kBM) == 0) && tc2_usable<D>();
   // per head the key/value tiles every query tile streams through
   p.group = head_group(two_tiles ? p.num_qtiles / 2 : p.num_qtiles, p.BH, 2.0 * a.N * D * 2, 60.0e6);
   if (two_tiles) {
@@ -779,6 +798,13 @@ int launch_d(const AttnArgs& a, void* out, float* lse, float* o_acc, float* lse_
 }
 
 }  // namespace
+
+const char* fwd_tc_kernel_name(int64_t L, int64_t D) {
+  const bool pair = L % (2 * kBM) == 0;
+  if (D == 64) return pair && tc2_usable<64>() ? "fwd_tc2_kernel" : "fwd_tc_kernel";
+  if (D == 128) return pair && tc2_usable<128>() ? "fwd_tc2_kernel" : "fwd_tc_kernel";
+  return nullptr;
+}
 
 int launch_fwd_tc(const AttnArgs& a, void* out, float* lse, float* o_acc, float* lse_acc, int step,
                   cudaStream_t stream) {

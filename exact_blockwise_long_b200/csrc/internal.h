@@ -36,13 +36,46 @@ int launch_fwd_simt(const AttnArgs& a, void* out, float* lse, float* o_acc, floa
 int launch_fwd_tc(const AttnArgs& a, void* out, float* lse, float* o_acc, float* lse_acc, int step,
                   cudaStream_t stream);
 
+// Name of the forward kernel launch_fwd_tc runs for shard length L and
+// head dimension D on the current device (nullptr for an unsupported D).
+const char* fwd_tc_kernel_name(int64_t L, int64_t D);
+
+// Names of the kernels the default backward (ringattn_bwd) launches for
+// head dimension D, joined by '+' (nullptr for an unsupported D).
+const char* bwd_tc_kernel_names(int64_t D);
+
 int launch_merge(float* o_a, float* lse_a, const float* o_b, const float* lse_b, int64_t rows, int64_t D,
                  cudaStream_t stream);
 
-// Backward: preprocess, KV-stationary tcgen05 main loop, dQ conversion.
-// phase_mask: bit 0 preprocess, bit 1 main loop, bit 2 dQ conversion.
+// Backward phases (bits of phase_mask):
+//   kPhasePre      D_i, lse_i*log2e into the workspace; zeroes the fp32 dQ
+//                  accumulator when the workspace holds one
+//   kPhaseKV       key/value-stationary pass writing dk, dv    } deterministic
+//   kPhaseQ        query-stationary pass writing dq            } split backward
+//   kPhaseFused    one key/value-stationary pass writing dk, dv and adding
+//                  dQ into the fp32 accumulator (D = 128)
+//   kPhaseConvert  dq = bf16(scale * accumulator)
+enum BwdPhase { kPhasePre = 1, kPhaseKV = 2, kPhaseQ = 4, kPhaseFused = 8, kPhaseConvert = 16, kPhaseAll = 31 };
+bool bwd_fused_supported(int64_t D);
+// Workspace bytes: two fp32 row vectors [B*H*N], each 256-byte aligned, then
+// (fused) the fp32 dQ accumulator [B*H*N, D].
+size_t bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t D, bool fused);
+// Phases of the default backward for head dimension D.
+int bwd_default_phases(int64_t D);
 int launch_bwd_tc(const AttnArgs& a, const void* out, const float* lse, const void* dout, void* dq, void* dk,
-                  void* dv, void* workspace, int phase_mask, cudaStream_t stream);
+                  void* dv, void* workspace, size_t workspace_bytes, int phase_mask, cudaStream_t stream);
+
+// Argument checks of the backward entry points (abi.cu), everything but the
+// workspace: RA_OK, kBwdEmpty (a valid empty problem: nothing to launch) or
+// a negative ra_status.  run_bwd launches the phases after the checks.
+constexpr int kBwdEmpty = 1;
+int check_bwd_args(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+                   const void* dq, const void* dk, const void* dv, int64_t B, int64_t H, int64_t Hkv, int64_t N,
+                   int64_t D, int dtype, int S, int q_chunk, int k_chunk, int causal, int phase_mask);
+int run_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+            void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t D, int S,
+            int q_chunk, int k_chunk, int causal, float scale, void* workspace, size_t workspace_bytes,
+            int phase_mask, void* stream);
 
 // Blockwise SwiGLU FFN on the tensor cores.
 // residual: optional bf16 [T, d_model] added to y before its rounding.

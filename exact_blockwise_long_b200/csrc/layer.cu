@@ -120,8 +120,7 @@ int mark(void* const* marks, int i, cudaStream_t st) {
 
 size_t bwd_ws_bytes(int64_t B, int64_t N, int64_t H, int64_t D, int64_t d_ff, int64_t ffn_chunk) {
   const size_t T = (size_t)B * N, dm = (size_t)(H * D), act = T * dm * 2;
-  size_t attn = (size_t)B * H * N * 4;
-  attn = 2 * up256(attn);
+  const size_t attn = bwd_workspace_bytes(B, H, N, D, bwd_fused_supported(D));
   return 7 * up256(act) + up256(attn) + up256(ffn_bwd_workspace_bytes(ffn_chunk, d_ff)) +
          up256(rmsnorm_dg_partial_floats((int64_t)T, (int64_t)dm) * 4);
 }
@@ -231,12 +230,13 @@ int blockwise_layer_bwd(const void* x, const void* g_attn, const void* wq, const
   auto* dk = c.take<__nv_bfloat16>(act);
   auto* dv = c.take<__nv_bfloat16>(act);
   auto* dxn = c.take<__nv_bfloat16>(act);
-  void* ws_attn = c.take<uint8_t>(2 * up256((size_t)B * H * N * 4));
+  const size_t ws_attn_bytes = bwd_workspace_bytes(B, H, N, D, bwd_fused_supported(D));
+  void* ws_attn = c.take<uint8_t>(ws_attn_bytes);
   void* ws_ffn = c.take<uint8_t>(ffn_bwd_workspace_bytes(ffn_chunk, d_ff));
   float* partial = c.take<float>(rmsnorm_dg_partial_floats(T, dm) * 4);
 
-  // steps (marks): 0 feed-forward, 1 norm, 2 dO, 3 dWo, 4-6 attention (preprocess, dK/dV pass, dQ pass),
-  // 7 dxn, 8 dWq/dWk/dWv, 9 norm
+  // steps (marks): 0 feed-forward, 1 norm, 2 dO, 3 dWo, 4-6 attention (preprocess; main pass or passes;
+  // dQ conversion or the query-stationary pass), 7 dxn, 8 dWq/dWk/dWv, 9 norm
   // feed-forward half: y = x2 + ffn(xn2)
   if ((rc = launch_ffn_bwd_tc(s.xn2, w1, w2, w3, dy, dxn2, dw1, dw2, dw3, T, dm, d_ff, ffn_chunk, ws_ffn, st)) !=
       RA_OK)
@@ -256,9 +256,15 @@ int blockwise_layer_bwd(const void* x, const void* g_attn, const void* wq, const
   }
   if ((rc = mark(marks, 3, st)) != RA_OK) return rc;
   AttnArgs a{s.q, s.k, s.v, B, H, N, D, RA_BF16, S, q_chunk, k_chunk, causal, 1.0f / sqrtf((float)D), H};
-  for (int ph = 0; ph < 3; ++ph) {
-    if ((rc = launch_bwd_tc(a, s.o, s.lse, dO, dq, dk, dv, ws_attn, 1 << ph, st)) != RA_OK) return rc;
-    if ((rc = mark(marks, 4 + ph, st)) != RA_OK) return rc;
+  {
+    // the default backward's phases, one mark after each
+    const int all = bwd_default_phases(D);
+    const int phases[3] = {kPhasePre, all & (kPhaseKV | kPhaseFused), all & (kPhaseQ | kPhaseConvert)};
+    for (int i = 0; i < 3; ++i) {
+      if ((rc = launch_bwd_tc(a, s.o, s.lse, dO, dq, dk, dv, ws_attn, ws_attn_bytes, phases[i], st)) != RA_OK)
+        return rc;
+      if ((rc = mark(marks, 4 + i, st)) != RA_OK) return rc;
+    }
   }
   {
     // dxn = dq Wq + dk Wk + dv Wv (one accumulation over three K ranges)

@@ -80,6 +80,9 @@ __global__ void __launch_bounds__(kWarps * 32) merge_kernel(float* __restrict__ 
                              (wa != 0.f ? wa * x1.w : 0.f) + (wb != 0.f ? wb * y1.w : 0.f));
       }
     }
+    // every lane has read lse_a of both rows (top of this iteration) before
+    // lane 0 overwrites them
+    __syncwarp();
     if (lane == 0) {
       float wa, wb, l;
       merge_weights(la0, lb0, wa, wb, l);

@@ -9,10 +9,12 @@
 // their hot path because cudaMalloc can synchronise the device and stall
 // other streams.  Such callers cannot hand ringattn_bwd its workspace.
 //
-// The backward's scratch (fp32 dQ accumulator plus the two fp32 row
-// vectors) lives instead in one file-scope device array of fixed size,
-// kNoallocScratchBytes.  Every GPU that loads this part of the library
-// keeps that array until the process exits.
+// It runs the deterministic two-pass backward (the key/value-stationary and
+// query-stationary passes), whose only scratch is two fp32 row vectors
+// [B*H*N] -- D_i = dO_i . O_i and lse_i * log2(e) -- rather than the fused
+// pass's fp32 dQ accumulator.  Those vectors live in one file-scope device
+// array of fixed size, kNoallocScratchBytes.  Every GPU that loads this
+// library keeps that array until the process exits.
 #include <mutex>
 
 #include "common.cuh"
@@ -55,20 +57,21 @@ int ringattn_bwd_noalloc(const void* q, const void* k, const void* v, const void
                          const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N,
                          int64_t D, int dtype, int S, int q_chunk, int k_chunk, int causal, float scale,
                          void* stream) {
-  const size_t need = ringattn_bwd_workspace_size(B, H, N, D);
-  if (need > ra::kNoallocScratchBytes) return RA_ERR_WORKSPACE;  // larger than the static scratch
-  if (need == 0) {
-    // empty or invalid extents: the regular entry point validates and answers
-    return ringattn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, H, N, D, dtype, S, q_chunk, k_chunk, causal,
-                        scale, nullptr, 0, stream);
-  }
-  void* scratch = nullptr;
-  const int rc = ra::scratch_address(&scratch);
+  constexpr int kPhases = ra::kPhasePre | ra::kPhaseKV | ra::kPhaseQ;
+  // the same argument checks, in the same order, as the workspace entry points
+  const int rc = ra::check_bwd_args(q, k, v, out, lse, dout, dq, dk, dv, B, H, H, N, D, dtype, S, q_chunk, k_chunk,
+                                    causal, kPhases);
+  if (rc == ra::kBwdEmpty) return RA_OK;
   if (rc != RA_OK) return rc;
-  // The preprocess phase clears the dQ accumulator and overwrites both row
-  // vectors, so nothing left in the array by an earlier call leaks in.
-  return ringattn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, H, N, D, dtype, S, q_chunk, k_chunk, causal, scale,
-                      scratch, ra::kNoallocScratchBytes, stream);
+  const size_t need = ra::bwd_workspace_bytes(B, H, N, D, false);
+  if (need > ra::kNoallocScratchBytes) return RA_ERR_WORKSPACE;  // larger than the static scratch
+  void* scratch = nullptr;
+  const int rs = ra::scratch_address(&scratch);
+  if (rs != RA_OK) return rs;
+  // The preprocess phase overwrites both row vectors in full before the two
+  // passes read them, so nothing an earlier call left in the array leaks in.
+  return ra::run_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, H, H, N, D, S, q_chunk, k_chunk, causal, scale,
+                     scratch, need, kPhases, stream);
 }
 
 }  // extern "C"

@@ -25,7 +25,9 @@
  * Conventions common to every call
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library
  *    never frees or retains them.  The library allocates nothing per call.
- *    Its only persistent device state is one status word per device.
+ *    Its persistent device state, on every device that loads it, is one
+ *    status word and the RINGATTN_NOALLOC_SCRATCH_BYTES array of
+ *    ringattn_bwd_noalloc (held whether or not that call is used).
  *  - Attention tensors are contiguous [B, H, N, D] (D innermost).  LSE and
  *    the backward's D-vector are contiguous fp32 [B, H, N].  Pointers must be
  *    16-byte aligned.
@@ -73,6 +75,22 @@ RA_API int ringattn_version(void);
 
 /* Human-readable text for an ra_status value (static storage). */
 RA_API const char* ringattn_status_string(int status);
+
+/*
+ * ringattn_kernel_plan -- names of the kernels a call would launch on the
+ * current device for a problem of N tokens in S shards with head dimension
+ * D and `dtype` (static strings, several names joined by '+'):
+ *   op 0: ringattn_fwd / ringattn_fwd_gqa, e.g. "fwd_tc2_kernel" (two
+ *         128-row query tiles per CTA, used when the shard length is a
+ *         multiple of 256 and this build's register split is usable on the
+ *         device), "fwd_tc_kernel" or "fwd_simt_kernel" (RA_F32);
+ *   op 1: ringattn_bwd / ringattn_bwd_gqa, e.g.
+ *         "bwd_preprocess_kernel+bwd_fused_kernel+bwd_dq_convert_kernel".
+ * NULL for an unknown op, a shape that breaks N % S, or an unsupported D or
+ * dtype.  Lets a caller (or a benchmark) name what actually runs; the choice
+ * is made once per device and does not change between calls.
+ */
+RA_API const char* ringattn_kernel_plan(int op, int64_t N, int64_t D, int dtype, int S);
 
 /*
  * ringattn_fwd -- exact ring blockwise attention forward.
@@ -150,7 +168,9 @@ RA_API int ringattn_merge(float* o_a, float* lse_a, const float* o_b, const floa
 
 /* Bytes of device workspace ringattn_bwd needs: two fp32 row vectors
  * [B,H,N] (D_i = dO_i . O_i and lse_i * log2(e)), each region 256-byte
- * aligned.  0 for empty problems. */
+ * aligned, followed for D = 128 by the fused pass's fp32 dQ accumulator
+ * [B,H,N,D].  Enough for every phase mask of ringattn_bwd_phase.  0 for
+ * empty problems. */
 RA_API size_t ringattn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D);
 
 /*
@@ -160,11 +180,16 @@ RA_API size_t ringattn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64
  *   dv_j = sum_i P_ij dout_i
  *   dS_ij = P_ij (dout_i . v_j - D_i)
  *   dq_i = scale sum_j dS_ij k_j ;  dk_j = scale sum_i dS_ij q_i
- * dK and dV keep each key/value tile stationary while the query shards
- * pass by in ring order i = (j + t) mod S; dQ keeps each query tile
- * stationary and visits the KV shards in ring order j = (i - t) mod S
- * (causal: pairs in the future skipped).  Every gradient accumulates on chip
- * and is written once: no atomics, bit-reproducible.
+ * Each key/value tile stays on chip while the query shards pass by in ring
+ * order i = (j + t) mod S (causal: pairs in the future skipped, the
+ * diagonal pair masked).  dK and dV accumulate on chip and are written once.
+ * D = 128: the same pass forms dQ's share of each tile pair and adds it
+ * into an fp32 accumulator in the workspace; the sum over key tiles runs in
+ * the order the CTAs reach memory, so dq is reproducible up to that fp32
+ * summation order (dk, dv are bit-reproducible).  D = 64, or
+ * ringattn_bwd_phase with mask 7 for any D: the deterministic split
+ * backward (a second, query-stationary pass recomputes S and dP per tile
+ * pair and writes dq once; every output bit-reproducible).
  *
  *   q,k,v,out,dout [B,H,N,D] of `dtype` (out and lse from ringattn_fwd)
  *   lse            [B,H,N] fp32
@@ -172,7 +197,10 @@ RA_API size_t ringattn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64
  *   workspace      device buffer of ringattn_bwd_workspace_size() bytes,
  *                  16-byte aligned; its contents on entry do not matter
  * Only RA_BF16 is implemented (RA_F32 returns RA_ERR_UNSUPPORTED).
- * Chunk rules as for ringattn_fwd with RA_BF16.
+ * Chunk rules as for ringattn_fwd with RA_BF16.  If a device cannot place
+ * the fused pass's shared-memory tile set, the pass latches
+ * RA_ERR_UNSUPPORTED in the status word (ringattn_get_error) and writes
+ * nothing.
  */
 RA_API int ringattn_bwd(const void* q, const void* k, const void* v, const void* out,
                  const float* lse, const void* dout,
@@ -195,14 +223,24 @@ RA_API int ringattn_bwd_gqa(const void* q, const void* k, const void* v, const v
                             void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * ringattn_bwd_phase -- ringattn_bwd split into its three launches, for
- * callers that schedule or time them separately.  phase_mask (1..7) selects
- * bit 0: preprocess (D_i and lse_i*log2(e) into workspace), bit 1: the
- * key/value-stationary tensor-core loop (writes dk, dv), bit 2: the
- * query-stationary tensor-core loop (writes dq).  Bits 1 and 2 read what bit
- * 0 wrote into the same workspace and are independent of each other; mask 7
- * is ringattn_bwd.  Arguments and errors as ringattn_bwd, plus RA_ERR_ARG
- * for a mask outside 1..7.
+ * ringattn_bwd_phase -- the backward's launches, selected by phase_mask
+ * (1..31), for callers that schedule or time them separately:
+ *   bit 0 (1)   preprocess: D_i and lse_i*log2(e) into the workspace; when
+ *               the workspace is ringattn_bwd_workspace_size() bytes (D =
+ *               128) it also zeroes the fp32 dQ accumulator
+ *   bit 1 (2)   key/value-stationary pass writing dk, dv     } the split,
+ *   bit 2 (4)   query-stationary pass writing dq             } deterministic
+ *                                                              backward
+ *   bit 3 (8)   fused pass (D = 128): dk, dv written, dQ added into the
+ *               accumulator
+ *   bit 4 (16)  dq = bf16(scale * accumulator) (D = 128)
+ * Later bits read what bit 0 wrote into the same workspace; bit 4 reads what
+ * bit 3 added.  Mask 7 is the deterministic backward, which needs only the
+ * two row vectors (2 x round_up(B*H*N*4, 256) bytes); masks with bit 3 or 4
+ * need the full ringattn_bwd_workspace_size().  ringattn_bwd runs mask 25
+ * (1 + 8 + 16) for D = 128 and mask 7 for D = 64.  Arguments and errors as
+ * ringattn_bwd, plus RA_ERR_ARG for a mask outside 1..31 and
+ * RA_ERR_UNSUPPORTED for bits 3-4 with D = 64.
  */
 RA_API int ringattn_bwd_phase(const void* q, const void* k, const void* v, const void* out,
                               const float* lse, const void* dout,
@@ -213,23 +251,26 @@ RA_API int ringattn_bwd_phase(const void* q, const void* k, const void* v, const
                               void* stream);
 
 /*
- * ringattn_bwd_noalloc -- ringattn_bwd that allocates nothing and takes no
- * workspace.  The paper has no counterpart; it serves callers that cannot
+ * ringattn_bwd_noalloc -- the backward without a workspace and without any
+ * allocation.  The paper has no counterpart; it serves callers that cannot
  * allocate device memory when they run the backward (an allocator owned by
  * another framework, a device-memory budget fixed at start-up, or a hot
  * path where a cudaMalloc that may synchronise the device is not allowed).
  *
- * The scratch ringattn_bwd would take from `workspace` comes from one
- * static device array of RINGATTN_NOALLOC_SCRATCH_BYTES (64 MiB) that every
- * GPU which loads this library keeps until the process exits.  Problems
- * whose ringattn_bwd_workspace_size() exceeds it return RA_ERR_WORKSPACE
- * (B*H*N up to about 8.3 million rows, e.g. H=32, N=262144).
+ * It runs the deterministic split backward (ringattn_bwd_phase, mask 7) and
+ * gives its bits.  That backward's scratch -- two fp32 row vectors [B,H,N]
+ * -- comes from one static device array of RINGATTN_NOALLOC_SCRATCH_BYTES
+ * (64 MiB) that every GPU which loads this library keeps until the process
+ * exits.  Arguments are checked first, exactly as by ringattn_bwd, with the
+ * same errors; then a problem whose two row vectors exceed the array
+ * returns RA_ERR_WORKSPACE (B*H*N up to about 8.3 million rows, e.g. H=32,
+ * N=262144).
  * The first call on a device looks up the array's device address; make that
  * first call before any stream capture.  All calls share the one array and
- * it keeps the last call's contents (each call re-clears what must start at
- * zero), so calls that overlap on the GPU -- on different streams, or from
- * different host threads -- race and corrupt each other's gradients:
- * serialise them.  Arguments, results and other errors as ringattn_bwd.
+ * it keeps the last call's contents (each call overwrites both vectors in
+ * full before reading them), so calls that overlap on the GPU -- on
+ * different streams, or from different host threads -- race and corrupt
+ * each other's gradients: serialise them.
  */
 #define RINGATTN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 RA_API int ringattn_bwd_noalloc(const void* q, const void* k, const void* v, const void* out,
@@ -381,8 +422,9 @@ RA_API int blockwise_layer_bwd(const void* x, const void* g_attn, const void* wq
 
 /*
  * ringattn_get_error -- synchronise `stream`, return the device status word
- * of the current device (RA_OK or RA_ERR_TIMEOUT) and clear it.  Also
- * reports a pending CUDA error as RA_ERR_CUDA.
+ * of the current device (RA_OK, RA_ERR_TIMEOUT, or RA_ERR_UNSUPPORTED from
+ * a kernel that could not place its shared-memory tiles) and clear it.
+ * Also reports a pending CUDA error as RA_ERR_CUDA.
  */
 RA_API int ringattn_get_error(void* stream);
 

@@ -23,13 +23,20 @@ def _lib():
     torch.cuda.set_device(0)
 
 
-def run_bwd(q, k, v, do, S, qc, kc, causal):
+DETERMINISTIC = 7  # phase mask of the split (key/value- then query-stationary) backward
+
+
+def run_bwd(q, k, v, do, S, qc, kc, causal, phases=None):
+    """ringattn_bwd (phases None) or the phases of ringattn_bwd_phase."""
     import exact_blockwise_long_b200 as ra
     o, lse = run_fwd(q, k, v, S, qc, kc, causal)
     B, H, N, D = q.shape
     ws = torch.empty(ra.ringattn_bwd_workspace_size(B, H, N, D), device="cuda", dtype=torch.uint8)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ra.ringattn_bwd(q, k, v, o, lse, do, dq, dk, dv, S, qc, kc, causal, ws)
+    dq, dk, dv = (torch.full_like(x, float("nan")) for x in (q, k, v))
+    if phases is None:
+        ra.ringattn_bwd(q, k, v, o, lse, do, dq, dk, dv, S, qc, kc, causal, ws)
+    else:
+        ra.ringattn_bwd_phase(q, k, v, o, lse, do, dq, dk, dv, S, qc, kc, causal, ws, phases)
     assert ra.ringattn_get_error() == 0
     return dq, dk, dv
 
@@ -46,23 +53,71 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("phases", [None, DETERMINISTIC], ids=["default", "deterministic"])
 @pytest.mark.parametrize("B,H,N,D,S,qc,kc,causal", CASES)
-def test_bwd_full_oracle(B, H, N, D, S, qc, kc, causal):
+def test_bwd_full_oracle(B, H, N, D, S, qc, kc, causal, phases):
     q, k, v, do = small_attention_inputs(B, H, N, D, 100 + N + D + S, k_scale=2.0 if causal else 1.0)
-    dq, dk, dv = run_bwd(q, k, v, do, S, qc, kc, causal)
+    dq, dk, dv = run_bwd(q, k, v, do, S, qc, kc, causal, phases)
     gq, gk, gv = oracle.attention_backward(to_f64(q), to_f64(k), to_f64(v), to_f64(do), causal)
     errs = [max_abs(to_f64(a), b) for a, b in ((dq, gq), (dk, gk), (dv, gv))]
     assert max(errs) <= TOL_BF16_GRAD, errs
 
 
-def test_bwd_bit_reproducible():
-    """Every gradient accumulates on chip and is written once (no atomics):
-    repeated runs give identical bits."""
+def test_bwd_deterministic_bit_reproducible():
+    """The split backward accumulates every gradient on chip and writes it
+    once (no atomics): repeated runs give identical bits."""
     q, k, v, do = small_attention_inputs(1, 2, 1024, 128, 5)
-    a = run_bwd(q, k, v, do, 4, 128, 128, True)
+    a = run_bwd(q, k, v, do, 4, 128, 128, True, DETERMINISTIC)
     for _ in range(3):
-        b = run_bwd(q, k, v, do, 4, 128, 128, True)
+        b = run_bwd(q, k, v, do, 4, 128, 128, True, DETERMINISTIC)
         assert all(torch.equal(x, y) for x, y in zip(a, b))
+
+
+def _bf16_order_close(a, b):
+    """Equal up to the order of an fp32 sum before one bf16 rounding: at most
+    one bf16 step (2^-8 relative) apart, plus fp32 noise near zero."""
+    a, b = a.float(), b.float()
+    return bool(((a - b).abs() <= 2.0 ** -7 * torch.maximum(a.abs(), b.abs()) + 1e-5).all())
+
+
+@pytest.mark.parametrize("D,S,causal", [(128, 4, True), (128, 2, False)])
+def test_bwd_default_vs_deterministic(D, S, causal):
+    """The default backward sums dQ over key tiles with fp32 additions in
+    whatever order the CTAs reach memory; dK and dV are the same matmuls in
+    the same order as the split backward's, so they agree to the bit; dQ
+    agrees up to summation order, and repeats of the default agree likewise."""
+    import exact_blockwise_long_b200 as ra
+    q, k, v, do = small_attention_inputs(2, 2, 1024, D, 9 + S, k_scale=2.0)
+    B, H, N, _ = q.shape
+    plan = ra.lib().ringattn_kernel_plan(1, N, D, 0, S).decode()
+    assert "bwd_fused_kernel" in plan, plan
+    ref = run_bwd(q, k, v, do, S, 128, 256, causal, DETERMINISTIC)
+    for _ in range(3):
+        got = run_bwd(q, k, v, do, S, 128, 256, causal)
+        assert torch.equal(got[1], ref[1]) and torch.equal(got[2], ref[2])
+        assert _bf16_order_close(got[0], ref[0])
+
+
+def test_bwd_phase_masks():
+    """Phase masks run alone, in the order the default backward runs them,
+    give the default backward's dk, dv (bit for bit) and dq (up to order)."""
+    import exact_blockwise_long_b200 as ra
+    q, k, v, do = small_attention_inputs(1, 2, 1024, 128, 21, k_scale=2.0)
+    ref = run_bwd(q, k, v, do, 4, 128, 128, True)
+    o, lse = run_fwd(q, k, v, 4, 128, 128, True)
+    ws = torch.empty(ra.ringattn_bwd_workspace_size(1, 2, 1024, 128), device="cuda", dtype=torch.uint8)
+    dq, dk, dv = (torch.full_like(x, float("nan")) for x in (q, k, v))
+    for m in (1, 8, 16):
+        ra.ringattn_bwd_phase(q, k, v, o, lse, do, dq, dk, dv, 4, 128, 128, True, ws, m)
+    assert ra.ringattn_get_error() == 0
+    assert torch.equal(dk, ref[1]) and torch.equal(dv, ref[2]) and _bf16_order_close(dq, ref[0])
+    # the split passes need only the two row vectors at the head of the workspace
+    small = torch.empty(2 * 2 * 1024 * 4, device="cuda", dtype=torch.uint8)
+    with pytest.raises(ra.RingAttnError):
+        ra.ringattn_bwd_phase(q, k, v, o, lse, do, dq, dk, dv, 4, 128, 128, True, small, 25)
+    ra.ringattn_bwd_phase(q, k, v, o, lse, do, dq, dk, dv, 4, 128, 128, True, small, DETERMINISTIC)
+    assert ra.ringattn_get_error() == 0
+    assert torch.equal(dk, ref[1]) and torch.equal(dv, ref[2]) and _bf16_order_close(dq, ref[0])
 
 
 @pytest.mark.parametrize("name", ["n8k_d64_causal", "n8k_d64_full", "n32k_d128"])

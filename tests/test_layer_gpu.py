@@ -134,13 +134,22 @@ def test_layer_empty_batch():
     assert all(torch.count_nonzero(g) == 0 for g in grads)
 
 
-def test_layer_bit_reproducible():
-    """Every reduction is in a fixed order (TMA adds in stream order, split-K
-    adds onto zero, ordered dg sums): repeated runs give identical bits."""
+def test_layer_repeatable():
+    """The forward reduces in a fixed order: repeated runs give identical
+    bits.  The backward's attention sums dQ over key tiles with fp32
+    additions in arrival order, so dx and the parameter gradients of repeats
+    differ only by that order's rounding: far below the layer's tolerance
+    (relative Frobenius 2^-6), bounded here by 2^-10."""
     w = LayerWorkload("t", 1, 1024, 2, 128, 384, 4, 128, 128, 256, 71, w_std=256 ** -0.5)
     x, params, dy = layer_inputs(w)
     a = run_layer(w, x, params, dy)
+
+    def rel(p, q):
+        p, q = p.float(), q.float()
+        return float((p - q).norm() / q.norm().clamp_min(1e-30))
+
     for _ in range(3):
         b = run_layer(w, x, params, dy)
-        assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
-        assert all(torch.equal(p, q) for p, q in zip(a[2], b[2]))
+        assert torch.equal(a[0], b[0])
+        assert rel(b[1], a[1]) <= 2.0 ** -10
+        assert all(rel(p, q) <= 2.0 ** -10 for p, q in zip(b[2], a[2]))
