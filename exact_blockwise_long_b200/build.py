@@ -13,6 +13,7 @@ import argparse
 import concurrent.futures as cf
 import glob
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -53,13 +54,52 @@ def needs_build() -> bool:
     return any(os.path.getmtime(p) > t for p in _deps())
 
 
+# Kernels whose warp roles re-split the launch's registers (setmaxnreg): the
+# split is sized for this many registers per thread at launch, so a compile
+# that lands on another count is a build error (the library also refuses to
+# launch such a kernel at run time).
+LAUNCH_REGS = {"fwd_tc.cu": {"fwd_tc2_kernel": 168}, "bwd_tc.cu": {"bwd_fused_kernel": 128}}
+
+
+def kernel_registers(ptxas_log: str) -> dict:
+    """{mangled entry name: registers} from `ptxas -v` output."""
+    regs, cur = {}, None
+    for line in ptxas_log.splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            cur = m.group(1)
+            continue
+        m = re.search(r"Used (\d+) registers", line)
+        if m and cur:
+            regs[cur] = int(m.group(1))
+            cur = None
+    return regs
+
+
+def check_launch_registers(src: str, ptxas_log: str) -> None:
+    want = LAUNCH_REGS.get(os.path.basename(src), {})
+    regs = kernel_registers(ptxas_log)
+    for kernel, n in want.items():
+        found = {name: r for name, r in regs.items() if kernel in name}
+        if not found:
+            raise RuntimeError(f"{src}: ptxas reported no registers for {kernel}")
+        bad = {name: r for name, r in found.items() if r != n}
+        if bad:
+            raise RuntimeError(f"{src}: {kernel} compiled to {sorted(set(bad.values()))} registers per thread; "
+                               f"its register split needs exactly {n}")
+
+
 def _compile(src: str, extra) -> str:
     obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
-    cmd = [nvcc()] + FLAGS + list(extra) + ["-c", src, "-o", obj]
+    checked = os.path.basename(src) in LAUNCH_REGS
+    flags = list(extra) + (["-Xptxas", "-v"] if checked and "-v" not in extra else [])
+    cmd = [nvcc()] + FLAGS + flags + ["-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed on {src}:\n{r.stdout}\n{r.stderr}")
-    if r.stderr.strip():
+    if checked:
+        check_launch_registers(src, r.stdout + r.stderr)
+    if r.stderr.strip() and (not checked or "-v" in extra):
         sys.stderr.write(r.stderr)
     return obj
 

@@ -30,10 +30,15 @@
 //                 dQ  += dS K     (dS bf16 over dP, A operand from TMEM)
 #include <math.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace ra {
+
+bool fused_usable();  // below: the fused pass's register split fits this build on this device
+
 namespace {
 
 constexpr int kT = 128;        // rows per tile (TMEM lanes)
@@ -432,21 +437,51 @@ __global__ void __launch_bounds__(kThreads, 1)
 // The dK/dV loop above plus a fifth matmul per tile pair,
 //   dQ^T_n = K^T dS^T_n   (M = d, N = 128 queries, K = 128 keys),
 // whose 128 x 128 fp32 result is added into an fp32 dQ accumulator in HBM
-// (L2-resident for the head group in flight) by the element-wise warps.  It
-// replaces the query-stationary pass, which recomputes S and dP (two of its
-// three matmuls) to avoid those additions.  The sum over key tiles then runs
-// in whatever order the CTAs reach L2, so dQ is reproducible only up to fp32
+// (L2-resident for the head group in flight).  It replaces the
+// query-stationary pass, which recomputes S and dP (two of its three
+// matmuls) to avoid those additions.  The sum over key tiles runs in
+// whatever order the CTAs reach L2, so dQ is reproducible only up to fp32
 // summation order; dK and dV are still written once per key tile.
+//
+// The additions are this pass's limiter: an SM moves fp32 reductions to L2
+// at about 22 bytes per clock, whichever instruction carries them (scalar
+// or vector reductions, or bulk reductions from shared memory, measured
+// with all SMs busy), and each tile pair adds 64 KB -- about 3000 clocks,
+// more than the pair's 2560 clocks of matmuls.  So a warpgroup of its own
+// (the drain warps) keeps that path busy without pause, and the element-wise
+// warps never wait on it.
 //
 // Both operands of dQ^T come from shared memory: K (stationary, read as an
 // MN-major A operand) and dS^T (MN-major B), which the element-wise warps
-// write beside their TMEM copy.  Tensor memory holds S^T [0,128),
-// dP^T [128,256), dK [256,384), dV [384,512): dQ^T has no columns of its own
-// and lands in the dP^T columns after dK has read dS^T from them; the next
-// dP^T is issued once the element-wise warps have loaded dQ^T out.
-// MMA order per step n: dV_n (two halves), dP_n, S_{n+1}, dK_n, dQ^T_n.
-// Element-wise order per step n: P^T_n, then dQ^T_{n-1} drained (loaded,
-// released, its 64 columns per thread reduced into HBM), then dS^T_n.
+// write beside their TMEM copy (the A operand of dK).  Tensor memory holds
+// S^T [0,128), dP^T [128,256), dK [256,384), dV [384,512): dQ^T has no
+// columns of its own and lands in the dP^T columns after dK has read dS^T
+// from them.  The drain warps load all of it into registers and free the
+// columns at once (dP^T of the next tile goes there), then add it into HBM
+// while the next tile is computed: the additions stay off the chain
+// dP -> dS -> dK, dQ^T -> next dP that sets the step time.  (Reading dK's
+// dS^T from shared memory as well, so that dQ^T could go first, was slower:
+// 32 KB more shared-memory reads per tile pair.)
+//
+// Warp roles (512 threads): warps 0-3 drain dQ^T (TMEM lane = d index),
+// warps 4-11 element-wise (as in the dK/dV pass), warp 12 TMA producer,
+// warp 13 MMA issuer, warp 14 TMEM allocator.
+// MMA order per step n: dP_n and the two halves of dV_n in the order their
+// inputs become ready (dP_n first when both are), S_{n+1}, dK_n, dQ^T_n.
+constexpr int kThreadsF = 512;
+// Register split: launched at kLaunchRegsF per thread (512 x 128 = 65536);
+// the element-wise warpgroups rise to kEwRegsF and the drain warpgroup (128
+// dQ^T values per thread) to kDrainRegsF, the producer/MMA warpgroup drops
+// to kRoleRegsF: 256 x 144 + 128 x 144 + 128 x 80 = 65536.  The host
+// launches this kernel only when the compiled register count equals
+// kLaunchRegsF.
+constexpr int kLaunchRegsF = 128;
+constexpr uint32_t kEwRegsF = 144;
+constexpr uint32_t kDrainRegsF = 144;
+constexpr uint32_t kRoleRegsF = 80;
+static_assert(256 * kEwRegsF + 128 * kDrainRegsF + 128 * kRoleRegsF <= kThreadsF * kLaunchRegsF,
+              "register split exceeds launch");
+
 template <int D>
 struct FusedLayout {
   static constexpr int kTile = kT * D * 2;
@@ -470,7 +505,7 @@ struct FusedLayout {
 static_assert(FusedLayout<128>::kBytes <= kMaxDynSmem, "fused backward tile set exceeds shared memory");
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsF, 1)
     bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                      const BParams p) {
@@ -506,14 +541,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_kv = bars;
   uint64_t* bar_qf = bar_kv + 1;
   uint64_t* bar_qe = bar_qf + kSt;
-  uint64_t* bar_sf = bar_qe + kSt;   // S^T computed
-  uint64_t* bar_dpf = bar_sf + 1;    // dP^T computed
-  uint64_t* bar_ph = bar_dpf + 1;    // first half of P^T written to TMEM
-  uint64_t* bar_pr = bar_ph + 1;     // all of P^T written to TMEM
-  uint64_t* bar_dsr = bar_pr + 1;    // dS^T written to TMEM and shared memory
-  uint64_t* bar_dqf = bar_dsr + 1;   // dQ^T computed (in the dP^T columns)
-  uint64_t* bar_dqe = bar_dqf + 1;   // dQ^T loaded out: the dP^T columns are free
-  uint64_t* bar_done = bar_dqe + 1;  // dK, dV final
+  uint64_t* bar_sf = bar_qe + kSt;    // S^T computed
+  uint64_t* bar_dpf = bar_sf + 1;     // dP^T computed
+  uint64_t* bar_ph = bar_dpf + 1;     // first half of P^T written to TMEM
+  uint64_t* bar_pr = bar_ph + 1;      // all of P^T written to TMEM
+  uint64_t* bar_dsr = bar_pr + 1;     // dS^T written to TMEM and shared memory
+  uint64_t* bar_dqf = bar_dsr + 1;    // dQ^T computed (in the dP^T columns)
+  uint64_t* bar_dqe = bar_dqf + 1;    // dQ^T loaded out of the dP^T columns: free again
+  uint64_t* bar_done = bar_dqe + 1;   // dK, dV final
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + LY::kTmemSlot);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LY::kAbort);
 
@@ -529,12 +564,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_pr, 2 * 128);
     mbar_init(bar_dsr, 2 * 128);
     mbar_init(bar_dqf, 1);
-    mbar_init(bar_dqe, 2 * 128);
+    mbar_init(bar_dqe, 128);
     mbar_init(bar_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 2) {
+  if (warp == 14) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -544,8 +579,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem, tDP = tmem + 128, tDK = tmem + 256, tDV = tmem + 384;
 
-  if (warp == 0) {
-    if (lane == 0) {
+  if (warp >= 12) {
+    regs_dec<kRoleRegsF>();
+    if (warp == 12 && lane == 0) {
+      // ---------------- TMA producer ----------------
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
@@ -566,9 +603,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++n;
         return true;
       });
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
+    } else if (warp == 13 && lane == 0) {
+      // ---------------- MMA issuer ----------------
       constexpr uint32_t idSS = idesc_bf16_f32(kT, kT, false, false);  // K-major x K-major
       constexpr uint32_t idTS = idesc_bf16_f32(kT, D, false, true);    // TMEM A x MN-major B
       constexpr uint32_t idDQ = idesc_bf16_f32(D, kT, true, true);     // MN-major K^T x MN-major dS^T
@@ -593,29 +629,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int n = 0; ok && n < n_total; ++n) {
         const int st = n % kSt;
         const uint32_t qb = q_base + st * LY::kTile, dob = do_base + st * LY::kTile;
-        // dV += P^T dO in two halves as the element-wise warps publish them
+        // dP^T = V dO^T (into the dP^T columns once the drain warps have loaded
+        // dQ^T_{n-1} out of them) and dV += P^T dO in two halves (as the
+        // element-wise warps publish P^T), each as soon as its input is ready;
+        // dP^T, on the step's critical chain, goes first when both are
+        auto issue_dp = [&]() {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          if (!(ok = mbar_wait(half ? bar_pr : bar_ph, n & 1, p.st, abort_flag))) break;
-          tc_fence_after();
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * LY::kSlab + (kk & 3) * 32;
+            mma_bf16_ss(tDP, sdesc_sw128(v_base + off, 16, 1024), sdesc_sw128(dob + off, 16, 1024), idSS,
+                        kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar_dpf);
+        };
+        auto issue_dv = [&](int half) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int kk = (j >> 1) * 4 + half * 2 + (j & 1);
             mma_bf16_ts(tDV, tS + a_col(kk), sdesc_sw128(dob + kk * 2048, LY::kSlab, 1024), idTS,
                         (n > 0 || half > 0 || j > 0) ? 1u : 0u);
           }
+        };
+        bool dp = false;
+        int dv = 0;
+        const unsigned long long t0 = globaltimer_ns();
+        while (!dp || dv < 2) {
+          if (!dp && (n == 0 || mbar_try_wait(bar_dqe, (n - 1) & 1))) {
+            tc_fence_after();
+            issue_dp();
+            dp = true;
+          } else if (dv < 2 && mbar_try_wait(dv ? bar_pr : bar_ph, n & 1)) {
+            tc_fence_after();
+            issue_dv(dv);
+            ++dv;
+          } else if (*abort_flag) {
+            ok = false;
+            break;
+          } else if (globaltimer_ns() - t0 > p.st.timeout_ns) {
+            atomicExch(p.st.word, (int)RA_ERR_TIMEOUT);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
         }
         if (!ok) break;
-        // dP^T = V dO^T into the dP^T columns, once dQ^T_{n-1} has left them
-        if (n > 0 && !(ok = mbar_wait(bar_dqe, (n - 1) & 1, p.st, abort_flag))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * LY::kSlab + (kk & 3) * 32;
-          mma_bf16_ss(tDP, sdesc_sw128(v_base + off, 16, 1024), sdesc_sw128(dob + off, 16, 1024), idSS,
-                      kk > 0 ? 1u : 0u);
-        }
-        mma_commit(bar_dpf);
         // S^T of the next query tile into the columns dV has read
         if (n + 1 < n_total) {
           const int st1 = (n + 1) % kSt;
@@ -640,37 +697,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       mma_commit(bar_done);
     }
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    regs_inc<kDrainRegsF>();
+    // ---------------- dQ drain: one d index (TMEM lane) per thread ----------------
+    const int r = warp * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    int m = 0;
+    walk.run([&](int qbh, int qt, bool) {
+      if (!__all_sync(FULL, mbar_wait(bar_dqf, m & 1, p.st, abort_flag))) return false;
+      tc_fence_after();
+      // all 128 query columns of this d index: load, free the columns, add
+      uint32_t a[4][32];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tmem_ld32(tDP + lane_off + 32 * i, a[i]);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(bar_dqe);
+      float* dst = p.dqacc + ((size_t)qbh * p.N + qt * kT) * D + r;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int c = 0; c < 32; ++c) red_add_f32(dst + (size_t)(32 * i + c) * D, __uint_as_float(a[i][c]));
+      ++m;
+      return true;
+    });
+  } else {
+    regs_inc<kEwRegsF>();
+    // ---------------- element-wise: P^T, dS^T; dK, dV epilogue ----------------
     const int h = (warp >> 2) - 1;          // query columns [64 h, 64 h + 64)
-    const int r = (warp & 3) * 32 + lane;   // key row of S^T, dP^T = TMEM lane; d index of dQ^T
+    const int r = (warp & 3) * 32 + lane;   // key row = TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t cS = tS + lane_off + h * kHalf, cDP = tDP + lane_off + h * kHalf;
     const float2 sl22 = make_float2(p.scale_log2, p.scale_log2);
     // this thread's row of the dS^T tile in shared memory: slab h, 128-byte
     // swizzled row r (16-byte chunk j stored at chunk j ^ (r % 8))
     const uint32_t ds_row = smem_u32(sDS) + h * LY::kSlab + r * 128;
-    // dQ^T of step m (query rows qrow .. qrow + 127): load this thread's 64
-    // columns, free the dP^T columns, then add them into the accumulator.
-    auto drain_dq = [&](int m, int qrow, bool release) -> bool {
-      if (!__all_sync(FULL, mbar_wait(bar_dqf, m & 1, p.st, abort_flag))) return false;
-      tc_fence_after();
-      uint32_t a[32], b[32];
-      tmem_ld32(cDP, a);
-      tmem_ld32(cDP + 32, b);
-      tmem_ld_wait();
-      if (release) {
-        tc_fence_before();
-        mbar_arrive(bar_dqe);
-      }
-      float* dst = p.dqacc + ((size_t)qrow + h * kHalf) * D + r;
-#pragma unroll
-      for (int c = 0; c < 32; ++c) red_add_f32(dst + (size_t)c * D, __uint_as_float(a[c]));
-#pragma unroll
-      for (int c = 0; c < 32; ++c) red_add_f32(dst + (size_t)(32 + c) * D, __uint_as_float(b[c]));
-      return true;
-    };
-    int n = 0, prev_qrow = 0;
-    const bool ok = walk.run([&](int qbh, int qt, bool diag) {
+    int n = 0;
+    const bool ok = walk.run([&](int, int, bool diag) {
       const int st = n % kSt;
       if (!__all_sync(FULL, mbar_wait(&bar_qf[st], (n / kSt) & 1, p.st, abort_flag))) return false;
       if (!__all_sync(FULL, mbar_wait(bar_sf, n & 1, p.st, abort_flag))) return false;
@@ -700,42 +763,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(half ? bar_pr : bar_ph);
       }
-      // the previous step's dQ^T: its columns are needed for this step's dP^T
-      if (n > 0 && !drain_dq(n - 1, prev_qrow, true)) return false;
-
+      // dP^T_n completes after dQ^T_{n-1} (in issue order), which was the
+      // last reader of the shared-memory dS^T tile written below
       if (!__all_sync(FULL, mbar_wait(bar_dpf, n & 1, p.st, abort_flag))) return false;
       tc_fence_after();
+      // dP^T columns of this group in; bf16 dS^T out over the first 32 of them
+      // (the A operand of dK) and to row r of slab h of the shared-memory tile
+      // (16-byte chunk j of the row at chunk j ^ (r % 8))
       {
         uint32_t a[32], b[32];
         tmem_ld32(cDP, a);
         tmem_ld32(cDP + 32, b);
         tmem_ld_wait();
-        uint32_t pk[32];
 #pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const int q = 2 * x;
-          pk[x] = pack_bf16x2(P[q] * (__uint_as_float(a[2 * x]) - dvec[q]),
-                              P[q + 1] * (__uint_as_float(a[2 * x + 1]) - dvec[q + 1]));
-          pk[16 + x] = pack_bf16x2(P[32 + q] * (__uint_as_float(b[2 * x]) - dvec[32 + q]),
-                                   P[33 + q] * (__uint_as_float(b[2 * x + 1]) - dvec[33 + q]));
+        for (int g = 0; g < 2; ++g) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            const int q = 32 * g + 2 * x;
+            const uint32_t d0 = g ? b[2 * x] : a[2 * x], d1 = g ? b[2 * x + 1] : a[2 * x + 1];
+            pk[x] = pack_bf16x2(P[q] * (__uint_as_float(d0) - dvec[q]), P[q + 1] * (__uint_as_float(d1) - dvec[q + 1]));
+          }
+          tmem_st16(cDP + 16 * g, pk);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            st_shared_v4(ds_row + (((4 * g + j) ^ (r & 7)) << 4), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2],
+                         pk[4 * j + 3]);
         }
-        tmem_st32(cDP, pk);  // bf16 dS^T over the first 32 of this group's dP^T columns
-        // the same 64 bf16 values as row r of slab h of the shared-memory dS^T
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          st_shared_v4(ds_row + ((j ^ (r & 7)) << 4), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
       }
       tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar_dsr);
-      prev_qrow = qbh * p.N + qt * kT;
       ++n;
       return true;
     });
-    bool fin = ok;
-    if (fin && n > 0) fin = drain_dq(n - 1, prev_qrow, false);
-    if (fin && __all_sync(FULL, mbar_wait(bar_done, 0, p.st, abort_flag))) {
+    if (ok && __all_sync(FULL, mbar_wait(bar_done, 0, p.st, abort_flag))) {
       tc_fence_after();
       const size_t row = (size_t)krow0 + r;
       store_acc_row<D / 2>(tDK + lane_off + h * (D / 2), p.scale, p.dk + row * D + h * (D / 2));
@@ -745,7 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == 14) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -1160,13 +1223,14 @@ int launch_passes(const AttnArgs& a, const void* dout, void* dq, void* dk, void*
   }
   if (phase_mask & kPhaseFused) {
     if constexpr (D == 128) {
+      if (!fused_usable()) return RA_ERR_UNSUPPORTED;
       // per key/value head: K, V, its query heads' Q, dO (bf16) and their
       // fp32 dQ accumulator rows stay in L2 while the head group is in flight
       p.group = head_group(p.num_tiles, p.BHkv, (double)a.N * D * (2.0 * (2 + 2 * p.G) + 4.0 * p.G), 100.0e6);
       p.smem_alloc = FusedLayout<D>::kAlloc;
       auto kern = bwd_fused_kernel<D>;
       if (set_smem_attr((const void*)kern, FusedLayout<D>::kAlloc) != RA_OK) return RA_ERR_CUDA;
-      kern<<<(unsigned)(p.BHkv * p.num_tiles), kThreads, FusedLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
+      kern<<<(unsigned)(p.BHkv * p.num_tiles), kThreadsF, FusedLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
       if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
     } else {
       return RA_ERR_UNSUPPORTED;
@@ -1179,6 +1243,33 @@ int launch_passes(const AttnArgs& a, const void* dout, void* dq, void* dk, void*
 
 bool bwd_fused_supported(int64_t D) { return D == 128; }
 
+// Whether bwd_fused_kernel may run on the current device: its register split
+// (setmaxnreg) is sized for exactly kLaunchRegsF registers per thread at
+// launch, so a build that compiled it to another count must not launch it
+// (the split would then wait for registers that were never allocated).
+// Decided once per device and cached.  Without a device nothing launches;
+// the answer is then the build's (its register count is checked when the
+// library is built).
+bool fused_usable() {
+  constexpr int kMaxDev = 64;
+  static std::mutex mu;
+  static signed char known[kMaxDev] = {};  // 0 unknown, 1 usable, -1 not
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return true;
+  }
+  if (dev < 0 || dev >= kMaxDev) return false;
+  std::lock_guard<std::mutex> lk(mu);
+  if (known[dev] == 0) {
+    cudaFuncAttributes fa;
+    const bool ok = cudaFuncGetAttributes(&fa, (const void*)bwd_fused_kernel<128>) == cudaSuccess &&
+                    fa.numRegs == kLaunchRegsF;
+    known[dev] = ok ? 1 : -1;
+  }
+  return known[dev] > 0;
+}
+
 size_t bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t D, bool fused) {
   if (B <= 0 || H <= 0 || N <= 0 || D <= 0) return 0;
   const size_t rows = (size_t)B * H * N;
@@ -1187,13 +1278,14 @@ size_t bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t D, bool fuse
 }
 
 int bwd_default_phases(int64_t D) {
-  return bwd_fused_supported(D) ? (kPhasePre | kPhaseFused | kPhaseConvert) : (kPhasePre | kPhaseKV | kPhaseQ);
+  return bwd_fused_supported(D) && fused_usable() ? (kPhasePre | kPhaseFused | kPhaseConvert)
+                                                  : (kPhasePre | kPhaseKV | kPhaseQ);
 }
 
 const char* bwd_tc_kernel_names(int64_t D) {
   if (D != 64 && D != 128) return nullptr;
-  return bwd_fused_supported(D) ? "bwd_preprocess_kernel+bwd_fused_kernel+bwd_dq_convert_kernel"
-                                : "bwd_preprocess_kernel+bwd_kv_kernel+bwd_q_kernel";
+  return (bwd_default_phases(D) & kPhaseFused) ? "bwd_preprocess_kernel+bwd_fused_kernel+bwd_dq_convert_kernel"
+                                               : "bwd_preprocess_kernel+bwd_kv_kernel+bwd_q_kernel";
 }
 
 int launch_bwd_tc(const AttnArgs& a, const void* out, const float* lse, const void* dout, void* dq, void* dk,

@@ -737,13 +737,19 @@ __global__ void __launch_bounds__(kThreads2, 1)
 // launch, so a build that compiled it to another count must not launch it
 // (a split larger than the launch's registers would wait forever).  Decided
 // once per device and cached; ringattn_kernel_plan reports the outcome.
+// Without a device nothing launches; the answer is then the build's (its
+// register count is checked when the library is built).
 template <int D>
 bool tc2_usable() {
   constexpr int kMaxDev = 64;
   static std::mutex mu;
   static signed char known[kMaxDev] = {};  // 0 unknown, 1 usable, -1 not
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return false;
+  if (cudaGetDevice(&dev) != cudaSuccess) {  // no device: nothing launches; the build checked the count
+    cudaGetLastError();
+    return true;
+  }
+  if (dev < 0 || dev >= kMaxDev) return false;
   std::lock_guard<std::mutex> lk(mu);
   if (known[dev] == 0) {
     cudaFuncAttributes fa;

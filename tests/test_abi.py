@@ -210,3 +210,21 @@ def test_accumulate_and_cast_contract(L):
     assert L.ringattn_cast(FAKE, None, 16, 0, None) == -1
     assert L.ringattn_cast(FAKE, MIS, 16, 0, None) == -4
     assert L.ringattn_cast(None, None, 0, 1, None) == 0
+
+
+def test_build_checks_launch_registers():
+    """A kernel whose register split needs an exact launch register count
+    fails the build when ptxas lands on another count."""
+    from exact_blockwise_long_b200 import build
+    log = ("ptxas info    : Compiling entry function '_ZN2ra_bwd_fused_kernelILi128EE' for 'sm_100a'\n"
+           "ptxas info    : Function properties for _ZN2ra_bwd_fused_kernelILi128EE\n"
+           "    0 bytes stack frame, 0 bytes spill stores, 0 bytes spill loads\n"
+           "ptxas info    : Used 128 registers, used 1 barriers\n"
+           "ptxas info    : Compiling entry function '_ZN2ra_bwd_kv_kernelILi128EE' for 'sm_100a'\n"
+           "ptxas info    : Used 161 registers, used 1 barriers\n")
+    assert build.kernel_registers(log) == {"_ZN2ra_bwd_fused_kernelILi128EE": 128, "_ZN2ra_bwd_kv_kernelILi128EE": 161}
+    build.check_launch_registers("csrc/bwd_tc.cu", log)
+    with pytest.raises(RuntimeError, match="exactly 128"):
+        build.check_launch_registers("csrc/bwd_tc.cu", log.replace("Used 128", "Used 120"))
+    with pytest.raises(RuntimeError, match="no registers"):
+        build.check_launch_registers("csrc/fwd_tc.cu", log)
