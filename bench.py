@@ -62,6 +62,9 @@ def parse():
                     choices=["n32k_d128", "n8k_d64_causal", "n8k_d64_full", "layer7b", "layer7b_full",
                              "n1m_d128", "n32k_d128_gqa8", "decode_n128k", "n32k_d128_step", "merge_n32k"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--ring", action="store_true",
+                    help="run the multi-device ring (one sequence shard per rank, key/value blocks passed "
+                         "rank to rank) on the workload's whole sequence instead of one batch per rank")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (smaller profiling cases)")
@@ -746,6 +749,75 @@ def run_layer(args, ra, dev, rank, world, dist):
     return line
 
 
+def run_ring(args, ra, dev, rank, world, dist):
+    """The workload's sequence cut into `world` contiguous shards, one per
+    rank; forward and backward by exact_blockwise_long_b200.ring (key/value
+    blocks and the dK/dV accumulators passed rank to rank by NCCL send/receive,
+    overlapped with each shard pair's compute).  The total work is fixed
+    (strong scaling)."""
+    import torch
+    from dataclasses import replace
+    from exact_blockwise_long_b200 import ring
+    from exact_blockwise_long_b200.synthetic import attention_inputs
+    aw, _ = workload(args.workload)
+    if args.heads:
+        aw = replace(aw, H=args.heads)
+    if aw.N % world or (aw.N // world) % aw.q_chunk or (aw.N // world) % aw.k_chunk:
+        raise SystemExit(f"--ring: {aw.N} tokens do not split into {world} shards of whole chunks")
+    L = aw.N // world
+    q, k, v, do = attention_inputs(aw, device=dev)  # the same full-sequence draw on every rank
+    sl = slice(rank * L, (rank + 1) * L)
+    q, k, v, do = (t[:, :, sl].contiguous() for t in (q, k, v, do))
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        out, lse = ring.ring_attention_forward(q, k, v, aw.causal, q_chunk=aw.q_chunk, k_chunk=aw.k_chunk)
+        ring.ring_attention_backward(q, k, v, out, lse, do, aw.causal, q_chunk=aw.q_chunk, k_chunk=aw.k_chunk)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if ra.ringattn_get_error() != 0:
+        raise RuntimeError("device status word set during warm-up")
+    clocks = ClockSampler(dev.index)
+    dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk = clocks.stop()
+    if ra.ringattn_get_error() != 0:
+        raise RuntimeError("device status word set during the timed region")
+    ms = max_over_ranks(a.elapsed_time(b) / args.steps, dist, dev)
+    flops = attn_step_flops(aw)
+    value = flops / (ms * 1e-3) / 1e12
+    pk = peaks()
+    peak, peak_kind, _ = tensor_peak(pk, ms * args.steps)
+    # this rank's launches per step: forward pairs and the cast; backward
+    # preparation, pairs, the accumulator additions after the first step, casts
+    vis = sum(1 for t in range(world) if not (aw.causal and (rank - t) % world > rank))
+    per_pair = 1 if "bwd_fused_kernel" in ra.ringattn_kernel_plan(1, L, aw.D, torch.bfloat16, 1) else 2
+    launches = (vis + 1) + (1 + per_pair * vis + 2 * (vis - 1) + 3)
+    return {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(describe(aw, None), workload=f"{aw.name} as a device ring: {world} shard(s) of {L} "
+                                                        f"tokens, one per rank, causal FLOPs counted once",
+                           parallelism=f"ring{world}"),
+            "tokens_per_s": aw.B * aw.N / (ms * 1e-3), "pct_of_bf16_peak": 100.0 * value / world / peak,
+            "roofline": {"bound": "tensor", "kernel": "ring (all per-pair launches)", "achieved": value / world,
+                         "peak": peak, "unit": "TFLOP/s", "frac": value / world / peak, "traffic": None,
+                         "peak_kind": peak_kind},
+            "gpu_launches": launches * args.steps, "clocks": clk, "e2e": None}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -763,6 +835,16 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
     else:
         torch.cuda.set_device(0)
+        if args.ring:  # a ring of one rank still runs through the process-group calls
+            import socket
+            from datetime import timedelta
+            sk = socket.socket()
+            sk.bind(("127.0.0.1", 0))
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", str(sk.getsockname()[1]))
+            sk.close()
+            dist.init_process_group("nccl", rank=0, world_size=1, timeout=timedelta(seconds=120),
+                                    device_id=torch.device("cuda", 0))
     dev = torch.device("cuda", torch.cuda.current_device())
 
     from exact_blockwise_long_b200 import build
@@ -774,11 +856,12 @@ def main():
     from dataclasses import replace
     from exact_blockwise_long_b200.synthetic import attention_inputs, ffn_inputs
 
-    if args.workload.startswith("decode") or args.workload in ("layer7b_full", "n32k_d128_step", "merge_n32k"):
-        runner = (run_decode if args.workload.startswith("decode") else
+    if args.ring or args.workload.startswith("decode") or args.workload in ("layer7b_full", "n32k_d128_step",
+                                                                            "merge_n32k"):
+        runner = (run_ring if args.ring else run_decode if args.workload.startswith("decode") else
                   run_layer if args.workload == "layer7b_full" else run_step_mode)
         line = runner(args, ra, dev, rank, world, dist)
-        if world > 1:
+        if dist.is_initialized():
             dist.barrier()
             dist.destroy_process_group()
         if rank == 0:

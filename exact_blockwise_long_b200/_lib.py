@@ -13,6 +13,7 @@ import threading
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libringattn.so")
+CHECKED_LIB_PATH = os.path.join(_HERE, "libringattn_checked.so")  # built with --checked
 
 RA_BF16 = 0
 RA_F32 = 1
@@ -20,6 +21,7 @@ RA_F32 = 1
 STATUS = {
     0: "RA_OK", -1: "RA_ERR_ARG", -2: "RA_ERR_SHAPE", -3: "RA_ERR_DTYPE", -4: "RA_ERR_ALIGN",
     -5: "RA_ERR_UNSUPPORTED", -6: "RA_ERR_CUDA", -7: "RA_ERR_TIMEOUT", -8: "RA_ERR_WORKSPACE",
+    -9: "RA_ERR_BOUNDS",
 }
 
 # name -> (restype, argtypes); the order mirrors include/ringattn.h
@@ -43,6 +45,10 @@ SIGNATURES = {
                           _P, _SZ, _P]),
     "ringattn_bwd_phase": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I,
                                 _F, _P, _SZ, _I, _P]),
+    "ringattn_bwd_prepare_size": (_SZ, [_I64, _I64, _I64]),
+    "ringattn_bwd_prepare": (_I, [_P, _P, _P, _P, _SZ, _I64, _I64, _I64, _I64, _I, _P]),
+    "ringattn_bwd_pair": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _F, _I,
+                               _P]),
     "ringattn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I,
                                   _F, _P]),
     "ringattn_decode_workspace_size": (_SZ, [_I64, _I64, _I64, _I64, _I, _I]),
@@ -74,21 +80,26 @@ class RingAttnError(RuntimeError):
         super().__init__(f"{fn} failed: {STATUS.get(status, status)}")
 
 
+def load(path: str) -> ctypes.CDLL:
+    """A handle on a build of the library at `path` with the ABI's signatures."""
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m exact_blockwise_long_b200.build` "
+            "(there is no fallback implementation)")
+    h = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        f = getattr(h, name)
+        f.restype = res
+        f.argtypes = args
+    return h
+
+
 def lib() -> ctypes.CDLL:
     """Load the shared library once; raise if it has not been built."""
     global _lib
     with _lock:
         if _lib is None:
-            if not os.path.exists(LIB_PATH):
-                raise RuntimeError(
-                    f"{LIB_PATH} is missing: build it with `python -m exact_blockwise_long_b200.build` "
-                    "(there is no fallback implementation)")
-            h = ctypes.CDLL(LIB_PATH)
-            for name, (res, args) in SIGNATURES.items():
-                f = getattr(h, name)
-                f.restype = res
-                f.argtypes = args
-            _lib = h
+            _lib = load(LIB_PATH)
     return _lib
 
 

@@ -162,6 +162,38 @@ def ringattn_bwd_phase(q, k, v, out, lse, dout, dq, dk, dv, S, q_chunk, k_chunk,
     return dq, dk, dv
 
 
+def ringattn_bwd_prepare_size(B, H, N) -> int:
+    return int(lib().ringattn_bwd_prepare_size(int(B), int(H), int(N)))
+
+
+def ringattn_bwd_prepare(out, lse, dout, prep, stream=None):
+    """prep <- D_n = dout_n . out_n and lse_n * log2(e) of one query block."""
+    B, H, N, D = _bhnd(out)
+    if dout.shape != out.shape or dout.dtype != out.dtype:
+        raise ValueError("out and dout must share shape and dtype")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N):
+        raise ValueError("lse must be float32 [B, H, N]")
+    call("ringattn_bwd_prepare", _dev(out, "out"), _dev(lse, "lse"), _dev(dout, "dout"), _dev(prep, "prep"),
+         prep.numel() * prep.element_size(), B, H, N, D, _dtype(out), _stream(stream))
+    return prep
+
+
+def ringattn_bwd_pair(q, k, v, dout, prep, dq_acc, dk_acc, dv_acc, q_chunk, k_chunk, diag, kv_accumulate=False,
+                      scale=0.0, stream=None):
+    """One shard pair's gradient: dq_acc += its dq share; dk_acc, dv_acc <- (or +=) its dk, dv share (fp32)."""
+    B, H, N, D = _bhnd(q)
+    for t in (k, v, dout):
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("q, k, v, dout must share shape and dtype")
+    for t in (dq_acc, dk_acc, dv_acc):
+        if t.dtype != torch.float32 or t.shape != q.shape:
+            raise ValueError("the accumulators are float32 [B, H, N, D]")
+    call("ringattn_bwd_pair", _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(dout, "dout"), _dev(prep, "prep"),
+         _dev(dq_acc, "dq_acc"), _dev(dk_acc, "dk_acc"), _dev(dv_acc, "dv_acc"), B, H, N, D, _dtype(q),
+         int(q_chunk), int(k_chunk), int(bool(diag)), float(scale), int(bool(kv_accumulate)), _stream(stream))
+    return dq_acc, dk_acc, dv_acc
+
+
 def ringattn_bwd_noalloc(q, k, v, out, lse, dout, dq, dk, dv, S, q_chunk, k_chunk, causal, scale=0.0, stream=None):
     """The deterministic backward without a workspace: the library's fixed
     static scratch is used instead, for callers that cannot allocate device

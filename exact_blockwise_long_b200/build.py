@@ -1,10 +1,15 @@
 """Build libringattn.so in-tree with nvcc for sm_100a.
 
-    python -m exact_blockwise_long_b200.build [--force]
+    python -m exact_blockwise_long_b200.build [--force] [--checked]
 
 Each .cu under csrc/ is compiled to an object under _build/ (in parallel),
 then linked into exact_blockwise_long_b200/libringattn.so.  A rebuild happens
 when the library is missing or older than any source or header.
+
+--checked builds libringattn_checked.so instead (objects under
+_build/checked/): the same sources with -DRA_CHECKED, whose kernels check
+every tile and row index against its tensor before the access and latch
+RA_ERR_BOUNDS in the device status word instead of making it.
 """
 
 from __future__ import annotations
@@ -24,6 +29,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libringattn.so")
+LIB_CHECKED = os.path.join(PKG, "libringattn_checked.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
@@ -47,10 +53,10 @@ def _deps():
         glob.glob(os.path.join(INCLUDE, "*.h")) + [os.path.abspath(__file__)]
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in _deps())
 
 
@@ -89,8 +95,8 @@ def check_launch_registers(src: str, ptxas_log: str) -> None:
                                f"its register split needs exactly {n}")
 
 
-def _compile(src: str, extra) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+def _compile(src: str, extra, out_dir: str = BUILD) -> str:
+    obj = os.path.join(out_dir, os.path.basename(src)[:-3] + ".o")
     checked = os.path.basename(src) in LAUNCH_REGS
     flags = list(extra) + (["-Xptxas", "-v"] if checked and "-v" not in extra else [])
     cmd = [nvcc()] + FLAGS + flags + ["-c", src, "-o", obj]
@@ -104,28 +110,31 @@ def _compile(src: str, extra) -> str:
     return obj
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and not needs_build():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
-    extra = ["-Xptxas", "-v"] if verbose_ptxas else []
+def build(force: bool = False, verbose_ptxas: bool = False, checked: bool = False) -> str:
+    lib = LIB_CHECKED if checked else LIB
+    out_dir = os.path.join(BUILD, "checked") if checked else BUILD
+    if not force and not needs_build(lib):
+        return lib
+    os.makedirs(out_dir, exist_ok=True)
+    extra = (["-Xptxas", "-v"] if verbose_ptxas else []) + (["-DRA_CHECKED"] if checked else [])
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, extra), _sources()))
-    tmp = LIB + ".tmp"
+        objs = list(ex.map(lambda s: _compile(s, extra, out_dir), _sources()))
+    tmp = lib + ".tmp"
     cmd = [nvcc()] + ARCH + ["-shared", "-o", tmp] + objs + ["-lcudart_static", "-lrt", "-ldl", "-lpthread"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--ptxas-v", action="store_true", help="print register/smem usage per kernel")
+    ap.add_argument("--checked", action="store_true", help="build the bounds-checked library (-DRA_CHECKED)")
     a = ap.parse_args()
-    print(build(force=a.force or a.ptxas_v, verbose_ptxas=a.ptxas_v))
+    print(build(force=a.force or a.ptxas_v, verbose_ptxas=a.ptxas_v, checked=a.checked))
 
 
 if __name__ == "__main__":

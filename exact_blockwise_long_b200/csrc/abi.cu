@@ -195,6 +195,7 @@ const char* ringattn_status_string(int status) {
     case RA_ERR_CUDA: return "CUDA runtime error";
     case RA_ERR_TIMEOUT: return "device-side bounded wait timed out";
     case RA_ERR_WORKSPACE: return "workspace missing or too small";
+    case RA_ERR_BOUNDS: return "bounds-checked build: an index fell outside its tensor";
     default: return "unknown status";
   }
 }
@@ -211,12 +212,14 @@ const char* ringattn_kernel_plan(int op, int64_t N, int64_t D, int dtype, int S)
 int ringattn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t H,
                  int64_t N, int64_t D, int dtype, int S, int q_chunk, int k_chunk, int causal, float scale,
                  void* stream) {
+  RA_NVTX_RANGE();
   return ringattn_fwd_gqa(q, k, v, out, lse, B, H, H, N, D, dtype, S, q_chunk, k_chunk, causal, scale, stream);
 }
 
 int ringattn_fwd_gqa(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t H,
                      int64_t Hkv, int64_t N, int64_t D, int dtype, int S, int q_chunk, int k_chunk, int causal,
                      float scale, void* stream) {
+  RA_NVTX_RANGE();
   if (Hkv < 0 || (Hkv == 0 && H != 0) || (Hkv > 0 && H % Hkv != 0)) return RA_ERR_ARG;
   int rc = check_attn(q, k, v, B, H, N, D, dtype, S, q_chunk, k_chunk, causal);
   if (rc == kEmpty) return RA_OK;
@@ -232,6 +235,7 @@ int ringattn_fwd_gqa(const void* q, const void* k, const void* v, void* out, flo
 int ringattn_fwd_step(const void* q, const void* k, const void* v, float* o_acc, float* lse_acc, int64_t B,
                       int64_t H, int64_t N, int64_t D, int dtype, int S, int q_chunk, int k_chunk, int causal,
                       float scale, int t, void* stream) {
+  RA_NVTX_RANGE();
   const int64_t Hkv = H;
   if (t < 0 || t >= S) return RA_ERR_ARG;
   int rc = check_attn(q, k, v, B, H, N, D, dtype, S, q_chunk, k_chunk, causal);
@@ -247,6 +251,7 @@ int ringattn_fwd_step(const void* q, const void* k, const void* v, float* o_acc,
 
 int ringattn_merge(float* o_a, float* lse_a, const float* o_b, const float* lse_b, int64_t rows, int64_t D,
                    void* stream) {
+  RA_NVTX_RANGE();
   if (!o_a || !lse_a || !o_b || !lse_b) return RA_ERR_ARG;
   if (rows < 0 || D <= 0) return RA_ERR_ARG;
   if (D % 4) return RA_ERR_SHAPE;
@@ -310,10 +315,50 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* out, const
 
 extern "C" {
 
+size_t ringattn_bwd_prepare_size(int64_t B, int64_t H, int64_t N) {
+  return bwd_workspace_bytes(B, H, N, 1, false);  // two fp32 row vectors; 0 for empty problems
+}
+
+int ringattn_bwd_prepare(const void* out, const float* lse, const void* dout, void* prep, size_t prep_bytes,
+                         int64_t B, int64_t H, int64_t N, int64_t D, int dtype, void* stream) {
+  RA_NVTX_RANGE();
+  if (B < 0 || H < 0 || N < 0) return RA_ERR_ARG;
+  if (dtype != RA_BF16 && dtype != RA_F32) return RA_ERR_DTYPE;
+  if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
+  if (dtype != RA_BF16) return RA_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || N == 0) return RA_OK;
+  if (!out || !lse || !dout) return RA_ERR_ARG;
+  if (!aligned16(out) || !aligned16(lse) || !aligned16(dout)) return RA_ERR_ALIGN;
+  if (!prep || prep_bytes < ringattn_bwd_prepare_size(B, H, N)) return RA_ERR_WORKSPACE;
+  if (!aligned16(prep)) return RA_ERR_ALIGN;
+  AttnArgs a{nullptr, nullptr, nullptr, B, H, N, D, dtype, 1, 128, 128, 0, resolve_scale(0.f, D), H};
+  return launch_bwd_tc(a, out, lse, dout, nullptr, nullptr, nullptr, prep, ringattn_bwd_prepare_size(B, H, N),
+                       kPhasePre, static_cast<cudaStream_t>(stream));
+}
+
+int ringattn_bwd_pair(const void* q, const void* k, const void* v, const void* dout, const void* prep,
+                      float* dq_acc, float* dk_acc, float* dv_acc, int64_t B, int64_t H, int64_t N, int64_t D,
+                      int dtype, int q_chunk, int k_chunk, int diag, float scale, int kv_accumulate,
+                      void* stream) {
+  RA_NVTX_RANGE();
+  if (kv_accumulate != 0 && kv_accumulate != 1) return RA_ERR_ARG;
+  int rc = check_attn(q, k, v, B, H, N, D, dtype, 1, q_chunk, k_chunk, diag);
+  if (rc == kEmpty) return dtype == RA_BF16 ? RA_OK : RA_ERR_UNSUPPORTED;
+  if (rc != RA_OK) return rc;
+  if (!dout || !dq_acc || !dk_acc || !dv_acc) return RA_ERR_ARG;
+  if (!aligned16(dout) || !aligned16(dq_acc) || !aligned16(dk_acc) || !aligned16(dv_acc)) return RA_ERR_ALIGN;
+  if (dtype != RA_BF16) return RA_ERR_UNSUPPORTED;
+  if (!prep) return RA_ERR_WORKSPACE;
+  if (!aligned16(prep)) return RA_ERR_ALIGN;
+  AttnArgs a{q, k, v, B, H, N, D, dtype, 1, q_chunk, k_chunk, diag, resolve_scale(scale, D), H};
+  return launch_bwd_pair(a, dout, prep, dq_acc, dk_acc, dv_acc, kv_accumulate, static_cast<cudaStream_t>(stream));
+}
+
 int ringattn_bwd_phase(const void* q, const void* k, const void* v, const void* out, const float* lse,
                        const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N, int64_t D,
                        int dtype, int S, int q_chunk, int k_chunk, int causal, float scale, void* workspace,
                        size_t workspace_bytes, int phase_mask, void* stream) {
+  RA_NVTX_RANGE();
   return bwd_impl(q, k, v, out, lse, dout, dq, dk, dv, B, H, H, N, D, dtype, S, q_chunk, k_chunk, causal, scale,
                   workspace, workspace_bytes, phase_mask, stream);
 }
@@ -322,6 +367,7 @@ int ringattn_bwd_gqa(const void* q, const void* k, const void* v, const void* ou
                      const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t Hkv, int64_t N,
                      int64_t D, int dtype, int S, int q_chunk, int k_chunk, int causal, float scale,
                      void* workspace, size_t workspace_bytes, void* stream) {
+  RA_NVTX_RANGE();
   return bwd_impl(q, k, v, out, lse, dout, dq, dk, dv, B, H, Hkv, N, D, dtype, S, q_chunk, k_chunk, causal, scale,
                   workspace, workspace_bytes, bwd_default_phases(D), stream);
 }
@@ -330,6 +376,7 @@ int ringattn_bwd(const void* q, const void* k, const void* v, const void* out, c
                  const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N, int64_t D,
                  int dtype, int S, int q_chunk, int k_chunk, int causal, float scale, void* workspace,
                  size_t workspace_bytes, void* stream) {
+  RA_NVTX_RANGE();
   return bwd_impl(q, k, v, out, lse, dout, dq, dk, dv, B, H, H, N, D, dtype, S, q_chunk, k_chunk, causal, scale,
                   workspace, workspace_bytes, bwd_default_phases(D), stream);
 }
@@ -344,6 +391,7 @@ size_t ringattn_decode_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D
 int ringattn_decode(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t H,
                     int64_t Hkv, int64_t N, int64_t D, int dtype, int S, int k_chunk, float scale, void* workspace,
                     size_t workspace_bytes, void* stream) {
+  RA_NVTX_RANGE();
   if (B < 0 || H < 0 || N < 0 || Hkv <= 0 || S <= 0 || k_chunk <= 0) return RA_ERR_ARG;
   if (dtype != RA_BF16 && dtype != RA_F32) return RA_ERR_DTYPE;
   if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
@@ -371,6 +419,7 @@ size_t blockwise_ffn_workspace_size(int64_t chunk, int64_t d_ff, int dtype) {
 int blockwise_ffn(const void* x, const void* w1, const void* w2, const void* w3, void* y, int64_t T,
                   int64_t d_model, int64_t d_ff, int64_t chunk, int dtype, void* workspace,
                   size_t workspace_bytes, void* stream) {
+  RA_NVTX_RANGE();
   if (T < 0 || d_model <= 0 || d_ff <= 0 || chunk <= 0) return RA_ERR_ARG;
   if (dtype != RA_BF16 && dtype != RA_F32) return RA_ERR_DTYPE;
   if (T == 0) return dtype == RA_BF16 ? RA_OK : RA_ERR_UNSUPPORTED;  // no tokens: nothing to compute
@@ -391,6 +440,7 @@ size_t blockwise_ffn_bwd_workspace_size(int64_t chunk, int64_t d_ff, int dtype) 
 int blockwise_ffn_bwd(const void* x, const void* w1, const void* w2, const void* w3, const void* dy, void* dx,
                       float* dw1, float* dw2, float* dw3, int64_t T, int64_t d_model, int64_t d_ff, int64_t chunk,
                       int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  RA_NVTX_RANGE();
   if (T < 0 || d_model <= 0 || d_ff <= 0 || chunk <= 0) return RA_ERR_ARG;
   if (dtype != RA_BF16 && dtype != RA_F32) return RA_ERR_DTYPE;
   if (dtype != RA_BF16) return RA_ERR_UNSUPPORTED;
@@ -414,6 +464,7 @@ int blockwise_ffn_bwd(const void* x, const void* w1, const void* w2, const void*
 }
 
 int ringattn_accumulate(float* acc, const void* x, int64_t n, int dtype, void* stream) {
+  RA_NVTX_RANGE();
   if (n < 0) return RA_ERR_ARG;
   if (dtype != RA_BF16 && dtype != RA_F32) return RA_ERR_DTYPE;
   if (n == 0) return RA_OK;
@@ -423,6 +474,7 @@ int ringattn_accumulate(float* acc, const void* x, int64_t n, int dtype, void* s
 }
 
 int ringattn_cast(const float* x, void* out, int64_t n, int dtype, void* stream) {
+  RA_NVTX_RANGE();
   if (n < 0) return RA_ERR_ARG;
   if (dtype != RA_BF16 && dtype != RA_F32) return RA_ERR_DTYPE;
   if (n == 0) return RA_OK;
@@ -445,6 +497,7 @@ int ringattn_get_error(void* stream) {
 }
 
 int ringattn_selftest_timeout(int timeout_us, void* stream) {
+  RA_NVTX_RANGE();
   if (timeout_us <= 0 || timeout_us > 10000000) return RA_ERR_ARG;
   return launch_selftest_timeout(timeout_us, static_cast<cudaStream_t>(stream));
 }

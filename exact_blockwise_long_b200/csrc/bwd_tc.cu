@@ -64,7 +64,11 @@ struct BParams {
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
-  float* dqacc;        // fused pass: fp32 dQ accumulator [BH*N, D] (unscaled)
+  float* dqacc;        // fused pass: fp32 dQ accumulator [BH*N, D] (scaled dQ added into it)
+  float* dq32;         // query-stationary pass: fp32 dq accumulator to add into instead of writing dq
+  float* dk32;         // key/value passes: fp32 dk, dv outputs instead of bf16 dk, dv
+  float* dv32;
+  int kv_add;          // with dk32, dv32: add into them (1) or overwrite them (0)
   int smem_alloc;      // fused pass: dynamic shared memory bytes of the launch
   int BH, N, S, L, causal, num_tiles;
   int H, G;            // query heads; query heads per key/value head
@@ -141,6 +145,48 @@ __device__ __forceinline__ void load_row64(uint32_t taddr, float (&s)[kHalf]) {
   for (int x = 0; x < 32; ++x) {
     s[x] = __uint_as_float(a[x]);
     s[32 + x] = __uint_as_float(b[x]);
+  }
+}
+
+template <int W>
+__device__ __forceinline__ void store_acc_row(uint32_t taddr, float mul, __nv_bfloat16* dst_row);
+
+// Store W fp32 columns of one TMEM row, times `mul`, as fp32 to global, or
+// add them to what is there (add != 0).
+template <int W>
+__device__ __forceinline__ void store_acc_row_f32(uint32_t taddr, float mul, float* dst_row, int add) {
+#pragma unroll
+  for (int c = 0; c < W / 32; ++c) {
+    uint32_t reg[32];
+    tmem_ld32(taddr + c * 32, reg);
+    tmem_ld_wait();
+    float4* dst = reinterpret_cast<float4*>(dst_row + c * 32);
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+      float4 o = make_float4(__uint_as_float(reg[4 * x]) * mul, __uint_as_float(reg[4 * x + 1]) * mul,
+                             __uint_as_float(reg[4 * x + 2]) * mul, __uint_as_float(reg[4 * x + 3]) * mul);
+      if (add) {
+        const float4 a = dst[x];
+        o.x += a.x;
+        o.y += a.y;
+        o.z += a.z;
+        o.w += a.w;
+      }
+      dst[x] = o;
+    }
+  }
+}
+
+// The dK and dV rows of one thread (key row `row`, half h of the d columns):
+// bf16 dk, dv, or fp32 dk32, dv32 (written or added) when those are given.
+template <int D>
+__device__ __forceinline__ void store_dkdv(uint32_t tDK, uint32_t tDV, size_t row, int h, const BParams& p) {
+  if (p.dk32) {
+    store_acc_row_f32<D / 2>(tDK, p.scale, p.dk32 + row * D + h * (D / 2), p.kv_add);
+    store_acc_row_f32<D / 2>(tDV, 1.f, p.dv32 + row * D + h * (D / 2), p.kv_add);
+  } else {
+    store_acc_row<D / 2>(tDK, p.scale, p.dk + row * D + h * (D / 2));
+    store_acc_row<D / 2>(tDV, 1.f, p.dv + row * D + h * (D / 2));
   }
 }
 
@@ -267,12 +313,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmDO);
       mbar_arrive_expect_tx(bar_kv, 2 * LY::kTile);
-      tma_load_tile(sK, &tmK, bar_kv, krow0);
-      tma_load_tile(sV, &tmV, bar_kv, krow0);
+      if (in_bounds(krow0 + kT <= p.BHkv * p.N, p.st, abort_flag)) {
+        tma_load_tile(sK, &tmK, bar_kv, krow0);
+        tma_load_tile(sV, &tmV, bar_kv, krow0);
+      }
       int n = 0;
       walk.run([&](int qbh, int qt, bool) {
         const int st = n % kSt;
         const int qrow = qbh * p.N + qt * kT;
+        if (!in_bounds(qrow + kT <= p.BH * p.N, p.st, abort_flag)) return false;
         if (!mbar_wait(&bar_qe[st], ((n / kSt) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_qf[st], 2 * LY::kTile + 1024);
         tma_load_tile(sQ + st * LY::kTile, &tmQ, &bar_qf[st], qrow);
@@ -417,9 +466,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     });
     if (ok && __all_sync(FULL, mbar_wait(bar_done, 0, p.st, abort_flag))) {
       tc_fence_after();
-      const size_t row = (size_t)krow0 + r;
-      store_acc_row<D / 2>(tDK + lane_off + h * (D / 2), p.scale, p.dk + row * D + h * (D / 2));
-      store_acc_row<D / 2>(tDV + lane_off + h * (D / 2), 1.f, p.dv + row * D + h * (D / 2));
+      if (in_bounds(krow0 + r < p.BHkv * p.N, p.st, abort_flag))
+        store_dkdv<D>(tDK + lane_off + h * (D / 2), tDV + lane_off + h * (D / 2), (size_t)krow0 + r, h, p);
     }
   }
 
@@ -588,12 +636,15 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmDO);
       mbar_arrive_expect_tx(bar_kv, 2 * LY::kTile);
-      tma_load_tile(sK, &tmK, bar_kv, krow0);
-      tma_load_tile(sV, &tmV, bar_kv, krow0);
+      if (in_bounds(krow0 + kT <= p.BHkv * p.N, p.st, abort_flag)) {
+        tma_load_tile(sK, &tmK, bar_kv, krow0);
+        tma_load_tile(sV, &tmV, bar_kv, krow0);
+      }
       int n = 0;
       walk.run([&](int qbh, int qt, bool) {
         const int st = n % kSt;
         const int qrow = qbh * p.N + qt * kT;
+        if (!in_bounds(qrow + kT <= p.BH * p.N, p.st, abort_flag)) return false;
         if (!mbar_wait(&bar_qe[st], ((n / kSt) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_qf[st], 2 * LY::kTile + 1024);
         tma_load_tile(sQ + st * LY::kTile, &tmQ, &bar_qf[st], qrow);
@@ -713,11 +764,12 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(bar_dqe);
+      if (!in_bounds((qbh * p.N + qt * kT) + kT <= p.BH * p.N, p.st, abort_flag)) return false;
       float* dst = p.dqacc + ((size_t)qbh * p.N + qt * kT) * D + r;
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int c = 0; c < 32; ++c) red_add_f32(dst + (size_t)(32 * i + c) * D, __uint_as_float(a[i][c]));
+        for (int c = 0; c < 32; ++c) red_add_f32(dst + (size_t)(32 * i + c) * D, __uint_as_float(a[i][c]) * p.scale);
       ++m;
       return true;
     });
@@ -800,9 +852,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     });
     if (ok && __all_sync(FULL, mbar_wait(bar_done, 0, p.st, abort_flag))) {
       tc_fence_after();
-      const size_t row = (size_t)krow0 + r;
-      store_acc_row<D / 2>(tDK + lane_off + h * (D / 2), p.scale, p.dk + row * D + h * (D / 2));
-      store_acc_row<D / 2>(tDV + lane_off + h * (D / 2), 1.f, p.dv + row * D + h * (D / 2));
+      if (in_bounds(krow0 + r < p.BHkv * p.N, p.st, abort_flag))
+        store_dkdv<D>(tDK + lane_off + h * (D / 2), tDV + lane_off + h * (D / 2), (size_t)krow0 + r, h, p);
     }
   }
 
@@ -814,14 +865,14 @@ __global__ void __launch_bounds__(kThreadsF, 1)
   }
 }
 
-// dq = bf16(scale * dQ accumulator), four elements per thread per step;
-// HBM-bound (reads 4 B, writes 2 B per element).
+// dq = bf16(dQ accumulator) (the accumulator holds scaled sums), four
+// elements per thread per step; HBM-bound (reads 4 B, writes 2 B per element).
 __global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const float4* __restrict__ acc,
-                                                             uint2* __restrict__ dq, float scale, int64_t n4) {
+                                                             uint2* __restrict__ dq, int64_t n4) {
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
     const float4 a = acc[i];
-    dq[i] = make_uint2(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale));
+    dq[i] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
   }
 }
 
@@ -929,6 +980,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       walk.run([&](int kt, bool) {
         const int ks = n % LY::kKSt, vs = n % LY::kVSt;
         const int krow = kv_head_of(bh, p.H, p.G) * p.N + kt * kT;
+        if (!in_bounds(krow + kT <= p.BHkv * p.N, p.st, abort_flag)) return false;
         if (!mbar_wait(&bar_ke[ks], ((n / LY::kKSt) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_kf[ks], LY::kTile);
         tma_load_tile(sK + ks * LY::kTile, &tmK, &bar_kf[ks], krow);
@@ -996,8 +1048,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = (warp >> 2) - 1;          // key columns [64 h, 64 h + 64)
     const int r = (warp & 3) * 32 + lane;   // query row = TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const float nl2 = -p.lse2[qrow0 + r];
-    const float Dr = p.dvec[qrow0 + r];
+    const bool row_ok = in_bounds(qrow0 + r < p.BH * p.N, p.st, abort_flag);
+    const float nl2 = row_ok ? -p.lse2[qrow0 + r] : 0.f;
+    const float Dr = row_ok ? p.dvec[qrow0 + r] : 0.f;
     const float2 sl22 = make_float2(p.scale_log2, p.scale_log2), nl22 = make_float2(nl2, nl2);
     // this row's Q and dO, d elements [D/2 h, D/2 h + D/2), into TMEM as bf16
     // pairs (column 8 kk + j holds elements 16 kk + 2 j, 16 kk + 2 j + 1)
@@ -1007,7 +1060,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t wq[D / 4], wd[D / 4];
 #pragma unroll
       for (int x = 0; x < D / 16; ++x) {
-        const uint4 a = __ldg(gq + x), b = __ldg(gd + x);
+        const uint4 a = row_ok ? __ldg(gq + x) : make_uint4(0, 0, 0, 0);
+        const uint4 b = row_ok ? __ldg(gd + x) : make_uint4(0, 0, 0, 0);
         wq[4 * x] = a.x; wq[4 * x + 1] = a.y; wq[4 * x + 2] = a.z; wq[4 * x + 3] = a.w;
         wd[4 * x] = b.x; wd[4 * x + 1] = b.y; wd[4 * x + 2] = b.z; wd[4 * x + 3] = b.w;
       }
@@ -1067,7 +1121,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     });
     if (ok && __all_sync(FULL, mbar_wait(bar_done, 0, p.st, abort_flag))) {
       tc_fence_after();
-      store_acc_row<D / 2>(tDQ + lane_off + h * (D / 2), p.scale, p.dq + ((size_t)qrow0 + r) * D + h * (D / 2));
+      const size_t qrow = (size_t)qrow0 + r;
+      if (!row_ok) {
+      } else if (p.dq32)
+        store_acc_row_f32<D / 2>(tDQ + lane_off + h * (D / 2), p.scale, p.dq32 + qrow * D + h * (D / 2), 1);
+      else
+        store_acc_row<D / 2>(tDQ + lane_off + h * (D / 2), p.scale, p.dq + qrow * D + h * (D / 2));
     }
   }
 
@@ -1131,9 +1190,18 @@ int sm_count() {
   return sms;
 }
 
+// fp32 outputs of one shard pair's gradient (ringattn_bwd_pair).
+struct PairOut {
+  float* dq;   // added into
+  float* dk;   // written, or added into with kv_add
+  float* dv;
+  int kv_add;
+};
+
 template <int D>
 int launch_passes(const AttnArgs& a, const void* dout, void* dq, void* dk, void* dv, const float* dvec,
-                  const float* lse2, float* dqacc, int phase_mask, cudaStream_t stream);
+                  const float* lse2, float* dqacc, int phase_mask, cudaStream_t stream,
+                  const PairOut* pair = nullptr);
 
 template <int D>
 int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* dout, void* dq, void* dk, void* dv,
@@ -1165,7 +1233,7 @@ int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* d
     const int64_t n4 = rows * D / 4;
     const int64_t want = (n4 + 255) / 256, cap = (int64_t)sm_count() * 8;
     bwd_dq_convert_kernel<<<(unsigned)(want < cap ? want : cap), 256, 0, stream>>>(
-        reinterpret_cast<const float4*>(dqacc), reinterpret_cast<uint2*>(dq), a.scale, n4);
+        reinterpret_cast<const float4*>(dqacc), reinterpret_cast<uint2*>(dq), n4);
     if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
   }
   return RA_OK;
@@ -1174,7 +1242,7 @@ int launch_d(const AttnArgs& a, const void* out, const float* lse, const void* d
 // The tensor-core passes selected by phase_mask (kPhaseKV, kPhaseQ, kPhaseFused).
 template <int D>
 int launch_passes(const AttnArgs& a, const void* dout, void* dq, void* dk, void* dv, const float* dvec,
-                  const float* lse2, float* dqacc, int phase_mask, cudaStream_t stream) {
+                  const float* lse2, float* dqacc, int phase_mask, cudaStream_t stream, const PairOut* pair) {
   const int64_t rows = a.B * a.H * a.N;
 
   alignas(64) CUtensorMap tq, tk, tv, tdo;
@@ -1205,6 +1273,12 @@ int launch_passes(const AttnArgs& a, const void* dout, void* dq, void* dk, void*
   int rc = current_status(&p.st);
   if (rc != RA_OK) return rc;
   p.dqacc = dqacc;
+  if (pair) {
+    p.dq32 = pair->dq;
+    p.dk32 = pair->dk;
+    p.dv32 = pair->dv;
+    p.kv_add = pair->kv_add;
+  }
   if (phase_mask & kPhaseKV) {
     // per key/value head: K, V and its query heads' Q, dO stream through L2
     p.group = head_group(p.num_tiles, p.BHkv, (double)a.N * D * 2 * (2 + 2 * p.G), 100.0e6);
@@ -1286,6 +1360,23 @@ const char* bwd_tc_kernel_names(int64_t D) {
   if (D != 64 && D != 128) return nullptr;
   return (bwd_default_phases(D) & kPhaseFused) ? "bwd_preprocess_kernel+bwd_fused_kernel+bwd_dq_convert_kernel"
                                                : "bwd_preprocess_kernel+bwd_kv_kernel+bwd_q_kernel";
+}
+
+int launch_bwd_pair(const AttnArgs& a, const void* dout, const void* prep, float* dq_acc, float* dk_acc,
+                    float* dv_acc, int kv_add, cudaStream_t stream) {
+  const size_t vec_bytes = ((size_t)(a.B * a.H * a.N) * 4 + 255) & ~(size_t)255;
+  const float* dvec = static_cast<const float*>(prep);
+  const float* lse2 = reinterpret_cast<const float*>(static_cast<const uint8_t*>(prep) + vec_bytes);
+  const PairOut po{dq_acc, dk_acc, dv_acc, kv_add};
+  // the fused pass adds the scaled dQ into dq_acc itself; the split passes
+  // add it in the query-stationary pass's epilogue
+  if (a.D == 128 && fused_usable())
+    return launch_passes<128>(a, dout, nullptr, nullptr, nullptr, dvec, lse2, dq_acc, kPhaseFused, stream, &po);
+  if (a.D == 128)
+    return launch_passes<128>(a, dout, nullptr, nullptr, nullptr, dvec, lse2, nullptr, kPhaseKV | kPhaseQ, stream, &po);
+  if (a.D == 64)
+    return launch_passes<64>(a, dout, nullptr, nullptr, nullptr, dvec, lse2, nullptr, kPhaseKV | kPhaseQ, stream, &po);
+  return RA_ERR_UNSUPPORTED;
 }
 
 int launch_bwd_tc(const AttnArgs& a, const void* out, const float* lse, const void* dout, void* dq, void* dk,

@@ -89,6 +89,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
 }
 
 // ---------------------------------------------------------------------------
+// Bounds checks (built with -DRA_CHECKED)
+// ---------------------------------------------------------------------------
+#ifdef RA_CHECKED
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+
+// In a checked build: whether an access is inside its tensor.  A failed
+// check latches RA_ERR_BOUNDS in the device status word (the first error
+// stays), raises the CTA's abort flag so the other warps' bounded waits end,
+// and returns false: the caller skips the access.  In other builds it is
+// always true and costs nothing.
+__device__ __forceinline__ bool in_bounds(bool ok, const DevStatus& st, volatile int* abort_flag) {
+  if constexpr (kChecked) {
+    if (!ok) {
+      atomicCAS(st.word, 0, (int)RA_ERR_BOUNDS);
+      if (abort_flag) *abort_flag = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------------------
 // Fences
 // ---------------------------------------------------------------------------
 // Make generic-proxy shared-memory writes visible to the async proxy

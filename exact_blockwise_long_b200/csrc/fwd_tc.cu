@@ -340,11 +340,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       mbar_arrive_expect_tx(bar_q, LY::kTileBytes);
-      tma_load_tile(sQ, &tmQ, bar_q, qrow0);
+      if (in_bounds(qrow0 + kBM <= p.BH * p.N, p.st, abort_flag)) tma_load_tile(sQ, &tmQ, bar_q, qrow0);
       int n = 0;
       walk.run([&](int kt, bool) {
         const int krow = kv_head_of(bh, p.H, p.G) * p.N + kt * kBN;
         const int ks = n % kKSt, vs = n % kVSt;
+        if (!in_bounds(krow + kBN <= (p.BH / p.G) * p.N, p.st, abort_flag)) return false;
         if (!mbar_wait(&bar_ke[ks], ((n / kKSt) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_kf[ks], LY::kTileBytes);
         tma_load_tile(sK + ks * LY::kTileBytes, &tmK, &bar_kf[ks], krow);
@@ -442,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     });
     if (ok && __all_sync(0xffffffffu, mbar_wait(bar_od, (n - 1) & 1, p.st, abort_flag))) {
       tc_fence_after();
-      store_row<D>(tO + lane_off, m_run, l_run, qrow0 + r, p);
+      if (in_bounds(qrow0 + r < p.BH * p.N, p.st, abort_flag)) store_row<D>(tO + lane_off, m_run, l_run, qrow0 + r, p);
     }
   }
 
@@ -607,11 +608,13 @@ __global__ void __launch_bounds__(kThreads2, 1)
       mbar_arrive_expect_tx(bar_q, 2 * LY::kTileBytes);
 #pragma unroll
       for (int t = 0; t < 2; ++t)
-        tma_load_tile(sQ + t * LY::kTileBytes, &tmQ, bar_q, qrow0 + t * kBM);
+        if (in_bounds(qrow0 + (t + 1) * kBM <= p.BH * p.N, p.st, abort_flag))
+          tma_load_tile(sQ + t * LY::kTileBytes, &tmQ, bar_q, qrow0 + t * kBM);
       int n = 0;
       walk.run([&](int kt, bool, bool, bool) {
         const int krow = kv_head_of(bh, p.H, p.G) * p.N + kt * kBN;
         const int ks = n % kKSt, vs = n % kVSt;
+        if (!in_bounds(krow + kBN <= (p.BH / p.G) * p.N, p.st, abort_flag)) return false;
         if (!mbar_wait(&bar_ke[ks], ((n / kKSt) & 1) ^ 1, p.st, abort_flag)) return false;
         mbar_arrive_expect_tx(&bar_kf[ks], LY::kTileBytes);
         tma_load_tile(sK + ks * LY::kTileBytes, &tmK, &bar_kf[ks], krow);
@@ -720,7 +723,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
     });
     if (ok && __all_sync(FULL, mbar_wait(bar_done, 0, p.st, abort_flag))) {
       tc_fence_after();
-      store_row<D>(tO, m_run, l_run, qrow0 + tile * kBM + r, p);
+      if (in_bounds(qrow0 + tile * kBM + r < p.BH * p.N, p.st, abort_flag))
+        store_row<D>(tO, m_run, l_run, qrow0 + tile * kBM + r, p);
     }
   }
 

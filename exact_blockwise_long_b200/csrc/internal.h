@@ -5,9 +5,22 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "ringattn.h"
 
 namespace ra {
+
+// An NVTX range over one ABI call's host-side work (argument checks and the
+// enqueue of its kernels), named after the call; visible in profilers that
+// attach an NVTX collector, free otherwise.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define RA_NVTX_RANGE() const ::ra::NvtxRange ra_nvtx_range_(__func__)
 
 struct DevStatus;
 
@@ -64,6 +77,12 @@ size_t bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t D, bool fuse
 int bwd_default_phases(int64_t D);
 int launch_bwd_tc(const AttnArgs& a, const void* out, const float* lse, const void* dout, void* dq, void* dk,
                   void* dv, void* workspace, size_t workspace_bytes, int phase_mask, cudaStream_t stream);
+
+// One shard pair's gradient into fp32 accumulators (ringattn_bwd_pair):
+// a.N is the pair's block length, a.S = 1, a.causal the diagonal mask; prep
+// holds the query block's two row vectors (kPhasePre output).
+int launch_bwd_pair(const AttnArgs& a, const void* dout, const void* prep, float* dq_acc, float* dk_acc,
+                    float* dv_acc, int kv_add, cudaStream_t stream);
 
 // Argument checks of the backward entry points (abi.cu), everything but the
 // workspace: RA_OK, kBwdEmpty (a valid empty problem: nothing to launch) or

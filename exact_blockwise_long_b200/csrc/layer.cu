@@ -150,6 +150,7 @@ int blockwise_layer_fwd(const void* x, const void* g_attn, const void* wq, const
                         void* saved, size_t saved_size, int64_t B, int64_t N, int64_t H, int64_t D, int64_t d_ff,
                         int S, int q_chunk, int k_chunk, int causal, int ffn_chunk, float eps, void* workspace,
                         size_t workspace_bytes, void* const* marks, void* stream) {
+  RA_NVTX_RANGE();
   int rc = check_layer(B, N, H, D, d_ff, S, q_chunk, k_chunk, ffn_chunk, causal);
   if (rc == kNoTokens) return RA_OK;  // no tokens: nothing to compute
   if (rc != RA_OK) return rc;
@@ -196,6 +197,7 @@ int blockwise_layer_bwd(const void* x, const void* g_attn, const void* wq, const
                         int64_t B, int64_t N, int64_t H, int64_t D, int64_t d_ff, int S, int q_chunk, int k_chunk,
                         int causal, int ffn_chunk, void* workspace, size_t workspace_bytes, void* const* marks,
                         void* stream) {
+  RA_NVTX_RANGE();
   int rc = check_layer(B, N, H, D, d_ff, S, q_chunk, k_chunk, ffn_chunk, causal);
   if (rc == kNoTokens) {  // no tokens: every parameter gradient is zero
     const size_t dm = (size_t)(H * D), ff = (size_t)d_ff;

@@ -57,6 +57,7 @@ int ringattn_bwd_noalloc(const void* q, const void* k, const void* v, const void
                          const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N,
                          int64_t D, int dtype, int S, int q_chunk, int k_chunk, int causal, float scale,
                          void* stream) {
+  RA_NVTX_RANGE();
   constexpr int kPhases = ra::kPhasePre | ra::kPhaseKV | ra::kPhaseQ;
   // the same argument checks, in the same order, as the workspace entry points
   const int rc = ra::check_bwd_args(q, k, v, out, lse, dout, dq, dk, dv, B, H, H, N, D, dtype, S, q_chunk, k_chunk,

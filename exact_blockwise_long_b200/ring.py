@@ -17,9 +17,14 @@ when j > i (causal).  Meanwhile the key/value block moves on to rank i+1
 and the next arrives from rank i-1 (peer-to-peer send/receive through
 torch.distributed, NCCL on GPUs, issued before the step's compute so the
 transfer overlaps it).  The forward merges each pair into fp32 (O, LSE)
-accumulators; the backward sums each pair's dq locally and lets the dk, dv
-accumulators travel with their key/value block, which returns to its owner
-after the last step.
+accumulators.  The backward adds each pair's dq share into a local fp32
+accumulator; each key/value block's dk, dv accumulators follow the block
+one step behind it: at step t a rank computes its share of the block it
+holds into a buffer of its own while the block's accumulator -- finished by
+the previous rank at step t - 1 -- is on its way, and adds the two once both
+are there.  So the key/value blocks and the accumulators both move while
+pairs are computed; after the last step the accumulators take one more hop,
+home to their blocks' owners.
 
 The per-pair computations go through an `ops` object; `DeviceOps` (the
 default) calls the C ABI.  Tests substitute reference arithmetic to check
@@ -39,20 +44,21 @@ class DeviceOps:
         from . import api
         self.api = api
         self.q_chunk, self.k_chunk = int(q_chunk), int(k_chunk)
-        self._ws = None
 
     def fwd_pair(self, q, k, v, o_acc, lse_acc, causal):
         """Merge the attention of q against (k, v) -- one shard pair, the
         causal mask only on the diagonal pair -- into (o_acc, lse_acc)."""
         self.api.ringattn_fwd_step(q, k, v, o_acc, lse_acc, 1, self.q_chunk, self.k_chunk, causal, 0)
 
-    def bwd_pair(self, q, k, v, o, lse, do, dq, dk, dv, causal):
-        """This pair's share of the gradients, with the global o and lse."""
-        B, H, L, D = q.shape
-        n = self.api.ringattn_bwd_workspace_size(B, H, L, D)
-        if self._ws is None or self._ws.numel() < n:
-            self._ws = torch.empty(n, device=q.device, dtype=torch.uint8)
-        self.api.ringattn_bwd(q, k, v, o, lse, do, dq, dk, dv, 1, self.q_chunk, self.k_chunk, causal, self._ws)
+    def bwd_prepare(self, o, lse, do):
+        """The query block's row statistics (D_n = dO_n . O_n, lse), once per backward."""
+        B, H, L, D = o.shape
+        prep = torch.empty(self.api.ringattn_bwd_prepare_size(B, H, L), device=o.device, dtype=torch.uint8)
+        return self.api.ringattn_bwd_prepare(o, lse, do, prep)
+
+    def bwd_pair(self, q, k, v, do, prep, dq_acc, dk, dv, causal):
+        """dq_acc += this pair's dq share; dk, dv <- its dk, dv share (fp32)."""
+        self.api.ringattn_bwd_pair(q, k, v, do, prep, dq_acc, dk, dv, self.q_chunk, self.k_chunk, causal)
 
     def accumulate(self, acc, x):
         self.api.ringattn_accumulate(acc, x)
@@ -105,40 +111,55 @@ def ring_attention_backward(q, k, v, out, lse, dout, causal=True, ops=None, grou
     """dq, dk, dv of sum(dout * out) for this rank's shards.
 
     out and lse are this rank's rows of the global forward result.  Each
-    key/value block carries fp32 dk, dv accumulators around the ring; after
-    the last step they take one more hop, back to the block's owner.
+    key/value block's fp32 dk, dv accumulators follow it around the ring one
+    step behind; after the last step they take one more hop, back to the
+    block's owner.
     """
     ops = ops or DeviceOps(q_chunk, k_chunk)
     rank, world = dist.get_rank(group), dist.get_world_size(group)
     shape = q.shape
     f32 = dict(device=q.device, dtype=torch.float32)
+    prep = ops.bwd_prepare(out, lse, dout)
     dq_acc = torch.zeros(shape, **f32)
-    # k, v of the caller are only read (see ring_attention_forward); blocks
-    # and their gradient accumulators arrive alternately in two buffer sets
-    cur = [k.contiguous(), v.contiguous(), torch.zeros(shape, **f32), torch.zeros(shape, **f32)]
-    bufs = [[torch.empty_like(x) for x in cur] for _ in range(2)]
-    dq_p, dk_p, dv_p = (torch.empty_like(q) for _ in range(3))
+    # k, v of the caller are only read (see ring_attention_forward)
+    kv = [k.contiguous(), v.contiguous()]
+    kv_bufs = [[torch.empty_like(kv[0]), torch.empty_like(kv[1])] for _ in range(2 if world > 2 else 1)]
+    # dk, dv accumulator pairs in three roles: `part` takes this step's share,
+    # `recv` receives the accumulator of the block held now, `done` is the
+    # finished accumulator of the previous step's block (being sent on)
+    part = [torch.empty(shape, **f32), torch.empty(shape, **f32)]
+    recv = [torch.empty(shape, **f32), torch.empty(shape, **f32)]
+    spare = [torch.empty(shape, **f32), torch.empty(shape, **f32)]
+    done = None
     for t in range(world):
         j = (rank - t) % world
-        if not (causal and j > rank):
-            ops.bwd_pair(q, cur[0], cur[1], out, lse, dout, dq_p, dk_p, dv_p, causal and j == rank)
-            ops.accumulate(dq_acc, dq_p)
-            ops.accumulate(cur[2], dk_p)
-            ops.accumulate(cur[3], dv_p)
-        if world == 1:
-            break
-        # the block (with its gradients) moves on; after the last step only
-        # the gradients travel, home to the block's owner
-        nxt = bufs[t % 2]
-        if t < world - 1:
-            reqs = _exchange(cur, nxt, rank, world, group)
-        else:
-            reqs = _exchange(cur[2:], nxt[2:], rank, world, group)
+        reqs = []
+        if t < world - 1:  # the block moves on while this step computes with it
+            nxt = kv_bufs[t % len(kv_bufs)]
+            reqs += _exchange(kv, nxt, rank, world, group)
+        if t > 0:  # the previous step's finished accumulator on; this block's in
+            reqs += _exchange(done, recv, rank, world, group)
+        visible = not (causal and j > rank)  # always true at t == 0 (the diagonal pair)
+        if visible:
+            ops.bwd_pair(q, kv[0], kv[1], dout, prep, dq_acc, part[0], part[1], causal and j == rank)
         for r in reqs:
             r.wait()
-        cur = nxt
+        if t == 0:
+            done, part, spare = part, spare, None  # the block's first share is its accumulator
+        else:
+            if visible:
+                ops.accumulate(recv[0], part[0])
+                ops.accumulate(recv[1], part[1])
+            done, recv = recv, done  # the sent buffer is free again: it receives next
+        if t < world - 1:
+            kv = nxt
+    if world > 1:
+        # the finished accumulators go home: this rank's block comes from rank - 1
+        for r in _exchange(done, recv, rank, world, group):
+            r.wait()
+        done = recv
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ops.cast(dq_acc, dq)
-    ops.cast(cur[2], dk)
-    ops.cast(cur[3], dv)
+    ops.cast(done[0], dk)
+    ops.cast(done[1], dv)
     return dq, dk, dv

@@ -67,7 +67,9 @@ typedef enum {
   RA_ERR_UNSUPPORTED = -5, /* valid request this build does not implement   */
   RA_ERR_CUDA = -6,        /* a CUDA runtime call failed                    */
   RA_ERR_TIMEOUT = -7,     /* a kernel's bounded wait ran out (device word) */
-  RA_ERR_WORKSPACE = -8    /* workspace missing or smaller than required    */
+  RA_ERR_WORKSPACE = -8,   /* workspace missing or smaller than required    */
+  RA_ERR_BOUNDS = -9       /* a bounds-checked build (RA_CHECKED) caught an
+                              index outside its tensor (device word)        */
 } ra_status;
 
 /* Library ABI version (major*100 + minor). */
@@ -251,6 +253,39 @@ RA_API int ringattn_bwd_phase(const void* q, const void* k, const void* v, const
                               void* stream);
 
 /*
+ * ringattn_bwd_prepare, ringattn_bwd_pair -- the backward one shard pair at
+ * a time, for a ring spread over devices (chapterpal "Ring Attention",
+ * definition: key/value blocks circulate while each device keeps its query
+ * block; darcstar note, DarcStar commentary, paragraph one: per-block
+ * results combine exactly).  A device holding query block i (N tokens of
+ * [B,H,N,D] q, out, dout and [B,H,N] lse, all from the whole-sequence
+ * forward) prepares once:
+ *   prep <- D_n = dout_n . out_n and lse_n * log2(e), two fp32 row vectors
+ *   [B,H,N], each region 256-byte aligned (ringattn_bwd_prepare_size bytes)
+ * and then, for each key/value block j it holds in turn (same N):
+ *   dq_acc += dq share of the pair   (fp32 [B,H,N,D], added into)
+ *   dk_acc, dv_acc (fp32 [B,H,N,D])  = the pair's dk, dv share, or += with
+ *                                      kv_accumulate = 1
+ * with P, dS from the prepared lse and D (the global softmax statistics):
+ * summed over all pairs these are ringattn_bwd's gradients.  diag = 1 is
+ * the diagonal pair of a causal ring (mask j > i inside it); 0 is an
+ * unmasked pair (the caller skips pairs that lie wholly in the future).
+ * Chunk rules as ringattn_fwd with S = 1; only RA_BF16.  dq_acc additions
+ * run in arrival order for D = 128 (fp32 summation order, as ringattn_bwd).
+ * Errors: RA_ERR_ARG, RA_ERR_SHAPE, RA_ERR_ALIGN, RA_ERR_UNSUPPORTED,
+ * RA_ERR_WORKSPACE (prep missing or too small), RA_ERR_CUDA.
+ */
+RA_API size_t ringattn_bwd_prepare_size(int64_t B, int64_t H, int64_t N);
+RA_API int ringattn_bwd_prepare(const void* out, const float* lse, const void* dout, void* prep,
+                                size_t prep_bytes, int64_t B, int64_t H, int64_t N, int64_t D, int dtype,
+                                void* stream);
+RA_API int ringattn_bwd_pair(const void* q, const void* k, const void* v, const void* dout, const void* prep,
+                             float* dq_acc, float* dk_acc, float* dv_acc,
+                             int64_t B, int64_t H, int64_t N, int64_t D, int dtype,
+                             int q_chunk, int k_chunk, int diag, float scale, int kv_accumulate,
+                             void* stream);
+
+/*
  * ringattn_bwd_noalloc -- the backward without a workspace and without any
  * allocation.  The paper has no counterpart; it serves callers that cannot
  * allocate device memory when they run the backward (an allocator owned by
@@ -422,8 +457,10 @@ RA_API int blockwise_layer_bwd(const void* x, const void* g_attn, const void* wq
 
 /*
  * ringattn_get_error -- synchronise `stream`, return the device status word
- * of the current device (RA_OK, RA_ERR_TIMEOUT, or RA_ERR_UNSUPPORTED from
- * a kernel that could not place its shared-memory tiles) and clear it.
+ * of the current device (RA_OK, RA_ERR_TIMEOUT, RA_ERR_UNSUPPORTED from a
+ * kernel that could not place its shared-memory tiles, or, in a library
+ * built with RA_CHECKED, RA_ERR_BOUNDS from an index check that failed: the
+ * access was skipped and the kernel wound down) and clear it.
  * Also reports a pending CUDA error as RA_ERR_CUDA.
  */
 RA_API int ringattn_get_error(void* stream);

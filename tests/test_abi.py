@@ -228,3 +228,12 @@ def test_build_checks_launch_registers():
         build.check_launch_registers("csrc/bwd_tc.cu", log.replace("Used 128", "Used 120"))
     with pytest.raises(RuntimeError, match="no registers"):
         build.check_launch_registers("csrc/fwd_tc.cu", log)
+
+
+def test_checked_build_exports_the_abi():
+    """The bounds-checked build (-DRA_CHECKED) compiles from the same sources
+    and exports the same entry points."""
+    from exact_blockwise_long_b200 import _lib, build
+    h = _lib.load(build.build(checked=True))
+    for name in declared_symbols():
+        assert hasattr(h, name), name

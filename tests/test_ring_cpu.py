@@ -4,8 +4,8 @@ the gloo backend.  The per-pair work is done by fp64 reference arithmetic
 softmax statistics), so this checks the driver itself: the ring order
 (i - t) mod S, the causal skip and diagonal mask per shard pair, the
 send/receive pairing, the exact merge of the forward partials, and the
-key/value gradients travelling with their blocks and returning to their
-owners.  Gathered over the ranks, the results equal full-sequence
+key/value gradient accumulators following their blocks one step behind and
+returning to their owners.  Gathered over the ranks, the results equal full-sequence
 attention and its gradient from the oracle."""
 
 import os
@@ -39,18 +39,22 @@ class ReferenceOps:
         o_acc.copy_(torch.from_numpy(o_new))
         lse_acc.copy_(torch.from_numpy(l_new))
 
-    def bwd_pair(self, q, k, v, o, lse, do, dq, dk, dv, causal):
-        q, k, v, o, lse, do = (t.double().numpy() for t in (q, k, v, o, lse, do))
+    def bwd_prepare(self, o, lse, do):
+        o, lse, do = (t.double().numpy() for t in (o, lse, do))
+        return np.sum(do * o, axis=-1), lse                   # D_i with the global output; global lse
+
+    def bwd_pair(self, q, k, v, do, prep, dq_acc, dk, dv, causal):
+        dvec, lse = prep
+        q, k, v, do = (t.double().numpy() for t in (q, k, v, do))
         scale = 1.0 / np.sqrt(q.shape[-1])
         s = np.einsum("bhid,bhjd->bhij", q, k) * scale
         if causal:
             L = q.shape[2]
             s = np.where(np.tril(np.ones((L, L), bool)), s, -np.inf)
         p = np.exp(s - lse[..., None])                       # global softmax statistics
-        dvec = np.sum(do * o, axis=-1)                       # D_i with the global output
         dp = np.einsum("bhid,bhjd->bhij", do, v)
         ds = p * (dp - dvec[..., None])
-        dq.copy_(torch.from_numpy(np.einsum("bhij,bhjd->bhid", ds, k) * scale))
+        dq_acc += torch.from_numpy(np.einsum("bhij,bhjd->bhid", ds, k) * scale).to(dq_acc.dtype)
         dk.copy_(torch.from_numpy(np.einsum("bhij,bhid->bhjd", ds, q) * scale))
         dv.copy_(torch.from_numpy(np.einsum("bhij,bhid->bhjd", p, do)))
 

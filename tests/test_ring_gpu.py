@@ -73,21 +73,52 @@ def test_device_ops_over_an_emulated_ring(S, causal):
     dq = [torch.zeros((B, H, L, D), **f32) for _ in range(S)]
     dk = [torch.zeros((B, H, L, D), **f32) for _ in range(S)]
     dv = [torch.zeros((B, H, L, D), **f32) for _ in range(S)]
-    pq, pk, pv = (torch.empty((B, H, L, D), device="cuda", dtype=torch.bfloat16) for _ in range(3))
+    pk, pv = (torch.empty((B, H, L, D), **f32) for _ in range(2))
     for i in range(S):
+        prep = ops.bwd_prepare(sh(out, i), sh(lse, i), sh(do, i))
         for t in range(S):
             j = (i - t) % S
             if causal and j > i:
                 continue
-            ops.bwd_pair(sh(q, i), sh(k, j), sh(v, j), sh(out, i), sh(lse, i), sh(do, i), pq, pk, pv,
-                         causal and j == i)
-            ops.accumulate(dq[i], pq)
+            ops.bwd_pair(sh(q, i), sh(k, j), sh(v, j), sh(do, i), prep, dq[i], pk, pv, causal and j == i)
             ops.accumulate(dk[j], pk)
             ops.accumulate(dv[j], pv)
     gq, gk, gv = oracle.attention_backward(to_f64(q), to_f64(k), to_f64(v), to_f64(do), causal)
     for got, ref in ((dq, gq), (dk, gk), (dv, gv)):
         assert max_abs(to_f64(torch.cat(got, 2)), ref) <= TOL_BF16_GRAD
     import exact_blockwise_long_b200 as ra
+    assert ra.ringattn_get_error() == 0
+
+
+@pytest.mark.parametrize("D", [128, 64])
+def test_pair_over_whole_sequence_equals_backward(D):
+    """One diagonal pair over the whole sequence is the whole backward: its
+    fp32 dk, dv round to ringattn_bwd's bf16 bits (same matmuls, same order),
+    dq agrees up to fp32 summation order; kv_accumulate adds onto dk, dv."""
+    import exact_blockwise_long_b200 as ra
+    B, H, N = 1, 2, 1024
+    q, k, v, do = small_attention_inputs(B, H, N, D, 61 + D, k_scale=2.0)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), device="cuda", dtype=torch.float32)
+    ra.ringattn_fwd(q, k, v, o, lse, 1, 128, 256, True)
+    ws = torch.empty(ra.ringattn_bwd_workspace_size(B, H, N, D), device="cuda", dtype=torch.uint8)
+    ref = [torch.empty_like(q) for _ in range(3)]
+    ra.ringattn_bwd(q, k, v, o, lse, do, *ref, 1, 128, 256, True, ws)
+    prep = torch.empty(ra.ringattn_bwd_prepare_size(B, H, N), device="cuda", dtype=torch.uint8)
+    ra.ringattn_bwd_prepare(o, lse, do, prep)
+    f32 = dict(device="cuda", dtype=torch.float32)
+    dq_acc = torch.zeros((B, H, N, D), **f32)
+    dk_acc, dv_acc = (torch.full((B, H, N, D), float("nan"), **f32) for _ in range(2))
+    ra.ringattn_bwd_pair(q, k, v, do, prep, dq_acc, dk_acc, dv_acc, 128, 256, True)
+    assert ra.ringattn_get_error() == 0
+    assert torch.equal(dk_acc.to(torch.bfloat16), ref[1]) and torch.equal(dv_acc.to(torch.bfloat16), ref[2])
+    a, b = dq_acc.to(torch.bfloat16).float(), ref[0].float()
+    assert bool(((a - b).abs() <= 2.0 ** -7 * torch.maximum(a.abs(), b.abs()) + 1e-5).all())
+    # the second call adds the same shares again: dq and (with kv_accumulate) dk, dv double
+    dk1, dv1, dq1 = dk_acc.clone(), dv_acc.clone(), dq_acc.clone()
+    ra.ringattn_bwd_pair(q, k, v, do, prep, dq_acc, dk_acc, dv_acc, 128, 256, True, kv_accumulate=True)
+    assert torch.equal(dk_acc, 2 * dk1) and torch.equal(dv_acc, 2 * dv1)
+    assert torch.allclose(dq_acc, 2 * dq1, rtol=1e-5, atol=1e-6)
     assert ra.ringattn_get_error() == 0
 
 
