@@ -41,15 +41,12 @@ METRIC = "ring-attn fwd+bwd TFLOP/s & tokens/s on 1 B200; % of BF16 tensor peak"
 # Captured on 8 heads of the n32k_d128 workload and scaled x4 to its 32 heads
 # (heads are independent units).
 NCU_TRAFFIC = {
-    ("bwd_kv_kernel", "n32k_d128"): {
-        "bytes": 4 * (272.243200e6 + 101.754624e6),
-        "sha256": "cbc4330a94949a94c161a59bf5be8c407f2ec2c6336d4b56842b3501eb8472a5"},
-    ("bwd_q_kernel", "n32k_d128"): {
-        "bytes": 4 * (271.136512e6 + 49.010432e6),
-        "sha256": "cbc4330a94949a94c161a59bf5be8c407f2ec2c6336d4b56842b3501eb8472a5"},
+    ("bwd_fused_kernel", "n32k_d128"): {
+        "bytes": 4 * (419.497984e6 + 235.424512e6),
+        "sha256": "e436b176d802aa147e4026c819bbec41ac0999797e4562fea83b4894d1469f4a"},
     ("fwd_tc2_kernel", "n32k_d128"): {
-        "bytes": 4 * (201.815040e6 + 47.820032e6),
-        "sha256": "b9611e372d9d56c91c6de605248d55ae1557c659a94ef3f86ba6439a0cbf8bbd"},
+        "bytes": 4 * (202.440192e6 + 50.114304e6),
+        "sha256": "403d50d00a6aea6d2c63fe48b573641de9619642750527beae2b4454b4d71ed0"},
 }
 
 
