@@ -1041,14 +1041,54 @@ def main():
             "roofline": roof, "gpu_launches": launches, "clocks": clk,
             "kernel_plan": {"fwd": fwd_name, "bwd": bwd_plan or None}}
 
-    # End to end through the public API: every step copies its inputs from
-    # pinned host memory and reads its results back.  Two device buffer sets
+    # End to end through the C ABI's host-buffer step (plain attention
+    # workloads): every step's inputs come from pinned host memory and its
+    # results go back to it inside ringattn_step_host; two device buffer sets
+    # are used in turn, each guarded by the event that marks its last copy
+    # out, so one step's copies overlap the neighbouring steps' compute.
+    if not args.no_e2e and aw.bwd and fw is None and not gqa:
+        hin = [t.cpu().pin_memory() for t in (q, k, v, do)]
+        hout = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse, dq, dk, dv)]
+                for _ in range(2)]
+        devs = [torch.empty(ra.ringattn_step_host_size(B, H, N, D), device=dev, dtype=torch.uint8) for _ in range(2)]
+        h2d = sum(t.numel() * t.element_size() for t in hin)
+        d2h = sum(t.numel() * t.element_size() for t in hout[0])
+        e2e_steps = max(3, args.steps)
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        done = [event(), event()]
+        for e_ in done:
+            e_.record(stream)  # create the events before their handles are passed on
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a, b = event(), event()
+        a.record(stream)
+        s_in.wait_event(a)
+        s_out.wait_event(a)
+        for j in range(e2e_steps):
+            bi = j % 2
+            ra.ringattn_step_host(*hin, *hout[bi], devs[bi], *cfg, stream, s_in, s_out,
+                                  wait_event=done[bi] if j >= 2 else None, done_event=done[bi])
+        stream.wait_event(done[(e2e_steps - 1) % 2])
+        stream.wait_event(done[(e2e_steps - 2) % 2])
+        b.record(stream)
+        torch.cuda.synchronize()
+        if ra.ringattn_get_error() != 0:
+            raise RuntimeError("device status word set during the end-to-end run")
+        e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, dist if world > 1 else None, dev)
+        line["e2e"] = {"value": whole_job_tflops(flops_step, world, e_ms), "unit": "TFLOP/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
+                       "steps": e2e_steps, "api": "ringattn_step_host (C ABI, host buffers)",
+                       "copies": "pinned host, on two copy streams inside the C call, overlapped with compute"}
+
+    # End to end through the public API (the other workloads): every step
+    # copies its inputs from pinned host memory and reads its results back.  Two device buffer sets
     # let step j+1's host-to-device copies and step j-1's device-to-host
     # copies run on their own streams while step j computes.  Each tensor
     # moves as soon as it can: q, k, v first and dO (and the FFN's x, dy)
     # behind them while the forward runs; O and LSE go back while the
     # backward runs, dK and dV while the dQ pass runs, dQ last.
-    if not args.no_e2e:
+    if not args.no_e2e and "e2e" not in line:
         in_f0 = [q, k, v]
         in_b0 = ([do] if aw.bwd else []) + ([x, dy] if fw is not None else [])
         out_f0 = [o, lse]

@@ -21,6 +21,8 @@ from .api import (  # noqa: F401
     ringattn_bwd_prepare,
     ringattn_bwd_prepare_size,
     ringattn_bwd_pair,
+    ringattn_step_host,
+    ringattn_step_host_size,
     ringattn_decode,
     ringattn_decode_workspace_size,
     blockwise_ffn,
@@ -40,7 +42,8 @@ from .api import (  # noqa: F401
 
 __all__ = [
     "ringattn_fwd", "ringattn_fwd_gqa", "ringattn_bwd_gqa", "ringattn_fwd_step", "ringattn_merge", "ringattn_bwd", "ringattn_bwd_phase", "ringattn_bwd_noalloc", "ringattn_bwd_workspace_size",
-    "ringattn_kernel_plan", "ringattn_bwd_prepare", "ringattn_bwd_prepare_size", "ringattn_bwd_pair",
+    "ringattn_kernel_plan", "ringattn_bwd_prepare", "ringattn_bwd_prepare_size", "ringattn_bwd_pair", "ringattn_step_host",
+    "ringattn_step_host_size",
     "ringattn_decode", "ringattn_decode_workspace_size", "blockwise_ffn", "blockwise_ffn_bwd", "ringattn_accumulate", "ringattn_cast", "blockwise_layer_fwd", "blockwise_layer_bwd", "blockwise_layer_saved_size",
     "blockwise_layer_fwd_workspace_size", "blockwise_layer_bwd_workspace_size", "blockwise_ffn_bwd_workspace_size", "blockwise_ffn_workspace_size", "ringattn_get_error", "ringattn_selftest_timeout",
     "RA_BF16", "RA_F32", "RingAttnError", "lib",

@@ -208,6 +208,36 @@ def ringattn_bwd_noalloc(q, k, v, out, lse, dout, dq, dk, dv, S, q_chunk, k_chun
     return dq, dk, dv
 
 
+def ringattn_step_host_size(B, H, N, D) -> int:
+    return int(lib().ringattn_step_host_size(int(B), int(H), int(N), int(D)))
+
+
+def ringattn_step_host(h_q, h_k, h_v, h_dout, h_out, h_lse, h_dq, h_dk, h_dv, dev, S, q_chunk, k_chunk, causal,
+                       compute_stream, in_stream, out_stream, wait_event=None, done_event=None, scale=0.0):
+    """One forward + backward step on host tensors (pinned), every copy inside
+    the C call: inputs in on in_stream, kernels on compute_stream, results out
+    on out_stream.  wait_event guards the reuse of `dev`; done_event is
+    recorded once the last result is on the host."""
+    B, H, N, D = _bhnd(h_q)
+    for t in (h_q, h_k, h_v, h_dout, h_out, h_dq, h_dk, h_dv):
+        if t.is_cuda or t.shape != h_q.shape or t.dtype != h_q.dtype or not t.is_contiguous():
+            raise ValueError("host tensors [B, H, N, D] of one dtype, contiguous")
+    if h_lse.is_cuda or h_lse.dtype != torch.float32 or tuple(h_lse.shape) != (B, H, N):
+        raise ValueError("h_lse must be a float32 host tensor [B, H, N]")
+
+    def ev(e):
+        if e is None:
+            return None
+        if e.cuda_event == 0:
+            e.record()
+        return e.cuda_event
+
+    call("ringattn_step_host", *[t.data_ptr() for t in (h_q, h_k, h_v, h_dout, h_out, h_lse, h_dq, h_dk, h_dv)],
+         _dev(dev, "dev"), _nbytes(dev), B, H, N, D, _dtype(h_q), int(S), int(q_chunk), int(k_chunk),
+         int(bool(causal)), float(scale), int(compute_stream.cuda_stream), int(in_stream.cuda_stream),
+         int(out_stream.cuda_stream), ev(wait_event), ev(done_event))
+
+
 def ringattn_decode_workspace_size(B, H, N, D, S, k_chunk) -> int:
     return int(lib().ringattn_decode_workspace_size(int(B), int(H), int(N), int(D), int(S), int(k_chunk)))
 

@@ -315,6 +315,43 @@ RA_API int ringattn_bwd_noalloc(const void* q, const void* k, const void* v, con
                                 int S, int q_chunk, int k_chunk, int causal, float scale,
                                 void* stream);
 
+/*
+ * ringattn_step_host -- one training step (ringattn_fwd, then ringattn_bwd)
+ * on data in HOST memory, with every copy inside the call.  For callers whose
+ * sequences and gradients live on the host (a data loader, an optimizer on
+ * the CPU): the paper's training use (abstract) end to end.
+ *
+ *   h_q, h_k, h_v, h_dout    host [B,H,N,D] bf16 inputs (page-locked memory
+ *                            lets the copies overlap compute)
+ *   h_out, h_dq, h_dk, h_dv  host [B,H,N,D] bf16 results; h_lse host [B,H,N]
+ *   dev                      device buffer of ringattn_step_host_size()
+ *                            bytes (inputs, results and the backward's
+ *                            workspace), 16-byte aligned
+ *   compute_stream, in_stream, out_stream  cudaStream_t: kernels, host to
+ *                            device copies, device to host copies
+ *   wait_event               cudaEvent_t or NULL: the copies into `dev`
+ *                            start after it (the caller's guard on reusing
+ *                            `dev`, e.g. the done_event of the step that last
+ *                            used it)
+ *   done_event               cudaEvent_t or NULL: recorded on out_stream once
+ *                            the last result is on the host
+ * q, k, v are copied first and the forward starts when they are in; dout
+ * follows while the forward runs; out and lse go back while the backward
+ * runs; dq, dk, dv go back last.  Asynchronous like every call: read the
+ * host results after done_event.  Other arguments, rules and errors as
+ * ringattn_fwd and ringattn_bwd; RA_ERR_WORKSPACE if `dev` is missing or
+ * too small.  The call creates and releases a few CUDA events; it
+ * allocates no memory.
+ */
+RA_API size_t ringattn_step_host_size(int64_t B, int64_t H, int64_t N, int64_t D);
+RA_API int ringattn_step_host(const void* h_q, const void* h_k, const void* h_v, const void* h_dout,
+                              void* h_out, float* h_lse, void* h_dq, void* h_dk, void* h_dv,
+                              void* dev, size_t dev_bytes,
+                              int64_t B, int64_t H, int64_t N, int64_t D, int dtype,
+                              int S, int q_chunk, int k_chunk, int causal, float scale,
+                              void* compute_stream, void* in_stream, void* out_stream,
+                              void* wait_event, void* done_event);
+
 /* Bytes of device workspace ringattn_decode needs: an fp32 partial output
  * and log-sum-exp per (batch, head, split). */
 RA_API size_t ringattn_decode_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D, int S, int k_chunk);
