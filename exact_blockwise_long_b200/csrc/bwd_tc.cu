@@ -37,7 +37,7 @@
 
 namespace ra {
 
-bool fused_usable();  // below: the fused pass's register split fits this build on this device
+bool fused_usable(int64_t D);  // below: the fused pass's register split fits this build on this device
 
 namespace {
 
@@ -511,6 +511,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 // dS^T from shared memory as well, so that dQ^T could go first, was slower:
 // 32 KB more shared-memory reads per tile pair.)
 //
+// d = 64 (TMEM has room): dQ = dS K in its own columns (M = 128 queries,
+// N = 64), double-buffered, so dP^T never waits for the drain.  The drain
+// warps (TMEM lane = query row) stage each dQ tile into shared memory, 128-byte
+// swizzled, and one thread adds it into the accumulator with two TMA tensor
+// reductions (boxes of 32 fp32 columns x 128 rows).
+//
 // Warp roles (512 threads): warps 0-3 drain dQ^T (TMEM lane = d index),
 // warps 4-11 element-wise (as in the dK/dV pass), warp 12 TMA producer,
 // warp 13 MMA issuer, warp 14 TMEM allocator.
@@ -532,16 +538,20 @@ static_assert(256 * kEwRegsF + 128 * kDrainRegsF + 128 * kRoleRegsF <= kThreadsF
 
 template <int D>
 struct FusedLayout {
+  static constexpr int kStF = D == 64 ? 3 : 2;  // Q/dO stages
   static constexpr int kTile = kT * D * 2;
   static constexpr int kSlab = kT * 128;
   static constexpr int kK = 0;
   static constexpr int kV = kK + kTile;
   static constexpr int kQ = kV + kTile;
-  static constexpr int kDO = kQ + kSt * kTile;
-  static constexpr int kDS = kDO + kSt * kTile;  // dS^T bf16 [128 keys x 128 queries], two 64-query slabs
-  static constexpr int kVec = kDS + kT * kT * 2;  // per stage: lse*log2e [128], D [128]
-  static constexpr int kBar = kVec + kSt * 1024;
-  static constexpr int kNumBars = 1 + 2 * kSt + 8;
+  static constexpr int kDO = kQ + kStF * kTile;
+  static constexpr int kDS = kDO + kStF * kTile;  // dS^T bf16 [128 keys x 128 queries], two 64-query slabs
+  // d = 64: the dQ tile staged for its TMA reduction, fp32 [128 rows x 64]
+  // as two 128-byte swizzled boxes of 32 columns
+  static constexpr int kStage = kDS + kT * kT * 2;
+  static constexpr int kVec = kStage + (D == 64 ? kT * D * 4 : 0);  // per stage: lse*log2e [128], D [128]
+  static constexpr int kBar = kVec + kStF * 1024;
+  static constexpr int kNumBars = 1 + 2 * kStF + 10;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4;
@@ -551,14 +561,17 @@ struct FusedLayout {
   static constexpr int kAlloc = kBytes + 1024 <= kMaxDynSmem ? kBytes + 1024 : kMaxDynSmem;
 };
 static_assert(FusedLayout<128>::kBytes <= kMaxDynSmem, "fused backward tile set exceeds shared memory");
+static_assert(FusedLayout<64>::kBytes <= kMaxDynSmem, "fused backward tile set exceeds shared memory");
 
 template <int D>
 __global__ void __launch_bounds__(kThreadsF, 1)
     bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                     const BParams p) {
-  static_assert(D == 128, "dQ^T takes all 128 TMEM lanes: M = d = 128");
+                     const __grid_constant__ CUtensorMap tmDQ, const BParams p) {
+  static_assert(D == 128 || D == 64, "head dimension 64 or 128");
   using LY = FusedLayout<D>;
+  constexpr int kSt = LY::kStF;
+  constexpr bool kD64 = D == 64;
   extern __shared__ uint8_t smem_fu[];
   const uint32_t pad = (1024 - (smem_u32(smem_fu) & 1023)) & 1023;
   if (pad + LY::kBytes > (uint32_t)p.smem_alloc) {
@@ -594,9 +607,9 @@ __global__ void __launch_bounds__(kThreadsF, 1)
   uint64_t* bar_ph = bar_dpf + 1;     // first half of P^T written to TMEM
   uint64_t* bar_pr = bar_ph + 1;      // all of P^T written to TMEM
   uint64_t* bar_dsr = bar_pr + 1;     // dS^T written to TMEM and shared memory
-  uint64_t* bar_dqf = bar_dsr + 1;    // dQ^T computed (in the dP^T columns)
-  uint64_t* bar_dqe = bar_dqf + 1;    // dQ^T loaded out of the dP^T columns: free again
-  uint64_t* bar_done = bar_dqe + 1;   // dK, dV final
+  uint64_t* bar_dqf = bar_dsr + 1;    // [2] dQ^T (d = 128: in the dP^T columns) / dQ buffer b computed
+  uint64_t* bar_dqe = bar_dqf + 2;    // [2] ... loaded out: its columns free again
+  uint64_t* bar_done = bar_dqe + 2;   // dK, dV final
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + LY::kTmemSlot);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LY::kAbort);
 
@@ -611,8 +624,10 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     mbar_init(bar_ph, 2 * 128);
     mbar_init(bar_pr, 2 * 128);
     mbar_init(bar_dsr, 2 * 128);
-    mbar_init(bar_dqf, 1);
-    mbar_init(bar_dqe, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar_dqf[b], 1);
+      mbar_init(&bar_dqe[b], 128);
+    }
     mbar_init(bar_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -625,7 +640,10 @@ __global__ void __launch_bounds__(kThreadsF, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tDP = tmem + 128, tDK = tmem + 256, tDV = tmem + 384;
+  // d = 128: S^T, dP^T (shared with dQ^T), dK, dV, 128 columns each;
+  // d = 64: S^T, dP^T, dK, dV (64), dQ buffers 0, 1 (64 each)
+  const uint32_t tS = tmem, tDP = tmem + 128, tDK = tmem + 256, tDV = tmem + 256 + D;
+  const uint32_t tDQ = tmem + 384;
 
   if (warp >= 12) {
     regs_dec<kRoleRegsF>();
@@ -658,7 +676,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       // ---------------- MMA issuer ----------------
       constexpr uint32_t idSS = idesc_bf16_f32(kT, kT, false, false);  // K-major x K-major
       constexpr uint32_t idTS = idesc_bf16_f32(kT, D, false, true);    // TMEM A x MN-major B
-      constexpr uint32_t idDQ = idesc_bf16_f32(D, kT, true, true);     // MN-major K^T x MN-major dS^T
+      constexpr uint32_t idDQ = kD64 ? idesc_bf16_f32(kT, D, true, true)   // MN-major dS x MN-major K
+                                     : idesc_bf16_f32(D, kT, true, true);  // MN-major K^T x MN-major dS^T
       const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV);
       const uint32_t q_base = smem_u32(sQ), do_base = smem_u32(sDO), ds_base = smem_u32(sDS);
       auto a_col = [](int kk) -> uint32_t { return kk < 4 ? kk * 8 : 64 + (kk - 4) * 8; };
@@ -705,7 +724,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         int dv = 0;
         const unsigned long long t0 = globaltimer_ns();
         while (!dp || dv < 2) {
-          if (!dp && (n == 0 || mbar_try_wait(bar_dqe, (n - 1) & 1))) {
+          if (!dp && (kD64 || n == 0 || mbar_try_wait(&bar_dqe[0], (n - 1) & 1))) {
             tc_fence_after();
             issue_dp();
             dp = true;
@@ -739,15 +758,71 @@ __global__ void __launch_bounds__(kThreadsF, 1)
           mma_bf16_ts(tDK, tDP + a_col(kk), sdesc_sw128(qb + kk * 2048, LY::kSlab, 1024), idTS,
                       (n > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bar_qe[st]);  // Q_n and dO_n are no longer read
-        // dQ^T = K^T dS^T over the dP^T columns (dK has been issued before it)
+        if constexpr (kD64) {
+          // dQ = dS K into buffer n % 2 once the drain has loaded step n - 2 out of it
+          const int b = n & 1;
+          if (n >= 2 && !(ok = mbar_wait(&bar_dqe[b], ((n - 2) >> 1) & 1, p.st, abort_flag))) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kT / 16; ++kk)
-          mma_bf16_ss(tDP, sdesc_sw128(k_base + kk * 2048, LY::kSlab, 1024),
-                      sdesc_sw128(ds_base + kk * 2048, LY::kSlab, 1024), idDQ, kk > 0 ? 1u : 0u);
-        mma_commit(bar_dqf);
+          for (int kk = 0; kk < kT / 16; ++kk)
+            mma_bf16_ss(tDQ + b * D, sdesc_sw128(ds_base + kk * 2048, LY::kSlab, 1024),
+                        sdesc_sw128(k_base + kk * 2048, LY::kSlab, 1024), idDQ, kk > 0 ? 1u : 0u);
+          mma_commit(&bar_dqf[b]);
+        } else {
+          // dQ^T = K^T dS^T over the dP^T columns (dK has been issued before it)
+#pragma unroll
+          for (int kk = 0; kk < kT / 16; ++kk)
+            mma_bf16_ss(tDP, sdesc_sw128(k_base + kk * 2048, LY::kSlab, 1024),
+                        sdesc_sw128(ds_base + kk * 2048, LY::kSlab, 1024), idDQ, kk > 0 ? 1u : 0u);
+          mma_commit(&bar_dqf[0]);
+        }
       }
       mma_commit(bar_done);
     }
+  } else if (warp < 4 && kD64) {
+    regs_inc<kDrainRegsF>();
+    // ---------------- dQ drain, d = 64: one query row (TMEM lane) per thread ----------------
+    const int r = warp * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    // this thread's row of the two staging boxes (columns [0,32), [32,64)):
+    // 128-byte row r, 16-byte chunk j at chunk j ^ (r % 8)
+    const uint32_t stage_row = smem_u32(smem + LY::kStage) + r * 128;
+    int m = 0;
+    walk.run([&](int qbh, int qt, bool) {
+      const int b = m & 1;
+      if (!__all_sync(FULL, mbar_wait(&bar_dqf[b], (m >> 1) & 1, p.st, abort_flag))) return false;
+      tc_fence_after();
+      uint32_t a[2][32];
+      tmem_ld32(tDQ + b * D + lane_off, a[0]);
+      tmem_ld32(tDQ + b * D + lane_off + 32, a[1]);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&bar_dqe[b]);
+      const int qrow = qbh * p.N + qt * kT;
+      if (!in_bounds(qrow + kT <= p.BH * p.N, p.st, abort_flag)) return false;
+      // the previous tile's reductions have read the staging boxes
+      if (threadIdx.x == 0) bulk_wait_read_all();
+      named_bar_sync(1, 128);
+#pragma unroll
+      for (int bx = 0; bx < 2; ++bx)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          st_shared_v4(stage_row + bx * kT * 128 + ((j ^ (r & 7)) << 4),
+                       __float_as_uint(__uint_as_float(a[bx][4 * j]) * p.scale),
+                       __float_as_uint(__uint_as_float(a[bx][4 * j + 1]) * p.scale),
+                       __float_as_uint(__uint_as_float(a[bx][4 * j + 2]) * p.scale),
+                       __float_as_uint(__uint_as_float(a[bx][4 * j + 3]) * p.scale));
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (threadIdx.x == 0) {
+        tma_add_2d(&tmDQ, smem + LY::kStage, 0, qrow);
+        tma_add_2d(&tmDQ, smem + LY::kStage + kT * 128, 32, qrow);
+        bulk_commit_group();
+      }
+      ++m;
+      return true;
+    });
+    if (threadIdx.x == 0) bulk_wait_all();  // the staging boxes stay in use until the reductions are done
   } else if (warp < 4) {
     regs_inc<kDrainRegsF>();
     // ---------------- dQ drain: one d index (TMEM lane) per thread ----------------
@@ -755,7 +830,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     int m = 0;
     walk.run([&](int qbh, int qt, bool) {
-      if (!__all_sync(FULL, mbar_wait(bar_dqf, m & 1, p.st, abort_flag))) return false;
+      if (!__all_sync(FULL, mbar_wait(&bar_dqf[0], m & 1, p.st, abort_flag))) return false;
       tc_fence_after();
       // all 128 query columns of this d index: load, free the columns, add
       uint32_t a[4][32];
@@ -763,7 +838,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       for (int i = 0; i < 4; ++i) tmem_ld32(tDP + lane_off + 32 * i, a[i]);
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(bar_dqe);
+      mbar_arrive(&bar_dqe[0]);
       if (!in_bounds((qbh * p.N + qt * kT) + kT <= p.BH * p.N, p.st, abort_flag)) return false;
       float* dst = p.dqacc + ((size_t)qbh * p.N + qt * kT) * D + r;
 #pragma unroll
@@ -799,8 +874,9 @@ __global__ void __launch_bounds__(kThreadsF, 1)
 #pragma unroll
         for (int c = 32 * half; c < 32 * half + 32; c += 2) {
           const float2 t = fma2(make_float2(P[c], P[c + 1]), sl22, make_float2(-lse2[c], -lse2[c + 1]));
-          P[c] = ex2_approx(t.x);
-          P[c + 1] = ex2_approx(t.y);
+          const float2 e = (kD64 && (c / 2) % 2 == 1) ? ex2_poly2(t) : make_float2(ex2_approx(t.x), ex2_approx(t.y));
+          P[c] = e.x;
+          P[c + 1] = e.y;
         }
         if (diag) {
 #pragma unroll
@@ -1296,26 +1372,27 @@ int launch_passes(const AttnArgs& a, const void* dout, void* dq, void* dk, void*
     if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
   }
   if (phase_mask & kPhaseFused) {
-    if constexpr (D == 128) {
-      if (!fused_usable()) return RA_ERR_UNSUPPORTED;
-      // per key/value head: K, V, its query heads' Q, dO (bf16) and their
-      // fp32 dQ accumulator rows stay in L2 while the head group is in flight
-      p.group = head_group(p.num_tiles, p.BHkv, (double)a.N * D * (2.0 * (2 + 2 * p.G) + 4.0 * p.G), 100.0e6);
-      p.smem_alloc = FusedLayout<D>::kAlloc;
-      auto kern = bwd_fused_kernel<D>;
-      if (set_smem_attr((const void*)kern, FusedLayout<D>::kAlloc) != RA_OK) return RA_ERR_CUDA;
-      kern<<<(unsigned)(p.BHkv * p.num_tiles), kThreadsF, FusedLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
-      if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
-    } else {
-      return RA_ERR_UNSUPPORTED;
-    }
+    if (!fused_usable(D)) return RA_ERR_UNSUPPORTED;
+    // d = 64: the dQ tiles reach the accumulator by TMA tensor reductions
+    // (boxes of 32 fp32 columns x 128 rows); d = 128 adds with scalar
+    // reductions and takes no map (tq stands in for it)
+    alignas(64) CUtensorMap tdq = tq;
+    if (D == 64 && make_tmap_f32_2d(&tdq, dqacc, D, rows, D * 4, 32, kT) != RA_OK) return RA_ERR_CUDA;
+    // per key/value head: K, V, its query heads' Q, dO (bf16) and their
+    // fp32 dQ accumulator rows stay in L2 while the head group is in flight
+    p.group = head_group(p.num_tiles, p.BHkv, (double)a.N * D * (2.0 * (2 + 2 * p.G) + 4.0 * p.G), 100.0e6);
+    p.smem_alloc = FusedLayout<D>::kAlloc;
+    auto kern = bwd_fused_kernel<D>;
+    if (set_smem_attr((const void*)kern, FusedLayout<D>::kAlloc) != RA_OK) return RA_ERR_CUDA;
+    kern<<<(unsigned)(p.BHkv * p.num_tiles), kThreadsF, FusedLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, tdq, p);
+    if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
   }
   return RA_OK;
 }
 
 }  // namespace
 
-bool bwd_fused_supported(int64_t D) { return D == 128; }
+bool bwd_fused_supported(int64_t D) { return D == 128 || D == 64; }
 
 // Whether bwd_fused_kernel may run on the current device: its register split
 // (setmaxnreg) is sized for exactly kLaunchRegsF registers per thread at
@@ -1324,24 +1401,26 @@ bool bwd_fused_supported(int64_t D) { return D == 128; }
 // Decided once per device and cached.  Without a device nothing launches;
 // the answer is then the build's (its register count is checked when the
 // library is built).
-bool fused_usable() {
+bool fused_usable(int64_t D) {
   constexpr int kMaxDev = 64;
   static std::mutex mu;
-  static signed char known[kMaxDev] = {};  // 0 unknown, 1 usable, -1 not
+  static signed char known[kMaxDev][2] = {};  // [device][d = 64, 128]: 0 unknown, 1 usable, -1 not
+  if (D != 64 && D != 128) return false;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
     cudaGetLastError();
     return true;
   }
   if (dev < 0 || dev >= kMaxDev) return false;
+  const int i = D == 128;
   std::lock_guard<std::mutex> lk(mu);
-  if (known[dev] == 0) {
+  if (known[dev][i] == 0) {
     cudaFuncAttributes fa;
-    const bool ok = cudaFuncGetAttributes(&fa, (const void*)bwd_fused_kernel<128>) == cudaSuccess &&
-                    fa.numRegs == kLaunchRegsF;
-    known[dev] = ok ? 1 : -1;
+    const void* f = D == 128 ? (const void*)bwd_fused_kernel<128> : (const void*)bwd_fused_kernel<64>;
+    const bool ok = cudaFuncGetAttributes(&fa, f) == cudaSuccess && fa.numRegs == kLaunchRegsF;
+    known[dev][i] = ok ? 1 : -1;
   }
-  return known[dev] > 0;
+  return known[dev][i] > 0;
 }
 
 size_t bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t D, bool fused) {
@@ -1352,8 +1431,8 @@ size_t bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t D, bool fuse
 }
 
 int bwd_default_phases(int64_t D) {
-  return bwd_fused_supported(D) && fused_usable() ? (kPhasePre | kPhaseFused | kPhaseConvert)
-                                                  : (kPhasePre | kPhaseKV | kPhaseQ);
+  return bwd_fused_supported(D) && fused_usable(D) ? (kPhasePre | kPhaseFused | kPhaseConvert)
+                                                   : (kPhasePre | kPhaseKV | kPhaseQ);
 }
 
 const char* bwd_tc_kernel_names(int64_t D) {
@@ -1370,12 +1449,12 @@ int launch_bwd_pair(const AttnArgs& a, const void* dout, const void* prep, float
   const PairOut po{dq_acc, dk_acc, dv_acc, kv_add};
   // the fused pass adds the scaled dQ into dq_acc itself; the split passes
   // add it in the query-stationary pass's epilogue
-  if (a.D == 128 && fused_usable())
-    return launch_passes<128>(a, dout, nullptr, nullptr, nullptr, dvec, lse2, dq_acc, kPhaseFused, stream, &po);
+  const int phases = fused_usable(a.D) ? kPhaseFused : (kPhaseKV | kPhaseQ);
+  float* acc = (phases & kPhaseFused) ? dq_acc : nullptr;
   if (a.D == 128)
-    return launch_passes<128>(a, dout, nullptr, nullptr, nullptr, dvec, lse2, nullptr, kPhaseKV | kPhaseQ, stream, &po);
+    return launch_passes<128>(a, dout, nullptr, nullptr, nullptr, dvec, lse2, acc, phases, stream, &po);
   if (a.D == 64)
-    return launch_passes<64>(a, dout, nullptr, nullptr, nullptr, dvec, lse2, nullptr, kPhaseKV | kPhaseQ, stream, &po);
+    return launch_passes<64>(a, dout, nullptr, nullptr, nullptr, dvec, lse2, acc, phases, stream, &po);
   return RA_ERR_UNSUPPORTED;
 }
 

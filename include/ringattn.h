@@ -170,9 +170,9 @@ RA_API int ringattn_merge(float* o_a, float* lse_a, const float* o_b, const floa
 
 /* Bytes of device workspace ringattn_bwd needs: two fp32 row vectors
  * [B,H,N] (D_i = dO_i . O_i and lse_i * log2(e)), each region 256-byte
- * aligned, followed for D = 128 by the fused pass's fp32 dQ accumulator
- * [B,H,N,D].  Enough for every phase mask of ringattn_bwd_phase.  0 for
- * empty problems. */
+ * aligned, followed by the fused pass's fp32 dQ accumulator [B,H,N,D].
+ * Enough for every phase mask of ringattn_bwd_phase.  0 for empty
+ * problems. */
 RA_API size_t ringattn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D);
 
 /*
@@ -185,13 +185,13 @@ RA_API size_t ringattn_bwd_workspace_size(int64_t B, int64_t H, int64_t N, int64
  * Each key/value tile stays on chip while the query shards pass by in ring
  * order i = (j + t) mod S (causal: pairs in the future skipped, the
  * diagonal pair masked).  dK and dV accumulate on chip and are written once.
- * D = 128: the same pass forms dQ's share of each tile pair and adds it
- * into an fp32 accumulator in the workspace; the sum over key tiles runs in
- * the order the CTAs reach memory, so dq is reproducible up to that fp32
- * summation order (dk, dv are bit-reproducible).  D = 64, or
- * ringattn_bwd_phase with mask 7 for any D: the deterministic split
- * backward (a second, query-stationary pass recomputes S and dP per tile
- * pair and writes dq once; every output bit-reproducible).
+ * The same pass forms dQ's share of each tile pair and adds it into an
+ * fp32 accumulator in the workspace; the sum over key tiles runs in the
+ * order the CTAs reach memory, so dq is reproducible up to that fp32
+ * summation order (dk, dv are bit-reproducible).  ringattn_bwd_phase with
+ * mask 7 runs the deterministic split backward instead (a second,
+ * query-stationary pass recomputes S and dP per tile pair and writes dq
+ * once; every output bit-reproducible).
  *
  *   q,k,v,out,dout [B,H,N,D] of `dtype` (out and lse from ringattn_fwd)
  *   lse            [B,H,N] fp32
@@ -228,21 +228,20 @@ RA_API int ringattn_bwd_gqa(const void* q, const void* k, const void* v, const v
  * ringattn_bwd_phase -- the backward's launches, selected by phase_mask
  * (1..31), for callers that schedule or time them separately:
  *   bit 0 (1)   preprocess: D_i and lse_i*log2(e) into the workspace; when
- *               the workspace is ringattn_bwd_workspace_size() bytes (D =
- *               128) it also zeroes the fp32 dQ accumulator
+ *               the workspace is ringattn_bwd_workspace_size() bytes it
+ *               also zeroes the fp32 dQ accumulator
  *   bit 1 (2)   key/value-stationary pass writing dk, dv     } the split,
  *   bit 2 (4)   query-stationary pass writing dq             } deterministic
  *                                                              backward
- *   bit 3 (8)   fused pass (D = 128): dk, dv written, dQ added into the
+ *   bit 3 (8)   fused pass: dk, dv written, scale * dQ added into the
  *               accumulator
- *   bit 4 (16)  dq = bf16(scale * accumulator) (D = 128)
+ *   bit 4 (16)  dq = bf16(accumulator)
  * Later bits read what bit 0 wrote into the same workspace; bit 4 reads what
  * bit 3 added.  Mask 7 is the deterministic backward, which needs only the
  * two row vectors (2 x round_up(B*H*N*4, 256) bytes); masks with bit 3 or 4
  * need the full ringattn_bwd_workspace_size().  ringattn_bwd runs mask 25
- * (1 + 8 + 16) for D = 128 and mask 7 for D = 64.  Arguments and errors as
- * ringattn_bwd, plus RA_ERR_ARG for a mask outside 1..31 and
- * RA_ERR_UNSUPPORTED for bits 3-4 with D = 64.
+ * (1 + 8 + 16).  Arguments and errors as ringattn_bwd, plus RA_ERR_ARG for
+ * a mask outside 1..31.
  */
 RA_API int ringattn_bwd_phase(const void* q, const void* k, const void* v, const void* out,
                               const float* lse, const void* dout,
@@ -271,7 +270,7 @@ RA_API int ringattn_bwd_phase(const void* q, const void* k, const void* v, const
  * the diagonal pair of a causal ring (mask j > i inside it); 0 is an
  * unmasked pair (the caller skips pairs that lie wholly in the future).
  * Chunk rules as ringattn_fwd with S = 1; only RA_BF16.  dq_acc additions
- * run in arrival order for D = 128 (fp32 summation order, as ringattn_bwd).
+ * run in arrival order (fp32 summation order, as ringattn_bwd).
  * Errors: RA_ERR_ARG, RA_ERR_SHAPE, RA_ERR_ALIGN, RA_ERR_UNSUPPORTED,
  * RA_ERR_WORKSPACE (prep missing or too small), RA_ERR_CUDA.
  */

@@ -91,8 +91,7 @@ def test_bwd_workspace_contract(L):
     ws = L.ringattn_bwd_workspace_size(1, 32, 32768, 128)
     # D_i and lse*log2(e) (fp32 rows), then the fused pass's fp32 dQ accumulator
     assert ws == 2 * rows * 4 + rows * 128 * 4
-    # d = 64 runs the split passes: the two row vectors only
-    assert L.ringattn_bwd_workspace_size(1, 32, 32768, 64) == 2 * rows * 4
+    assert L.ringattn_bwd_workspace_size(1, 32, 32768, 64) == 2 * rows * 4 + rows * 64 * 4
     assert L.ringattn_bwd_workspace_size(0, 1, 1, 1) == 0
     b = L.ringattn_bwd
     ws = L.ringattn_bwd_workspace_size(1, 1, 1024, 128)
@@ -105,8 +104,7 @@ def test_bwd_workspace_contract(L):
     assert ph(*args, FAKE, ws, 32, None) == -1          # unknown phase bit
     assert ph(*args, FAKE, 2 * 1024 * 4, 8, None) == -8  # the fused pass needs the dQ accumulator
     args64 = args[:12] + [64] + args[13:]
-    assert ph(*args64, FAKE, ws, 8, None) == -5         # no fused pass at d = 64
-    assert ph(*args64, FAKE, ws, 16, None) == -5
+    assert ph(*args64, FAKE, 2 * 1024 * 4, 8, None) == -8  # d = 64 fused pass: the accumulator too
 
 
 def test_kernel_plan(L):
@@ -114,7 +112,7 @@ def test_kernel_plan(L):
     plan = L.ringattn_kernel_plan
     assert plan(0, 1024, 64, 1, 4) == b"fwd_simt_kernel"
     assert plan(1, 32768, 128, 0, 16) == b"bwd_preprocess_kernel+bwd_fused_kernel+bwd_dq_convert_kernel"
-    assert plan(1, 8192, 64, 0, 8) == b"bwd_preprocess_kernel+bwd_kv_kernel+bwd_q_kernel"
+    assert plan(1, 8192, 64, 0, 8) == b"bwd_preprocess_kernel+bwd_fused_kernel+bwd_dq_convert_kernel"
     assert plan(1, 1024, 64, 1, 4) is None              # no fp32 backward
     assert plan(0, 1000, 128, 0, 16) is None            # N % S
     assert plan(0, 1024, 96, 0, 4) is None              # D

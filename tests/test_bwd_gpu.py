@@ -80,22 +80,34 @@ def _bf16_order_close(a, b):
     return bool(((a - b).abs() <= 2.0 ** -7 * torch.maximum(a.abs(), b.abs()) + 1e-5).all())
 
 
-@pytest.mark.parametrize("D,S,causal", [(128, 4, True), (128, 2, False)])
+@pytest.mark.parametrize("D,S,causal", [(128, 4, True), (128, 2, False), (64, 4, True), (64, 2, False)])
 def test_bwd_default_vs_deterministic(D, S, causal):
     """The default backward sums dQ over key tiles with fp32 additions in
     whatever order the CTAs reach memory; dK and dV are the same matmuls in
     the same order as the split backward's, so they agree to the bit; dQ
-    agrees up to summation order, and repeats of the default agree likewise."""
+    agrees up to summation order, and repeats of the default agree likewise.
+    At d = 64 the fused pass forms P as the split dK/dV pass does (every
+    second exponential on the FMA pipe, relative error 1e-4), while the split
+    dQ pass recomputes P on the hardware exponential alone; that can move the
+    bf16 rounding of single dS values by one step, so there dQ is held to
+    2^-7 of its largest magnitude instead (the oracle bound is 5e-2)."""
     import exact_blockwise_long_b200 as ra
     q, k, v, do = small_attention_inputs(2, 2, 1024, D, 9 + S, k_scale=2.0)
     B, H, N, _ = q.shape
     plan = ra.lib().ringattn_kernel_plan(1, N, D, 0, S).decode()
     assert "bwd_fused_kernel" in plan, plan
     ref = run_bwd(q, k, v, do, S, 128, 256, causal, DETERMINISTIC)
+    first = None
     for _ in range(3):
         got = run_bwd(q, k, v, do, S, 128, 256, causal)
         assert torch.equal(got[1], ref[1]) and torch.equal(got[2], ref[2])
-        assert _bf16_order_close(got[0], ref[0])
+        if D == 128:
+            assert _bf16_order_close(got[0], ref[0])
+        else:
+            a, b = got[0].float(), ref[0].float()
+            assert (a - b).abs().max() <= 2.0 ** -7 * b.abs().max()
+        first = got[0] if first is None else first
+        assert _bf16_order_close(got[0], first)  # repeats: summation order only
 
 
 def test_bwd_phase_masks():

@@ -65,7 +65,7 @@ CASES = [
     # (B, H, Hkv, N, D, S, qc, kc, causal)
     (1, 2, 2, 1024, 128, 4, 128, 256, 1),   # two-tile forward, fused backward
     (1, 2, 2, 640, 128, 5, 128, 128, 1),    # one-tile forward (shard of 128)
-    (2, 2, 2, 768, 64, 3, 128, 256, 0),     # d = 64: split backward
+    (2, 2, 2, 768, 64, 3, 128, 256, 0),     # d = 64: fused backward, TMA-reduced dQ
     (1, 4, 1, 512, 128, 2, 256, 128, 1),    # MQA
 ]
 
@@ -82,7 +82,7 @@ def test_checked_build_is_clean_and_identical(libs, B, H, Hkv, N, D, S, qc, kc, 
         g1 = _bwd(plain, q, k, v, o1, l1, do, S, qc, kc, causal, mask, st)
         g2 = _bwd(checked, q, k, v, o1, l1, do, S, qc, kc, causal, mask, st)
         assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2])
-        assert torch.equal(g1[0], g2[0]) if mask == 7 or D == 64 else _close(g1[0], g2[0])
+        assert torch.equal(g1[0], g2[0]) if mask == 7 else _close(g1[0], g2[0])
     assert checked.ringattn_get_error(ctypes.c_void_p(st)) == 0
     assert plain.ringattn_get_error(ctypes.c_void_p(st)) == 0
 
