@@ -38,12 +38,15 @@ METRIC = "ring-attn fwd+bwd TFLOP/s & tokens/s on 1 B200; % of BF16 tensor peak"
 # DRAM traffic per launch of the dominant kernel, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
 # source it was taken on (sha256 of the source file).
-# Captured on 8 heads of the n32k_d128 workload and scaled x4 to its 32 heads
-# (heads are independent units).
+# n32k_d128: captured on 8 heads of the workload and scaled x4 to its 32
+# heads (heads are independent units); n8k_d64_causal: the whole workload.
 NCU_TRAFFIC = {
     ("bwd_fused_kernel", "n32k_d128"): {
-        "bytes": 4 * (419.497984e6 + 235.424512e6),
-        "sha256": "e436b176d802aa147e4026c819bbec41ac0999797e4562fea83b4894d1469f4a"},
+        "bytes": 4 * (416.6848e6 + 228.141824e6),
+        "sha256": "297dde69d985a79b83ed2f20cca49e6c6098d38c6524aa6bdd52d2f33d56607d"},
+    ("bwd_fused_kernel", "n8k_d64_causal"): {
+        "bytes": 206.919936e6 + 93.923072e6,
+        "sha256": "297dde69d985a79b83ed2f20cca49e6c6098d38c6524aa6bdd52d2f33d56607d"},
     ("fwd_tc2_kernel", "n32k_d128"): {
         "bytes": 4 * (202.440192e6 + 50.114304e6),
         "sha256": "403d50d00a6aea6d2c63fe48b573641de9619642750527beae2b4454b4d71ed0"},
