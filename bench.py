@@ -1047,8 +1047,10 @@ def main():
     # End to end through the C ABI's host-buffer step (plain attention
     # workloads): every step's inputs come from pinned host memory and its
     # results go back to it inside ringattn_step_host; two device buffer sets
-    # are used in turn, each guarded by the event that marks its last copy
-    # out, so one step's copies overlap the neighbouring steps' compute.
+    # are used in turn.  A set's inputs are refilled once the backward that
+    # read them has run (its consumed event) and its results overwritten once
+    # they are on the host (its done event), so one step's copies overlap the
+    # neighbouring steps' compute.
     if not args.no_e2e and aw.bwd and fw is None and not gqa:
         hin = [t.cpu().pin_memory() for t in (q, k, v, do)]
         hout = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse, dq, dk, dv)]
@@ -1058,8 +1060,8 @@ def main():
         d2h = sum(t.numel() * t.element_size() for t in hout[0])
         e2e_steps = max(3, args.steps)
         s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-        done = [event(), event()]
-        for e_ in done:
+        done, consumed = [event(), event()], [event(), event()]
+        for e_ in done + consumed:
             e_.record(stream)  # create the events before their handles are passed on
         torch.cuda.synchronize()
         if world > 1:
@@ -1071,7 +1073,9 @@ def main():
         for j in range(e2e_steps):
             bi = j % 2
             ra.ringattn_step_host(*hin, *hout[bi], devs[bi], *cfg, stream, s_in, s_out,
-                                  wait_event=done[bi] if j >= 2 else None, done_event=done[bi])
+                                  inputs_free_event=consumed[bi] if j >= 2 else None,
+                                  outputs_free_event=done[bi] if j >= 2 else None,
+                                  consumed_event=consumed[bi], done_event=done[bi])
         stream.wait_event(done[(e2e_steps - 1) % 2])
         stream.wait_event(done[(e2e_steps - 2) % 2])
         b.record(stream)

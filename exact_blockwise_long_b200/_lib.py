@@ -52,7 +52,7 @@ SIGNATURES = {
     "ringattn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I,
                                   _F, _P]),
     "ringattn_step_host_size": (_SZ, [_I64, _I64, _I64, _I64]),
-    "ringattn_step_host": (_I, [_P] * 10 + [_SZ, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P]),
+    "ringattn_step_host": (_I, [_P] * 10 + [_SZ, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _F] + [_P] * 7),
     "ringattn_decode_workspace_size": (_SZ, [_I64, _I64, _I64, _I64, _I, _I]),
     "ringattn_decode": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I, _I, _I, _F, _P, _SZ, _P]),
     "blockwise_ffn_workspace_size": (_SZ, [_I64, _I64, _I]),

@@ -213,11 +213,14 @@ def ringattn_step_host_size(B, H, N, D) -> int:
 
 
 def ringattn_step_host(h_q, h_k, h_v, h_dout, h_out, h_lse, h_dq, h_dk, h_dv, dev, S, q_chunk, k_chunk, causal,
-                       compute_stream, in_stream, out_stream, wait_event=None, done_event=None, scale=0.0):
+                       compute_stream, in_stream, out_stream, inputs_free_event=None, outputs_free_event=None,
+                       consumed_event=None, done_event=None, scale=0.0):
     """One forward + backward step on host tensors (pinned), every copy inside
     the C call: inputs in on in_stream, kernels on compute_stream, results out
-    on out_stream.  wait_event guards the reuse of `dev`; done_event is
-    recorded once the last result is on the host."""
+    on out_stream.  inputs_free_event and outputs_free_event guard the reuse
+    of `dev` (pass the consumed_event and done_event of the step that last
+    used it); consumed_event is recorded once the backward has run,
+    done_event once the last result is on the host."""
     B, H, N, D = _bhnd(h_q)
     for t in (h_q, h_k, h_v, h_dout, h_out, h_dq, h_dk, h_dv):
         if t.is_cuda or t.shape != h_q.shape or t.dtype != h_q.dtype or not t.is_contiguous():
@@ -235,7 +238,8 @@ def ringattn_step_host(h_q, h_k, h_v, h_dout, h_out, h_lse, h_dq, h_dk, h_dv, de
     call("ringattn_step_host", *[t.data_ptr() for t in (h_q, h_k, h_v, h_dout, h_out, h_lse, h_dq, h_dk, h_dv)],
          _dev(dev, "dev"), _nbytes(dev), B, H, N, D, _dtype(h_q), int(S), int(q_chunk), int(k_chunk),
          int(bool(causal)), float(scale), int(compute_stream.cuda_stream), int(in_stream.cuda_stream),
-         int(out_stream.cuda_stream), ev(wait_event), ev(done_event))
+         int(out_stream.cuda_stream), ev(inputs_free_event), ev(outputs_free_event), ev(consumed_event),
+         ev(done_event))
 
 
 def ringattn_decode_workspace_size(B, H, N, D, S, k_chunk) -> int:

@@ -4,7 +4,9 @@
 // The forward's output and log-sum-exp go back while the backward runs; dO
 // comes in while the forward runs.  With two device buffer sets used in
 // turn and the caller's events ordering their reuse, one step's copies
-// overlap the neighbouring steps' compute.
+// overlap the neighbouring steps' compute: a set's inputs may be refilled
+// as soon as the backward that read them has run, its results overwritten
+// once they have been copied out.
 #include "common.cuh"
 #include "internal.h"
 
@@ -49,8 +51,8 @@ size_t ringattn_step_host_size(int64_t B, int64_t H, int64_t N, int64_t D) {
 int ringattn_step_host(const void* h_q, const void* h_k, const void* h_v, const void* h_dout, void* h_out,
                        float* h_lse, void* h_dq, void* h_dk, void* h_dv, void* dev, size_t dev_bytes, int64_t B,
                        int64_t H, int64_t N, int64_t D, int dtype, int S, int q_chunk, int k_chunk, int causal,
-                       float scale, void* compute_stream, void* in_stream, void* out_stream, void* wait_event,
-                       void* done_event) {
+                       float scale, void* compute_stream, void* in_stream, void* out_stream,
+                       void* inputs_free_event, void* outputs_free_event, void* consumed_event, void* done_event) {
   RA_NVTX_RANGE();
   if (B < 0 || H < 0 || N < 0) return RA_ERR_ARG;
   if (dtype != RA_BF16 && dtype != RA_F32) return RA_ERR_DTYPE;
@@ -82,7 +84,10 @@ int ringattn_step_host(const void* h_q, const void* h_k, const void* h_v, const 
     return rc;
   };
   auto ok = [](cudaError_t e) { return e == cudaSuccess; };
-  if (wait_event && !ok(cudaStreamWaitEvent(is, static_cast<cudaEvent_t>(wait_event), 0))) return release(RA_ERR_CUDA);
+  if (inputs_free_event && !ok(cudaStreamWaitEvent(is, static_cast<cudaEvent_t>(inputs_free_event), 0)))
+    return release(RA_ERR_CUDA);
+  if (outputs_free_event && !ok(cudaStreamWaitEvent(cs, static_cast<cudaEvent_t>(outputs_free_event), 0)))
+    return release(RA_ERR_CUDA);
   // q, k, v in; then dO, which the forward does not need
   for (int i = 0; i < 3; ++i)
     if (!ok(cudaMemcpyAsync(b.t[i], host[i], act, cudaMemcpyHostToDevice, is))) return release(RA_ERR_CUDA);
@@ -104,6 +109,7 @@ int ringattn_step_host(const void* h_q, const void* h_k, const void* h_v, const 
                     q_chunk, k_chunk, causal, scale, b.ws, b.ws_bytes, cs);
   if (rc != RA_OK) return release(rc);
   if (!ok(cudaEventRecord(ev[3], cs)) || !ok(cudaStreamWaitEvent(os, ev[3], 0))) return release(RA_ERR_CUDA);
+  if (consumed_event && !ok(cudaEventRecord(static_cast<cudaEvent_t>(consumed_event), cs))) return release(RA_ERR_CUDA);
   void* hg[3] = {h_dq, h_dk, h_dv};
   for (int i = 0; i < 3; ++i)
     if (!ok(cudaMemcpyAsync(hg[i], b.t[5 + i], act, cudaMemcpyDeviceToHost, os))) return release(RA_ERR_CUDA);

@@ -328,10 +328,15 @@ RA_API int ringattn_bwd_noalloc(const void* q, const void* k, const void* v, con
  *                            workspace), 16-byte aligned
  *   compute_stream, in_stream, out_stream  cudaStream_t: kernels, host to
  *                            device copies, device to host copies
- *   wait_event               cudaEvent_t or NULL: the copies into `dev`
- *                            start after it (the caller's guard on reusing
- *                            `dev`, e.g. the done_event of the step that last
- *                            used it)
+ *   inputs_free_event        cudaEvent_t or NULL: the copies of the inputs
+ *                            into `dev` start after it (the consumed_event of
+ *                            the step that last used `dev`)
+ *   outputs_free_event       cudaEvent_t or NULL: the forward writes results
+ *                            into `dev` after it (the done_event of the step
+ *                            that last used `dev`)
+ *   consumed_event           cudaEvent_t or NULL: recorded on compute_stream
+ *                            once the backward has run (the inputs in `dev`
+ *                            are no longer read)
  *   done_event               cudaEvent_t or NULL: recorded on out_stream once
  *                            the last result is on the host
  * q, k, v are copied first and the forward starts when they are in; dout
@@ -349,7 +354,8 @@ RA_API int ringattn_step_host(const void* h_q, const void* h_k, const void* h_v,
                               int64_t B, int64_t H, int64_t N, int64_t D, int dtype,
                               int S, int q_chunk, int k_chunk, int causal, float scale,
                               void* compute_stream, void* in_stream, void* out_stream,
-                              void* wait_event, void* done_event);
+                              void* inputs_free_event, void* outputs_free_event,
+                              void* consumed_event, void* done_event);
 
 /* Bytes of device workspace ringattn_decode needs: an fp32 partial output
  * and log-sum-exp per (batch, head, split). */

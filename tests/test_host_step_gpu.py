@@ -2,7 +2,7 @@
 inside the C call, must give the same results as the device-path calls
 (forward, lse, dk, dv to the bit; dq up to the fp32 summation order of the
 fused backward), also over several steps that use two device buffer sets in
-turn with the done events guarding their reuse."""
+turn with the consumed and done events guarding their reuse."""
 
 import pytest
 import torch
@@ -45,10 +45,13 @@ def test_host_step_matches_device_path(D, S, qc, kc, causal):
     outs = [[torch.full(t.shape, float("nan"), dtype=t.dtype).pin_memory() for t in steps[0][1]] for _ in steps]
     cs, s_in, s_out = torch.cuda.current_stream(), torch.cuda.Stream(), torch.cuda.Stream()
     done = [torch.cuda.Event(), torch.cuda.Event()]
+    consumed = [torch.cuda.Event(), torch.cuda.Event()]
     for j, (hin, _) in enumerate(steps):
         bi = j % 2
         ra.ringattn_step_host(*hin, *outs[j], devs[bi], S, qc, kc, causal, cs, s_in, s_out,
-                              wait_event=done[bi] if j >= 2 else None, done_event=done[bi])
+                              inputs_free_event=consumed[bi] if j >= 2 else None,
+                              outputs_free_event=done[bi] if j >= 2 else None,
+                              consumed_event=consumed[bi], done_event=done[bi])
     for e in done:
         e.synchronize()
     assert ra.ringattn_get_error() == 0
@@ -68,7 +71,7 @@ def test_host_step_rejects_bad_arguments():
     assert need > 0 and L.ringattn_step_host_size(0, H, N, D) == 0
     h = [0x10000] * 9
     dev = torch.empty(need, device="cuda", dtype=torch.uint8)
-    base = [B, H, N, D, 0, 2, 128, 128, 1, 0.0, None, None, None, None, None]
+    base = [B, H, N, D, 0, 2, 128, 128, 1, 0.0] + [None] * 7
     assert L.ringattn_step_host(*h, dev.data_ptr(), need - 1, *base) == -8         # device buffer too small
     assert L.ringattn_step_host(*h, None, need, *base) == -8                       # device buffer missing
     assert L.ringattn_step_host(*([None] + h[1:]), dev.data_ptr(), need, *base) == -1
