@@ -3,6 +3,8 @@
 // shared-memory matrix descriptors.  Hand-written inline PTX.
 #pragma once
 
+#include <utility>
+#include <type_traits>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -294,6 +296,56 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   d |= (uint64_t)2 << 61;  // SWIZZLE_128B
   return d;
 }
+
+// A single thread issues every MMA of a CTA, and the latency of its own
+// dependent instructions sits between consecutive MMAs.  For short matmuls
+// a group of K steps builds its operand descriptors once and adds the steps'
+// compile-time offsets inside the MMA instructions (the start-address field
+// holds address / 16 in bits 0-13, and shared-memory addresses stay below
+// 256 KB, so the sum never carries out of the field).  The offsets are
+// immediates added inside the asm: one add per operand between MMAs, and
+// nothing for the compiler to hoist into registers.
+template <uint32_t AOFF, uint32_t BOFF>
+__device__ __forceinline__ void mma_bf16_ss_at(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 ra, rb;\n\t"
+      "add.s64 ra, %1, %5;\n\t"
+      "add.s64 rb, %2, %6;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ra, rb, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(AOFF >> 4), "n"(BOFF >> 4)
+      : "memory");
+}
+
+template <uint32_t BOFF>
+__device__ __forceinline__ void mma_bf16_ts_at(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 rb;\n\t"
+      "add.s64 rb, %2, %5;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], rb, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(BOFF >> 4)
+      : "memory");
+}
+
+// f(std::integral_constant<int, i>{}) for i = 0 .. N-1, each i a constant
+// expression inside f.
+template <typename F, int... I>
+__device__ __forceinline__ void static_for_impl(F& f, std::integer_sequence<int, I...>) {
+  (f(std::integral_constant<int, I>{}), ...);
+}
+template <int N, typename F>
+__device__ __forceinline__ void static_for(F&& f) {
+  static_for_impl(f, std::make_integer_sequence<int, N>{});
+}
+
+// Byte offset of K step kk (16 bf16 along K) in a 128-byte-swizzled tile:
+// K-major, rows of 64 elements in slabs of `slab` bytes (32 bytes per step
+// inside a slab); MN-major, K rows of 128 bytes (16 rows per step).
+__host__ __device__ constexpr uint32_t kmajor_step(int kk, int slab) { return (kk >> 2) * slab + (kk & 3) * 32; }
+__host__ __device__ constexpr uint32_t mnmajor_step(int kk) { return kk * 2048; }
 
 // 32 lanes x 32 columns of 32-bit TMEM words: thread i of the warp gets
 // lane (32*(warp%4) + i), columns [col, col+32).
