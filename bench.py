@@ -42,11 +42,11 @@ METRIC = "ring-attn fwd+bwd TFLOP/s & tokens/s on 1 B200; % of BF16 tensor peak"
 # heads (heads are independent units); n8k_d64_causal: the whole workload.
 NCU_TRAFFIC = {
     ("bwd_fused_kernel", "n32k_d128"): {
-        "bytes": 4 * (416.6848e6 + 228.141824e6),
-        "sha256": "297dde69d985a79b83ed2f20cca49e6c6098d38c6524aa6bdd52d2f33d56607d"},
+        "bytes": 4 * (418.488064e6 + 236.270592e6),
+        "sha256": "7be4f91bd244f6a2659f1db49f2fec56d6c6810b02dfd1ea6341c582cfdd2d77"},
     ("bwd_fused_kernel", "n8k_d64_causal"): {
-        "bytes": 206.919936e6 + 93.923072e6,
-        "sha256": "297dde69d985a79b83ed2f20cca49e6c6098d38c6524aa6bdd52d2f33d56607d"},
+        "bytes": 206.973696e6 + 93.997568e6,
+        "sha256": "7be4f91bd244f6a2659f1db49f2fec56d6c6810b02dfd1ea6341c582cfdd2d77"},
     ("fwd_tc2_kernel", "n32k_d128"): {
         "bytes": 4 * (202.440192e6 + 50.114304e6),
         "sha256": "403d50d00a6aea6d2c63fe48b573641de9619642750527beae2b4454b4d71ed0"},
