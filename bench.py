@@ -37,20 +37,49 @@ METRIC = "ring-attn fwd+bwd TFLOP/s & tokens/s on 1 B200; % of BF16 tensor peak"
 
 # DRAM traffic per launch of the dominant kernel, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
-# source it was taken on (sha256 of the source file).
+# code it was taken on: the sha256 of the source file with its comments and
+# blank lines removed (code_fingerprint), so that any change to the code
+# voids the figure and a change to a comment does not.
 # n32k_d128: captured on 8 heads of the workload and scaled x4 to its 32
 # heads (heads are independent units); n8k_d64_causal: the whole workload.
 NCU_TRAFFIC = {
     ("bwd_fused_kernel", "n32k_d128"): {
         "bytes": 4 * (418.488064e6 + 236.270592e6),
-        "sha256": "7be4f91bd244f6a2659f1db49f2fec56d6c6810b02dfd1ea6341c582cfdd2d77"},
+        "code_sha256": "4a7e542d5ea8f821cedeb8f71d9f4428d80b751d8e8d7b1e4fe037036d5a7de9"},
     ("bwd_fused_kernel", "n8k_d64_causal"): {
         "bytes": 206.973696e6 + 93.997568e6,
-        "sha256": "7be4f91bd244f6a2659f1db49f2fec56d6c6810b02dfd1ea6341c582cfdd2d77"},
+        "code_sha256": "4a7e542d5ea8f821cedeb8f71d9f4428d80b751d8e8d7b1e4fe037036d5a7de9"},
     ("fwd_tc2_kernel", "n32k_d128"): {
         "bytes": 4 * (202.440192e6 + 50.114304e6),
-        "sha256": "403d50d00a6aea6d2c63fe48b573641de9619642750527beae2b4454b4d71ed0"},
+        "code_sha256": "c488625a208af031ae2481df9d6dd97427efc681e42ec2e1e105e4c354ca19e5"},
 }
+
+
+def code_fingerprint(path: str) -> str:
+    """sha256 of a C/C++/CUDA source with // and /* */ comments and blank
+    lines removed and trailing blanks stripped (string and character
+    literals are kept as they are)."""
+    src = open(path, encoding="utf-8").read()
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":  # literal: copy up to the matching unescaped quote
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = [ln.rstrip() for ln in "".join(out).split("\n")]
+    return hashlib.sha256("\n".join(ln for ln in lines if ln).encode()).hexdigest()
 
 
 def parse():
@@ -672,12 +701,12 @@ def run_layer(args, ra, dev, rank, world, dist):
     pk = peaks()
     achieved = kflops / (kms * 1e-3) / 1e12
     src = os.path.join(ROOT, "exact_blockwise_long_b200", "csrc", ksrc)
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    sha = code_fingerprint(src)
     tr = NCU_TRAFFIC.get((kname, args.workload))
     peak, peak_kind, other = tensor_peak(pk, ms * args.steps)
     roof = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": peak,
             "unit": "TFLOP/s", "frac": achieved / peak,
-            "traffic": tr["bytes"] if tr and tr["sha256"] == sha else None,
+            "traffic": tr["bytes"] if tr and tr["code_sha256"] == sha else None,
             "peak_kind": peak_kind, "frac_of_other_peak": achieved / other,
             "kernel_ms": kms,
             "kernels": {k_: {"ms": v_[0], "algorithmic_tflops": v_[1] / (v_[0] * 1e-3) / 1e12}
@@ -1025,9 +1054,9 @@ def main():
     kms, kflops, ksrc = kernels[kname]
     achieved = kflops / (kms * 1e-3) / 1e12
     src = os.path.join(ROOT, "exact_blockwise_long_b200", "csrc", ksrc)
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    sha = code_fingerprint(src)
     tr = NCU_TRAFFIC.get((kname, args.workload))
-    traffic = tr["bytes"] if tr and tr["sha256"] == sha else None
+    traffic = tr["bytes"] if tr and tr["code_sha256"] == sha else None
     peak, peak_kind, other = tensor_peak(pk, ms_step * args.steps)
     roof = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": peak,
             "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,

@@ -7,24 +7,34 @@
 //   dV_j = sum_i P_ij dO_i            dS_ij = P_ij (dO_i . V_j - D_i)
 //   dK_j = scale sum_i dS_ij Q_i      dQ_i = scale sum_j dS_ij K_j
 //
-// Both sides of the ring: the key/value gradients keep a KV tile stationary
-// while the query shards pass by in ring order i = (j + t) mod S (the
-// forward's pairs, loop nest turned around); the query gradient keeps a
-// query tile stationary and visits the KV shards in ring order
-// j = (i - t) mod S, exactly like the forward.  Under the causal mask pairs
-// of shards in the future are skipped and the diagonal pair is masked inside
-// its tiles.  Each gradient accumulates in tensor memory and is written to
-// HBM once, so there are no atomics and the result is deterministic.
+// The default backward (ringattn_bwd) is three launches:
+//   preprocess  D_i = dO_i . O_i and lse_i * log2(e); zeroes the fp32 dQ
+//               accumulator                                         (HBM-bound)
+//   fused pass  a key/value tile stays on chip while the query shards pass
+//               by in ring order i = (j + t) mod S (the forward's pairs, loop
+//               nest turned around; under the causal mask pairs of shards in
+//               the future are skipped and the diagonal pair is masked inside
+//               its tiles).  Per (key tile, query tile) 5 tcgen05 MMAs:
+//                 S^T  = K Q^T, dP^T = V dO^T       (into TMEM)
+//                 dV  += P^T dO, dK += dS^T Q       (A operands from TMEM)
+//                 dQ^T = K^T dS^T (d = 128) or dQ = dS K (d = 64), added in
+//                 fp32 into the accumulator by a drain warpgroup
+//               dK and dV are written once per key tile; dQ sums over key
+//               tiles in arrival order (reproducible up to fp32 order).
+//   conversion  dq = bf16(accumulator)                               (HBM-bound)
 //
-// Three launches:
-//   preprocess  D_i = dO_i . O_i and lse_i * log2(e)             (HBM-bound)
+// The deterministic backward (ringattn_bwd_phase mask 7, ringattn_bwd_noalloc)
+// splits the work in two passes, each gradient accumulated in tensor memory
+// and written once (no additions in memory, every output bit-reproducible):
 //   dK/dV       per (key tile, query tile) 4 tcgen05 MMAs:
 //                 S^T  = K Q^T    (TMEM [0,128))
 //                 dP^T = V dO^T   (TMEM [128,256))
 //                 dV  += P^T dO   (P^T bf16 over S^T, A operand from TMEM)
 //                 dK  += dS^T Q   (dS^T bf16 over dP^T, A operand from TMEM)
-//   dQ          per (query tile, key tile) 3 tcgen05 MMAs, Q and dO held in
-//               TMEM as their A operands:
+//   dQ          the query tile stationary, the KV shards visited in ring
+//               order j = (i - t) mod S exactly like the forward; per
+//               (query tile, key tile) 3 tcgen05 MMAs, Q and dO held in TMEM
+//               as their A operands:
 //                 S    = Q K^T    (TMEM [0,128))
 //                 dP   = dO V^T   (TMEM [128,256))
 //                 dQ  += dS K     (dS bf16 over dP, A operand from TMEM)
