@@ -50,6 +50,8 @@ CASES = [
     (1, 1, 128, 128, 1, 128, 128, True),    # a single tile
     (1, 1, 2048, 128, 16, 128, 128, True),  # one tile per shard
     (1, 2, 1536, 64, 1, 512, 1536, True),   # no ring
+    (1, 1, 128, 64, 1, 128, 128, True),     # d = 64, a single tile: one dQ buffer used once
+    (1, 2, 1024, 64, 8, 128, 128, True),    # d = 64, one tile per shard: walks of 1 to 8 tiles
 ]
 
 
