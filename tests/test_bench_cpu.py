@@ -1,4 +1,5 @@
-"""bench.py host logic on CPU: the clock sampler against a fake NVML."""
+"""bench.py host logic on CPU: the clock sampler against a fake NVML, and the
+code fingerprint that ties the committed ncu traffic figures to kernel code."""
 
 import sys
 import time
@@ -82,3 +83,32 @@ def test_clocks_rejected_rules():
     assert bench.clocks_rejected({"sm_mhz": 1000.0, "sm_max_mhz": 1965.0, "reasons": []})
     # no samples at all is not a rejection
     assert not bench.clocks_rejected({"sm_mhz": None, "sm_max_mhz": None, "reasons": []})
+
+
+def test_code_fingerprint_ignores_comments_only(tmp_path):
+    src = tmp_path / "k.cu"
+    base = 'int f(int x) {\n  // a comment\n  return x + 1;  /* another */\n}\nconst char* s = "a // b /* c";\n'
+    src.write_text(base)
+    ref = bench.code_fingerprint(str(src))
+    # comments, blank lines and trailing blanks do not count
+    src.write_text(base.replace("// a comment", "// reworded, longer comment").replace("/* another */", "") + "\n\n")
+    assert bench.code_fingerprint(str(src)) == ref
+    src.write_text("/* header\n   block */\n" + base.replace("return x + 1;", "return x + 1;   "))
+    assert bench.code_fingerprint(str(src)) == ref
+    # code does, including text inside a string literal that looks like a comment
+    src.write_text(base.replace("x + 1", "x + 2"))
+    assert bench.code_fingerprint(str(src)) != ref
+    src.write_text(base.replace('"a // b /* c"', '"a // b /* d"'))
+    assert bench.code_fingerprint(str(src)) != ref
+
+
+def test_traffic_figures_match_the_kernel_code():
+    """Every committed ncu traffic figure names the code it was taken on; the
+    bench reports it only while that code is unchanged (null otherwise).  The
+    committed figures are for the current kernel sources."""
+    import os
+    root = os.path.dirname(bench.__file__)
+    for (kernel, _), entry in bench.NCU_TRAFFIC.items():
+        src = os.path.join(root, "exact_blockwise_long_b200", "csrc", "bwd_tc.cu" if kernel.startswith("bwd") else "fwd_tc.cu")
+        assert entry["code_sha256"] == bench.code_fingerprint(src), kernel
+
