@@ -41,15 +41,15 @@ def test_accumulate_and_cast_are_exact():
     assert ra.ringattn_get_error() == 0
 
 
-@pytest.mark.parametrize("S,causal", [(3, True), (4, True), (2, False)])
-def test_device_ops_over_an_emulated_ring(S, causal):
+@pytest.mark.parametrize("S,causal,D", [(3, True, 128), (4, True, 128), (2, False, 128), (3, True, 64), (2, False, 64)])
+def test_device_ops_over_an_emulated_ring(S, causal, D):
     """Each rank's schedule run in turn on one GPU: shard pairs in ring
     order with the causal skip and diagonal mask, exact merge, gradients
     summed per pair -- equal to full-sequence attention."""
     from exact_blockwise_long_b200.ring import DeviceOps
-    B, H, D, L = 1, 2, 128, 512
+    B, H, L = 1, 2, 512
     N = S * L
-    q, k, v, do = small_attention_inputs(B, H, N, D, 40 + S, k_scale=2.0 if causal else 1.0)
+    q, k, v, do = small_attention_inputs(B, H, N, D, 40 + S + D, k_scale=2.0 if causal else 1.0)
     ops = DeviceOps(128, 256)
     sh = lambda t, i: t[:, :, i * L:(i + 1) * L].contiguous()  # noqa: E731
     outs, lses = [], []
